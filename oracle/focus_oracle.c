@@ -1,0 +1,507 @@
+/*
+ * focus_oracle.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, scalar CPU reference of the FOCUS NVFP4 weight
+ * fake-quantizer: per-tensor scale s2, forward, straight-through backward for
+ * the scale parameters m and q, AdamW on m and q, and the NVFP4 export pack.
+ * Only the tests, the package's smoke check and the benchmark's CPU-baseline
+ * leg may load this code.  The CUDA library shares nothing with it: no header,
+ * table, helper or constant.
+ *
+ * Sources (page title, then the part of the page):
+ *  [card]  "FOCUS NVFP4 scales for Llama-3.2-1B-Instruct (our reproduction)",
+ *          section "What this is": the field table (m per 16-element block,
+ *          q per 8-element sub-block, s2 = amax(|W|)/(6*448)), the row-major
+ *          layout sentence, and the three equations for S_b, c_i and w'_i with
+ *          the two rules after them (E2M1 rounds to nearest, ties to even; a
+ *          block whose scaled maximum is 0 gets scale 1 before the clamp).
+ *          Section "Calibration": AdamW, betas 0.9/0.999, weight decay 0,
+ *          lr 5e-3 for m and 1e-3 for q, m starts at 1 and q at 6.
+ *  [gist]  "Technische Samenvatting: FOCUS ...", section "Methodologie",
+ *          item 1 (scales learned through the straight-through estimator).
+ *
+ * Readings of points the pages leave open (each also listed in the design
+ * notes of the repository):
+ *  - Forward arithmetic is IEEE binary32, round to nearest even, one rounding
+ *    per operation, no fused multiply-add: m, q and s2 are FP32 on the card,
+ *    and a code that depends on a rounding must be decided in the same
+ *    precision on both sides.  Build with -ffp-contract=off.
+ *  - x_b = fl(fl(A_b*m_b) / fl(6*s2)); "scaled maximum is 0" means x_b == 0.
+ *  - e4m3() is round to nearest even (the plain cast).
+ *  - sigmoid(q) is the binary32 rounding of 1/(1+exp(-q)) evaluated in
+ *    binary64.
+ *  - y_i = fl(w_i / D_k) with D_k = fl(fl(S_b*sigma_k)*s2);
+ *    w'_i = bf16_rne(fl(fl(c_i*S_b)*s2)).
+ *  - E2M1 keeps the sign of zero: a negative input that rounds to 0 gives
+ *    code 0x8 and w' = -0.0.
+ *  - Straight-through backward: rounding is the identity inside the clamps,
+ *    clamps pass the gradient at their end points and block it outside,
+ *    and the substitution x == 0 -> 1 blocks it.  The gradient sums are
+ *    accumulated in binary64 and rounded to binary32 once.
+ *  - AdamW follows the algorithm with decoupled weight decay and bias
+ *    correction, step counted from 1, eps 1e-8; evaluated in binary64 from
+ *    the binary32 inputs, results rounded to binary32.
+ *  - NVFP4 byte layout: element 2j in the low nibble and 2j+1 in the high
+ *    nibble of byte j of a row; one E4M3 byte per block, row-major
+ *    [out, in/16]; the tensor scale stored is s2 itself.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define FO_OK 0
+#define FO_ERR_SHAPE 1
+#define FO_ERR_VALUE 2
+#define FO_ERR_NONFINITE 3
+
+/* ------------------------------------------------------------------------ */
+/* scalar formats                                                            */
+/* ------------------------------------------------------------------------ */
+
+static float f32_from_bits(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t bits_from_f32(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* bf16 is the upper half of a binary32. */
+float fo_bf16_to_f32(uint16_t h) { return f32_from_bits((uint32_t)h << 16); }
+
+/* Round a binary32 to bf16, nearest with ties to even, by looking at the
+ * 16 bits that are dropped. */
+uint16_t fo_f32_to_bf16(float f)
+{
+    uint32_t u = bits_from_f32(f);
+    if (isnan(f)) return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t keep = u >> 16;
+    uint32_t dropped = u & 0xFFFFu;
+    if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u)))
+        keep += 1u; /* the next bf16 up in magnitude (may become inf) */
+    return (uint16_t)keep;
+}
+
+/* Nearest integer to v >= 0, ties to the even integer. */
+static double round_half_even(double v)
+{
+    double lo = floor(v);
+    double frac = v - lo;
+    if (frac > 0.5) return lo + 1.0;
+    if (frac < 0.5) return lo;
+    return (fmod(lo, 2.0) == 0.0) ? lo : lo + 1.0;
+}
+
+/* E4M3 ("fn": bias 7, no infinities, 0x7F/0xFF are NaN, max 448) decode. */
+double fo_e4m3_decode(int byte)
+{
+    int sign = (byte >> 7) & 1;
+    int e = (byte >> 3) & 0xF;
+    int mant = byte & 7;
+    double v;
+    if (e == 15 && mant == 7) return NAN;
+    if (e == 0) v = ldexp((double)mant, -9);               /* subnormal: mant * 2^-9 */
+    else v = ldexp(1.0 + mant / 8.0, e - 7);                /* normal */
+    return sign ? -v : v;
+}
+
+/* E4M3 encode of a non-negative finite x: round to nearest, ties to even,
+ * values above 448 saturate to 448.  Returns -1 outside the domain.  The
+ * quantizer only ever passes x in [2^-6, 448] (the clamp of the S_b
+ * equation), where every result is a normal number. */
+int fo_e4m3_encode(float xf)
+{
+    double x = (double)xf;
+    if (!(x >= 0.0) || isinf(x)) return -1;
+    if (x > 448.0) return 0x7E;
+    if (x < ldexp(1.0, -6)) {
+        double k = round_half_even(x / ldexp(1.0, -9));     /* 0..8 */
+        return (int)k;                                      /* k == 8 is 2^-6 = 0x08 */
+    }
+    int E;
+    frexp(x, &E);                 /* x = f * 2^E, f in [0.5, 1) */
+    int e = E - 1;                /* x in [2^e, 2^(e+1)) */
+    double k = round_half_even(ldexp(x, -e) * 8.0);         /* 8..16 */
+    if (k == 16.0) { e += 1; k = 8.0; }
+    if (e > 8 || (e == 8 && k > 14.0)) return 0x7E;        /* cannot happen for x <= 448 */
+    return ((e + 7) << 3) | ((int)k - 8);
+}
+
+/* E2M1 magnitudes by code 0..7. */
+static const double e2m1_mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double fo_e2m1_decode(int code)
+{
+    double v = e2m1_mag[code & 7];
+    return (code & 8) ? -v : v;
+}
+
+/* E2M1 encode of u in [-6, 6]: nearest magnitude, ties to the even code
+ * (the card's "ties to even"); the sign bit is kept, so -0.1 gives 0x8.
+ * The seven midpoints between neighbouring magnitudes decide the code: the
+ * code is the number of midpoints below |u|, and at a midpoint the even of
+ * the two neighbouring codes wins.  Magnitudes above 6 saturate to 6. */
+int fo_e2m1_encode(float uf)
+{
+    static const double mid[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+    double a = fabs((double)uf);
+    int sign = signbit(uf) ? 8 : 0;
+    int code = 0;
+    for (int j = 0; j < 7; ++j) {
+        if (a > mid[j]) code = j + 1;
+        else if (a == mid[j]) code = ((j & 1) == 0) ? j : j + 1; /* even of j, j+1 */
+    }
+    return sign | code;
+}
+
+/* sigmoid(q) as a binary32: 1/(1+exp(-q)) in binary64, rounded once. */
+float fo_sigmoid(float q)
+{
+    double e = exp(-(double)q);
+    return (float)(1.0 / (1.0 + e));
+}
+
+/* ------------------------------------------------------------------------ */
+/* the quantizer, block by block                                             */
+/* ------------------------------------------------------------------------ */
+
+/* Everything the forward decides for one 16-element block. */
+typedef struct {
+    float A;          /* max |w| over the block */
+    float x;          /* fl(fl(A*m)/fl(6*s2)), before the zero rule and the clamp */
+    int inS;          /* 1 when the clamp of S_b passes the gradient */
+    int sb;           /* E4M3 byte of S_b */
+    float S;          /* value of S_b */
+    float sigma[2];   /* sigmoid(q_k) for the two sub-blocks */
+    float D[2];       /* fl(fl(S*sigma_k)*s2) */
+    float y[16];      /* fl(w_i / D_k) */
+    int in[16];       /* 1 when -6 <= y_i <= 6 */
+    int code[16];     /* E2M1 code of clamp(y_i, -6, 6) */
+    float c[16];      /* its value */
+    float wq[16];     /* fl(fl(c*S)*s2) before the bf16 cast */
+    int band[16];     /* 1: |y| within 2^-20 relative of a code boundary or of 6; 2: exactly on a midpoint */
+} fo_block;
+
+/* Boundaries of the code decision and of the clamp, in |y|. */
+static const double y_edges[8] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0};
+
+static int band_of(float y)
+{
+    double a = fabs((double)y);
+    for (int j = 0; j < 8; ++j) {
+        if (a == y_edges[j] && j < 7) return 2;
+        if (fabs(a - y_edges[j]) <= ldexp(y_edges[j], -20)) return 1;
+    }
+    return 0;
+}
+
+/* The three equations of the card for one block of 16 weights w (given as
+ * bf16 bits), with its block factor m_b and its two sub-block logits q2. */
+static void quantize_block(const uint16_t *w16, float m_b, const float *q2, float s2, fo_block *B)
+{
+    float w[16];
+    float A = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        w[i] = fo_bf16_to_f32(w16[i]);
+        float a = fabsf(w[i]);
+        if (a > A) A = a;
+    }
+    B->A = A;
+
+    /* S_b = e4m3(clamp(max|w_b| * m_b / (6*s2), 2^-6, 448)); scale 1 when the scaled max is 0 */
+    float num = A * m_b;
+    float den = 6.0f * s2;
+    float x = num / den;
+    B->x = x;
+    B->inS = (x != 0.0f) && (x >= 0x1p-6f) && (x <= 448.0f);
+    float xc = x;
+    if (xc == 0.0f) xc = 1.0f;
+    if (xc < 0x1p-6f) xc = 0x1p-6f;
+    if (xc > 448.0f) xc = 448.0f;
+    B->sb = fo_e4m3_encode(xc);
+    B->S = (float)fo_e4m3_decode(B->sb);
+
+    /* c_i = E2M1(clamp(w_i / (S_b * sigmoid(q_k) * s2), -6, 6)); w'_i = c_i * S_b * s2 */
+    for (int k = 0; k < 2; ++k) {
+        float sig = fo_sigmoid(q2[k]);
+        float Ssig = B->S * sig;
+        float D = Ssig * s2;
+        B->sigma[k] = sig;
+        B->D[k] = D;
+        for (int j = 0; j < 8; ++j) {
+            int i = 8 * k + j;
+            float y = w[i] / D;
+            float u = y;
+            if (u < -6.0f) u = -6.0f;
+            if (u > 6.0f) u = 6.0f;
+            B->y[i] = y;
+            B->in[i] = (y >= -6.0f) && (y <= 6.0f);
+            B->code[i] = fo_e2m1_encode(u);
+            B->c[i] = (float)fo_e2m1_decode(B->code[i]);
+            float cS = B->c[i] * B->S;
+            B->wq[i] = cS * s2;
+            B->band[i] = band_of(y);
+        }
+    }
+}
+
+/* Straight-through gradients of one block, given the upstream gradient g of
+ * w' (bf16 bits).  With y = w/(S*sigma*s2), c = R(clamp(y)), dR/du = 1,
+ * S = E4M3(clamp(x)) with dE/dx = 1 and x = A*m/(6*s2):
+ *   dw'/dS = s2*(c - in*y),   dS/dm = inS*A/(6*s2)
+ *     => dL/dm = inS * (A/6) * sum_i g_i*(c_i - in_i*y_i)
+ *   dw'/dsigma = -in*S*s2*y/sigma,   dsigma/dq = sigma*(1-sigma)
+ *     => dL/dq_k = -(1-sigma_k) * S * s2 * sum_{i in k} in_i*g_i*y_i          */
+static void block_grads(const fo_block *B, const uint16_t *g16, float s2, double *dm, double dq[2])
+{
+    double sm = 0.0;
+    double sq[2] = {0.0, 0.0};
+    for (int i = 0; i < 16; ++i) {
+        double g = (double)fo_bf16_to_f32(g16[i]);
+        double t = B->in[i] ? ((double)B->c[i] - (double)B->y[i]) : (double)B->c[i];
+        sm += g * t;
+        if (B->in[i]) sq[i / 8] += g * (double)B->y[i];
+    }
+    *dm = B->inS ? ((double)B->A / 6.0) * sm : 0.0;
+    for (int k = 0; k < 2; ++k)
+        dq[k] = -(1.0 - (double)B->sigma[k]) * (double)B->S * (double)s2 * sq[k];
+}
+
+static int check_shape(int64_t out, int64_t in)
+{
+    if (out < 0 || in < 0 || (in % 16) != 0) return FO_ERR_SHAPE;
+    return FO_OK;
+}
+
+static int check_s2(float s2)
+{
+    if (!(s2 > 0.0f) || isinf(s2)) return FO_ERR_VALUE;
+    return FO_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* public entry points (used through ctypes by the tests)                    */
+/* ------------------------------------------------------------------------ */
+
+int fo_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void fo_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* s2 = amax(|W|) / (6*448), one binary32 division (6*448 = 2688 exactly).
+ * Card, field table, row s2. */
+int fo_s2(const uint16_t *W, int64_t n, float *s2_out)
+{
+    float A = 0.0f;
+    int bad = 0;
+#pragma omp parallel for reduction(max : A) reduction(| : bad)
+    for (int64_t i = 0; i < n; ++i) {
+        float w = fo_bf16_to_f32(W[i]);
+        if (!isfinite(w)) bad = 1;
+        float a = fabsf(w);
+        if (a > A) A = a;
+    }
+    if (bad) return FO_ERR_NONFINITE;
+    *s2_out = A / 2688.0f;
+    return FO_OK;
+}
+
+/* Counters the forward reports. */
+typedef struct {
+    int64_t zero_blocks;   /* x == 0 (scale forced to 1) */
+    int64_t clamp_low;     /* 0 < x < 2^-6, or x < 0 */
+    int64_t clamp_high;    /* x > 448 */
+    int64_t out_of_range;  /* |y| > 6 */
+    int64_t band;          /* |y| within 2^-20 relative of a boundary (ties included) */
+    int64_t exact_ties;    /* |y| exactly on one of the seven midpoints */
+} fo_stats;
+
+/* Forward over a row-major [out, in] tensor.  Every output may be NULL.
+ *   Wq     bf16 bits [out, in]   w'
+ *   codes  u8 [out, in]          one E2M1 code per element (unpacked)
+ *   scales u8 [out, in/16]       E4M3 byte of S_b
+ *   band   u8 [out, in]          0 / 1 (near a boundary) / 2 (exactly on a midpoint)
+ *   ys     f32 [out, in]         y_i = w_i / D_k                                       */
+int fo_fwd(const uint16_t *W, const float *m, const float *q, float s2, int64_t out, int64_t in,
+           uint16_t *Wq, uint8_t *codes, uint8_t *scales, uint8_t *band, float *ys, fo_stats *st)
+{
+    int rc = check_shape(out, in);
+    if (rc) return rc;
+    if ((rc = check_s2(s2))) return rc;
+    const int64_t nb = in / 16;
+    int64_t zb = 0, lo = 0, hi = 0, oor = 0, bd = 0, ties = 0;
+    int bad = 0;
+#pragma omp parallel for reduction(+ : zb, lo, hi, oor, bd, ties) reduction(| : bad) schedule(static)
+    for (int64_t r = 0; r < out; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t blk = r * nb + b;
+            const int64_t e0 = r * in + 16 * b;
+            if (!isfinite(m[blk]) || !isfinite(q[2 * blk]) || !isfinite(q[2 * blk + 1])) bad = 1;
+            for (int i = 0; i < 16; ++i)
+                if (!isfinite(fo_bf16_to_f32(W[e0 + i]))) bad = 1;
+            fo_block B;
+            quantize_block(W + e0, m[blk], q + 2 * blk, s2, &B);
+            if (B.x == 0.0f) zb++;
+            else if (B.x < 0x1p-6f) lo++;
+            else if (B.x > 448.0f) hi++;
+            if (scales) scales[blk] = (uint8_t)B.sb;
+            for (int i = 0; i < 16; ++i) {
+                if (!B.in[i]) oor++;
+                if (B.band[i]) bd++;
+                if (B.band[i] == 2) ties++;
+                if (Wq) Wq[e0 + i] = fo_f32_to_bf16(B.wq[i]);
+                if (codes) codes[e0 + i] = (uint8_t)B.code[i];
+                if (band) band[e0 + i] = (uint8_t)B.band[i];
+                if (ys) ys[e0 + i] = B.y[i];
+            }
+        }
+    }
+    if (bad) return FO_ERR_NONFINITE;
+    if (st) {
+        st->zero_blocks = zb; st->clamp_low = lo; st->clamp_high = hi;
+        st->out_of_range = oor; st->band = bd; st->exact_ties = ties;
+    }
+    return FO_OK;
+}
+
+/* Straight-through backward: dm [out, in/16], dq [out, in/8] as binary32.
+ * accumulate = 1 adds to what dm and dq hold (the sum is formed in binary64
+ * and rounded once). */
+int fo_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, const float *q, float s2,
+               int64_t out, int64_t in, float *dm, float *dq, int accumulate)
+{
+    int rc = check_shape(out, in);
+    if (rc) return rc;
+    if ((rc = check_s2(s2))) return rc;
+    const int64_t nb = in / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < out; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t blk = r * nb + b;
+            const int64_t e0 = r * in + 16 * b;
+            fo_block B;
+            quantize_block(W + e0, m[blk], q + 2 * blk, s2, &B);
+            double gm, gq[2];
+            block_grads(&B, dWq + e0, s2, &gm, gq);
+            if (accumulate) {
+                dm[blk] = (float)((double)dm[blk] + gm);
+                dq[2 * blk] = (float)((double)dq[2 * blk] + gq[0]);
+                dq[2 * blk + 1] = (float)((double)dq[2 * blk + 1] + gq[1]);
+            } else {
+                dm[blk] = (float)gm;
+                dq[2 * blk] = (float)gq[0];
+                dq[2 * blk + 1] = (float)gq[1];
+            }
+        }
+    }
+    return FO_OK;
+}
+
+/* AdamW with decoupled weight decay (Loshchilov & Hutter), bias-corrected
+ * moments, step t counted from 1:
+ *   p   <- p * (1 - lr*wd)
+ *   v1  <- b1*v1 + (1-b1)*g
+ *   v2  <- b2*v2 + (1-b2)*g^2
+ *   p   <- p - (lr/(1-b1^t)) * v1 / (sqrt(v2)/sqrt(1-b2^t) + eps)
+ * Card, "Calibration": betas 0.9/0.999, weight decay 0, constant lr. */
+int fo_adamw(float *p, const float *g, float *v1, float *v2, int64_t n, double lr, double b1, double b2,
+             double eps, double wd, int64_t step)
+{
+    if (n < 0) return FO_ERR_SHAPE;
+    if (step < 1 || !(lr >= 0.0) || !(eps >= 0.0) || !(b1 >= 0.0 && b1 < 1.0) || !(b2 >= 0.0 && b2 < 1.0))
+        return FO_ERR_VALUE;
+    const double bc1 = 1.0 - pow(b1, (double)step);
+    const double bc2 = 1.0 - pow(b2, (double)step);
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        double pi = (double)p[i] * (1.0 - lr * wd);
+        double gi = (double)g[i];
+        double a = b1 * (double)v1[i] + (1.0 - b1) * gi;
+        double s = b2 * (double)v2[i] + (1.0 - b2) * gi * gi;
+        pi -= (lr / bc1) * a / (sqrt(s) / sqrt(bc2) + eps);
+        v1[i] = (float)a;
+        v2[i] = (float)s;
+        p[i] = (float)pi;
+    }
+    return FO_OK;
+}
+
+/* One calibration step of one tensor, as the composition of the three parts
+ * above: forward (w' written when Wq is not NULL), straight-through backward
+ * (added to dm_acc / dq_acc when they are not NULL), then AdamW on m and q.
+ * gm_out / gq_out (may be NULL) receive the binary32 gradients used. */
+int fo_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, float *m_v1, float *m_v2,
+            float *q_v1, float *q_v2, float s2, int64_t out, int64_t in, double lr_m, double lr_q,
+            double b1, double b2, double eps, double wd, int64_t step, uint16_t *Wq,
+            const float *dm_acc, const float *dq_acc, float *gm_out, float *gq_out)
+{
+    int rc = check_shape(out, in);
+    if (rc) return rc;
+    if ((rc = check_s2(s2))) return rc;
+    const int64_t nb = out * (in / 16);
+    float *gm = gm_out, *gq = gq_out;
+    float *own = NULL;
+    if (!gm || !gq) {
+        own = (float *)malloc(sizeof(float) * 3 * (size_t)(nb > 0 ? nb : 1));
+        if (!own) return FO_ERR_VALUE;
+        gm = own;
+        gq = own + nb;
+    }
+    if (Wq) {
+        rc = fo_fwd(W, m, q, s2, out, in, Wq, NULL, NULL, NULL, NULL, NULL);
+        if (rc) goto done;
+    }
+    if (dm_acc && dq_acc) {
+        memcpy(gm, dm_acc, sizeof(float) * (size_t)nb);
+        memcpy(gq, dq_acc, sizeof(float) * 2 * (size_t)nb);
+        rc = fo_ste_bwd(W, dWq, m, q, s2, out, in, gm, gq, 1);
+    } else {
+        rc = fo_ste_bwd(W, dWq, m, q, s2, out, in, gm, gq, 0);
+    }
+    if (rc) goto done;
+    rc = fo_adamw(m, gm, m_v1, m_v2, nb, lr_m, b1, b2, eps, wd, step);
+    if (rc) goto done;
+    rc = fo_adamw(q, gq, q_v1, q_v2, 2 * nb, lr_q, b1, b2, eps, wd, step);
+done:
+    free(own);
+    return rc;
+}
+
+/* NVFP4 export: codes u8 [out, in/2] (element 2j low nibble, 2j+1 high),
+ * scales u8 [out, in/16] (E4M3 bytes of S_b), tensor scale = s2.
+ * Card, "What this is": E2M1 elements, one E4M3 scale per 16 elements, one
+ * FP32 scale per tensor. */
+int fo_pack(const uint16_t *W, const float *m, const float *q, float s2, int64_t out, int64_t in,
+            uint8_t *codes, uint8_t *scales, float *tensor_scale)
+{
+    int rc = check_shape(out, in);
+    if (rc) return rc;
+    if ((rc = check_s2(s2))) return rc;
+    const int64_t nb = in / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < out; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t blk = r * nb + b;
+            const int64_t e0 = r * in + 16 * b;
+            fo_block B;
+            quantize_block(W + e0, m[blk], q + 2 * blk, s2, &B);
+            scales[blk] = (uint8_t)B.sb;
+            for (int j = 0; j < 8; ++j)
+                codes[e0 / 2 + j] = (uint8_t)((B.code[2 * j] & 0xF) | ((B.code[2 * j + 1] & 0xF) << 4));
+        }
+    }
+    *tensor_scale = s2;
+    return FO_OK;
+}
