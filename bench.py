@@ -1,0 +1,438 @@
+"""Benchmark of the FOCUS NVFP4 weight fake-quantizer on B200.
+
+Workload: every linear weight of Llama-3.1-8B (32 layers x q, k, v, o, gate,
+up, down: 224 tensors, 6,979,321,856 weights), synthetic: W ~ N(0, 0.02) bf16,
+m = 1, q = 6, dW' ~ N(0, 1e-3) bf16, zero AdamW moments at step 1.  One step
+is one pass of the whole hot path over all 224 tensors:
+  s2 of every tensor (two launches),
+  the fused forward + straight-through backward + AdamW step (one launch,
+  W' written, W read once),
+  the NVFP4 export pack of the updated parameters (one launch).
+Metric: Gelem/s = weights per second of whole steps (all ranks).  The
+roofline object reports the fused step kernel against the measured HBM copy
+bandwidth.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 it is launched by torch.distributed.run, one rank per GPU; every
+rank steps its own model (seeded by rank: weak scaling, no data-path
+collective), the time is the max over ranks.  The reference arm times the CPU
+oracle on the host cores (rank 0 only), on a bounded row sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Gelem/s FOCUS fwd+STE-bwd+AdamW and % of B200 HBM roofline (ncu)"
+WORKLOAD = "Llama-3.1-8B all 224 linear weights (32 layers x q,o[4096,4096] k,v[1024,4096] " \
+           "gate,up[14336,4096] down[4096,14336]); step = s2 + fused fwd/STE-bwd/AdamW (W' written) + NVFP4 pack"
+# algorithmic bytes per weight of one step: s2 reads W (2); the fused step reads W, dW' (2+2), m (0.25),
+# q (0.5), four moments (1.5) and writes W' (2), m, q, moments (2.25); the pack reads W, m, q (2.75) and
+# writes codes (0.5) and scales (0.0625)
+BYTES_S2 = 2.0
+BYTES_STEP = 10.5
+BYTES_PACK = 3.3125
+KERNEL_SOURCES = ("fp4_post_weight_b200/csrc/focus_kernels.cuh", "fp4_post_weight_b200/csrc/focus_capi.cu")
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the fused step kernel from the committed ncu summary,
+    valid only while the kernel sources are unchanged."""
+    p = os.path.join(ROOT, "profiles", "focus_step_fused_llama8b.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch_full_workload")
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def init_dist(world, local):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = "clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," \
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except Exception:
+            self.proc.kill()
+        self.out.flush()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.out.name) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) < 8:
+                    continue
+                try:
+                    sm.append(float(p[0])); mx.append(float(p[1]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, p[4:8]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.out.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the workload
+# ---------------------------------------------------------------------------
+
+def build_model(rank: int, device):
+    import torch
+
+    from fp4_post_weight_b200 import dist as D
+    import synth
+    from fp4_post_weight_b200.table import Entry
+    ents = []
+    for j, (_, sh) in enumerate(synth.LLAMA_8B.tensors()):
+        t = synth.llama_8b_tensor(j, sh, device, seed_base=D.seed_base(rank))
+        o, i = sh
+        e = Entry(W=t.W, m=t.m, q=t.q, s2=torch.zeros(1, device=device), dWq=t.dWq,
+                  Wq=torch.empty_like(t.W), m_exp_avg=torch.zeros_like(t.m), m_exp_avg_sq=torch.zeros_like(t.m),
+                  q_exp_avg=torch.zeros_like(t.q), q_exp_avg_sq=torch.zeros_like(t.q),
+                  codes=torch.empty((o, i // 2), dtype=torch.uint8, device=device),
+                  scales=torch.empty((o, i // 16), dtype=torch.uint8, device=device))
+        ents.append(e)
+    return ents
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import synth
+    from fp4_post_weight_b200 import dist as D
+    from fp4_post_weight_b200 import focus as F
+    from fp4_post_weight_b200.table import FocusTable, hparams
+
+    init_dist(world, local)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ents = build_model(rank, dev)
+    N = synth.LLAMA_8B.n_elements()
+    # the step writes W' (no codes: the export pack after the update writes those)
+    step_tab = FocusTable([dataclasses.replace(e, codes=None, scales=None) for e in ents])
+    pack_tab = FocusTable(ents)
+    hp = hparams()
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+
+    t_counter = [0]
+
+    def one_step(ev=None):
+        t_counter[0] += 1
+        step_tab.s2()
+        if ev is not None:
+            ev[0].record(stream)
+        step_tab.step(t_counter[0], hp)
+        if ev is not None:
+            ev[1].record(stream)
+        pack_tab.pack()
+
+    for _ in range(args.warmup):
+        one_step()
+    st = F.focus_get_error()
+    if st != 0:
+        raise SystemExit(f"device status after warm-up: {F.focus_status_string(st)}")
+    torch.cuda.synchronize()
+    D.barrier()
+
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid).replace("GPU-", "")
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    D.barrier()
+    start.record(stream)
+    for k in range(args.steps):
+        one_step(kev[k])
+    end.record(stream)
+    torch.cuda.synchronize()
+    D.barrier()
+    clk = clocks.stop()
+    ms = start.elapsed_time(end)
+    step_kernel_ms = sum(a.elapsed_time(b) for a, b in kev) / args.steps
+    ms_max = D.max_over_ranks(ms)
+    st = F.focus_get_error()
+    if st != 0:
+        raise SystemExit(f"device status after timing: {F.focus_status_string(st)}")
+    ms_per_step = ms_max / args.steps
+    value = N * world / (ms_per_step * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, ents, N, world, dev)
+
+    peaks = measured_peaks()
+    achieved = N * BYTES_STEP / (step_kernel_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "kernel": "tile_kernel<KIND_STEP> (focus_step_fused)", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)",
+            "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(),
+            "bytes_per_elem": BYTES_STEP, "launch_ms": round(step_kernel_ms, 4)}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.cpu_seconds)
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 2), "unit": "Gelem/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded N(0,0.02) bf16 weights of the Llama-3.1-8B linear shapes; "
+                        "no checkpoint)",
+                "config": {"workload": WORKLOAD, "tensors": len(ents), "elements_per_gpu": N,
+                           "l2": "inputs larger than L2 (57.6 GB resident per GPU vs 126 MB L2)",
+                           "parallelism": f"dp{world} (one model per GPU, no collective)",
+                           "bytes_per_elem_step": BYTES_S2 + BYTES_STEP + BYTES_PACK},
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": 4 * args.steps, "clocks": clk,
+                "kernel_ms": {"fused_step": round(step_kernel_ms, 4)}}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(args, ents, N, world, dev):
+    """The same step through the C ABI with host buffers: per step every input
+    (W, dW', m, q, moments) is copied from pinned host memory and every output
+    (W', m, q, moments, codes, scales, s2) is copied back, tensor by tensor on
+    two copy streams overlapping the compute stream."""
+    import torch
+
+    from fp4_post_weight_b200 import dist as D
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    ins = ("W", "dWq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq")
+    outs = ("Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq", "codes", "scales", "s2")
+    hosts = []
+    for e in ents:
+        h = {}
+        for n in set(ins) | set(outs):
+            t = getattr(e, n)
+            h[n] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            h[n].copy_(t)
+        hosts.append(h)
+    tabs = [FocusTable([e]) for e in ents]
+    h2d, comp, d2h = torch.cuda.Stream(dev), torch.cuda.current_stream(dev), torch.cuda.Stream(dev)
+    hp = hparams()
+    bi = sum(h[n].numel() * h[n].element_size() for h in hosts for n in ins)
+    bo = sum(h[n].numel() * h[n].element_size() for h in hosts for n in outs)
+
+    def step(t):
+        done_in, done_c = [], []
+        for e, h in zip(ents, hosts):
+            with torch.cuda.stream(h2d):
+                for n in ins:
+                    getattr(e, n).copy_(h[n], non_blocking=True)
+                ev = torch.cuda.Event(); ev.record(h2d); done_in.append(ev)
+        for e, tab, ev in zip(ents, tabs, done_in):
+            comp.wait_event(ev)
+            tab.s2(stream=comp)
+            tab.step(t, hp, stream=comp)
+            tab.pack(stream=comp)
+            ec = torch.cuda.Event(); ec.record(comp); done_c.append(ec)
+        for e, h, ec in zip(ents, hosts, done_c):
+            d2h.wait_event(ec)
+            with torch.cuda.stream(d2h):
+                for n in outs:
+                    h[n].copy_(getattr(e, n), non_blocking=True)
+        # the next step's uploads must not overwrite tensors still being read back
+        h2d.wait_stream(d2h)
+
+    steps = max(1, args.e2e_steps)
+    step(1)
+    torch.cuda.synchronize()
+    D.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(h2d)
+    for k in range(steps):
+        step(2 + k)
+    d2h.synchronize()
+    e.record(d2h)
+    torch.cuda.synchronize()
+    ms = D.max_over_ranks(s.elapsed_time(e)) / steps
+    del hosts
+    return {"value": round(N * world / (ms * 1e-3) / 1e9, 3), "unit": "Gelem/s", "h2d_bytes_per_step": bi,
+            "d2h_bytes_per_step": bo, "ms_per_step": round(ms, 2), "steps": steps}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_inputs(rows: int, seed: int = 0):
+    """A row sample of the Llama-3.1-8B shapes: `rows` rows of each of the seven
+    projection shapes, generated on the host with the workload's recipe."""
+    import numpy as np
+
+    import synth
+    res = []
+    for j, (_, (o, i)) in enumerate(synth.LLAMA_8B.layer_shapes()):
+        t = synth.llama_8b_tensor(1000 + j + seed, (rows, i), "cpu")
+        z = np.zeros((rows, i // 16), np.float32)
+        zq = np.zeros((rows, i // 8), np.float32)
+        res.append([synth.bits(t.W), synth.bits(t.dWq), t.m.numpy().copy(), t.q.numpy().copy(),
+                    z.copy(), z.copy(), zq.copy(), zq.copy()])
+    return res
+
+
+def oracle_step(sample):
+    import oracle
+    n = 0
+    for W, G, m, q, a, b, c, d in sample:
+        s2 = oracle.s2(W)
+        oracle.step(W, G, m, q, a, b, c, d, s2, 1, want_wq=True)
+        oracle.pack(W, m, q, s2)
+        n += W.size
+    return n
+
+
+def cpu_baseline(seconds: float) -> dict:
+    import oracle
+    oracle.build()
+    threads = oracle.num_threads()
+    rows = 16
+    t0 = time.time()
+    n = oracle_step(oracle_sample_inputs(rows))
+    dt = time.time() - t0
+    # scale the sample to about `seconds` of work
+    rows = max(16, int(rows * seconds / max(dt, 1e-3)))
+    rows = min(rows, 4096)
+    sample = oracle_sample_inputs(rows)
+    t0 = time.time()
+    n = oracle_step(sample)
+    dt = time.time() - t0
+    return {"value": round(n / dt / 1e9, 5), "unit": "Gelem/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows} rows of each Llama-3.1-8B projection shape ({n} weights): s2 + fwd + "
+                      f"STE-bwd + AdamW + pack, {dt:.1f} s on {threads} OpenMP threads"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    threads = oracle.num_threads()
+    rows = 16
+    t0 = time.time()
+    oracle_step(oracle_sample_inputs(rows))
+    dt = time.time() - t0
+    per_step = args.reference_seconds
+    rows = min(4096, max(16, int(rows * per_step / max(dt, 1e-3))))
+    for w in range(args.warmup):
+        oracle_step(oracle_sample_inputs(rows, seed=w))
+    samples = [oracle_sample_inputs(rows, seed=100 + k) for k in range(args.steps)]
+    t0 = time.time()
+    n = 0
+    for smp in samples:
+        n += oracle_step(smp)
+    dt = time.time() - t0
+    value = n / dt / 1e9
+    desc = (f"{rows} rows of each Llama-3.1-8B projection shape per step: s2 + fwd + STE-bwd + AdamW + pack "
+            f"on {threads} OpenMP threads")
+    line = {"metric": METRIC, "value": round(value, 5), "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64-accumulate/f32", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample_rows_per_shape": rows},
+            "cpu_baseline": {"value": round(value, 5), "unit": "Gelem/s", "cores": threads, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(value, 5), "unit": "Gelem/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=4.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: at least 3 warm-up steps are used", file=sys.stderr)
+        args.warmup = 3
+    from fp4_post_weight_b200 import dist as D
+    world, rank, local = D.env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

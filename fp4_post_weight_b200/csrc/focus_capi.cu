@@ -1,0 +1,365 @@
+// focus_capi.cu -- the extern "C" boundary of libfocus.so (declared in focus.h).
+//
+// Every entry point checks its arguments on the host, then enqueues kernels on
+// the caller's stream; nothing is allocated and nothing synchronizes except
+// focus_get_error().  Launch sizes: a persistent grid of (SM count) x (CTAs
+// resident per SM, from the occupancy calculator), cached per device.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "focus.h"
+#include "focus_kernels.cuh"
+
+namespace focus {
+
+static_assert(sizeof(focus_tensor_desc) == 144, "descriptor layout is part of the ABI");
+
+namespace {
+
+constexpr int MAX_DEVICES = 64;
+
+struct DeviceInfo {
+    int sms = 0;
+    int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_amax = 0, occ_adam = 0;
+};
+
+std::once_flag g_once[MAX_DEVICES];
+DeviceInfo g_info[MAX_DEVICES];
+
+int device_info(DeviceInfo **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return FOCUS_ERR_CUDA;
+    std::call_once(g_once[dev], [dev] {
+        DeviceInfo &d = g_info[dev];
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_fwd, tile_kernel<KIND_FWD>, THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_bwd, tile_kernel<KIND_BWD>, THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_step, tile_kernel<KIND_STEP>, THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_amax, amax_tiles_kernel, THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_adam, adamw_kernel, THREADS, 0);
+    });
+    DeviceInfo &d = g_info[dev];
+    if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0)
+        return FOCUS_ERR_CUDA;
+    *out = &d;
+    return FOCUS_OK;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int64_t out, int64_t in) {
+    if (out < 0 || in < 0 || (in % 16) != 0) return FOCUS_ERR_SHAPE;
+    if (in > 0 && out > (INT64_C(1) << 58) / in) return FOCUS_ERR_SHAPE;
+    return FOCUS_OK;
+}
+
+int check_s2(float s2) { return (s2 > 0.0f && std::isfinite(s2)) ? FOCUS_OK : FOCUS_ERR_VALUE; }
+
+int64_t tiles_of(int64_t out, int64_t in) {
+    const int64_t nblk = out * (in / 16);
+    return (nblk + TILE_BLOCKS - 1) / TILE_BLOCKS;
+}
+
+int64_t grid_for(int64_t tiles, int sms, int occ) {
+    int64_t g = (int64_t)sms * occ;
+    return tiles < g ? tiles : g;
+}
+
+int launch_status() {
+    return cudaGetLastError() == cudaSuccess ? FOCUS_OK : FOCUS_ERR_CUDA;
+}
+
+focus_tensor_desc one_desc(const uint16_t *W, const uint16_t *dWq, uint16_t *Wq, const float *m, const float *q,
+                           int64_t out, int64_t in) {
+    focus_tensor_desc d;
+    std::memset(&d, 0, sizeof d);
+    d.W = W;
+    d.dWq = dWq;
+    d.Wq = Wq;
+    d.m = const_cast<float *>(m);
+    d.q = const_cast<float *>(q);
+    d.out = out;
+    d.in = in;
+    d.block_begin = 0;
+    d.tile_begin = 0;
+    return d;
+}
+
+Hyper make_hyper(float lr_m, float lr_q, float beta1, float beta2, float eps, float wd, int64_t step) {
+    const double bc1 = 1.0 - std::pow((double)beta1, (double)step);
+    const double bc2 = 1.0 - std::pow((double)beta2, (double)step);
+    Hyper h;
+    h.lr_m_step = (float)((double)lr_m / bc1);
+    h.lr_q_step = (float)((double)lr_q / bc1);
+    h.decay_m = (float)(1.0 - (double)lr_m * wd);
+    h.decay_q = (float)(1.0 - (double)lr_q * wd);
+    h.beta1 = beta1;
+    h.one_m_beta1 = (float)(1.0 - (double)beta1);
+    h.beta2 = beta2;
+    h.one_m_beta2 = (float)(1.0 - (double)beta2);
+    h.bc2_sqrt = (float)std::sqrt(bc2);
+    h.eps = eps;
+    return h;
+}
+
+int check_hyper(float lr, float beta1, float beta2, float eps, float wd, int64_t step) {
+    if (!(lr >= 0.0f) || !std::isfinite(lr)) return FOCUS_ERR_VALUE;
+    if (!(beta1 >= 0.0f && beta1 < 1.0f) || !(beta2 >= 0.0f && beta2 < 1.0f)) return FOCUS_ERR_VALUE;
+    if (!(eps >= 0.0f) || !std::isfinite(eps) || !(wd >= 0.0f) || !std::isfinite(wd)) return FOCUS_ERR_VALUE;
+    if (step < 1) return FOCUS_ERR_VALUE;
+    return FOCUS_OK;
+}
+
+}  // namespace
+}  // namespace focus
+
+using namespace focus;
+
+namespace {
+template <int KIND>
+int launch_on(const Args &a, cudaStream_t s) {
+    DeviceInfo *di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    if (a.total_tiles == 0 && !a.one_scale_out) return FOCUS_OK;
+    const int occ = KIND == KIND_FWD ? di->occ_fwd : (KIND == KIND_BWD ? di->occ_bwd : di->occ_step);
+    int64_t grid = grid_for(a.total_tiles, di->sms, occ);
+    if (grid < 1) grid = 1;   // the pack of an empty tensor still writes its tensor scale
+    tile_kernel<KIND><<<(unsigned)grid, THREADS, 0, s>>>(a);
+    return launch_status();
+}
+
+int launch_s2(const Args &a, uint32_t *partial, float *one_out, int n_finish, cudaStream_t s) {
+    DeviceInfo *di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    if (a.total_tiles > 0) {
+        const int64_t grid = grid_for(a.total_tiles, di->sms, di->occ_amax);
+        amax_tiles_kernel<<<(unsigned)grid, THREADS, 0, s>>>(a, partial);
+        if ((rc = launch_status())) return rc;
+    }
+    if (n_finish > 0) {
+        s2_finish_kernel<<<(unsigned)n_finish, THREADS, 0, s>>>(a, partial, one_out);
+        return launch_status();
+    }
+    return FOCUS_OK;
+}
+}  // namespace
+
+extern "C" {
+
+const char *focus_status_string(int status) {
+    switch (status) {
+    case FOCUS_OK: return "FOCUS_OK";
+    case FOCUS_ERR_NULL: return "FOCUS_ERR_NULL: a required pointer is NULL";
+    case FOCUS_ERR_SHAPE: return "FOCUS_ERR_SHAPE: in must be a multiple of 16, sizes non-negative";
+    case FOCUS_ERR_ALIGN: return "FOCUS_ERR_ALIGN: tensor base addresses must be 16-byte aligned";
+    case FOCUS_ERR_VALUE: return "FOCUS_ERR_VALUE: a scalar argument is out of range";
+    case FOCUS_ERR_WORKSPACE: return "FOCUS_ERR_WORKSPACE: workspace missing or too small";
+    case FOCUS_ERR_CUDA: return "FOCUS_ERR_CUDA: a CUDA call or launch failed";
+    case FOCUS_ERR_NONFINITE_INPUT: return "FOCUS_ERR_NONFINITE_INPUT: a kernel met a non-finite input";
+    default: return "FOCUS_ERR_UNKNOWN";
+    }
+}
+
+const char *focus_version(void) { return "0.1.0"; }
+
+size_t focus_s2_workspace_bytes(int64_t out, int64_t in) {
+    if (check_shape(out, in)) return 0;
+    const int64_t t = tiles_of(out, in);
+    return (size_t)(t > 0 ? t : 1) * sizeof(uint32_t);
+}
+
+int focus_s2(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, void *ws_dev, size_t ws_bytes,
+             focus_stream_t stream) {
+    int rc = check_shape(out, in);
+    if (rc) return rc;
+    if (!s2_dev || !ws_dev || (!W && out * in > 0)) return FOCUS_ERR_NULL;
+    if (!aligned16(W) || !aligned16(ws_dev)) return FOCUS_ERR_ALIGN;
+    if (ws_bytes < focus_s2_workspace_bytes(out, in)) return FOCUS_ERR_WORKSPACE;
+    Args a{};
+    a.table = nullptr;
+    a.n_tensors = 1;
+    a.one = one_desc(W, nullptr, nullptr, nullptr, nullptr, out, in);
+    a.total_tiles = tiles_of(out, in);
+    return launch_s2(a, static_cast<uint32_t *>(ws_dev), s2_dev, 1, (cudaStream_t)stream);
+}
+
+int focus_fwd(const uint16_t *W, const float *m, const float *q, float s2, int64_t out, int64_t in, uint16_t *Wq,
+              focus_stream_t stream) {
+    int rc = check_shape(out, in);
+    if (rc) return rc;
+    if ((rc = check_s2(s2))) return rc;
+    if (out * in == 0) return FOCUS_OK;
+    if (!W || !m || !q || !Wq) return FOCUS_ERR_NULL;
+    if (!aligned16(W) || !aligned16(m) || !aligned16(q) || !aligned16(Wq)) return FOCUS_ERR_ALIGN;
+    Args a{};
+    a.one = one_desc(W, nullptr, Wq, m, q, out, in);
+    a.write_wq = 1;
+    a.one_s2 = s2;
+    a.n_tensors = 1;
+    a.total_tiles = tiles_of(out, in);
+    return launch_on<KIND_FWD>(a, (cudaStream_t)stream);
+}
+
+int focus_pack_nvfp4(const uint16_t *W, const float *m, const float *q, float s2, int64_t out, int64_t in,
+                     uint8_t *codes, uint8_t *scales, float *tensor_scale_dev, focus_stream_t stream) {
+    int rc = check_shape(out, in);
+    if (rc) return rc;
+    if ((rc = check_s2(s2))) return rc;
+    if (!tensor_scale_dev) return FOCUS_ERR_NULL;
+    if (out * in > 0) {
+        if (!W || !m || !q || !codes || !scales) return FOCUS_ERR_NULL;
+        if (!aligned16(W) || !aligned16(m) || !aligned16(q) || !aligned16(codes) || !aligned16(scales))
+            return FOCUS_ERR_ALIGN;
+    }
+    Args a{};
+    a.one_scale_out = tensor_scale_dev;
+    a.one = one_desc(W, nullptr, nullptr, m, q, out, in);
+    a.one.codes = codes;
+    a.one.scales = scales;
+    a.one_s2 = s2;
+    a.n_tensors = 1;
+    a.total_tiles = tiles_of(out, in);
+    return launch_on<KIND_FWD>(a, (cudaStream_t)stream);
+}
+
+int focus_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, const float *q, float s2, int64_t out,
+                  int64_t in, float *dm, float *dq, int accumulate, focus_stream_t stream) {
+    int rc = check_shape(out, in);
+    if (rc) return rc;
+    if ((rc = check_s2(s2))) return rc;
+    if (accumulate != 0 && accumulate != 1) return FOCUS_ERR_VALUE;
+    if (out * in == 0) return FOCUS_OK;
+    if (!W || !dWq || !m || !q || !dm || !dq) return FOCUS_ERR_NULL;
+    if (!aligned16(W) || !aligned16(dWq) || !aligned16(m) || !aligned16(q) || !aligned16(dm) || !aligned16(dq))
+        return FOCUS_ERR_ALIGN;
+    Args a{};
+    a.one = one_desc(W, dWq, nullptr, m, q, out, in);
+    a.one.dm = dm;
+    a.one.dq = dq;
+    a.one_s2 = s2;
+    a.n_tensors = 1;
+    a.accumulate = accumulate;
+    a.total_tiles = tiles_of(out, in);
+    return launch_on<KIND_BWD>(a, (cudaStream_t)stream);
+}
+
+int focus_adamw_step(float *p, const float *g, float *exp_avg, float *exp_avg_sq, int64_t n, float lr, float beta1,
+                     float beta2, float eps, float weight_decay, int64_t step, focus_stream_t stream) {
+    if (n < 0) return FOCUS_ERR_SHAPE;
+    int rc = check_hyper(lr, beta1, beta2, eps, weight_decay, step);
+    if (rc) return rc;
+    if (n == 0) return FOCUS_OK;
+    if (!p || !g || !exp_avg || !exp_avg_sq) return FOCUS_ERR_NULL;
+    if (!aligned16(p) || !aligned16(g) || !aligned16(exp_avg) || !aligned16(exp_avg_sq)) return FOCUS_ERR_ALIGN;
+    DeviceInfo *di;
+    if ((rc = device_info(&di))) return rc;
+    const Hyper h = make_hyper(lr, lr, beta1, beta2, eps, weight_decay, step);
+    const int64_t per_cta = (int64_t)THREADS * 4;
+    const int64_t grid = grid_for((n + per_cta - 1) / per_cta, di->sms, di->occ_adam);
+    adamw_kernel<<<(unsigned)(grid > 0 ? grid : 1), THREADS, 0, (cudaStream_t)stream>>>(
+        p, g, exp_avg, exp_avg_sq, n, h.lr_m_step, h.decay_m, h);
+    return launch_status();
+}
+
+int focus_table_prepare(focus_tensor_desc *d, int n, int purpose, int64_t *total_tiles) {
+    if (!d || !total_tiles) return FOCUS_ERR_NULL;
+    if (n < 0 || (purpose != 0 && purpose != 1)) return FOCUS_ERR_VALUE;
+    int64_t tiles = 0, blocks = 0;
+    for (int i = 0; i < n; ++i) {
+        focus_tensor_desc &e = d[i];
+        int rc = check_shape(e.out, e.in);
+        if (rc) return rc;
+        if (!e.s2) return FOCUS_ERR_NULL;
+        if (!aligned16(e.s2)) return FOCUS_ERR_ALIGN;
+        const int64_t nblk = e.out * (e.in / 16);
+        if (nblk > 0) {
+            if (!e.W || !e.m || !e.q) return FOCUS_ERR_NULL;
+            const void *ptrs[] = {e.W, e.m, e.q, e.Wq, e.codes, e.scales, e.dm, e.dq, e.dWq,
+                                  e.m_exp_avg, e.m_exp_avg_sq, e.q_exp_avg, e.q_exp_avg_sq};
+            for (const void *p : ptrs)
+                if (p && !aligned16(p)) return FOCUS_ERR_ALIGN;
+            if ((e.codes == nullptr) != (e.scales == nullptr)) return FOCUS_ERR_NULL;
+            if (purpose == 1 && (!e.dWq || !e.m_exp_avg || !e.m_exp_avg_sq || !e.q_exp_avg || !e.q_exp_avg_sq))
+                return FOCUS_ERR_NULL;
+            if ((e.dm == nullptr) != (e.dq == nullptr)) return FOCUS_ERR_NULL;
+        }
+        e.block_begin = blocks;
+        e.tile_begin = tiles;
+        blocks += nblk;
+        tiles += (nblk + TILE_BLOCKS - 1) / TILE_BLOCKS;
+    }
+    *total_tiles = tiles;
+    return FOCUS_OK;
+}
+
+size_t focus_s2_multi_workspace_bytes(int64_t total_tiles) {
+    return (size_t)(total_tiles > 0 ? total_tiles : 1) * sizeof(uint32_t);
+}
+
+int focus_s2_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, void *ws_dev, size_t ws_bytes,
+                   focus_stream_t stream) {
+    if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
+    if (n == 0) return FOCUS_OK;
+    if (!descs_dev || !ws_dev) return FOCUS_ERR_NULL;
+    if (!aligned16(descs_dev) || !aligned16(ws_dev)) return FOCUS_ERR_ALIGN;
+    if (ws_bytes < focus_s2_multi_workspace_bytes(total_tiles)) return FOCUS_ERR_WORKSPACE;
+    Args a{};
+    a.table = descs_dev;
+    a.n_tensors = n;
+    a.total_tiles = total_tiles;
+    return launch_s2(a, static_cast<uint32_t *>(ws_dev), nullptr, n, (cudaStream_t)stream);
+}
+
+int focus_step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, const focus_hparams *hp,
+                     int64_t step, unsigned flags, focus_stream_t stream) {
+    if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
+    if (!hp) return FOCUS_ERR_NULL;
+    int rc = check_hyper(hp->lr_m, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
+    if (rc) return rc;
+    if ((rc = check_hyper(hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
+    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD)) return FOCUS_ERR_VALUE;
+    if (n == 0) return FOCUS_OK;
+    if (!descs_dev) return FOCUS_ERR_NULL;
+    if (!aligned16(descs_dev)) return FOCUS_ERR_ALIGN;
+    Args a{};
+    a.table = descs_dev;
+    a.n_tensors = n;
+    a.total_tiles = total_tiles;
+    a.write_wq = 1;
+    a.accumulate = (flags & FOCUS_STEP_ACCUMULATE) ? 1 : 0;
+    a.write_grad = (flags & FOCUS_STEP_WRITE_GRAD) ? 1 : 0;
+    a.hp = make_hyper(hp->lr_m, hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
+    return launch_on<KIND_STEP>(a, (cudaStream_t)stream);
+}
+
+int focus_pack_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {
+    if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
+    if (n == 0) return FOCUS_OK;
+    if (!descs_dev) return FOCUS_ERR_NULL;
+    if (!aligned16(descs_dev)) return FOCUS_ERR_ALIGN;
+    Args a{};
+    a.table = descs_dev;
+    a.n_tensors = n;
+    a.total_tiles = total_tiles;
+    return launch_on<KIND_FWD>(a, (cudaStream_t)stream);
+}
+
+int focus_get_error(focus_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FOCUS_ERR_CUDA;
+    unsigned int flags = 0;
+    if (cudaMemcpyFromSymbol(&flags, g_error_flags, sizeof flags) != cudaSuccess) return FOCUS_ERR_CUDA;
+    if (flags) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_flags, &zero, sizeof zero) != cudaSuccess) return FOCUS_ERR_CUDA;
+        return FOCUS_ERR_NONFINITE_INPUT;
+    }
+    return FOCUS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,206 @@
+"""Thin ctypes binding of libfocus.so (include/focus.h): argument marshalling only.
+
+Each function has the name of its C entry point, takes CUDA torch tensors (or
+raw device addresses as ints), passes their addresses and the current CUDA
+stream, and raises FocusError on a non-zero status.  Every computation runs in
+the library's kernels; there is no fallback: a missing libfocus.so raises at
+import time.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfocus.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"libfocus.so is not built ({_LIB_PATH}); run fp4_post_weight_b200.build.build()")
+_lib = ctypes.CDLL(_LIB_PATH)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+FOCUS_OK = 0
+FOCUS_STEP_ACCUMULATE = 1
+FOCUS_STEP_WRITE_GRAD = 2
+
+
+class focus_tensor_desc(ctypes.Structure):
+    _fields_ = [("W", _P), ("dWq", _P), ("Wq", _P), ("m", _P), ("q", _P),
+                ("m_exp_avg", _P), ("m_exp_avg_sq", _P), ("q_exp_avg", _P), ("q_exp_avg_sq", _P),
+                ("s2", _P), ("codes", _P), ("scales", _P), ("dm", _P), ("dq", _P),
+                ("out", _I64), ("in_", _I64), ("block_begin", _I64), ("tile_begin", _I64)]
+
+
+assert ctypes.sizeof(focus_tensor_desc) == 144
+
+
+class focus_hparams(ctypes.Structure):
+    _fields_ = [("lr_m", _F), ("lr_q", _F), ("beta1", _F), ("beta2", _F), ("eps", _F),
+                ("weight_decay", _F)]
+
+
+_SIGS = {
+    "focus_status_string": ([_I], ctypes.c_char_p),
+    "focus_version": ([], ctypes.c_char_p),
+    "focus_s2_workspace_bytes": ([_I64, _I64], _SZ),
+    "focus_s2": ([_P, _I64, _I64, _P, _P, _SZ, _P], _I),
+    "focus_fwd": ([_P, _P, _P, _F, _I64, _I64, _P, _P], _I),
+    "focus_ste_bwd": ([_P, _P, _P, _P, _F, _I64, _I64, _P, _P, _I, _P], _I),
+    "focus_adamw_step": ([_P, _P, _P, _P, _I64, _F, _F, _F, _F, _F, _I64, _P], _I),
+    "focus_pack_nvfp4": ([_P, _P, _P, _F, _I64, _I64, _P, _P, _P, _P], _I),
+    "focus_table_prepare": ([ctypes.POINTER(focus_tensor_desc), _I, _I, ctypes.POINTER(_I64)], _I),
+    "focus_s2_multi_workspace_bytes": ([_I64], _SZ),
+    "focus_s2_multi": ([_P, _I, _I64, _P, _SZ, _P], _I),
+    "focus_step_fused": ([_P, _I, _I64, ctypes.POINTER(focus_hparams), _I64, ctypes.c_uint, _P], _I),
+    "focus_pack_multi": ([_P, _I, _I64, _P], _I),
+    "focus_get_error": ([_P], _I),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+EXPORTED = tuple(_SIGS)
+
+
+class FocusError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.focus_status_string(status).decode()}")
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != FOCUS_OK:
+        raise FocusError(rc, where)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, torch.Tensor):
+        if not x.is_cuda:
+            raise ValueError("device tensors only (the library computes on the GPU)")
+        if not x.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        return x.data_ptr()
+    raise TypeError(f"cannot pass {type(x)} as a device pointer")
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _bf16(t, name):
+    if isinstance(t, torch.Tensor) and t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16")
+
+
+def _f32(t, name):
+    if isinstance(t, torch.Tensor) and t.dtype != torch.float32:
+        raise TypeError(f"{name} must be float32")
+
+
+def _shape(W, out=None, in_=None):
+    if out is not None:
+        return int(out), int(in_)
+    if W.dim() != 2:
+        raise ValueError("W must be 2-D [out, in]")
+    return int(W.shape[0]), int(W.shape[1])
+
+
+def focus_version() -> str:
+    return _lib.focus_version().decode()
+
+
+def focus_status_string(status: int) -> str:
+    return _lib.focus_status_string(int(status)).decode()
+
+
+def focus_s2_workspace_bytes(out: int, in_: int) -> int:
+    return int(_lib.focus_s2_workspace_bytes(int(out), int(in_)))
+
+
+def focus_s2(W, s2_out, workspace, stream=None, out=None, in_=None):
+    """s2 = amax(|W|)/(6*448) into the one-float device tensor s2_out."""
+    _bf16(W, "W"); _f32(s2_out, "s2_out")
+    o, i = _shape(W, out, in_)
+    nbytes = workspace.numel() * workspace.element_size() if isinstance(workspace, torch.Tensor) else 1 << 62
+    _check(_lib.focus_s2(_ptr(W), o, i, _ptr(s2_out), _ptr(workspace), nbytes, _stream(stream)), "focus_s2")
+
+
+def focus_fwd(W, m, q, s2: float, Wq, stream=None, out=None, in_=None):
+    _bf16(W, "W"); _bf16(Wq, "Wq"); _f32(m, "m"); _f32(q, "q")
+    o, i = _shape(W, out, in_)
+    _check(_lib.focus_fwd(_ptr(W), _ptr(m), _ptr(q), float(s2), o, i, _ptr(Wq), _stream(stream)), "focus_fwd")
+
+
+def focus_ste_bwd(W, dWq, m, q, s2: float, dm, dq, accumulate: bool = False, stream=None, out=None, in_=None):
+    _bf16(W, "W"); _bf16(dWq, "dWq"); _f32(m, "m"); _f32(q, "q"); _f32(dm, "dm"); _f32(dq, "dq")
+    o, i = _shape(W, out, in_)
+    _check(_lib.focus_ste_bwd(_ptr(W), _ptr(dWq), _ptr(m), _ptr(q), float(s2), o, i, _ptr(dm), _ptr(dq),
+                              1 if accumulate else 0, _stream(stream)), "focus_ste_bwd")
+
+
+def focus_adamw_step(p, g, exp_avg, exp_avg_sq, lr: float, step: int, beta1=0.9, beta2=0.999, eps=1e-8,
+                     weight_decay=0.0, stream=None, n=None):
+    for t, nm in ((p, "p"), (g, "g"), (exp_avg, "exp_avg"), (exp_avg_sq, "exp_avg_sq")):
+        _f32(t, nm)
+    n = int(p.numel()) if n is None else int(n)
+    _check(_lib.focus_adamw_step(_ptr(p), _ptr(g), _ptr(exp_avg), _ptr(exp_avg_sq), n, float(lr), float(beta1),
+                                 float(beta2), float(eps), float(weight_decay), int(step), _stream(stream)),
+           "focus_adamw_step")
+
+
+def focus_pack_nvfp4(W, m, q, s2: float, codes, scales, tensor_scale, stream=None, out=None, in_=None):
+    _bf16(W, "W"); _f32(m, "m"); _f32(q, "q"); _f32(tensor_scale, "tensor_scale")
+    o, i = _shape(W, out, in_)
+    _check(_lib.focus_pack_nvfp4(_ptr(W), _ptr(m), _ptr(q), float(s2), o, i, _ptr(codes), _ptr(scales),
+                                 _ptr(tensor_scale), _stream(stream)), "focus_pack_nvfp4")
+
+
+def focus_table_prepare(descs, purpose: int) -> int:
+    """Checks a ctypes array of focus_tensor_desc in place; returns total_tiles."""
+    tiles = _I64(0)
+    _check(_lib.focus_table_prepare(descs, len(descs), int(purpose), ctypes.byref(tiles)), "focus_table_prepare")
+    return int(tiles.value)
+
+
+def focus_s2_multi_workspace_bytes(total_tiles: int) -> int:
+    return int(_lib.focus_s2_multi_workspace_bytes(int(total_tiles)))
+
+
+def focus_s2_multi(table_dev, n: int, total_tiles: int, workspace, stream=None):
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(_lib.focus_s2_multi(_ptr(table_dev), int(n), int(total_tiles), _ptr(workspace), nbytes,
+                               _stream(stream)), "focus_s2_multi")
+
+
+def focus_step_fused(table_dev, n: int, total_tiles: int, hp: focus_hparams, step: int, flags: int = 0,
+                     stream=None):
+    _check(_lib.focus_step_fused(_ptr(table_dev), int(n), int(total_tiles), ctypes.byref(hp), int(step),
+                                 int(flags), _stream(stream)), "focus_step_fused")
+
+
+def focus_pack_multi(table_dev, n: int, total_tiles: int, stream=None):
+    _check(_lib.focus_pack_multi(_ptr(table_dev), int(n), int(total_tiles), _stream(stream)), "focus_pack_multi")
+
+
+def focus_get_error(stream=None) -> int:
+    """Synchronizes the stream and returns (and clears) the sticky device status."""
+    return int(_lib.focus_get_error(_stream(stream)))
+
+
+def raw_call(name: str, *args):
+    """Call an entry point with raw ctypes arguments (addresses as ints); returns the status."""
+    return getattr(_lib, name)(*args)

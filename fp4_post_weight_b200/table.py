@@ -1,0 +1,78 @@
+"""Multi-tensor table: every linear weight of a model, stepped in one launch.
+
+Builds the focus_tensor_desc array (include/focus.h) from torch tensors, lets
+the library check it (focus_table_prepare), keeps the device copy, and calls
+the multi-tensor entry points.  Marshalling only: all arithmetic is in the
+library's kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+from . import focus as F
+
+_FIELDS = ("W", "dWq", "Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq", "s2",
+           "codes", "scales", "dm", "dq")
+
+PURPOSE_FORWARD = 0
+PURPOSE_STEP = 1
+
+
+@dataclass
+class Entry:
+    """One weight: W [out, in] bf16 plus whatever the calls in use need."""
+    W: torch.Tensor
+    m: torch.Tensor
+    q: torch.Tensor
+    s2: torch.Tensor                          # one float32 on the device
+    dWq: torch.Tensor | None = None
+    Wq: torch.Tensor | None = None
+    m_exp_avg: torch.Tensor | None = None
+    m_exp_avg_sq: torch.Tensor | None = None
+    q_exp_avg: torch.Tensor | None = None
+    q_exp_avg_sq: torch.Tensor | None = None
+    codes: torch.Tensor | None = None
+    scales: torch.Tensor | None = None
+    dm: torch.Tensor | None = None
+    dq: torch.Tensor | None = None
+    extra: dict = field(default_factory=dict)
+
+
+class FocusTable:
+    def __init__(self, entries: list[Entry], purpose: int = PURPOSE_STEP):
+        self.entries = list(entries)
+        n = len(self.entries)
+        self.n = n
+        descs = (F.focus_tensor_desc * max(n, 1))()
+        for i, e in enumerate(self.entries):
+            d = descs[i]
+            for name in _FIELDS:
+                t = getattr(e, name)
+                setattr(d, name, None if t is None else F._ptr(t))
+            d.out, d.in_ = int(e.W.shape[0]), int(e.W.shape[1])
+        self.total_tiles = F.focus_table_prepare((F.focus_tensor_desc * n).from_buffer(descs), purpose) if n else 0
+        self.descs = descs
+        dev = self.entries[0].W.device if n else torch.device("cuda")
+        raw = torch.frombuffer(bytearray(bytes(descs)), dtype=torch.uint8)
+        self.dev = raw.to(dev)                  # 256-byte aligned device copy
+        self._ws = None
+
+    def s2(self, stream=None):
+        need = F.focus_s2_multi_workspace_bytes(self.total_tiles)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.dev.device)
+        F.focus_s2_multi(self.dev, self.n, self.total_tiles, self._ws, stream)
+
+    def step(self, step: int, hp: F.focus_hparams | None = None, flags: int = 0, stream=None):
+        hp = hp or hparams()
+        F.focus_step_fused(self.dev, self.n, self.total_tiles, hp, step, flags, stream)
+
+    def pack(self, stream=None):
+        F.focus_pack_multi(self.dev, self.n, self.total_tiles, stream)
+
+
+def hparams(lr_m=5e-3, lr_q=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0) -> F.focus_hparams:
+    """The card's calibration setting: AdamW, lr 5e-3 for m and 1e-3 for q, betas 0.9/0.999, wd 0."""
+    return F.focus_hparams(lr_m, lr_q, beta1, beta2, eps, weight_decay)

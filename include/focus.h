@@ -1,0 +1,232 @@
+/*
+ * focus.h -- C ABI of libfocus.so: the FOCUS NVFP4 weight fake-quantizer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * FOCUS (Coupled-Relaxation and Dual-Granularity Scaling) learns, for every
+ * linear weight W[out, in] of a frozen BF16 model, one factor m per 16-element
+ * block and one logit q per 8-element sub-block.  The source of every formula
+ * is the model card "FOCUS NVFP4 scales for Llama-3.2-1B-Instruct (our
+ * reproduction)", section "What this is" (field table, layout sentence and the
+ * three equations with the rules that follow them) and section "Calibration"
+ * (optimizer and learning rates); the straight-through estimator is named in
+ * "Technische Samenvatting: FOCUS ...", section "Methodologie", item 1.
+ *
+ * Per block b (16 weights along in_features) with sub-blocks k = 0, 1 (8 each):
+ *   A_b  = max |w_i|
+ *   x_b  = fl(fl(A_b * m_b) / fl(6 * s2));  x_b == 0 -> 1
+ *   S_b  = e4m3_rne(clamp(x_b, 2^-6, 448))
+ *   D_k  = fl(fl(S_b * sigmoid(q_k)) * s2)
+ *   y_i  = fl(w_i / D_k)
+ *   c_i  = E2M1_rne(clamp(y_i, -6, 6))             (ties to even, sign kept)
+ *   w'_i = bf16_rne(fl(fl(c_i * S_b) * s2))
+ * All arithmetic is IEEE binary32 with one rounding per operation; sigmoid is
+ * the binary32 rounding of 1/(1+exp(-q)) evaluated in binary64.
+ *
+ * Conventions for every call:
+ *  - Tensors are dense row-major.  W, dW' and W' are bf16, passed as uint16_t
+ *    bit patterns.  m is float[out][in/16], q is float[out][in/8]: m[r][b]
+ *    belongs to W[r][16b..16b+15], q[r][2b+k] to W[r][16b+8k..16b+8k+7].
+ *  - Pointers named *_dev, and every tensor pointer, are device pointers
+ *    (cudaMalloc / PyTorch CUDA memory) on the current device; their base
+ *    addresses must be 16-byte aligned.  Parameters passed by value or through
+ *    a host pointer are read before the call returns.
+ *  - The caller owns every buffer and the stream.  The library allocates no
+ *    device or host memory; temporary storage is passed in as a workspace.
+ *  - Every call only enqueues work on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) and returns at once.  The return value reports the
+ *    argument checks (done on the host, before anything is enqueued) and the
+ *    launch status; a failed check enqueues nothing.
+ *  - Non-finite values in W, m or q, and an invalid s2 read from device
+ *    memory, are outside the contract: kernels never trap on them, they set a
+ *    sticky device flag that focus_get_error() reports.
+ *  - in must be a multiple of 16; out >= 0 (an empty tensor is a no-op).
+ */
+#ifndef FOCUS_H
+#define FOCUS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *focus_stream_t; /* a cudaStream_t */
+
+typedef enum focus_status {
+    FOCUS_OK = 0,
+    FOCUS_ERR_NULL = 1,             /* a required pointer is NULL */
+    FOCUS_ERR_SHAPE = 2,            /* in % 16 != 0, out < 0, n < 0, or a size overflows */
+    FOCUS_ERR_ALIGN = 3,            /* a tensor base address is not 16-byte aligned */
+    FOCUS_ERR_VALUE = 4,            /* s2 <= 0 or not finite, lr < 0, step < 1, beta outside [0,1) ... */
+    FOCUS_ERR_WORKSPACE = 5,        /* workspace missing or smaller than required */
+    FOCUS_ERR_CUDA = 6,             /* a CUDA runtime call or a launch failed */
+    FOCUS_ERR_NONFINITE_INPUT = 7   /* reported by focus_get_error(): the device flag was set */
+} focus_status;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *focus_status_string(int status);
+
+/* ---------------------------------------------------------------------------
+ * Per-tensor scale s2 = amax(|W|) / (6 * 448).
+ * Card, field table, row "s2": one FP32 scale per tensor, frozen, computed from
+ * the base weights.  Two passes: every CTA writes the max |w| of its tile into
+ * the workspace, then one CTA reduces those maxima and divides once by 2688.
+ * The result is exact (max is order-free; one correctly rounded division).
+ *   W       [out, in] bf16, device
+ *   s2_dev  one float, device, written
+ *   ws_dev  device workspace of at least focus_s2_workspace_bytes(out, in)
+ *           bytes, 16-byte aligned; its contents on entry do not matter.
+ * An all-zero W gives s2 = 0, which the other calls reject.
+ * ------------------------------------------------------------------------- */
+size_t focus_s2_workspace_bytes(int64_t out, int64_t in);
+int focus_s2(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, void *ws_dev,
+             size_t ws_bytes, focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Forward fake-quantization W -> W'.
+ * Card, "What this is": the S_b, c_i and w'_i equations.
+ *   W   [out, in] bf16, device (read)
+ *   m   [out, in/16] float, device (read)
+ *   q   [out, in/8] float, device (read)
+ *   s2  the tensor scale, by value: finite and > 0, else FOCUS_ERR_VALUE
+ *   Wq  [out, in] bf16, device (written; must not overlap W)
+ * ------------------------------------------------------------------------- */
+int focus_fwd(const uint16_t *W, const float *m, const float *q, float s2, int64_t out, int64_t in,
+              uint16_t *Wq, focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Straight-through backward for m and q.
+ * "Technische Samenvatting: FOCUS ...", "Methodologie" item 1 (scales learned
+ * through the straight-through estimator), applied to the card's equations:
+ * rounding (E2M1 and E4M3) acts as the identity; the clamps pass the gradient
+ * at and inside their bounds and block it outside; the zero-block rule blocks
+ * it.  With g_i the gradient of w'_i, in_i = [-6 <= y_i <= 6] and
+ * inS_b = [x_b != 0 and 2^-6 <= x_b <= 448]:
+ *   dL/dm_b   = inS_b * (A_b/6) * sum_{i in b} g_i * (in_i ? c_i - y_i : c_i)
+ *   dL/dq_k   = -(1 - sigmoid(q_k)) * S_b * s2 * sum_{i in k} in_i * g_i * y_i
+ *   W, dWq     [out, in] bf16, device (read); dWq is dL/dW'
+ *   m, q       as in focus_fwd (read)
+ *   dm         [out, in/16] float, device; dq [out, in/8] float, device
+ *   accumulate 0: dm, dq are overwritten; 1: the gradients are added to them
+ * Sums are formed in binary32 (order fixed per block).
+ * ------------------------------------------------------------------------- */
+int focus_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, const float *q, float s2,
+                  int64_t out, int64_t in, float *dm, float *dq, int accumulate, focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * AdamW update of a parameter vector, in place.
+ * Card, "Calibration": AdamW with betas 0.9/0.999, weight decay 0 and a
+ * constant learning rate (5e-3 for m, 1e-3 for q).  Decoupled weight decay and
+ * bias correction, step counted from 1:
+ *   p <- p*(1 - lr*wd); v1 <- b1*v1 + (1-b1)*g; v2 <- b2*v2 + (1-b2)*g^2
+ *   p <- p - (lr/(1-b1^t)) * v1 / (sqrt(v2)/sqrt(1-b2^t) + eps)
+ *   p, exp_avg, exp_avg_sq  n floats, device (read and written)
+ *   g                       n floats, device (read)
+ *   lr >= 0, 0 <= beta1, beta2 < 1, eps >= 0, weight_decay >= 0, step >= 1
+ * ------------------------------------------------------------------------- */
+int focus_adamw_step(float *p, const float *g, float *exp_avg, float *exp_avg_sq, int64_t n, float lr,
+                     float beta1, float beta2, float eps, float weight_decay, int64_t step,
+                     focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * NVFP4 export pack.
+ * Card, "What this is": the deployed model is plain NVFP4 -- E2M1 elements,
+ * one E4M3 scale per 16 elements, one FP32 scale per tensor.  Byte layout (the
+ * card gives none; this is the common one):
+ *   codes             [out, in/2] uint8, device: byte j of a row holds element
+ *                     2j in bits 0-3 and element 2j+1 in bits 4-7 (sign bit 3/7)
+ *   scales            [out, in/16] uint8, device: the E4M3 byte of S_b
+ *   tensor_scale_dev  one float, device: s2 (a dequantization multiplier,
+ *                     w' = c * S_b * s2)
+ * Other arguments as in focus_fwd.
+ * ------------------------------------------------------------------------- */
+int focus_pack_nvfp4(const uint16_t *W, const float *m, const float *q, float s2, int64_t out, int64_t in,
+                     uint8_t *codes, uint8_t *scales, float *tensor_scale_dev, focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Multi-tensor interface: every linear weight of a model in one launch.
+ *
+ * A table of focus_tensor_desc lives in DEVICE memory.  The caller fills the
+ * table on the host, calls focus_table_prepare() on it (which checks every
+ * entry and fills the two *_begin fields), copies it to device memory and then
+ * passes the device copy to the calls below, step after step.  The table must
+ * not change without being prepared again.
+ * ------------------------------------------------------------------------- */
+typedef struct focus_tensor_desc {
+    const uint16_t *W;     /* [out, in] bf16 base weight (read) */
+    const uint16_t *dWq;   /* [out, in] bf16 dL/dW' (read by focus_step_fused; may be NULL otherwise) */
+    uint16_t *Wq;          /* [out, in] bf16 W' (written when not NULL) */
+    float *m;              /* [out, in/16] */
+    float *q;              /* [out, in/8] */
+    float *m_exp_avg;      /* AdamW first moment of m  (focus_step_fused) */
+    float *m_exp_avg_sq;   /* AdamW second moment of m (focus_step_fused) */
+    float *q_exp_avg;      /* AdamW first moment of q  (focus_step_fused) */
+    float *q_exp_avg_sq;   /* AdamW second moment of q (focus_step_fused) */
+    float *s2;             /* one float: written by focus_s2_multi, read by the others */
+    uint8_t *codes;        /* [out, in/2] NVFP4 codes (written when not NULL) */
+    uint8_t *scales;       /* [out, in/16] E4M3 scale bytes (written when not NULL) */
+    float *dm;             /* [out, in/16] gradient buffer, see FOCUS_STEP_* flags (may be NULL) */
+    float *dq;             /* [out, in/8]  gradient buffer, see FOCUS_STEP_* flags (may be NULL) */
+    int64_t out;
+    int64_t in;
+    int64_t block_begin;   /* filled by focus_table_prepare: sum of out*in/16 over earlier entries */
+    int64_t tile_begin;    /* filled by focus_table_prepare: first work tile of this entry */
+} focus_tensor_desc;
+
+typedef struct focus_hparams {
+    float lr_m;            /* 5e-3 on the card */
+    float lr_q;            /* 1e-3 on the card */
+    float beta1;           /* 0.9 */
+    float beta2;           /* 0.999 */
+    float eps;             /* 1e-8 */
+    float weight_decay;    /* 0 */
+} focus_hparams;
+
+/* Flags of focus_step_fused. */
+#define FOCUS_STEP_ACCUMULATE 1u  /* add dm/dq (earlier micro-batches) to this step's gradients */
+#define FOCUS_STEP_WRITE_GRAD 2u  /* write the gradients used by the update into dm/dq */
+
+/* Checks every entry (pointers, alignment, shapes, which outputs are present
+ * for `purpose`: 0 = s2/forward/pack only, 1 = also focus_step_fused) and
+ * fills block_begin and tile_begin.  Host memory in, host memory out.
+ * *total_tiles receives the number of work tiles, passed to the calls below. */
+int focus_table_prepare(focus_tensor_desc *descs_host, int n_tensors, int purpose, int64_t *total_tiles);
+
+/* Workspace bytes focus_s2_multi needs for a prepared table. */
+size_t focus_s2_multi_workspace_bytes(int64_t total_tiles);
+
+/* s2 of every entry (two launches). */
+int focus_s2_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles, void *ws_dev,
+                   size_t ws_bytes, focus_stream_t stream);
+
+/* One calibration step of every entry in one launch, W read once:
+ * forward (W' when desc.Wq != NULL, codes/scales when present), straight-
+ * through backward, AdamW on m and q (lr_m for m, lr_q for q) at step `step`.
+ * hp is a host pointer.  flags: FOCUS_STEP_ACCUMULATE, FOCUS_STEP_WRITE_GRAD
+ * (both need desc.dm and desc.dq).  Outputs W', codes and scales are those
+ * of the forward, i.e. of m and q before the update. */
+int focus_step_fused(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
+                     const focus_hparams *hp, int64_t step, unsigned flags, focus_stream_t stream);
+
+/* NVFP4 pack of every entry with codes and scales present (desc.s2 holds the
+ * tensor scale, which the caller exports). */
+int focus_pack_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
+                     focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Synchronizes `stream`, then reports and clears the sticky device flag:
+ * FOCUS_ERR_NONFINITE_INPUT when any kernel since the last call met a
+ * non-finite W/m/q value or an invalid s2 read from a table, FOCUS_ERR_CUDA
+ * when the stream reports an error, else FOCUS_OK.
+ * ------------------------------------------------------------------------- */
+int focus_get_error(focus_stream_t stream);
+
+/* Library version, "major.minor.patch" (static storage). */
+const char *focus_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FOCUS_H */

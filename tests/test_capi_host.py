@@ -1,0 +1,119 @@
+"""The C-ABI library loads, exports every function include/focus.h declares,
+and rejects bad arguments on the host before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def F():
+    from fp4_post_weight_b200 import build
+    build.build()
+    from fp4_post_weight_b200 import focus
+    return focus
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "focus.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(focus_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_function(F):
+    names = declared_functions()
+    assert len(names) >= 14
+    lib = ctypes.CDLL(F._LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(F.EXPORTED)
+
+
+def test_status_strings(F):
+    for s in range(8):
+        assert F.focus_status_string(s).startswith("FOCUS_")
+    assert F.focus_version() == "0.1.0"
+
+
+P = 0x7f0000001000  # an aligned address that is never dereferenced: every call below fails its checks first
+U = 0x7f0000001004  # misaligned
+call = None
+
+
+def _c(F, name, *a):
+    return F.raw_call(name, *a)
+
+
+def test_shape_and_value_checks(F):
+    f32 = ctypes.c_float
+    E = F
+    assert _c(F, "focus_fwd", P, P, P, f32(1.0), 4, 15, P, None) == 2          # in % 16
+    assert _c(F, "focus_fwd", P, P, P, f32(1.0), -1, 16, P, None) == 2         # out < 0
+    assert _c(F, "focus_fwd", P, P, P, f32(0.0), 4, 16, P, None) == 4          # s2 <= 0
+    assert _c(F, "focus_fwd", P, P, P, f32(float("inf")), 4, 16, P, None) == 4
+    assert _c(F, "focus_fwd", P, P, P, f32(float("nan")), 4, 16, P, None) == 4
+    assert _c(F, "focus_fwd", None, P, P, f32(1.0), 4, 16, P, None) == 1       # NULL
+    assert _c(F, "focus_fwd", U, P, P, f32(1.0), 4, 16, P, None) == 3          # misaligned
+    assert _c(F, "focus_fwd", P, P, P, f32(1.0), 0, 16, P, None) == 0          # empty: no-op
+    assert _c(F, "focus_ste_bwd", P, P, P, P, f32(1.0), 4, 16, P, P, 2, None) == 4  # accumulate flag
+    assert _c(F, "focus_ste_bwd", P, None, P, P, f32(1.0), 4, 16, P, P, 0, None) == 1
+    assert _c(F, "focus_pack_nvfp4", P, P, P, f32(1.0), 4, 16, P, P, None, None) == 1
+    assert _c(F, "focus_s2", P, 4, 16, P, P, 0, None) == 5                     # workspace too small
+    assert _c(F, "focus_s2", P, 4, 24, P, P, 64, None) == 2
+    assert F.focus_s2_workspace_bytes(4, 16) == 4
+    assert F.focus_s2_workspace_bytes(2048, 2048) == 4 * (2048 * 128 // 256)
+
+
+def test_adamw_checks(F):
+    f = ctypes.c_float
+    args = lambda lr, b1, b2, eps, wd, step: (P, P, P, P, 8, f(lr), f(b1), f(b2), f(eps), f(wd), step, None)
+    assert _c(F, "focus_adamw_step", *args(1e-3, 0.9, 0.999, 1e-8, 0.0, 0)) == 4
+    assert _c(F, "focus_adamw_step", *args(-1e-3, 0.9, 0.999, 1e-8, 0.0, 1)) == 4
+    assert _c(F, "focus_adamw_step", *args(1e-3, 1.0, 0.999, 1e-8, 0.0, 1)) == 4
+    assert _c(F, "focus_adamw_step", *args(1e-3, 0.9, 0.999, -1.0, 0.0, 1)) == 4
+    assert _c(F, "focus_adamw_step", P, P, P, P, -1, f(1e-3), f(0.9), f(0.999), f(1e-8), f(0), 1, None) == 2
+    assert _c(F, "focus_adamw_step", U, P, P, P, 8, f(1e-3), f(0.9), f(0.999), f(1e-8), f(0), 1, None) == 3
+
+
+def test_table_prepare_on_host(F):
+    n = 3
+    shapes = [(4, 32), (1, 16), (300, 4096)]
+    descs = (F.focus_tensor_desc * n)()
+    for i, (o, k) in enumerate(shapes):
+        d = descs[i]
+        for name in ("W", "dWq", "Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq", "s2"):
+            setattr(d, name, P + 4096 * (i + 1))
+        d.out, d.in_ = o, k
+    tiles = F.focus_table_prepare(descs, 1)
+    nblk = [o * k // 16 for o, k in shapes]
+    assert [descs[i].block_begin for i in range(n)] == [0, nblk[0], nblk[0] + nblk[1]]
+    t = [(b + 255) // 256 for b in nblk]
+    assert [descs[i].tile_begin for i in range(n)] == [0, t[0], t[0] + t[1]]
+    assert tiles == sum(t)
+    # a step needs the moments and dW'
+    descs[1].q_exp_avg = None
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, 1)
+    assert e.value.status == 1
+    assert F.focus_table_prepare(descs, 0) == tiles
+    descs[2].in_ = 40
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, 0)
+    assert e.value.status == 2
+    descs[2].in_ = 4096
+    descs[2].m = U
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, 0)
+    assert e.value.status == 3
+
+
+def test_step_hparam_checks(F):
+    hp = F.focus_hparams(5e-3, 1e-3, 0.9, 0.999, 1e-8, 0.0)
+    assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(hp), 0, 0, None) == 4
+    assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(hp), 1, 8, None) == 4
+    assert F.raw_call("focus_step_fused", P, 1, 1, None, 1, 0, None) == 1
+    bad = F.focus_hparams(5e-3, -1e-3, 0.9, 0.999, 1e-8, 0.0)
+    assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(bad), 1, 0, None) == 4

@@ -1,0 +1,293 @@
+"""GPU parity of every C-ABI entry point against the oracle, on small shapes
+that span several tiles (4096 weights each) and end in ragged tails."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.parity import (assert_close, block_mask, check_forward, host, host_bits, unpack_codes)
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 16), (3, 48), (2, 4096), (37, 1040), (7, 4112), (128, 2048), (257, 160)]
+
+
+@pytest.fixture(scope="module")
+def F():
+    from fp4_post_weight_b200 import focus
+    return focus
+
+
+def make(shape, seed, q_mean=3.0, q_std=3.0, dev="cuda"):
+    g = torch.Generator(device=dev).manual_seed(seed)
+    o, i = shape
+    W = synth.add_outliers(synth.normal_bf16(shape, 0.02, g, dev), 2e-3, 20.0, g) if o * i else \
+        torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+    if o * i >= 64:
+        W.view(-1)[:16] = 0          # a zero block
+    m = synth.uniform((o, i // 16), 0.3, 2.5, g, dev)
+    q = synth.normal((o, i // 8), q_mean, q_std, g, dev)
+    dW = synth.normal_bf16(shape, 1e-3, g, dev)
+    return W, m, q, dW
+
+
+@pytest.mark.parametrize("shape", SHAPES + [(0, 64), (8, 0)])
+def test_s2(F, shape):
+    W, *_ = make(shape, 1)
+    o, i = shape
+    ws = torch.empty(max(F.focus_s2_workspace_bytes(o, i), 16), dtype=torch.uint8, device="cuda")
+    s2 = torch.full((1,), -1.0, device="cuda")
+    F.focus_s2(W, s2, ws)
+    want = oracle.s2(host_bits(W))
+    assert host(s2)[0] == want
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_fwd_and_pack(F, shape):
+    W, m, q, _ = make(shape, 2)
+    o, i = shape
+    s2 = float(oracle.s2(host_bits(W)))
+    Wq = torch.empty_like(W)
+    F.focus_fwd(W, m, q, s2, Wq)
+    codes = torch.empty((o, i // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((o, i // 16), dtype=torch.uint8, device="cuda")
+    ts = torch.zeros(1, device="cuda")
+    F.focus_pack_nvfp4(W, m, q, s2, codes, scales, ts)
+    assert F.focus_get_error() == 0
+    ref = oracle.fwd(host_bits(W), host(m), host(q), s2)
+    check_forward(ref, Wq=host_bits(Wq), codes=unpack_codes(host(codes)), scales=host(scales))
+    assert host(ts)[0] == np.float32(s2)
+    rc, rs, rt = oracle.pack(host_bits(W), host(m), host(q), s2)
+    assert rt == host(ts)[0]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_ste_bwd(F, shape):
+    W, m, q, dW = make(shape, 3)
+    o, i = shape
+    s2 = float(oracle.s2(host_bits(W)))
+    dm = torch.empty((o, i // 16), device="cuda")
+    dq = torch.empty((o, i // 8), device="cuda")
+    F.focus_ste_bwd(W, dW, m, q, s2, dm, dq)
+    ref_f = oracle.fwd(host_bits(W), host(m), host(q), s2)
+    codes = torch.empty((o, i // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((o, i // 16), dtype=torch.uint8, device="cuda")
+    F.focus_pack_nvfp4(W, m, q, s2, codes, scales, torch.zeros(1, device="cuda"))
+    mism = check_forward(ref_f, codes=unpack_codes(host(codes)))
+    skip = block_mask(mism)
+    rdm, rdq = oracle.ste_bwd(host_bits(W), host_bits(dW), host(m), host(q), s2)
+    assert_close(host(dm), rdm, "dm", skip)
+    assert_close(host(dq), rdq, "dq", np.repeat(skip, 2, axis=1))
+    # accumulate: add a second gradient
+    F.focus_ste_bwd(W, dW, m, q, s2, dm, dq, accumulate=True)
+    rdm2, rdq2 = oracle.ste_bwd(host_bits(W), host_bits(dW), host(m), host(q), s2, dm=rdm.copy(), dq=rdq.copy())
+    assert_close(host(dm), rdm2, "dm (accumulated)", skip)
+    assert_close(host(dq), rdq2, "dq (accumulated)", np.repeat(skip, 2, axis=1))
+    assert F.focus_get_error() == 0
+
+
+@pytest.mark.parametrize("n,wd", [(1, 0.0), (7, 0.0), (4099, 0.0), (4099, 0.01), (100000, 0.0)])
+def test_adamw(F, n, wd):
+    g = torch.Generator(device="cuda").manual_seed(n)
+    p = synth.normal((n,), 6.0, 2.0, g, "cuda")
+    v1 = torch.zeros(n, device="cuda"); v2 = torch.zeros(n, device="cuda")
+    hp, hv1, hv2 = host(p).copy(), host(v1).copy(), host(v2).copy()
+    for t in range(1, 6):
+        gr = synth.normal((n,), 0.0, 1e-4, g, "cuda")
+        F.focus_adamw_step(p, gr, v1, v2, 1e-3, t, weight_decay=wd)
+        oracle.adamw(hp, host(gr), hv1, hv2, 1e-3, t, weight_decay=wd)
+    assert_close(host(p), hp, "p")
+    assert_close(host(v1), hv1, "exp_avg")
+    assert_close(host(v2), hv2, "exp_avg_sq")
+
+
+def _entries(shapes, seed, with_pack=True, warm=False):
+    from fp4_post_weight_b200.table import Entry
+    ents = []
+    for j, sh in enumerate(shapes):
+        W, m, q, dW = make(sh, seed + j)
+        o, i = sh
+        e = Entry(W=W, m=m, q=q, s2=torch.zeros(1, device="cuda"), dWq=dW, Wq=torch.empty_like(W))
+        g = torch.Generator(device="cuda").manual_seed(100 + j)
+        if warm:
+            e.m_exp_avg = synth.normal(m.shape, 0, 1e-4, g, "cuda"); e.m_exp_avg_sq = synth.normal(m.shape, 0, 1e-4, g, "cuda") ** 2
+            e.q_exp_avg = synth.normal(q.shape, 0, 1e-6, g, "cuda"); e.q_exp_avg_sq = synth.normal(q.shape, 0, 1e-6, g, "cuda") ** 2
+        else:
+            e.m_exp_avg = torch.zeros_like(m); e.m_exp_avg_sq = torch.zeros_like(m)
+            e.q_exp_avg = torch.zeros_like(q); e.q_exp_avg_sq = torch.zeros_like(q)
+        if with_pack:
+            e.codes = torch.empty((o, i // 2), dtype=torch.uint8, device="cuda")
+            e.scales = torch.empty((o, i // 16), dtype=torch.uint8, device="cuda")
+        e.dm = torch.zeros_like(m); e.dq = torch.zeros_like(q)
+        ents.append(e)
+    return ents
+
+
+@pytest.mark.parametrize("warm,step", [(False, 1), (True, 5)])
+def test_step_fused_table(F, warm, step):
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    shapes = SHAPES + [(0, 32)]
+    ents = _entries(shapes, 10, warm=warm)
+    host_in = [(host_bits(e.W), host_bits(e.dWq), host(e.m).copy(), host(e.q).copy(),
+                [host(x).copy() for x in (e.m_exp_avg, e.m_exp_avg_sq, e.q_exp_avg, e.q_exp_avg_sq)])
+               for e in ents]
+    tab = FocusTable(ents)
+    tab.s2()
+    tab.step(step, hparams(), flags=F.FOCUS_STEP_WRITE_GRAD)
+    assert F.focus_get_error() == 0
+    for e, (Wb, Gb, m, q, st) in zip(ents, host_in):
+        if Wb.size == 0:
+            continue
+        s2 = oracle.s2(Wb)
+        assert host(e.s2)[0] == s2
+        ref_f = oracle.fwd(Wb, m, q, s2)
+        mism = check_forward(ref_f, Wq=host_bits(e.Wq), codes=unpack_codes(host(e.codes)), scales=host(e.scales))
+        skip = block_mask(mism)
+        skq = np.repeat(skip, 2, axis=1)
+        _, gm, gq = oracle.step(Wb, Gb, m, q, *st, s2, step, want_wq=False)
+        assert_close(host(e.dm), gm, "dm", skip)
+        assert_close(host(e.dq), gq, "dq", skq)
+        assert_close(host(e.m), m, "m", skip)
+        assert_close(host(e.q), q, "q", skq)
+        assert_close(host(e.m_exp_avg), st[0], "m exp_avg", skip)
+        assert_close(host(e.m_exp_avg_sq), st[1], "m exp_avg_sq", skip)
+        assert_close(host(e.q_exp_avg), st[2], "q exp_avg", skq)
+        assert_close(host(e.q_exp_avg_sq), st[3], "q exp_avg_sq", skq)
+
+
+def test_step_accumulate_and_pack_multi(F):
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    shapes = [(37, 1040), (64, 512)]
+    ents = _entries(shapes, 40)
+    g = torch.Generator(device="cuda").manual_seed(7)
+    for e in ents:
+        e.dm.copy_(synth.normal(e.dm.shape, 0, 1e-5, g, "cuda"))
+        e.dq.copy_(synth.normal(e.dq.shape, 0, 1e-7, g, "cuda"))
+    host_in = [(host_bits(e.W), host_bits(e.dWq), host(e.m).copy(), host(e.q).copy(), host(e.dm).copy(),
+                host(e.dq).copy()) for e in ents]
+    tab = FocusTable(ents)
+    tab.s2()
+    tab.pack()          # codes/scales of the generated m, q; W' is not written by the pack
+    torch.cuda.synchronize()
+    for e, (Wb, _, m, q, _, _) in zip(ents, host_in):
+        s2 = oracle.s2(Wb)
+        codes, scales, _ = oracle.pack(Wb, m, q, s2)
+        np.testing.assert_array_equal(host(e.scales), scales)
+        ref = oracle.fwd(Wb, m, q, s2)
+        check_forward(ref, codes=unpack_codes(host(e.codes)))
+    tab.step(1, hparams(), flags=F.FOCUS_STEP_ACCUMULATE | F.FOCUS_STEP_WRITE_GRAD)
+    assert F.focus_get_error() == 0
+    for e, (Wb, Gb, m, q, dm0, dq0) in zip(ents, host_in):
+        s2 = oracle.s2(Wb)
+        z = [np.zeros_like(m), np.zeros_like(m), np.zeros_like(q), np.zeros_like(q)]
+        _, gm, gq = oracle.step(Wb, Gb, m, q, *z, s2, 1, want_wq=False, dm_acc=dm0, dq_acc=dq0)
+        assert_close(host(e.dm), gm, "accumulated dm")
+        assert_close(host(e.dq), gq, "accumulated dq")
+        assert_close(host(e.m), m, "m"); assert_close(host(e.q), q, "q")
+
+
+def test_pack_multi_leaves_wq_alone(F):
+    from fp4_post_weight_b200.table import FocusTable
+    ents = _entries([(16, 256)], 60)
+    for e in ents:
+        e.Wq.fill_(3.0)
+    tab = FocusTable(ents)
+    tab.s2()
+    tab.pack()
+    torch.cuda.synchronize()
+    assert bool((ents[0].Wq == 3.0).all())
+
+
+def test_worked_example_on_gpu(F):
+    here = os.path.dirname(os.path.abspath(__file__))
+    gold = json.load(open(os.path.join(here, "golden", "worked_block.json")))
+    Wf = torch.tensor(gold["W"], dtype=torch.float32)
+    W = Wf.to(torch.bfloat16).cuda()
+    assert torch.equal(W.float().cpu(), Wf)
+    m = torch.tensor(gold["m"], dtype=torch.float32).cuda()
+    q = torch.tensor(gold["q"], dtype=torch.float32).cuda()
+    ex = gold["expected"]
+    ws = torch.empty(16, dtype=torch.uint8, device="cuda")
+    s2 = torch.zeros(1, device="cuda")
+    F.focus_s2(W, s2, ws)
+    assert host(s2)[0] == np.float32(ex["s2"])
+    Wq = torch.empty_like(W)
+    F.focus_fwd(W, m, q, ex["s2"], Wq)
+    want = torch.tensor(ex["Wq"], dtype=torch.float32).to(torch.bfloat16)
+    assert np.array_equal(host_bits(Wq), host_bits(want))
+    for r, c in ex["negative_zero_Wq"]:
+        assert host_bits(Wq)[r, c] == 0x8000
+    codes = torch.empty((2, 16), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((2, 2), dtype=torch.uint8, device="cuda")
+    F.focus_pack_nvfp4(W, m, q, ex["s2"], codes, scales, torch.zeros(1, device="cuda"))
+    np.testing.assert_array_equal(unpack_codes(host(codes)), np.array(ex["codes"], np.uint8))
+    np.testing.assert_array_equal(host(scales), np.array(ex["scales"], np.uint8))
+    ones = torch.ones_like(W)
+    dm = torch.empty((2, 2), device="cuda"); dq = torch.empty((2, 4), device="cuda")
+    F.focus_ste_bwd(W, ones, m, q, ex["s2"], dm, dq)
+    np.testing.assert_array_equal(host(dm), np.array(ex["dm"], np.float32))
+    np.testing.assert_array_equal(host(dq), np.array(ex["dq"], np.float32))
+
+
+def test_codec_sweep(F):
+    """E4M3 and E2M1 decisions on crafted blocks: x on every E4M3 midpoint and
+    its neighbours (A = 0.375 = 6*s2 with s2 = 2^-4, so x = fl(0.375*m)/0.375),
+    plus E2M1 ties and signed zeros through y = w/D."""
+    mids = []
+    for b in range(0x08, 0x7E):
+        e, mn = (b >> 3) & 15, b & 7
+        v = (1 + mn / 8) * 2.0 ** (e - 7)
+        e2, mn2 = (e, mn + 1) if mn < 7 else (e + 1, 0)
+        v2 = (1 + mn2 / 8) * 2.0 ** (e2 - 7)
+        mids.append((v + v2) / 2)
+    xs = []
+    for x in mids:
+        x32 = np.float32(x)
+        xs += [x32, np.nextafter(x32, np.float32(0)), np.nextafter(x32, np.float32(1e9))]
+    rng = np.random.default_rng(0)
+    xs += list(np.exp2(rng.uniform(-8, 10, 20000)).astype(np.float32))
+    n = len(xs)
+    m = torch.tensor(np.array(xs, np.float32)).view(n, 1).cuda()
+    Wf = torch.zeros(n, 16)
+    Wf[:, 0] = 0.375
+    tvals = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.0, 0.1, -0.1, 6.0, 7.0, -7.0, 3.0]
+    W = Wf.to(torch.bfloat16).cuda()
+    q = torch.zeros((n, 2), device="cuda")
+    s2 = 2.0 ** -4
+    codes = torch.empty((n, 8), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((n, 1), dtype=torch.uint8, device="cuda")
+    F.focus_pack_nvfp4(W, m, q, s2, codes, scales, torch.zeros(1, device="cuda"))
+    ref = oracle.fwd(host_bits(W), host(m), host(q), s2)
+    np.testing.assert_array_equal(host(scales), ref.scales)
+    # E2M1: elements t * D for every block scale reached above (D = S * 0.5 * s2)
+    S = np.array([oracle.e4m3_decode(int(b)) for b in ref.scales[:, 0]], np.float64)
+    D = S * 0.5 * s2
+    for j, t in enumerate(tvals):
+        val = np.float32(t) * D.astype(np.float32)
+        Wf[:, 1 + j] = torch.tensor(val)
+    W2 = Wf.to(torch.bfloat16).cuda()
+    F.focus_pack_nvfp4(W2, m, q, s2, codes, scales, torch.zeros(1, device="cuda"))
+    Wq = torch.empty_like(W2)
+    F.focus_fwd(W2, m, q, s2, Wq)
+    ref2 = oracle.fwd(host_bits(W2), host(m), host(q), s2)
+    np.testing.assert_array_equal(host(scales), ref2.scales)
+    np.testing.assert_array_equal(unpack_codes(host(codes)), ref2.codes)
+    np.testing.assert_array_equal(host_bits(Wq), ref2.Wq)
+
+
+def test_nonfinite_input_sets_flag(F):
+    W, m, q, _ = make((4, 64), 5)
+    W[1, 7] = float("nan")
+    Wq = torch.empty_like(W)
+    assert F.focus_get_error() == 0
+    F.focus_fwd(W, m, q, 1e-4, Wq)
+    assert F.focus_get_error() == F.FOCUS_OK + 7
+    assert F.focus_get_error() == 0          # cleared
+    W[1, 7] = 0.0
+    m[0, 0] = float("inf")
+    F.focus_fwd(W, m, q, 1e-4, Wq)
+    assert F.focus_get_error() == 7
