@@ -148,14 +148,19 @@ class ClockSampler:
 # the workload
 # ---------------------------------------------------------------------------
 
-def build_model(rank: int, device):
+def model_tensors(layers: int):
+    import synth
+    return synth.LLAMA_8B.tensors()[:7 * layers]
+
+
+def build_model(rank: int, device, layers: int = 32):
     import torch
 
     from fp4_post_weight_b200 import dist as D
     import synth
     from fp4_post_weight_b200.table import Entry
     ents = []
-    for j, (_, sh) in enumerate(synth.LLAMA_8B.tensors()):
+    for j, (_, sh) in enumerate(model_tensors(layers)):
         t = synth.llama_8b_tensor(j, sh, device, seed_base=D.seed_base(rank))
         o, i = sh
         e = Entry(W=t.W, m=t.m, q=t.q, s2=torch.zeros(1, device=device), dWq=t.dWq,
@@ -178,8 +183,8 @@ def run_ours(args, world, rank, local):
     init_dist(world, local)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    ents = build_model(rank, dev)
-    N = synth.LLAMA_8B.n_elements()
+    ents = build_model(rank, dev, args.layers)
+    N = sum(o * i for _, (o, i) in model_tensors(args.layers))
     # the step writes W' (no codes: the export pack after the update writes those)
     step_tab = FocusTable([dataclasses.replace(e, codes=None, scales=None) for e in ents])
     pack_tab = FocusTable(ents)
@@ -222,7 +227,11 @@ def run_ours(args, world, rank, local):
     D.barrier()
     clk = clocks.stop()
     ms = start.elapsed_time(end)
-    step_kernel_ms = sum(a.elapsed_time(b) for a, b in kev) / args.steps
+    kms = [a.elapsed_time(b) for a, b in kev]
+    step_kernel_ms = sum(kms) / args.steps
+    if max(kms) > 1.5 * min(kms):
+        print(f"warning: fused-step launch times vary from {min(kms):.2f} to {max(kms):.2f} ms "
+              "(another job on this GPU?)", file=sys.stderr)
     ms_max = D.max_over_ranks(ms)
     st = F.focus_get_error()
     if st != 0:
@@ -249,13 +258,15 @@ def run_ours(args, world, rank, local):
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded N(0,0.02) bf16 weights of the Llama-3.1-8B linear shapes; "
                         "no checkpoint)",
-                "config": {"workload": WORKLOAD, "tensors": len(ents), "elements_per_gpu": N,
-                           "l2": "inputs larger than L2 (57.6 GB resident per GPU vs 126 MB L2)",
+                "config": {"workload": WORKLOAD if args.layers == 32 else
+                           f"first {args.layers} layers of: " + WORKLOAD, "tensors": len(ents), "elements_per_gpu": N,
+                           "l2": f"inputs larger than L2 ({N * 8.25 / 1e9:.1f} GB resident per GPU vs 126 MB L2)",
                            "parallelism": f"dp{world} (one model per GPU, no collective)",
                            "bytes_per_elem_step": BYTES_S2 + BYTES_STEP + BYTES_PACK},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": 4 * args.steps, "clocks": clk,
-                "kernel_ms": {"fused_step": round(step_kernel_ms, 4)}}
+                "kernel_ms": {"fused_step": round(step_kernel_ms, 4), "fused_step_min": round(min(kms), 4),
+                              "fused_step_max": round(max(kms), 4)}}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -417,6 +428,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--layers", type=int, default=32, help="decoder layers of the 8B shapes (32 = all)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")

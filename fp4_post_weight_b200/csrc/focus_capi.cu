@@ -36,9 +36,18 @@ int device_info(DeviceInfo **out) {
     std::call_once(g_once[dev], [dev] {
         DeviceInfo &d = g_info[dev];
         cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_fwd, tile_kernel<KIND_FWD>, THREADS, 0);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_bwd, tile_kernel<KIND_BWD>, THREADS, 0);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_step, tile_kernel<KIND_STEP>, THREADS, 0);
+        cudaFuncSetAttribute(pipe_kernel<KIND_FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)stage_smem_bytes<KIND_FWD>());
+        cudaFuncSetAttribute(pipe_kernel<KIND_BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)stage_smem_bytes<KIND_BWD>());
+        cudaFuncSetAttribute(pipe_kernel<KIND_STEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)stage_smem_bytes<KIND_STEP>());
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_fwd, pipe_kernel<KIND_FWD>, CTA_THREADS,
+                                                      stage_smem_bytes<KIND_FWD>());
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_bwd, pipe_kernel<KIND_BWD>, CTA_THREADS,
+                                                      stage_smem_bytes<KIND_BWD>());
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_step, pipe_kernel<KIND_STEP>, CTA_THREADS,
+                                                      stage_smem_bytes<KIND_STEP>());
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_amax, amax_tiles_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_adam, adamw_kernel, THREADS, 0);
     });
@@ -51,9 +60,13 @@ int device_info(DeviceInfo **out) {
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// A tensor holds at most 2^31 - 2^16 blocks (about 3.4e10 weights), so that
+// block and sub-block indices within it fit 32-bit arithmetic in the kernels.
+constexpr int64_t MAX_BLOCKS = (INT64_C(1) << 31) - (INT64_C(1) << 16);
+
 int check_shape(int64_t out, int64_t in) {
     if (out < 0 || in < 0 || (in % 16) != 0) return FOCUS_ERR_SHAPE;
-    if (in > 0 && out > (INT64_C(1) << 58) / in) return FOCUS_ERR_SHAPE;
+    if (in > 0 && out > MAX_BLOCKS / (in / 16 > 0 ? in / 16 : 1)) return FOCUS_ERR_SHAPE;
     return FOCUS_OK;
 }
 
@@ -101,7 +114,7 @@ Hyper make_hyper(float lr_m, float lr_q, float beta1, float beta2, float eps, fl
     h.one_m_beta1 = (float)(1.0 - (double)beta1);
     h.beta2 = beta2;
     h.one_m_beta2 = (float)(1.0 - (double)beta2);
-    h.bc2_sqrt = (float)std::sqrt(bc2);
+    h.inv_bc2_sqrt = (float)(1.0 / std::sqrt(bc2));
     h.eps = eps;
     return h;
 }
@@ -129,7 +142,7 @@ int launch_on(const Args &a, cudaStream_t s) {
     const int occ = KIND == KIND_FWD ? di->occ_fwd : (KIND == KIND_BWD ? di->occ_bwd : di->occ_step);
     int64_t grid = grid_for(a.total_tiles, di->sms, occ);
     if (grid < 1) grid = 1;   // the pack of an empty tensor still writes its tensor scale
-    tile_kernel<KIND><<<(unsigned)grid, THREADS, 0, s>>>(a);
+    pipe_kernel<KIND><<<(unsigned)grid, CTA_THREADS, stage_smem_bytes<KIND>(), s>>>(a);
     return launch_status();
 }
 

@@ -9,14 +9,21 @@
 // Work decomposition.  A tensor W[out, in] with in % 16 == 0 is a flat array of
 // nblk = out*in/16 blocks: m[blk] and q[2*blk + k] index it directly, whatever
 // the row length.  Work is cut into tiles of TILE_BLOCKS blocks; a persistent
-// grid walks the tiles of every tensor of a table.  Inside a tile each 16-block
-// is owned by a pair of adjacent lanes, lane parity k = sub-block k: a lane
-// loads its 8 weights (16 bytes) of W and of dW', its q and q moments, and (with
-// its partner) the block's m.  A warp therefore reads 512 contiguous bytes of W
-// per slot, 128 bytes of q, 64 of m: every access is a full, coalesced sector.
-// The block maximum and the m-gradient are combined across the pair with one
-// shuffle each.  Nothing is staged through shared memory: every byte is used
-// once by the lane that loaded it.
+// grid walks the tiles of every tensor of a table.
+//
+// Staging.  Each CTA runs one producer warp and NC_WARPS consumer warps over a
+// ring of shared-memory stages (focus_pipeline.cuh).  For a full tile the
+// producer issues one 1-D bulk copy per input array (W, dW', m, q, the AdamW
+// moments), all completing on the stage's mbarrier; a partial tile (the ragged
+// end of a tensor) is read by the consumers straight from global memory.  The
+// prefetch depth is therefore set by the number of stages, not by registers.
+//
+// Inside a tile each 16-block is owned by a pair of adjacent consumer lanes,
+// lane parity k = sub-block k: a lane takes its 8 weights (16 bytes) of W and
+// of dW', its q and q moments, and (with its partner) the block's m.  The block
+// maximum and the m-gradient are combined across the pair with one shuffle
+// each.  Outputs go from registers straight to global memory, coalesced: a warp
+// writes 512 contiguous bytes of W', 128 of q.
 //
 // Exactness.  Forward decisions (S_b, codes, w') are taken in binary32 with
 // explicit round-to-nearest intrinsics (__fmul_rn / __fdiv_rn cannot be fused
@@ -30,13 +37,16 @@
 #include <cuda_runtime.h>
 
 #include "focus.h"
+#include "focus_device.cuh"
+#include "focus_pipeline.cuh"
 
 namespace focus {
 
-constexpr int TILE_BLOCKS = 256;                 // 16-blocks per tile (4096 weights)
-constexpr int THREADS = 256;                     // threads per CTA
-constexpr int PAIRS = THREADS / 2;               // blocks handled per slot
-constexpr int SLOTS = TILE_BLOCKS / PAIRS;       // slots per thread per tile
+constexpr int NC_WARPS = 8;                      // consumer warps per CTA
+constexpr int CONSUMERS = NC_WARPS * 32;         // consumer threads
+constexpr int CTA_THREADS = CONSUMERS + 32;      // plus one producer warp
+constexpr int THREADS = 256;                     // threads of the other kernels
+constexpr int TILE_BLOCKS = CONSUMERS;           // 16-blocks per tile (4096 weights): one per consumer thread
 constexpr unsigned FULL = 0xffffffffu;
 
 // Sticky error word read by focus_get_error(): bit 0 a non-finite input,
@@ -45,15 +55,6 @@ constexpr unsigned FULL = 0xffffffffu;
 __device__ unsigned int g_error_flags = 0;
 
 enum Kind : int { KIND_FWD = 0, KIND_BWD = 1, KIND_STEP = 2 };
-
-struct Hyper {
-    float lr_m_step, lr_q_step;   // lr / (1 - beta1^t)
-    float decay_m, decay_q;       // 1 - lr*wd
-    float beta1, one_m_beta1;
-    float beta2, one_m_beta2;
-    float bc2_sqrt;               // sqrt(1 - beta2^t)
-    float eps;
-};
 
 struct Args {
     const focus_tensor_desc *table;  // device table, or nullptr: use `one`
@@ -67,73 +68,6 @@ struct Args {
     int write_grad;                  // step: FOCUS_STEP_WRITE_GRAD
     Hyper hp;
 };
-
-// ---------------------------------------------------------------------------
-// scalar helpers
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
-
-// Two binary32 -> packed bf16x2, round to nearest even ("lo" in bits 0-15).
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    uint32_t r;
-    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
-// E4M3 byte of x, round to nearest even (x in [2^-6, 448]).
-__device__ __forceinline__ uint32_t e4m3_byte(float x) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
-    return (uint32_t)r & 0xffu;
-}
-
-// Value of a normal E4M3 byte: exponent field e -> 2^(e-7), mantissa bits
-// shifted into the binary32 mantissa: bits = (byte << 20) + (120 << 23).
-__device__ __forceinline__ float e4m3_normal_value(uint32_t b) {
-    return __uint_as_float((b << 20) + 0x3C000000u);
-}
-
-// Two E2M1 codes (nearest, ties to even, saturating at +-6): lo in bits 0-3,
-// hi in bits 4-7.  The sign bit of each code is then set from the sign of its
-// input, so a negative value that rounds to zero keeps its sign (-0 = 0x8).
-__device__ __forceinline__ uint32_t e2m1_pair(float lo, float hi) {
-    uint32_t r;
-    asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u32.u8 %0, t; }"
-        : "=r"(r) : "f"(hi), "f"(lo));
-    r |= ((__float_as_uint(lo) >> 31) << 3) | ((__float_as_uint(hi) >> 31) << 7);
-    return r;
-}
-
-// Values of the two E2M1 codes in a byte, as binary32 (exact).
-__device__ __forceinline__ void e2m1_pair_values(uint32_t byte, float &lo, float &hi) {
-    uint32_t h2;
-    asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "r"(byte));
-    float a, b;
-    asm("{ .reg .b16 l, h; mov.b32 {l, h}, %2; cvt.f32.f16 %0, l; cvt.f32.f16 %1, h; }"
-        : "=f"(a), "=f"(b) : "r"(h2));
-    lo = a;
-    hi = b;
-}
-
-// sigmoid(q) rounded once to binary32 from a binary64 evaluation of 1/(1+e^-q).
-__device__ __forceinline__ float sigmoid_rn(float q) {
-    double t = exp(-(double)q);
-    return (float)(1.0 / (1.0 + t));
-}
-
-__device__ __forceinline__ bool finitef(float x) { return (__float_as_uint(x) & 0x7f800000u) != 0x7f800000u; }
-
-// One AdamW update in binary32: decoupled decay, bias-corrected moments.
-__device__ __forceinline__ void adamw_one(float &p, float g, float &v1, float &v2, float step_size,
-                                          float decay, const Hyper &h) {
-    p = p * decay;
-    v1 = h.beta1 * v1 + h.one_m_beta1 * g;
-    v2 = h.beta2 * v2 + h.one_m_beta2 * (g * g);
-    float denom = __fdiv_rn(sqrtf(v2), h.bc2_sqrt) + h.eps;
-    p = p - step_size * __fdiv_rn(v1, denom);
-}
 
 // ---------------------------------------------------------------------------
 // tensor lookup
@@ -166,176 +100,389 @@ __device__ __forceinline__ void load_tensor(const Args &a, int t, TensorRef &r) 
 // the tile engine
 // ---------------------------------------------------------------------------
 
-struct Slot {
-    uint4 w, g;
+// One 16-block's inputs as its consumer thread holds them.
+struct Block {
+    uint32_t w[8];          // W, bf16 pairs
+    uint32_t g[8];          // dW', bf16 pairs
     float m, mv1, mv2;
-    float q, qv1, qv2;
-    float gm_in, gq_in;
-    int64_t blk;
+    float q[2], qv1[2], qv2[2];
+    float gm_in, gq_in[2];
+    uint32_t blk;           // block index within its tensor (tensors hold fewer than 2^31 blocks)
     bool valid;
 };
 
+// A block's inputs straight from global memory (ragged tiles).
 template <int KIND>
-__device__ __forceinline__ void load_slot(const TensorRef &T, const Args &a, Slot &s, int64_t blk, int k) {
-    s.blk = blk;
-    s.valid = blk < T.nblk;
-    const int64_t sb = 2 * blk + k;                    // sub-block index
-    if (s.valid) {
-        s.w = __ldcs(reinterpret_cast<const uint4 *>(T.d.W) + sb);
-        if (KIND != KIND_FWD) s.g = __ldcs(reinterpret_cast<const uint4 *>(T.d.dWq) + sb);
-        s.m = T.d.m[blk];
-        s.q = T.d.q[sb];
-        if (KIND == KIND_STEP) {
-            s.mv1 = T.d.m_exp_avg[blk];
-            s.mv2 = T.d.m_exp_avg_sq[blk];
-            s.qv1 = T.d.q_exp_avg[sb];
-            s.qv2 = T.d.q_exp_avg_sq[sb];
-        }
-        if (KIND != KIND_FWD && a.accumulate) {
-            s.gm_in = T.d.dm[blk];
-            s.gq_in = T.d.dq[sb];
-        }
-    } else {
-        s.w = make_uint4(0, 0, 0, 0);
-        s.g = make_uint4(0, 0, 0, 0);
-        s.m = 1.0f; s.q = 0.0f;
-        s.mv1 = s.mv2 = s.qv1 = s.qv2 = 0.0f;
-        s.gm_in = s.gq_in = 0.0f;
+__device__ __forceinline__ void load_block_global(const TensorRef &T, const Args &a, Block &B, uint32_t blk) {
+    B.blk = blk;
+    B.valid = blk < (uint32_t)T.nblk;
+    if (!B.valid) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) B.w[j] = B.g[j] = 0u;
+        B.m = 1.0f; B.mv1 = B.mv2 = 0.0f; B.gm_in = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 2; ++k) { B.q[k] = 0.0f; B.qv1[k] = B.qv2[k] = 0.0f; B.gq_in[k] = 0.0f; }
+        return;
+    }
+    const uint4 *W = reinterpret_cast<const uint4 *>(T.d.W) + 2u * blk;
+    const uint4 w0 = __ldcs(W), w1 = __ldcs(W + 1);
+    B.w[0] = w0.x; B.w[1] = w0.y; B.w[2] = w0.z; B.w[3] = w0.w;
+    B.w[4] = w1.x; B.w[5] = w1.y; B.w[6] = w1.z; B.w[7] = w1.w;
+    if (KIND != KIND_FWD) {
+        const uint4 *G = reinterpret_cast<const uint4 *>(T.d.dWq) + 2u * blk;
+        const uint4 g0 = __ldcs(G), g1 = __ldcs(G + 1);
+        B.g[0] = g0.x; B.g[1] = g0.y; B.g[2] = g0.z; B.g[3] = g0.w;
+        B.g[4] = g1.x; B.g[5] = g1.y; B.g[6] = g1.z; B.g[7] = g1.w;
+    }
+    B.m = T.d.m[blk];
+    const float2 q = reinterpret_cast<const float2 *>(T.d.q)[blk];
+    B.q[0] = q.x; B.q[1] = q.y;
+    if (KIND == KIND_STEP) {
+        B.mv1 = T.d.m_exp_avg[blk];
+        B.mv2 = T.d.m_exp_avg_sq[blk];
+        const float2 v1 = reinterpret_cast<const float2 *>(T.d.q_exp_avg)[blk];
+        const float2 v2 = reinterpret_cast<const float2 *>(T.d.q_exp_avg_sq)[blk];
+        B.qv1[0] = v1.x; B.qv1[1] = v1.y; B.qv2[0] = v2.x; B.qv2[1] = v2.y;
+    }
+    if (KIND != KIND_FWD && a.accumulate) {
+        B.gm_in = T.d.dm[blk];
+        const float2 gq = reinterpret_cast<const float2 *>(T.d.dq)[blk];
+        B.gq_in[0] = gq.x; B.gq_in[1] = gq.y;
     }
 }
 
+// The forward, the straight-through gradients and the AdamW update of one block.
 template <int KIND>
-__device__ __forceinline__ void compute_slot(const TensorRef &T, const Args &a, Slot &s, int k) {
-    const uint32_t wv[4] = {s.w.x, s.w.y, s.w.z, s.w.w};
-
-    // A_b = max |w| over the block: max of the bf16 magnitude bit patterns of this
-    // lane's 8 weights, then of the pair.  (A NaN or infinity sorts above every
-    // finite magnitude, which is how it is detected.)
-    uint32_t amax2 = __vmaxu2(__vmaxu2(wv[0] & 0x7fff7fffu, wv[1] & 0x7fff7fffu),
-                              __vmaxu2(wv[2] & 0x7fff7fffu, wv[3] & 0x7fff7fffu));
-    uint32_t abits = max(amax2 & 0xffffu, amax2 >> 16);
-    abits = max(abits, __shfl_xor_sync(FULL, abits, 1));
+__device__ __forceinline__ void compute_block(const TensorRef &T, const Args &a, Block &B) {
+    // A_b = max |w| over the block: max of the bf16 magnitude bit patterns (a NaN
+    // or an infinity sorts above every finite magnitude, which is how it is found)
+    uint32_t am = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) am = __vmaxu2(am, B.w[j] & 0x7fff7fffu);
+    const uint32_t abits = max(am & 0xffffu, am >> 16);
     const float A = __uint_as_float(abits << 16);
-    bool bad = s.valid && (abits >= 0x7f80u || !finitef(s.m) || !finitef(s.q));
+    const bool bad = B.valid && (abits >= 0x7f80u || !finitef(B.m) || !finitef(B.q[0]) || !finitef(B.q[1]));
 
     // S_b = e4m3(clamp(fl(fl(A*m)/fl(6*s2)), 2^-6, 448)), scale 1 when the scaled max is 0
-    const float x = __fdiv_rn(__fmul_rn(A, s.m), T.den);
+    const float x = __fdiv_rn(__fmul_rn(A, B.m), T.den);
     const bool inS = (x != 0.0f) && (x >= 0x1p-6f) && (x <= 448.0f);
     float xc = (x == 0.0f) ? 1.0f : x;
     xc = fminf(fmaxf(xc, 0x1p-6f), 448.0f);
     const uint32_t sbyte = e4m3_byte(xc);
-    const float S = e4m3_normal_value(sbyte);
+    const float S = e4m3_normal_f32(sbyte);
+    const uint16_t S_h = (uint16_t)e4m3_normal_f16_bits(sbyte);
+    const uint64_t s2_2 = f2_pack(T.s2, T.s2);
 
-    // D_k = fl(fl(S*sigmoid(q_k))*s2); y_i = fl(w_i/D_k); c_i = E2M1(clamp(y_i, -6, 6))
-    const float sig = sigmoid_rn(s.q);
-    const float D = __fmul_rn(__fmul_rn(S, sig), T.s2);
-    float y[8];
+    const bool want_wq = KIND != KIND_BWD && a.write_wq && T.d.Wq != nullptr && B.valid;
+    float sig[2], sq[2];
+    uint64_t gcs2 = 0ull;                       // sum of g * (c*S), pairwise
+    uint32_t codes[2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        y[2 * j] = __fdiv_rn(bf16_lo(wv[j]), D);
-        y[2 * j + 1] = __fdiv_rn(bf16_hi(wv[j]), D);
-    }
-    uint32_t codes = 0;
+    for (int k = 0; k < 2; ++k) {
+        // D_k = fl(fl(S*sigmoid(q_k))*s2); y_i = fl(w_i/D_k); c_i = E2M1(clamp(y_i, -6, 6))
+        sig[k] = sigmoid_rn(B.q[k]);
+        const float D = __fmul_rn(__fmul_rn(S, sig[k]), T.s2);
+        uint64_t y2[4];
+        if (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f) {
+            const float nr = -__frcp_rn(D);
+            const uint64_t D2 = f2_pack(D, D), nr2 = f2_pack(nr, nr);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) codes |= e2m1_pair(y[2 * j], y[2 * j + 1]) << (8 * j);
-    float c[8];
+            for (int j = 0; j < 4; ++j) y2[j] = div_by_f2(bf16x2_neg_f2(B.w[4 * k + j]), D2, nr2);
+        } else {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) e2m1_pair_values((codes >> (8 * j)) & 0xffu, c[2 * j], c[2 * j + 1]);
-
-    // forward outputs: w' = bf16(fl(fl(c*S)*s2)), NVFP4 codes and scale byte
-    if (s.valid) {
-        if (a.write_wq && T.d.Wq) {
-            uint4 o;
-            o.x = pack_bf16x2(__fmul_rn(__fmul_rn(c[0], S), T.s2), __fmul_rn(__fmul_rn(c[1], S), T.s2));
-            o.y = pack_bf16x2(__fmul_rn(__fmul_rn(c[2], S), T.s2), __fmul_rn(__fmul_rn(c[3], S), T.s2));
-            o.z = pack_bf16x2(__fmul_rn(__fmul_rn(c[4], S), T.s2), __fmul_rn(__fmul_rn(c[5], S), T.s2));
-            o.w = pack_bf16x2(__fmul_rn(__fmul_rn(c[6], S), T.s2), __fmul_rn(__fmul_rn(c[7], S), T.s2));
-            __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + (2 * s.blk + k), o);
+            for (int j = 0; j < 4; ++j)
+                y2[j] = f2_pack(__fdiv_rn(bf16_lo(B.w[4 * k + j]), D), __fdiv_rn(bf16_hi(B.w[4 * k + j]), D));
         }
-        if (T.d.codes) reinterpret_cast<uint32_t *>(T.d.codes)[2 * s.blk + k] = codes;
-        if (T.d.scales && k == 0) T.d.scales[s.blk] = (uint8_t)sbyte;
+        uint32_t code = 0u;
+        uint64_t cs2[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t byte = e2m1_pair(f2_lo(y2[j]), f2_hi(y2[j]));
+            code |= byte << (8 * j);
+            const uint32_t h2 = e2m1_pair_f16x2(byte);
+            cs2[j] = f2_pack(mul_f16_exact(lo16(h2), S_h), mul_f16_exact(hi16(h2), S_h));   // c*S, exact
+        }
+        codes[k] = code;
+        // w' = bf16(fl(fl(c*S)*s2))
+        if (want_wq) {
+            uint4 o;
+            uint64_t p;
+            p = f2_mul(cs2[0], s2_2); o.x = pack_bf16x2(f2_lo(p), f2_hi(p));
+            p = f2_mul(cs2[1], s2_2); o.y = pack_bf16x2(f2_lo(p), f2_hi(p));
+            p = f2_mul(cs2[2], s2_2); o.z = pack_bf16x2(f2_lo(p), f2_hi(p));
+            p = f2_mul(cs2[3], s2_2); o.w = pack_bf16x2(f2_lo(p), f2_hi(p));
+            __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + (2u * B.blk + (uint32_t)k), o);
+        }
+        sq[k] = 0.0f;
+        if (KIND != KIND_FWD) {
+            // straight-through sums: sum g*c*S over the block, sum g*y inside the clamp per sub-block
+            uint64_t sq2 = 0ull;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint64_t g2 = bf16x2_f2(B.g[4 * k + j]);
+                gcs2 = f2_fma(g2, cs2[j], gcs2);
+                const float ylo = f2_lo(y2[j]), yhi = f2_hi(y2[j]);
+                const uint64_t yin2 = f2_pack(fabsf(ylo) <= 6.0f ? ylo : 0.0f, fabsf(yhi) <= 6.0f ? yhi : 0.0f);
+                sq2 = f2_fma(g2, yin2, sq2);
+            }
+            sq[k] = f2_lo(sq2) + f2_hi(sq2);
+        }
+    }
+    if (B.valid) {
+        if (T.d.codes) {
+            uint2 cc; cc.x = codes[0]; cc.y = codes[1];
+            reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
+        }
+        if (T.d.scales) T.d.scales[B.blk] = (uint8_t)sbyte;
     }
 
     if (KIND != KIND_FWD) {
-        // straight-through gradients: t_i = in_i ? c_i - y_i : c_i
-        const uint32_t gv[4] = {s.g.x, s.g.y, s.g.z, s.g.w};
-        float sm = 0.0f, sq = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float g = (j & 1) ? bf16_hi(gv[j >> 1]) : bf16_lo(gv[j >> 1]);
-            const bool in = fabsf(y[j]) <= 6.0f;
-            const float t = in ? c[j] - y[j] : c[j];
-            sm = fmaf(g, t, sm);
-            sq = in ? fmaf(g, y[j], sq) : sq;
-        }
-        const float sm_pair = sm + __shfl_xor_sync(FULL, sm, 1);
-        float gm = inS ? (A * (1.0f / 6.0f)) * sm_pair : 0.0f;
-        float gq = -((((1.0f - sig) * S) * T.s2) * sq);
+        // dL/dm = inS*(A/6)*sum g*(c - y_in) = inS*(A/6)*(sum g*c - sum g*y_in)
+        // dL/dq_k = -(1 - sigma_k)*S*s2*sum_k g*y_in
+        const float gc = __fdiv_rn(f2_lo(gcs2) + f2_hi(gcs2), S);
+        float gm = inS ? (A * (1.0f / 6.0f)) * (gc - (sq[0] + sq[1])) : 0.0f;
+        float gq0 = -((((1.0f - sig[0]) * S) * T.s2) * sq[0]);
+        float gq1 = -((((1.0f - sig[1]) * S) * T.s2) * sq[1]);
         if (a.accumulate) {
-            gm = s.gm_in + gm;
-            gq = s.gq_in + gq;
+            gm = B.gm_in + gm;
+            gq0 = B.gq_in[0] + gq0;
+            gq1 = B.gq_in[1] + gq1;
         }
-        if (s.valid && (!finitef(gm) || !finitef(gq)) && !bad) atomicOr(&g_error_flags, 4u);
-
-        if (KIND == KIND_BWD) {
-            if (s.valid) {
-                if (k == 0) T.d.dm[s.blk] = gm;
-                T.d.dq[2 * s.blk + k] = gq;
-            }
-        } else {
-            if (s.valid && a.write_grad) {
-                if (k == 0) T.d.dm[s.blk] = gm;
-                T.d.dq[2 * s.blk + k] = gq;
-            }
-            // AdamW: both lanes of a pair update m identically, lane 0 stores it
-            adamw_one(s.m, gm, s.mv1, s.mv2, a.hp.lr_m_step, a.hp.decay_m, a.hp);
-            adamw_one(s.q, gq, s.qv1, s.qv2, a.hp.lr_q_step, a.hp.decay_q, a.hp);
-            if (s.valid) {
-                const int64_t sb = 2 * s.blk + k;
-                T.d.q[sb] = s.q;
-                T.d.q_exp_avg[sb] = s.qv1;
-                T.d.q_exp_avg_sq[sb] = s.qv2;
-                if (k == 0) {
-                    T.d.m[s.blk] = s.m;
-                    T.d.m_exp_avg[s.blk] = s.mv1;
-                    T.d.m_exp_avg_sq[s.blk] = s.mv2;
-                }
+        if (B.valid && !bad && !(finitef(gm) && finitef(gq0) && finitef(gq1))) atomicOr(&g_error_flags, 4u);
+        if (B.valid && (KIND == KIND_BWD || a.write_grad)) {
+            T.d.dm[B.blk] = gm;
+            reinterpret_cast<float2 *>(T.d.dq)[B.blk] = make_float2(gq0, gq1);
+        }
+        if (KIND == KIND_STEP) {
+            adamw_one(B.m, gm, B.mv1, B.mv2, a.hp.lr_m_step, a.hp.decay_m, a.hp);
+            uint64_t qp = f2_pack(B.q[0], B.q[1]);
+            uint64_t v1 = f2_pack(B.qv1[0], B.qv1[1]), v2 = f2_pack(B.qv2[0], B.qv2[1]);
+            adamw_pair(qp, f2_pack(gq0, gq1), v1, v2, a.hp.lr_q_step, a.hp.decay_q, a.hp);
+            if (B.valid) {
+                T.d.m[B.blk] = B.m;
+                T.d.m_exp_avg[B.blk] = B.mv1;
+                T.d.m_exp_avg_sq[B.blk] = B.mv2;
+                reinterpret_cast<float2 *>(T.d.q)[B.blk] = make_float2(f2_lo(qp), f2_hi(qp));
+                reinterpret_cast<float2 *>(T.d.q_exp_avg)[B.blk] = make_float2(f2_lo(v1), f2_hi(v1));
+                reinterpret_cast<float2 *>(T.d.q_exp_avg_sq)[B.blk] = make_float2(f2_lo(v2), f2_hi(v2));
             }
         }
     }
     if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_error_flags, 1u);
 }
 
+// ---------------------------------------------------------------------------
+// shared-memory stage layout and pipeline depth per kind
+// ---------------------------------------------------------------------------
+
 template <int KIND>
-__global__ void __launch_bounds__(THREADS, 2) tile_kernel(const Args a) {
-    const int k = threadIdx.x & 1;
-    const int pair = threadIdx.x >> 1;
-    if (a.one_scale_out && blockIdx.x == 0 && threadIdx.x == 0) *a.one_scale_out = a.one_s2;
+struct Layout {
+    static constexpr bool G_ = KIND != KIND_FWD;         // dW' and the gradient accumulators
+    static constexpr bool ST = KIND == KIND_STEP;        // AdamW moments
+    static constexpr uint32_t W = 0;
+    static constexpr uint32_t G = W + TILE_BLOCKS * 32;
+    static constexpr uint32_t M = G + (G_ ? TILE_BLOCKS * 32 : 0);
+    static constexpr uint32_t Q = M + TILE_BLOCKS * 4;
+    static constexpr uint32_t MV1 = Q + TILE_BLOCKS * 8;
+    static constexpr uint32_t MV2 = MV1 + (ST ? TILE_BLOCKS * 4 : 0);
+    static constexpr uint32_t QV1 = MV2 + (ST ? TILE_BLOCKS * 4 : 0);
+    static constexpr uint32_t QV2 = QV1 + (ST ? TILE_BLOCKS * 8 : 0);
+    static constexpr uint32_t GM = QV2 + (ST ? TILE_BLOCKS * 8 : 0);
+    static constexpr uint32_t GQ = GM + (G_ ? TILE_BLOCKS * 4 : 0);
+    static constexpr uint32_t BYTES = GQ + (G_ ? TILE_BLOCKS * 8 : 0);   // one stage
+    // bytes the bulk copies of one full tile deliver
+    static __device__ __forceinline__ uint32_t tx_bytes(bool accumulate) {
+        return (accumulate || !G_) ? BYTES : GM;
+    }
+};
+
+template <int KIND> struct Depth;
+template <> struct Depth<KIND_FWD> { static constexpr int STAGES = 6, MIN_CTAS = 3; };
+template <> struct Depth<KIND_BWD> { static constexpr int STAGES = 4, MIN_CTAS = 2; };
+template <> struct Depth<KIND_STEP> { static constexpr int STAGES = 3, MIN_CTAS = 2; };
+
+template <int KIND>
+constexpr uint32_t stage_smem_bytes() { return Depth<KIND>::STAGES * Layout<KIND>::BYTES; }
+
+enum : uint32_t { MODE_BULK = 0, MODE_DIRECT = 1, MODE_SKIP = 2 };
+
+struct StageInfo {
+    int t;             // tensor of the tile
+    uint32_t first;    // first block of the tile within the tensor
+    uint32_t nb;       // blocks in the tile
+    uint32_t mode;     // MODE_*
+};
+
+// A block's inputs from a staged tile (local block lb of the tile).
+template <int KIND>
+__device__ __forceinline__ void load_block_smem(const Args &a, const unsigned char *stage, Block &B, uint32_t lb,
+                                                uint32_t blk) {
+    using L = Layout<KIND>;
+    B.blk = blk;
+    B.valid = true;
+    const uint4 *W = reinterpret_cast<const uint4 *>(stage + L::W) + 2u * lb;
+    const uint4 w0 = W[0], w1 = W[1];
+    B.w[0] = w0.x; B.w[1] = w0.y; B.w[2] = w0.z; B.w[3] = w0.w;
+    B.w[4] = w1.x; B.w[5] = w1.y; B.w[6] = w1.z; B.w[7] = w1.w;
+    if (KIND != KIND_FWD) {
+        const uint4 *G = reinterpret_cast<const uint4 *>(stage + L::G) + 2u * lb;
+        const uint4 g0 = G[0], g1 = G[1];
+        B.g[0] = g0.x; B.g[1] = g0.y; B.g[2] = g0.z; B.g[3] = g0.w;
+        B.g[4] = g1.x; B.g[5] = g1.y; B.g[6] = g1.z; B.g[7] = g1.w;
+    }
+    B.m = reinterpret_cast<const float *>(stage + L::M)[lb];
+    const float2 q = reinterpret_cast<const float2 *>(stage + L::Q)[lb];
+    B.q[0] = q.x; B.q[1] = q.y;
+    if (KIND == KIND_STEP) {
+        B.mv1 = reinterpret_cast<const float *>(stage + L::MV1)[lb];
+        B.mv2 = reinterpret_cast<const float *>(stage + L::MV2)[lb];
+        const float2 v1 = reinterpret_cast<const float2 *>(stage + L::QV1)[lb];
+        const float2 v2 = reinterpret_cast<const float2 *>(stage + L::QV2)[lb];
+        B.qv1[0] = v1.x; B.qv1[1] = v1.y; B.qv2[0] = v2.x; B.qv2[1] = v2.y;
+    }
+    if (KIND != KIND_FWD && a.accumulate) {
+        B.gm_in = reinterpret_cast<const float *>(stage + L::GM)[lb];
+        const float2 gq = reinterpret_cast<const float2 *>(stage + L::GQ)[lb];
+        B.gq_in[0] = gq.x; B.gq_in[1] = gq.y;
+    } else {
+        B.gm_in = 0.0f; B.gq_in[0] = B.gq_in[1] = 0.0f;
+    }
+}
+
+// Next tensor holding `tile`, scanning forward from T (tiles only increase).
+// Returns false when the table has no tensor for it.
+__device__ __forceinline__ bool seek_tensor(const Args &a, int64_t tile, int &t, TensorRef &T, bool &have) {
+    if (have && tile < T.tile_end) return true;
+    const int n = a.table ? a.n_tensors : 1;
+    if (have && t + 1 < n) ++t;
+    for (;;) {
+        load_tensor(a, t, T);
+        if (tile < T.tile_end || t + 1 >= n) break;
+        ++t;
+    }
+    have = true;
+    return tile < T.tile_end;
+}
+
+// The producer: one thread feeding the ring.
+template <int KIND>
+__device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint64_t *full, uint64_t *empty,
+                                        StageInfo *info) {
+    using L = Layout<KIND>;
+    constexpr int S = Depth<KIND>::STAGES;
     int t = 0;
     TensorRef T;
     bool have = false;
-    for (int64_t tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x) {
-        if (!have || tile >= T.tile_end) {
-            // tiles only increase: scan forward from the current tensor, never past the table
-            const int n = a.table ? a.n_tensors : 1;
-            if (have && t + 1 < n) ++t;
-            for (;;) {
-                load_tensor(a, t, T);
-                if (tile < T.tile_end || t + 1 >= n) break;
-                ++t;
-            }
-            have = true;
-            if (tile >= T.tile_end) break;      // total_tiles larger than the table: nothing left
-            if (!T.ok && threadIdx.x == 0) atomicOr(&g_error_flags, 2u);
+    uint32_t pending = 0;             // stages whose last use was filled by bulk copies
+    uint32_t pending_parity = 0;      // and the parity of that use
+    uint32_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++it) {
+        const uint32_t st = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        if (!mbar_wait(smem_u32(&empty[st]), ph ^ 1u)) {
+            atomicOr(&g_error_flags, 8u);
+            break;
         }
-        if (!T.ok) continue;
-        const int64_t first = (tile - T.d.tile_begin) * TILE_BLOCKS;
-        Slot s[SLOTS];
-#pragma unroll
-        for (int u = 0; u < SLOTS; ++u) load_slot<KIND>(T, a, s[u], first + u * PAIRS + pair, k);
-#pragma unroll
-        for (int u = 0; u < SLOTS; ++u) compute_slot<KIND>(T, a, s[u], k);
+        pending &= ~(1u << st);       // the consumers released it: its copies have landed
+        StageInfo inf;
+        const bool found = seek_tensor(a, tile, t, T, have);
+        inf.t = t;
+        inf.first = found ? (uint32_t)(tile - T.d.tile_begin) * TILE_BLOCKS : 0u;
+        const int64_t left = T.nblk - (int64_t)inf.first;
+        inf.nb = found ? (uint32_t)(left < TILE_BLOCKS ? left : TILE_BLOCKS) : 0u;
+        inf.mode = (!found || !T.ok) ? MODE_SKIP : (inf.nb == (uint32_t)TILE_BLOCKS ? MODE_BULK : MODE_DIRECT);
+        if (found && !T.ok) atomicOr(&g_error_flags, 2u);
+        info[st] = inf;
+        const uint32_t bar = smem_u32(&full[st]);
+        if (inf.mode == MODE_BULK) {
+            unsigned char *stage = smem + st * L::BYTES;
+            const uint32_t f = inf.first;
+            mbar_arrive_expect_tx(bar, L::tx_bytes(a.accumulate != 0));
+            bulk_g2s(smem_u32(stage + L::W), reinterpret_cast<const uint4 *>(T.d.W) + 2u * f, TILE_BLOCKS * 32, bar);
+            if (KIND != KIND_FWD)
+                bulk_g2s(smem_u32(stage + L::G), reinterpret_cast<const uint4 *>(T.d.dWq) + 2u * f, TILE_BLOCKS * 32,
+                         bar);
+            bulk_g2s(smem_u32(stage + L::M), T.d.m + f, TILE_BLOCKS * 4, bar);
+            bulk_g2s(smem_u32(stage + L::Q), T.d.q + 2u * f, TILE_BLOCKS * 8, bar);
+            if (KIND == KIND_STEP) {
+                bulk_g2s(smem_u32(stage + L::MV1), T.d.m_exp_avg + f, TILE_BLOCKS * 4, bar);
+                bulk_g2s(smem_u32(stage + L::MV2), T.d.m_exp_avg_sq + f, TILE_BLOCKS * 4, bar);
+                bulk_g2s(smem_u32(stage + L::QV1), T.d.q_exp_avg + 2u * f, TILE_BLOCKS * 8, bar);
+                bulk_g2s(smem_u32(stage + L::QV2), T.d.q_exp_avg_sq + 2u * f, TILE_BLOCKS * 8, bar);
+            }
+            if (KIND != KIND_FWD && a.accumulate) {
+                bulk_g2s(smem_u32(stage + L::GM), T.d.dm + f, TILE_BLOCKS * 4, bar);
+                bulk_g2s(smem_u32(stage + L::GQ), T.d.dq + 2u * f, TILE_BLOCKS * 8, bar);
+            }
+            pending |= 1u << st;
+            pending_parity = (pending_parity & ~(1u << st)) | (ph << st);
+        } else {
+            mbar_arrive(bar);
+        }
     }
+    // Before the CTA may exit, every bulk copy it issued must have landed (normally
+    // the consumers already waited for all of them; this matters after a timeout).
+    for (int st = 0; st < S; ++st)
+        if ((pending >> st) & 1u)
+            if (!mbar_wait(smem_u32(&full[st]), (pending_parity >> st) & 1u)) atomicOr(&g_error_flags, 8u);
+}
+
+// The consumers: NC_WARPS warps computing from the ring.
+template <int KIND>
+__device__ __forceinline__ void consume(const Args &a, const unsigned char *smem, uint64_t *full, uint64_t *empty,
+                                        const StageInfo *info) {
+    using L = Layout<KIND>;
+    constexpr int S = Depth<KIND>::STAGES;
+    const int lane = threadIdx.x & 31;
+    int tcur = -1;
+    TensorRef T;
+    uint32_t it = 0;
+    for (int64_t tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++it) {
+        const uint32_t st = it % S;
+        const uint32_t ph = (it / S) & 1u;
+        if (!mbar_wait(smem_u32(&full[st]), ph)) {
+            if (lane == 0) atomicOr(&g_error_flags, 8u);
+            break;
+        }
+        const StageInfo inf = info[st];
+        if (inf.mode != MODE_SKIP) {
+            if (inf.t != tcur) {
+                load_tensor(a, inf.t, T);
+                tcur = inf.t;
+            }
+            const unsigned char *stage = smem + st * L::BYTES;
+            const uint32_t lb = threadIdx.x;
+            Block B;
+            if (inf.mode == MODE_BULK) load_block_smem<KIND>(a, stage, B, lb, inf.first + lb);
+            else load_block_global<KIND>(T, a, B, inf.first + lb);
+            compute_block<KIND>(T, a, B);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+    }
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(CTA_THREADS, Depth<KIND>::MIN_CTAS) pipe_kernel(const Args a) {
+    constexpr int S = Depth<KIND>::STAGES;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full[S];
+    __shared__ __align__(8) uint64_t empty[S];
+    __shared__ StageInfo info[S];
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < S; ++st) {
+            mbar_init(smem_u32(&full[st]), 1);
+            mbar_init(smem_u32(&empty[st]), NC_WARPS);
+        }
+        mbar_fence_init();
+        if (a.one_scale_out && blockIdx.x == 0) *a.one_scale_out = a.one_s2;
+    }
+    __syncthreads();
+    if (threadIdx.x >= CONSUMERS) {
+        if (threadIdx.x == CONSUMERS) produce<KIND>(a, smem, full, empty, info);
+        return;
+    }
+    consume<KIND>(a, smem, full, empty, info);
 }
 
 // ---------------------------------------------------------------------------
@@ -361,12 +508,12 @@ __global__ void __launch_bounds__(THREADS) amax_tiles_kernel(const Args a, uint3
             have = true;
             if (tile >= T.tile_end) break;      // uniform across the CTA: no barrier is skipped by some threads only
         }
-        // 256 blocks x 32 bytes = 8 KB per tile: two 16-byte loads per thread
+        // TILE_BLOCKS blocks x 32 bytes per tile: two 16-byte loads per thread
         const int64_t first_sb = (tile - T.d.tile_begin) * TILE_BLOCKS * 2;
         const int64_t nsb = 2 * T.nblk;
         uint32_t mx = 0;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < 2 * TILE_BLOCKS / THREADS; ++u) {
             const int64_t sb = first_sb + u * THREADS + threadIdx.x;
             if (sb < nsb) {
                 const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(T.d.W) + sb);

@@ -1,0 +1,66 @@
+"""Exhaustive checks of the kernels' device arithmetic (focus_device.cuh).
+
+* The quotient fl(w/D) from one reciprocal per sub-block with one Markstein
+  correction (scalar and packed f32x2 forms) equals the IEEE division, bit
+  for bit (signed zeros included),
+  for every bf16 significand of w (both signs, and +-0) and every binary32
+  significand of D, at several exponent pairs inside the range the kernels
+  use it for.
+* fl(c*S) through the mixed-precision FMA equals the binary32 product for
+  every E2M1 value and every normal E4M3 scale, and c - y likewise.
+* The E2M1 conversion keeps the sign of negative values that round to zero
+  (code 0x8), which the kernels rely on for the signed-zero reading.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "cuda", "device_checks.cu")
+LIB = os.path.join(HERE, "cuda", "libdevice_checks.so")
+HDR = os.path.join(os.path.dirname(HERE), "fp4_post_weight_b200", "csrc", "focus_device.cuh")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(SRC), os.path.getmtime(HDR)):
+        subprocess.run(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-Xcompiler",
+                        "-fPIC", "-shared", SRC, "-o", LIB], check=True)
+    L = ctypes.CDLL(LIB)
+    L.check_div.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_ulonglong),
+                            ctypes.POINTER(ctypes.c_float), ctypes.c_int]
+    L.check_mixed.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
+    L.e2m1_raw_bytes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    return L
+
+
+@pytest.mark.parametrize("variant", [0, 2], ids=["scalar", "packed"])
+@pytest.mark.parametrize("we,de", [(0, 0), (-7, 3), (-20, -13), (10, -40), (-40, 10), (59, 0), (0, 59), (0, -59),
+                                   (-59, 0), (30, -30), (-30, 29)])
+def test_division_exhaustive(lib, we, de, variant):
+    n = ctypes.c_ulonglong(0)
+    ex = (ctypes.c_float * 4)()
+    assert lib.check_div(we, de, ctypes.byref(n), ex, variant) == 0
+    assert n.value == 0, f"{n.value} quotients differ, e.g. w={ex[0]!r} D={ex[1]!r} got {ex[2]!r} want {ex[3]!r}"
+
+
+def test_mixed_precision_helpers(lib):
+    bad = ctypes.c_ulonglong(0)
+    assert lib.check_mixed(ctypes.byref(bad)) == 0
+    assert bad.value == 0
+
+
+def test_e2m1_conversion_zero_sign(lib):
+    lo = np.array([-0.1, -0.0, -0.25, 0.1, -1e-30, -0.2], np.float32)
+    hi = np.array([0.0, -0.1, 0.2, -0.24, -0.0, -1e-20], np.float32)
+    out = np.zeros(len(lo), np.uint32)
+    assert lib.e2m1_raw_bytes(lo.ctypes.data, hi.ctypes.data, out.ctypes.data, len(lo)) == 0
+    mags = out & 0x77
+    assert np.all(mags == 0)            # every value rounds to a zero magnitude
+    want = (np.signbit(lo).astype(np.uint32) << 3) | (np.signbit(hi).astype(np.uint32) << 7)
+    np.testing.assert_array_equal(out, want)
