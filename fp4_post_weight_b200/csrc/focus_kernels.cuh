@@ -112,8 +112,8 @@ struct Block {
 };
 
 // A block's inputs straight from global memory (ragged tiles).
-template <int KIND>
-__device__ __forceinline__ void load_block_global(const TensorRef &T, const Args &a, Block &B, uint32_t blk) {
+template <int KIND, class TV>
+__device__ __forceinline__ void load_block_global(const TV &T, const Args &a, Block &B, uint32_t blk) {
     B.blk = blk;
     B.valid = blk < (uint32_t)T.nblk;
     if (!B.valid) {
@@ -152,8 +152,11 @@ __device__ __forceinline__ void load_block_global(const TensorRef &T, const Args
 }
 
 // The forward, the straight-through gradients and the AdamW update of one block.
-template <int KIND>
-__device__ __forceinline__ void compute_block(const TensorRef &T, const Args &a, Block &B) {
+// TV is any view of a tensor with members d (descriptor), s2, den and nblk:
+// the consumer warps pass the stage record in shared memory, so the
+// descriptor's pointers are read where used instead of held in registers.
+template <int KIND, class TV>
+__device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block &B) {
     // A_b = max |w| over the block: max of the bf16 magnitude bit patterns (a NaN
     // or an infinity sorts above every finite magnitude, which is how it is found)
     uint32_t am = 0u;
@@ -306,11 +309,17 @@ constexpr uint32_t stage_smem_bytes() { return Depth<KIND>::STAGES * Layout<KIND
 
 enum : uint32_t { MODE_BULK = 0, MODE_DIRECT = 1, MODE_SKIP = 2 };
 
+// The producer's record of one staged tile, read by the consumers from shared
+// memory: the tile's tensor (descriptor, s2, fl(6*s2), block count) and place.
 struct StageInfo {
-    int t;             // tensor of the tile
+    focus_tensor_desc d;
+    int64_t nblk;
+    float s2;
+    float den;
     uint32_t first;    // first block of the tile within the tensor
     uint32_t nb;       // blocks in the tile
     uint32_t mode;     // MODE_*
+    uint32_t pad;
 };
 
 // A block's inputs from a staged tile (local block lb of the tile).
@@ -384,19 +393,24 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
             break;
         }
         pending &= ~(1u << st);       // the consumers released it: its copies have landed
-        StageInfo inf;
+        StageInfo &inf = info[st];
         const bool found = seek_tensor(a, tile, t, T, have);
-        inf.t = t;
-        inf.first = found ? (uint32_t)(tile - T.d.tile_begin) * TILE_BLOCKS : 0u;
-        const int64_t left = T.nblk - (int64_t)inf.first;
-        inf.nb = found ? (uint32_t)(left < TILE_BLOCKS ? left : TILE_BLOCKS) : 0u;
-        inf.mode = (!found || !T.ok) ? MODE_SKIP : (inf.nb == (uint32_t)TILE_BLOCKS ? MODE_BULK : MODE_DIRECT);
+        const uint32_t first = found ? (uint32_t)(tile - T.d.tile_begin) * TILE_BLOCKS : 0u;
+        const int64_t left = T.nblk - (int64_t)first;
+        const uint32_t nb = found ? (uint32_t)(left < TILE_BLOCKS ? left : TILE_BLOCKS) : 0u;
+        const uint32_t mode = (!found || !T.ok) ? MODE_SKIP : (nb == (uint32_t)TILE_BLOCKS ? MODE_BULK : MODE_DIRECT);
         if (found && !T.ok) atomicOr(&g_error_flags, 2u);
-        info[st] = inf;
+        inf.d = T.d;
+        inf.nblk = T.nblk;
+        inf.s2 = T.s2;
+        inf.den = T.den;
+        inf.first = first;
+        inf.nb = nb;
+        inf.mode = mode;
         const uint32_t bar = smem_u32(&full[st]);
-        if (inf.mode == MODE_BULK) {
+        if (mode == MODE_BULK) {
             unsigned char *stage = smem + st * L::BYTES;
-            const uint32_t f = inf.first;
+            const uint32_t f = first;
             mbar_arrive_expect_tx(bar, L::tx_bytes(a.accumulate != 0));
             bulk_g2s(smem_u32(stage + L::W), reinterpret_cast<const uint4 *>(T.d.W) + 2u * f, TILE_BLOCKS * 32, bar);
             if (KIND != KIND_FWD)
@@ -434,8 +448,6 @@ __device__ __forceinline__ void consume(const Args &a, const unsigned char *smem
     using L = Layout<KIND>;
     constexpr int S = Depth<KIND>::STAGES;
     const int lane = threadIdx.x & 31;
-    int tcur = -1;
-    TensorRef T;
     uint32_t it = 0;
     for (int64_t tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++it) {
         const uint32_t st = it % S;
@@ -444,18 +456,15 @@ __device__ __forceinline__ void consume(const Args &a, const unsigned char *smem
             if (lane == 0) atomicOr(&g_error_flags, 8u);
             break;
         }
-        const StageInfo inf = info[st];
-        if (inf.mode != MODE_SKIP) {
-            if (inf.t != tcur) {
-                load_tensor(a, inf.t, T);
-                tcur = inf.t;
-            }
+        const StageInfo &inf = info[st];
+        const uint32_t mode = inf.mode;
+        if (mode != MODE_SKIP) {
             const unsigned char *stage = smem + st * L::BYTES;
             const uint32_t lb = threadIdx.x;
             Block B;
-            if (inf.mode == MODE_BULK) load_block_smem<KIND>(a, stage, B, lb, inf.first + lb);
-            else load_block_global<KIND>(T, a, B, inf.first + lb);
-            compute_block<KIND>(T, a, B);
+            if (mode == MODE_BULK) load_block_smem<KIND>(a, stage, B, lb, inf.first + lb);
+            else load_block_global<KIND>(inf, a, B, inf.first + lb);
+            compute_block<KIND>(inf, a, B);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
