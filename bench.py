@@ -37,14 +37,15 @@ sys.path.insert(0, ROOT)
 
 METRIC = "Gelem/s FOCUS fwd+STE-bwd+AdamW and % of B200 HBM roofline (ncu)"
 WORKLOAD = "Llama-3.1-8B all 224 linear weights (32 layers x q,o[4096,4096] k,v[1024,4096] " \
-           "gate,up[14336,4096] down[4096,14336]); step = s2 + fused fwd/STE-bwd/AdamW (W' written) + NVFP4 pack"
+           "gate,up[14336,4096] down[4096,14336]); step = s2 + one fused kernel: fwd (W' written), STE-bwd, " \
+           "AdamW, NVFP4 export pack of the updated m and q"
 # algorithmic bytes per weight of one step: s2 reads W (2); the fused step reads W, dW' (2+2), m (0.25),
-# q (0.5), four moments (1.5) and writes W' (2), m, q, moments (2.25); the pack reads W, m, q (2.75) and
-# writes codes (0.5) and scales (0.0625)
+# q (0.5), four moments (1.5) and writes W' (2), m, q, moments (2.25), NVFP4 codes (0.5) and scales (0.0625)
 BYTES_S2 = 2.0
-BYTES_STEP = 10.5
-BYTES_PACK = 3.3125
-KERNEL_SOURCES = ("fp4_post_weight_b200/csrc/focus_kernels.cuh", "fp4_post_weight_b200/csrc/focus_capi.cu")
+BYTES_STEP = 11.0625
+KERNEL_SOURCES = ("fp4_post_weight_b200/csrc/focus_kernels.cuh", "fp4_post_weight_b200/csrc/focus_device.cuh",
+                  "fp4_post_weight_b200/csrc/focus_pipeline.cuh", "fp4_post_weight_b200/csrc/focus_capi.cu")
+TRAFFIC_RECORD = "profiles/focus_step_fused_export_llama8b_2layers.md"
 
 
 def kernel_source_hash() -> str:
@@ -65,12 +66,13 @@ def measured_peaks() -> dict:
 
 
 def recorded_traffic():
-    """DRAM bytes per launch of the fused step kernel from the committed ncu summary,
-    valid only while the kernel sources are unchanged."""
-    p = os.path.join(ROOT, "profiles", "focus_step_fused_llama8b.json")
+    """DRAM bytes per launch of the fused step kernel on the full workload, from the
+    `bench-traffic:` line of the committed ncu summary; None once the kernel sources
+    differ from those the counters were taken with."""
     try:
-        with open(p) as f:
-            d = json.load(f)
+        with open(os.path.join(ROOT, TRAFFIC_RECORD)) as f:
+            line = next(l for l in f if l.startswith("bench-traffic:"))
+        d = json.loads(line.split(":", 1)[1])
     except Exception:
         return None
     if d.get("kernel_source_hash") != kernel_source_hash():
@@ -185,10 +187,10 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(dev)
     ents = build_model(rank, dev, args.layers)
     N = sum(o * i for _, (o, i) in model_tensors(args.layers))
-    # the step writes W' (no codes: the export pack after the update writes those)
-    step_tab = FocusTable([dataclasses.replace(e, codes=None, scales=None) for e in ents])
-    pack_tab = FocusTable(ents)
+    # one table: the step writes W' and exports the updated parameters as NVFP4
+    step_tab = FocusTable(ents)
     hp = hparams()
+    flags = F.FOCUS_STEP_PACK_UPDATED
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
 
@@ -199,10 +201,9 @@ def run_ours(args, world, rank, local):
         step_tab.s2()
         if ev is not None:
             ev[0].record(stream)
-        step_tab.step(t_counter[0], hp)
+        step_tab.step(t_counter[0], hp, flags)
         if ev is not None:
             ev[1].record(stream)
-        pack_tab.pack()
 
     for _ in range(args.warmup):
         one_step()
@@ -245,7 +246,7 @@ def run_ours(args, world, rank, local):
 
     peaks = measured_peaks()
     achieved = N * BYTES_STEP / (step_kernel_ms * 1e-3) / 1e9
-    roof = {"bound": "hbm", "kernel": "tile_kernel<KIND_STEP> (focus_step_fused)", "achieved": round(achieved, 1),
+    roof = {"bound": "hbm", "kernel": "pipe_kernel<KIND_STEP> (focus_step_fused with the export pack)", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)",
             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(),
             "bytes_per_elem": BYTES_STEP, "launch_ms": round(step_kernel_ms, 4)}
@@ -262,9 +263,9 @@ def run_ours(args, world, rank, local):
                            f"first {args.layers} layers of: " + WORKLOAD, "tensors": len(ents), "elements_per_gpu": N,
                            "l2": f"inputs larger than L2 ({N * 8.25 / 1e9:.1f} GB resident per GPU vs 126 MB L2)",
                            "parallelism": f"dp{world} (one model per GPU, no collective)",
-                           "bytes_per_elem_step": BYTES_S2 + BYTES_STEP + BYTES_PACK},
+                           "bytes_per_elem_step": BYTES_S2 + BYTES_STEP},
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": 4 * args.steps, "clocks": clk,
+                "gpu_launches": 3 * args.steps, "clocks": clk,
                 "kernel_ms": {"fused_step": round(step_kernel_ms, 4), "fused_step_min": round(min(kms), 4),
                               "fused_step_max": round(max(kms), 4)}}
         print(json.dumps(line), flush=True)
@@ -281,6 +282,7 @@ def run_e2e(args, ents, N, world, dev):
     import torch
 
     from fp4_post_weight_b200 import dist as D
+    from fp4_post_weight_b200 import focus as F
     from fp4_post_weight_b200.table import FocusTable, hparams
     ins = ("W", "dWq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq")
     outs = ("Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq", "codes", "scales", "s2")
@@ -308,8 +310,7 @@ def run_e2e(args, ents, N, world, dev):
         for e, tab, ev in zip(ents, tabs, done_in):
             comp.wait_event(ev)
             tab.s2(stream=comp)
-            tab.step(t, hp, stream=comp)
-            tab.pack(stream=comp)
+            tab.step(t, hp, F.FOCUS_STEP_PACK_UPDATED, stream=comp)
             ec = torch.cuda.Event(); ec.record(comp); done_c.append(ec)
         for e, h, ec in zip(ents, hosts, done_c):
             d2h.wait_event(ec)
@@ -340,23 +341,34 @@ def run_e2e(args, ents, N, world, dev):
 # the CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_inputs(rows: int, seed: int = 0):
-    """A row sample of the Llama-3.1-8B shapes: `rows` rows of each of the seven
-    projection shapes, generated on the host with the workload's recipe."""
+def oracle_sample_inputs(target: int, seed: int = 0):
+    """A sample of about `target` weights with the Llama-3.1-8B shapes and the
+    workload's recipe, generated on the host: the same fraction of the rows of
+    each of the seven projection shapes, over as many layers as needed."""
+    import math
+
     import numpy as np
 
     import synth
+    shapes = synth.LLAMA_8B.layer_shapes()
+    per_layer = sum(o * i for _, (o, i) in shapes)
+    layers = max(1, math.ceil(target / per_layer))
+    frac = min(1.0, target / (layers * per_layer))
     res = []
-    for j, (_, (o, i)) in enumerate(synth.LLAMA_8B.layer_shapes()):
-        t = synth.llama_8b_tensor(1000 + j + seed, (rows, i), "cpu")
-        z = np.zeros((rows, i // 16), np.float32)
-        zq = np.zeros((rows, i // 8), np.float32)
-        res.append([synth.bits(t.W), synth.bits(t.dWq), t.m.numpy().copy(), t.q.numpy().copy(),
-                    z.copy(), z.copy(), zq.copy(), zq.copy()])
-    return res
+    for l in range(layers):
+        for j, (_, (o, i)) in enumerate(shapes):
+            rows = max(1, int(round(o * frac)))
+            t = synth.llama_8b_tensor(1000 + 7 * l + j + seed, (rows, i), "cpu")
+            z = np.zeros((rows, i // 16), np.float32)
+            zq = np.zeros((rows, i // 8), np.float32)
+            res.append([synth.bits(t.W), synth.bits(t.dWq), t.m.numpy().copy(), t.q.numpy().copy(),
+                        z.copy(), z.copy(), zq.copy(), zq.copy()])
+    return res, layers, frac
 
 
 def oracle_step(sample):
+    """The whole path on the CPU oracle: s2, forward + straight-through backward +
+    AdamW, and the NVFP4 pack of the updated parameters, tensor by tensor."""
     import oracle
     n = 0
     for W, G, m, q, a, b, c, d in sample:
@@ -367,54 +379,55 @@ def oracle_step(sample):
     return n
 
 
+def _oracle_rate() -> float:
+    """Weights per second of oracle_step on this host (a small calibration sample)."""
+    sample, _, _ = oracle_sample_inputs(4_000_000, seed=77)
+    t0 = time.time()
+    n = oracle_step(sample)
+    return n / max(time.time() - t0, 1e-6)
+
+
 def cpu_baseline(seconds: float) -> dict:
     import oracle
     oracle.build()
     threads = oracle.num_threads()
-    rows = 16
-    t0 = time.time()
-    n = oracle_step(oracle_sample_inputs(rows))
-    dt = time.time() - t0
-    # scale the sample to about `seconds` of work
-    rows = max(16, int(rows * seconds / max(dt, 1e-3)))
-    rows = min(rows, 4096)
-    sample = oracle_sample_inputs(rows)
+    target = int(_oracle_rate() * seconds)
+    sample, layers, frac = oracle_sample_inputs(target)
     t0 = time.time()
     n = oracle_step(sample)
     dt = time.time() - t0
     return {"value": round(n / dt / 1e9, 5), "unit": "Gelem/s", "cores": threads, "kind": "oracle",
-            "sample": f"{rows} rows of each Llama-3.1-8B projection shape ({n} weights): s2 + fwd + "
-                      f"STE-bwd + AdamW + pack, {dt:.1f} s on {threads} OpenMP threads"}
+            "sample": f"{frac:.3f} of the rows of each Llama-3.1-8B projection shape over {layers} layer(s) "
+                      f"({n} weights): s2 + fwd + STE-bwd + AdamW + pack, {dt:.1f} s on {threads} OpenMP threads"}
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, timed on the host cores, on the same
+    metric; each step is a bounded sample of the workload (about
+    --reference-seconds of CPU work)."""
     if rank != 0:
         return
     import oracle
     oracle.build()
     threads = oracle.num_threads()
-    rows = 16
-    t0 = time.time()
-    oracle_step(oracle_sample_inputs(rows))
-    dt = time.time() - t0
-    per_step = args.reference_seconds
-    rows = min(4096, max(16, int(rows * per_step / max(dt, 1e-3))))
+    target = int(_oracle_rate() * args.reference_seconds)
     for w in range(args.warmup):
-        oracle_step(oracle_sample_inputs(rows, seed=w))
-    samples = [oracle_sample_inputs(rows, seed=100 + k) for k in range(args.steps)]
+        oracle_step(oracle_sample_inputs(max(target // 8, 1), seed=w)[0])
+    samples = [oracle_sample_inputs(target, seed=100 + k) for k in range(args.steps)]
     t0 = time.time()
     n = 0
-    for smp in samples:
+    for smp, _, _ in samples:
         n += oracle_step(smp)
     dt = time.time() - t0
     value = n / dt / 1e9
-    desc = (f"{rows} rows of each Llama-3.1-8B projection shape per step: s2 + fwd + STE-bwd + AdamW + pack "
-            f"on {threads} OpenMP threads")
+    _, layers, frac = samples[0]
+    desc = (f"{frac:.3f} of the rows of each Llama-3.1-8B projection shape over {layers} layer(s) per step "
+            f"({n // args.steps} weights): s2 + fwd + STE-bwd + AdamW + pack on {threads} OpenMP threads")
     line = {"metric": METRIC, "value": round(value, 5), "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * dt / args.steps, 2), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64-accumulate/f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32 forward, f64 sums", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": WORKLOAD, "sample_rows_per_shape": rows},
+            "config": {"workload": WORKLOAD, "sample_weights_per_step": n // args.steps},
             "cpu_baseline": {"value": round(value, 5), "unit": "Gelem/s", "cores": threads, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": round(value, 5), "unit": "Gelem/s", "h2d_bytes_per_step": 0,

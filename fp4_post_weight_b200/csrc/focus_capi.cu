@@ -175,6 +175,7 @@ const char *focus_status_string(int status) {
     case FOCUS_ERR_WORKSPACE: return "FOCUS_ERR_WORKSPACE: workspace missing or too small";
     case FOCUS_ERR_CUDA: return "FOCUS_ERR_CUDA: a CUDA call or launch failed";
     case FOCUS_ERR_NONFINITE_INPUT: return "FOCUS_ERR_NONFINITE_INPUT: a kernel met a non-finite input";
+    case FOCUS_ERR_DEVICE_TIMEOUT: return "FOCUS_ERR_DEVICE_TIMEOUT: a kernel's pipeline wait ran out";
     default: return "FOCUS_ERR_UNKNOWN";
     }
 }
@@ -336,7 +337,8 @@ int focus_step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_ti
     int rc = check_hyper(hp->lr_m, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
     if (rc) return rc;
     if ((rc = check_hyper(hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
-    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD)) return FOCUS_ERR_VALUE;
+    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD | FOCUS_STEP_PACK_UPDATED))
+        return FOCUS_ERR_VALUE;
     if (n == 0) return FOCUS_OK;
     if (!descs_dev) return FOCUS_ERR_NULL;
     if (!aligned16(descs_dev)) return FOCUS_ERR_ALIGN;
@@ -347,6 +349,7 @@ int focus_step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_ti
     a.write_wq = 1;
     a.accumulate = (flags & FOCUS_STEP_ACCUMULATE) ? 1 : 0;
     a.write_grad = (flags & FOCUS_STEP_WRITE_GRAD) ? 1 : 0;
+    a.pack_updated = (flags & FOCUS_STEP_PACK_UPDATED) ? 1 : 0;
     a.hp = make_hyper(hp->lr_m, hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
     return launch_on<KIND_STEP>(a, (cudaStream_t)stream);
 }
@@ -370,7 +373,7 @@ int focus_get_error(focus_stream_t stream) {
     if (flags) {
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbol(g_error_flags, &zero, sizeof zero) != cudaSuccess) return FOCUS_ERR_CUDA;
-        return FOCUS_ERR_NONFINITE_INPUT;
+        return (flags & 8u) ? FOCUS_ERR_DEVICE_TIMEOUT : FOCUS_ERR_NONFINITE_INPUT;
     }
     return FOCUS_OK;
 }

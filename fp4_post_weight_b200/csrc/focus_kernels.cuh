@@ -50,7 +50,8 @@ constexpr int TILE_BLOCKS = CONSUMERS;           // 16-blocks per tile (4096 wei
 constexpr unsigned FULL = 0xffffffffu;
 
 // Sticky error word read by focus_get_error(): bit 0 a non-finite input,
-// bit 1 an invalid tensor scale read from a table, bit 2 a non-finite gradient.
+// bit 1 an invalid tensor scale read from a table, bit 2 a non-finite
+// gradient, bit 3 a pipeline wait that ran out.
 // (This header is compiled into exactly one translation unit.)
 __device__ unsigned int g_error_flags = 0;
 
@@ -66,6 +67,7 @@ struct Args {
     int write_wq;                    // forward and step: write W' where the descriptor has it
     int accumulate;                  // bwd: add into dm/dq; step: FOCUS_STEP_ACCUMULATE
     int write_grad;                  // step: FOCUS_STEP_WRITE_GRAD
+    int pack_updated;                // step: FOCUS_STEP_PACK_UPDATED
     Hyper hp;
 };
 
@@ -151,6 +153,37 @@ __device__ __forceinline__ void load_block_global(const TV &T, const Args &a, Bl
     }
 }
 
+// NVFP4 codes and E4M3 scale byte of one block for block factor m and
+// sub-block logits q0, q1 (the forward's decisions only).
+template <class TV>
+__device__ __forceinline__ void encode_block(const TV &T, const uint32_t *w, float A, float m, float q0, float q1,
+                                             uint32_t &sbyte, uint32_t codes[2]) {
+    const float x = __fdiv_rn(__fmul_rn(A, m), T.den);
+    float xc = (x == 0.0f) ? 1.0f : x;
+    xc = fminf(fmaxf(xc, 0x1p-6f), 448.0f);
+    sbyte = e4m3_byte(xc);
+    const float S = e4m3_normal_f32(sbyte);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const float D = __fmul_rn(__fmul_rn(S, sigmoid_rn(k ? q1 : q0)), T.s2);
+        uint32_t code = 0u;
+        if (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f) {
+            const float nr = -__frcp_rn(D);
+            const uint64_t D2 = f2_pack(D, D), nr2 = f2_pack(nr, nr);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint64_t y2 = div_by_f2(bf16x2_neg_f2(w[4 * k + j]), D2, nr2);
+                code |= e2m1_pair(f2_lo(y2), f2_hi(y2)) << (8 * j);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                code |= e2m1_pair(__fdiv_rn(bf16_lo(w[4 * k + j]), D), __fdiv_rn(bf16_hi(w[4 * k + j]), D)) << (8 * j);
+        }
+        codes[k] = code;
+    }
+}
+
 // The forward, the straight-through gradients and the AdamW update of one block.
 // TV is any view of a tensor with members d (descriptor), s2, den and nblk:
 // the consumer warps pass the stage record in shared memory, so the
@@ -231,7 +264,8 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
             sq[k] = f2_lo(sq2) + f2_hi(sq2);
         }
     }
-    if (B.valid) {
+    // the forward's NVFP4 codes and scale (unless the step exports the updated parameters instead)
+    if (B.valid && !(KIND == KIND_STEP && a.pack_updated)) {
         if (T.d.codes) {
             uint2 cc; cc.x = codes[0]; cc.y = codes[1];
             reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
@@ -268,6 +302,14 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
                 reinterpret_cast<float2 *>(T.d.q)[B.blk] = make_float2(f2_lo(qp), f2_hi(qp));
                 reinterpret_cast<float2 *>(T.d.q_exp_avg)[B.blk] = make_float2(f2_lo(v1), f2_hi(v1));
                 reinterpret_cast<float2 *>(T.d.q_exp_avg_sq)[B.blk] = make_float2(f2_lo(v2), f2_hi(v2));
+            }
+            // NVFP4 export of the updated m and q: what a pack after this step would write
+            if (a.pack_updated && B.valid && T.d.codes) {
+                uint32_t sb2, codes2[2];
+                encode_block(T, B.w, A, B.m, f2_lo(qp), f2_hi(qp), sb2, codes2);
+                uint2 cc; cc.x = codes2[0]; cc.y = codes2[1];
+                reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
+                T.d.scales[B.blk] = (uint8_t)sb2;
             }
         }
     }

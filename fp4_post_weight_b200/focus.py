@@ -27,6 +27,7 @@ _SZ = ctypes.c_size_t
 FOCUS_OK = 0
 FOCUS_STEP_ACCUMULATE = 1
 FOCUS_STEP_WRITE_GRAD = 2
+FOCUS_STEP_PACK_UPDATED = 4
 
 
 class focus_tensor_desc(ctypes.Structure):

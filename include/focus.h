@@ -38,7 +38,8 @@
  *    launch status; a failed check enqueues nothing.
  *  - Non-finite values in W, m or q, and an invalid s2 read from device
  *    memory, are outside the contract: kernels never trap on them, they set a
- *    sticky device flag that focus_get_error() reports.
+ *    sticky device flag that focus_get_error() reports.  Every wait inside a
+ *    kernel is bounded in time; a wait that runs out sets the flag too.
  *  - in must be a multiple of 16; out >= 0 (an empty tensor is a no-op).
  */
 #ifndef FOCUS_H
@@ -56,12 +57,16 @@ typedef void *focus_stream_t; /* a cudaStream_t */
 typedef enum focus_status {
     FOCUS_OK = 0,
     FOCUS_ERR_NULL = 1,             /* a required pointer is NULL */
-    FOCUS_ERR_SHAPE = 2,            /* in % 16 != 0, out < 0, n < 0, or a size overflows */
+    FOCUS_ERR_SHAPE = 2,            /* in % 16 != 0, out < 0, n < 0, or a tensor of more than
+                                       2^31 - 2^16 blocks (out*in/16) */
     FOCUS_ERR_ALIGN = 3,            /* a tensor base address is not 16-byte aligned */
     FOCUS_ERR_VALUE = 4,            /* s2 <= 0 or not finite, lr < 0, step < 1, beta outside [0,1) ... */
     FOCUS_ERR_WORKSPACE = 5,        /* workspace missing or smaller than required */
     FOCUS_ERR_CUDA = 6,             /* a CUDA runtime call or a launch failed */
-    FOCUS_ERR_NONFINITE_INPUT = 7   /* reported by focus_get_error(): the device flag was set */
+    FOCUS_ERR_NONFINITE_INPUT = 7,  /* reported by focus_get_error(): a kernel met a non-finite input
+                                       or gradient, or an invalid s2 in a table */
+    FOCUS_ERR_DEVICE_TIMEOUT = 8    /* reported by focus_get_error(): a kernel's staging pipeline
+                                       gave up waiting (2 s) and left its work unfinished */
 } focus_status;
 
 /* Human-readable name of a status code (static storage; never NULL). */
@@ -186,6 +191,9 @@ typedef struct focus_hparams {
 /* Flags of focus_step_fused. */
 #define FOCUS_STEP_ACCUMULATE 1u  /* add dm/dq (earlier micro-batches) to this step's gradients */
 #define FOCUS_STEP_WRITE_GRAD 2u  /* write the gradients used by the update into dm/dq */
+#define FOCUS_STEP_PACK_UPDATED 4u /* codes/scales receive the NVFP4 export of the UPDATED m and q (what
+                                      focus_pack_multi would write after this call) instead of the
+                                      forward's; W is not read again */
 
 /* Checks every entry (pointers, alignment, shapes, which outputs are present
  * for `purpose`: 0 = s2/forward/pack only, 1 = also focus_step_fused) and
@@ -204,8 +212,9 @@ int focus_s2_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t to
  * forward (W' when desc.Wq != NULL, codes/scales when present), straight-
  * through backward, AdamW on m and q (lr_m for m, lr_q for q) at step `step`.
  * hp is a host pointer.  flags: FOCUS_STEP_ACCUMULATE, FOCUS_STEP_WRITE_GRAD
- * (both need desc.dm and desc.dq).  Outputs W', codes and scales are those
- * of the forward, i.e. of m and q before the update. */
+ * (both need desc.dm and desc.dq), FOCUS_STEP_PACK_UPDATED.  W' is the
+ * forward's, i.e. of m and q before the update; codes and scales are the
+ * forward's too unless FOCUS_STEP_PACK_UPDATED is set. */
 int focus_step_fused(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
                      const focus_hparams *hp, int64_t step, unsigned flags, focus_stream_t stream);
 
@@ -216,9 +225,10 @@ int focus_pack_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t 
 
 /* ---------------------------------------------------------------------------
  * Synchronizes `stream`, then reports and clears the sticky device flag:
+ * FOCUS_ERR_DEVICE_TIMEOUT when a kernel's pipeline wait ran out,
  * FOCUS_ERR_NONFINITE_INPUT when any kernel since the last call met a
- * non-finite W/m/q value or an invalid s2 read from a table, FOCUS_ERR_CUDA
- * when the stream reports an error, else FOCUS_OK.
+ * non-finite W/m/q value or gradient or an invalid s2 read from a table,
+ * FOCUS_ERR_CUDA when the stream reports an error, else FOCUS_OK.
  * ------------------------------------------------------------------------- */
 int focus_get_error(focus_stream_t stream);
 

@@ -33,7 +33,7 @@ def test_exports_every_declared_function(F):
 
 
 def test_status_strings(F):
-    for s in range(8):
+    for s in range(9):
         assert F.focus_status_string(s).startswith("FOCUS_")
     assert F.focus_version() == "0.1.0"
 
@@ -114,6 +114,7 @@ def test_step_hparam_checks(F):
     hp = F.focus_hparams(5e-3, 1e-3, 0.9, 0.999, 1e-8, 0.0)
     assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(hp), 0, 0, None) == 4
     assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(hp), 1, 8, None) == 4
+    assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(hp), 1, 16, None) == 4
     assert F.raw_call("focus_step_fused", P, 1, 1, None, 1, 0, None) == 1
     bad = F.focus_hparams(5e-3, -1e-3, 0.9, 0.999, 1e-8, 0.0)
     assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(bad), 1, 0, None) == 4

@@ -190,6 +190,26 @@ def test_step_accumulate_and_pack_multi(F):
         assert_close(host(e.m), m, "m"); assert_close(host(e.q), q, "q")
 
 
+def test_step_pack_updated_equals_pack_after_step(F):
+    """FOCUS_STEP_PACK_UPDATED: the step's codes and scales are bit for bit what
+    focus_pack_multi writes after the step (the pack is checked against the
+    oracle on generated inputs elsewhere); everything else is unchanged."""
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    shapes = [(37, 1040), (64, 512), (128, 2048), (3, 48)]
+    ea = _entries(shapes, 70)
+    eb = _entries(shapes, 70)
+    ta, tb = FocusTable(ea), FocusTable(eb)
+    ta.s2(); tb.s2()
+    ta.step(1, hparams(), flags=F.FOCUS_STEP_PACK_UPDATED)
+    tb.step(1, hparams())
+    tb.pack()
+    assert F.focus_get_error() == 0
+    for a, b in zip(ea, eb):
+        for name in ("codes", "scales", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"):
+            assert torch.equal(getattr(a, name), getattr(b, name)), name
+        assert np.array_equal(host_bits(a.Wq), host_bits(b.Wq))
+
+
 def test_pack_multi_leaves_wq_alone(F):
     from fp4_post_weight_b200.table import FocusTable
     ents = _entries([(16, 256)], 60)
