@@ -211,7 +211,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
 
     const bool want_wq = KIND != KIND_BWD && a.write_wq && T.d.Wq != nullptr && B.valid;
     float sig[2], sq[2];
-    uint64_t gcs2 = 0ull;                       // sum of g * (c*S), pairwise
+    uint64_t sm2 = 0ull;                        // sum of g * (in ? c - y : c), pairwise
     uint32_t codes[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -230,13 +230,14 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
                 y2[j] = f2_pack(__fdiv_rn(bf16_lo(B.w[4 * k + j]), D), __fdiv_rn(bf16_hi(B.w[4 * k + j]), D));
         }
         uint32_t code = 0u;
+        uint32_t ch2[4];
         uint64_t cs2[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint32_t byte = e2m1_pair(f2_lo(y2[j]), f2_hi(y2[j]));
             code |= byte << (8 * j);
-            const uint32_t h2 = e2m1_pair_f16x2(byte);
-            cs2[j] = f2_pack(mul_f16_exact(lo16(h2), S_h), mul_f16_exact(hi16(h2), S_h));   // c*S, exact
+            ch2[j] = e2m1_pair_f16x2(byte);
+            cs2[j] = f2_pack(mul_f16_exact(lo16(ch2[j]), S_h), mul_f16_exact(hi16(ch2[j]), S_h));   // c*S, exact
         }
         codes[k] = code;
         // w' = bf16(fl(fl(c*S)*s2))
@@ -251,15 +252,18 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
         }
         sq[k] = 0.0f;
         if (KIND != KIND_FWD) {
-            // straight-through sums: sum g*c*S over the block, sum g*y inside the clamp per sub-block
+            // straight-through sums, element by element: g*t with t = c - y inside the
+            // clamp and c outside (c - y is exact near the code, so the sum is well
+            // conditioned), and g*y inside the clamp, per sub-block
             uint64_t sq2 = 0ull;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const uint64_t g2 = bf16x2_f2(B.g[4 * k + j]);
-                gcs2 = f2_fma(g2, cs2[j], gcs2);
                 const float ylo = f2_lo(y2[j]), yhi = f2_hi(y2[j]);
-                const uint64_t yin2 = f2_pack(fabsf(ylo) <= 6.0f ? ylo : 0.0f, fabsf(yhi) <= 6.0f ? yhi : 0.0f);
-                sq2 = f2_fma(g2, yin2, sq2);
+                const float ilo = fabsf(ylo) <= 6.0f ? ylo : 0.0f, ihi = fabsf(yhi) <= 6.0f ? yhi : 0.0f;
+                const uint64_t t2 = f2_pack(sub_f16_f32(lo16(ch2[j]), ilo), sub_f16_f32(hi16(ch2[j]), ihi));
+                sm2 = f2_fma(g2, t2, sm2);
+                sq2 = f2_fma(g2, f2_pack(ilo, ihi), sq2);
             }
             sq[k] = f2_lo(sq2) + f2_hi(sq2);
         }
@@ -274,10 +278,8 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
     }
 
     if (KIND != KIND_FWD) {
-        // dL/dm = inS*(A/6)*sum g*(c - y_in) = inS*(A/6)*(sum g*c - sum g*y_in)
-        // dL/dq_k = -(1 - sigma_k)*S*s2*sum_k g*y_in
-        const float gc = __fdiv_rn(f2_lo(gcs2) + f2_hi(gcs2), S);
-        float gm = inS ? (A * (1.0f / 6.0f)) * (gc - (sq[0] + sq[1])) : 0.0f;
+        // dL/dm = inS*(A/6)*sum g*t;  dL/dq_k = -(1 - sigma_k)*S*s2*sum_k g*y_in
+        float gm = inS ? (A * (1.0f / 6.0f)) * (f2_lo(sm2) + f2_hi(sm2)) : 0.0f;
         float gq0 = -((((1.0f - sig[0]) * S) * T.s2) * sq[0]);
         float gq1 = -((((1.0f - sig[1]) * S) * T.s2) * sq[1]);
         if (a.accumulate) {
