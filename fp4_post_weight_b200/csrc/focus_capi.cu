@@ -163,6 +163,34 @@ int launch_s2(const Args &a, uint32_t *partial, float *one_out, int n_finish, cu
 }
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// s2 without a caller workspace
+//
+// Some callers of this library have no way to hand it device memory: a
+// runtime whose fixed memory pool owns every device allocation and forbids
+// any other, or a latency-critical path that must never enter cudaMalloc (it
+// can synchronize the device).  focus_s2_noalloc serves them: its per-tile
+// maxima live in the array below, which is part of the library's device image
+// (every GPU that loads the library keeps it until the process exits), so the
+// call allocates nothing.  One word per 4096-weight tile: NOALLOC_TILES words
+// cover a tensor of FOCUS_S2_NOALLOC_MAX_WEIGHTS weights.  The amax kernel
+// writes every word the finishing kernel reads, so nothing has to be cleared
+// between calls; two calls whose work overlaps on the GPU share the array and
+// race.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t NOALLOC_TILES = FOCUS_S2_NOALLOC_MAX_WEIGHTS / (TILE_BLOCKS * 16);
+static_assert(NOALLOC_TILES * TILE_BLOCKS * 16 == FOCUS_S2_NOALLOC_MAX_WEIGHTS, "whole tiles");
+
+static __device__ __align__(256) uint32_t g_s2_noalloc_scratch[NOALLOC_TILES];
+
+std::once_flag g_noalloc_once[MAX_DEVICES];
+uint32_t *g_noalloc_ptr[MAX_DEVICES];
+cudaError_t g_noalloc_status[MAX_DEVICES];
+
+}  // namespace
+
 extern "C" {
 
 const char *focus_status_string(int status) {
@@ -201,6 +229,31 @@ int focus_s2(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, void *ws
     a.one = one_desc(W, nullptr, nullptr, nullptr, nullptr, out, in);
     a.total_tiles = tiles_of(out, in);
     return launch_s2(a, static_cast<uint32_t *>(ws_dev), s2_dev, 1, (cudaStream_t)stream);
+}
+
+int focus_s2_noalloc(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, focus_stream_t stream) {
+    int rc = check_shape(out, in);
+    if (rc) return rc;
+    if (!s2_dev || (!W && out * in > 0)) return FOCUS_ERR_NULL;
+    if (!aligned16(W)) return FOCUS_ERR_ALIGN;
+    const int64_t tiles = tiles_of(out, in);
+    if (tiles > NOALLOC_TILES) return FOCUS_ERR_WORKSPACE;   // larger than the built-in scratch covers
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return FOCUS_ERR_CUDA;
+    // The first call on a device, with that device current, looks up the device
+    // address of the scratch array (its name in host code is only a stand-in).
+    std::call_once(g_noalloc_once[dev], [dev] {
+        void *p = nullptr;
+        g_noalloc_status[dev] = cudaGetSymbolAddress(&p, g_s2_noalloc_scratch);
+        g_noalloc_ptr[dev] = static_cast<uint32_t *>(p);
+    });
+    if (g_noalloc_status[dev] != cudaSuccess || g_noalloc_ptr[dev] == nullptr) return FOCUS_ERR_CUDA;
+    Args a{};
+    a.table = nullptr;
+    a.n_tensors = 1;
+    a.one = one_desc(W, nullptr, nullptr, nullptr, nullptr, out, in);
+    a.total_tiles = tiles;
+    return launch_s2(a, g_noalloc_ptr[dev], s2_dev, 1, (cudaStream_t)stream);
 }
 
 int focus_fwd(const uint16_t *W, const float *m, const float *q, float s2, int64_t out, int64_t in, uint16_t *Wq,

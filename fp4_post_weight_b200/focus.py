@@ -50,6 +50,7 @@ _SIGS = {
     "focus_version": ([], ctypes.c_char_p),
     "focus_s2_workspace_bytes": ([_I64, _I64], _SZ),
     "focus_s2": ([_P, _I64, _I64, _P, _P, _SZ, _P], _I),
+    "focus_s2_noalloc": ([_P, _I64, _I64, _P, _P], _I),
     "focus_fwd": ([_P, _P, _P, _F, _I64, _I64, _P, _P], _I),
     "focus_ste_bwd": ([_P, _P, _P, _P, _F, _I64, _I64, _P, _P, _I, _P], _I),
     "focus_adamw_step": ([_P, _P, _P, _P, _I64, _F, _F, _F, _F, _F, _I64, _P], _I),
@@ -138,6 +139,19 @@ def focus_s2(W, s2_out, workspace, stream=None, out=None, in_=None):
     o, i = _shape(W, out, in_)
     nbytes = workspace.numel() * workspace.element_size() if isinstance(workspace, torch.Tensor) else 1 << 62
     _check(_lib.focus_s2(_ptr(W), o, i, _ptr(s2_out), _ptr(workspace), nbytes, _stream(stream)), "focus_s2")
+
+
+FOCUS_S2_NOALLOC_MAX_WEIGHTS = 268435456
+
+
+def focus_s2_noalloc(W, s2_out, stream=None, out=None, in_=None):
+    """s2 into the one-float device tensor s2_out, without a workspace: for callers
+    that cannot hand the library device memory (the per-tile maxima live in a
+    fixed array inside the library; tensors of up to FOCUS_S2_NOALLOC_MAX_WEIGHTS
+    weights; calls that may overlap on the GPU must not be issued)."""
+    _bf16(W, "W"); _f32(s2_out, "s2_out")
+    o, i = _shape(W, out, in_)
+    _check(_lib.focus_s2_noalloc(_ptr(W), o, i, _ptr(s2_out), _stream(stream)), "focus_s2_noalloc")
 
 
 def focus_fwd(W, m, q, s2: float, Wq, stream=None, out=None, in_=None):

@@ -89,6 +89,25 @@ int focus_s2(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, void *ws
              size_t ws_bytes, focus_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * s2 without a workspace: the same result as focus_s2, for callers that
+ * cannot give the library device memory (a runtime whose own memory pool owns
+ * every device allocation, or a path that must never call cudaMalloc, which
+ * can synchronize the device).  The pages describe nothing like it; it only
+ * changes where the per-tile maxima live: in a 256 KB array inside the
+ * library's device image, held on every GPU that loads the library until the
+ * process exits.  This call allocates nothing.
+ *   W       [out, in] bf16, device; at most FOCUS_S2_NOALLOC_MAX_WEIGHTS
+ *           weights, else FOCUS_ERR_WORKSPACE and nothing is enqueued
+ *   s2_dev  one float, device, written
+ * The first call on a device (with that device current) looks up the array's
+ * device address; make that first call before any stream capture.  All calls
+ * share the array: calls whose work may overlap on the GPU (different streams
+ * without ordering between them) race and must not be issued.
+ * ------------------------------------------------------------------------- */
+#define FOCUS_S2_NOALLOC_MAX_WEIGHTS 268435456 /* 65,536 tiles of 4096 weights */
+int focus_s2_noalloc(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Forward fake-quantization W -> W'.
  * Card, "What this is": the S_b, c_i and w'_i equations.
  *   W   [out, in] bf16, device (read)
