@@ -81,6 +81,8 @@ struct TensorRef {
     int64_t tile_end;
     float s2;
     float den;      // fl(6 * s2)
+    float rden;     // fl(1 / den)
+    bool den_ok;    // den inside the range where the quotient by rden is exact
     bool ok;        // s2 usable
 };
 
@@ -96,6 +98,8 @@ __device__ __forceinline__ void load_tensor(const Args &a, int t, TensorRef &r) 
     r.tile_end = r.d.tile_begin + (r.nblk + TILE_BLOCKS - 1) / TILE_BLOCKS;
     r.ok = (r.s2 > 0.0f) && finitef(r.s2);
     r.den = __fmul_rn(6.0f, r.s2);
+    r.den_ok = r.ok && r.den >= 0x1p-60f && r.den <= 0x1p60f;
+    r.rden = r.den_ok ? rcp_rn(r.den) : 0.0f;
 }
 
 // ---------------------------------------------------------------------------
@@ -153,22 +157,38 @@ __device__ __forceinline__ void load_block_global(const TV &T, const Args &a, Bl
     }
 }
 
+// x_b = fl(fl(A*m) / fl(6*s2)).  With |A*m| and 6*s2 in [2^-60, 2^60] the
+// quotient and every intermediate of the correction stay normal, and the
+// quotient comes from the tensor's reciprocal of 6*s2 (two Markstein
+// corrections, correctly rounded); elsewhere from the IEEE division.
+template <class TV>
+__device__ __forceinline__ float scaled_max(const TV &T, float A, float m) {
+    const float Am = __fmul_rn(A, m);
+    const float aAm = fabsf(Am);
+    if (T.den_ok && aAm <= 0x1p60f && (aAm >= 0x1p-60f || aAm == 0.0f)) return div_full(Am, T.den, T.rden);
+    return __fdiv_rn(Am, T.den);
+}
+
 // NVFP4 codes and E4M3 scale byte of one block for block factor m and
 // sub-block logits q0, q1 (the forward's decisions only).
+// The sub-block sigmoids come from sigmoid_near with the forward's e^-q (t0, t1
+// at the logits q0_old, q1_old), bit-identical to evaluating them afresh.
 template <class TV>
 __device__ __forceinline__ void encode_block(const TV &T, const uint32_t *w, float A, float m, float q0, float q1,
-                                             uint32_t &sbyte, uint32_t codes[2]) {
-    const float x = __fdiv_rn(__fmul_rn(A, m), T.den);
+                                             double t0, double t1, float q0_old, float q1_old, uint32_t &sbyte,
+                                             uint32_t codes[2]) {
+    const float x = scaled_max(T, A, m);
     float xc = (x == 0.0f) ? 1.0f : x;
     xc = fminf(fmaxf(xc, 0x1p-6f), 448.0f);
     sbyte = e4m3_byte(xc);
     const float S = e4m3_normal_f32(sbyte);
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-        const float D = __fmul_rn(__fmul_rn(S, sigmoid_rn(k ? q1 : q0)), T.s2);
+        const float sig = k ? sigmoid_near(t1, q1_old, q1) : sigmoid_near(t0, q0_old, q0);
+        const float D = __fmul_rn(__fmul_rn(S, sig), T.s2);
         uint32_t code = 0u;
         if (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f) {
-            const float nr = -__frcp_rn(D);
+            const float nr = -rcp_rn(D);
             const uint64_t D2 = f2_pack(D, D), nr2 = f2_pack(nr, nr);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -200,7 +220,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
     const bool bad = B.valid && (abits >= 0x7f80u || !finitef(B.m) || !finitef(B.q[0]) || !finitef(B.q[1]));
 
     // S_b = e4m3(clamp(fl(fl(A*m)/fl(6*s2)), 2^-6, 448)), scale 1 when the scaled max is 0
-    const float x = __fdiv_rn(__fmul_rn(A, B.m), T.den);
+    const float x = scaled_max(T, A, B.m);
     const bool inS = (x != 0.0f) && (x >= 0x1p-6f) && (x <= 448.0f);
     float xc = (x == 0.0f) ? 1.0f : x;
     xc = fminf(fmaxf(xc, 0x1p-6f), 448.0f);
@@ -211,16 +231,17 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
 
     const bool want_wq = KIND != KIND_BWD && a.write_wq && T.d.Wq != nullptr && B.valid;
     float sig[2], sq[2];
+    double et[2];                               // e^-q of the forward, reused by the export
     uint64_t sm2 = 0ull;                        // sum of g * (in ? c - y : c), pairwise
     uint32_t codes[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
         // D_k = fl(fl(S*sigmoid(q_k))*s2); y_i = fl(w_i/D_k); c_i = E2M1(clamp(y_i, -6, 6))
-        sig[k] = sigmoid_rn(B.q[k]);
+        sig[k] = sigmoid_rn_t(B.q[k], et[k]);
         const float D = __fmul_rn(__fmul_rn(S, sig[k]), T.s2);
         uint64_t y2[4];
         if (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f) {
-            const float nr = -__frcp_rn(D);
+            const float nr = -rcp_rn(D);
             const uint64_t D2 = f2_pack(D, D), nr2 = f2_pack(nr, nr);
 #pragma unroll
             for (int j = 0; j < 4; ++j) y2[j] = div_by_f2(bf16x2_neg_f2(B.w[4 * k + j]), D2, nr2);
@@ -294,6 +315,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
         }
         if (KIND == KIND_STEP) {
             adamw_one(B.m, gm, B.mv1, B.mv2, a.hp.lr_m_step, a.hp.decay_m, a.hp);
+            const float q_old0 = B.q[0], q_old1 = B.q[1];
             uint64_t qp = f2_pack(B.q[0], B.q[1]);
             uint64_t v1 = f2_pack(B.qv1[0], B.qv1[1]), v2 = f2_pack(B.qv2[0], B.qv2[1]);
             adamw_pair(qp, f2_pack(gq0, gq1), v1, v2, a.hp.lr_q_step, a.hp.decay_q, a.hp);
@@ -308,7 +330,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
             // NVFP4 export of the updated m and q: what a pack after this step would write
             if (a.pack_updated && B.valid && T.d.codes) {
                 uint32_t sb2, codes2[2];
-                encode_block(T, B.w, A, B.m, f2_lo(qp), f2_hi(qp), sb2, codes2);
+                encode_block(T, B.w, A, B.m, f2_lo(qp), f2_hi(qp), et[0], et[1], q_old0, q_old1, sb2, codes2);
                 uint2 cc; cc.x = codes2[0]; cc.y = codes2[1];
                 reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
                 T.d.scales[B.blk] = (uint8_t)sb2;
@@ -346,7 +368,7 @@ struct Layout {
 template <int KIND> struct Depth;
 template <> struct Depth<KIND_FWD> { static constexpr int STAGES = 6, MIN_CTAS = 3; };
 template <> struct Depth<KIND_BWD> { static constexpr int STAGES = 4, MIN_CTAS = 2; };
-template <> struct Depth<KIND_STEP> { static constexpr int STAGES = 3, MIN_CTAS = 2; };
+template <> struct Depth<KIND_STEP> { static constexpr int STAGES = 2, MIN_CTAS = 3; };
 
 template <int KIND>
 constexpr uint32_t stage_smem_bytes() { return Depth<KIND>::STAGES * Layout<KIND>::BYTES; }
@@ -360,10 +382,12 @@ struct StageInfo {
     int64_t nblk;
     float s2;
     float den;
+    float rden;
+    uint32_t den_ok;
     uint32_t first;    // first block of the tile within the tensor
     uint32_t nb;       // blocks in the tile
     uint32_t mode;     // MODE_*
-    uint32_t pad;
+    uint32_t pad[3];
 };
 
 // A block's inputs from a staged tile (local block lb of the tile).
@@ -448,6 +472,8 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
         inf.nblk = T.nblk;
         inf.s2 = T.s2;
         inf.den = T.den;
+        inf.rden = T.rden;
+        inf.den_ok = T.den_ok ? 1u : 0u;
         inf.first = first;
         inf.nb = nb;
         inf.mode = mode;

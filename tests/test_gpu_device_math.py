@@ -10,6 +10,12 @@
   every E2M1 value and every normal E4M3 scale, and c - y likewise.
 * The E2M1 conversion keeps the sign of negative values that round to zero
   (code 0x8), which the kernels rely on for the signed-zero reading.
+* The reciprocal from the hardware approximation and one Newton step equals
+  __frcp_rn for every significand; the twice-corrected quotient used for the
+  scaled block maximum equals __fdiv_rn (every divisor significand for 1024
+  pseudo-random numerators, and 2^30 pseudo-random pairs); the sigmoid of an
+  updated logit computed from the old e^-q equals sigmoid_rn (2^28 pairs,
+  logits up to +-100).
 """
 import ctypes
 import os
@@ -35,6 +41,11 @@ def lib():
     L.check_div.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_ulonglong),
                             ctypes.POINTER(ctypes.c_float), ctypes.c_int]
     L.check_mixed.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
+    L.check_rcp.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_ulonglong)]
+    L.check_div_full.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong),
+                                 ctypes.POINTER(ctypes.c_float)]
+    L.check_sigmoid_near.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong),
+                                     ctypes.POINTER(ctypes.c_float)]
     L.e2m1_raw_bytes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     return L
 
@@ -64,3 +75,26 @@ def test_e2m1_conversion_zero_sign(lib):
     assert np.all(mags == 0)            # every value rounds to a zero magnitude
     want = (np.signbit(lo).astype(np.uint32) << 3) | (np.signbit(hi).astype(np.uint32) << 7)
     np.testing.assert_array_equal(out, want)
+
+
+@pytest.mark.parametrize("e", [0, -20, 20, -59, 59, -100, 100])
+def test_reciprocal_exhaustive(lib, e):
+    n = ctypes.c_ulonglong(0)
+    assert lib.check_rcp(e, ctypes.byref(n)) == 0
+    assert n.value == 0
+
+
+@pytest.mark.parametrize("mode,seed", [(0, 1), (0, 2), (1, 3), (1, 4)])
+def test_full_quotient(lib, mode, seed):
+    n = ctypes.c_ulonglong(0)
+    ex = (ctypes.c_float * 4)()
+    assert lib.check_div_full(mode, 512, seed, ctypes.byref(n), ex) == 0
+    assert n.value == 0, f"{n.value} quotients differ, e.g. a={ex[0]!r} b={ex[1]!r} got {ex[2]!r} want {ex[3]!r}"
+
+
+@pytest.mark.parametrize("seed", [11, 12])
+def test_sigmoid_of_updated_logit(lib, seed):
+    n = ctypes.c_ulonglong(0)
+    ex = (ctypes.c_float * 4)()
+    assert lib.check_sigmoid_near(seed, ctypes.byref(n), ex) == 0
+    assert n.value == 0, f"{n.value} differ, e.g. q0={ex[0]!r} q1={ex[1]!r} got {ex[2]!r} want {ex[3]!r}"
