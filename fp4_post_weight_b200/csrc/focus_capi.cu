@@ -24,7 +24,7 @@ constexpr int MAX_DEVICES = 64;
 
 struct DeviceInfo {
     int sms = 0;
-    int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_amax = 0, occ_adam = 0;
+    int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_amax = 0, occ_adam = 0;
 };
 
 std::once_flag g_once[MAX_DEVICES];
@@ -42,17 +42,22 @@ int device_info(DeviceInfo **out) {
                              (int)stage_smem_bytes<KIND_BWD>());
         cudaFuncSetAttribute(pipe_kernel<KIND_STEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)stage_smem_bytes<KIND_STEP>());
+        cudaFuncSetAttribute(pipe_kernel<KIND_STEP, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)stage_smem_bytes<KIND_STEP>());
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_fwd, pipe_kernel<KIND_FWD>, CTA_THREADS,
                                                       stage_smem_bytes<KIND_FWD>());
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_bwd, pipe_kernel<KIND_BWD>, CTA_THREADS,
                                                       stage_smem_bytes<KIND_BWD>());
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_step, pipe_kernel<KIND_STEP>, CTA_THREADS,
                                                       stage_smem_bytes<KIND_STEP>());
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_step_wqu, pipe_kernel<KIND_STEP, true>, CTA_THREADS,
+                                                      stage_smem_bytes<KIND_STEP>());
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_amax, amax_tiles_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_adam, adamw_kernel, THREADS, 0);
     });
     DeviceInfo &d = g_info[dev];
-    if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0)
+    if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_step_wqu <= 0 || d.occ_amax <= 0 ||
+        d.occ_adam <= 0)
         return FOCUS_ERR_CUDA;
     *out = &d;
     return FOCUS_OK;
@@ -133,16 +138,18 @@ int check_hyper(float lr, float beta1, float beta2, float eps, float wd, int64_t
 using namespace focus;
 
 namespace {
-template <int KIND>
+template <int KIND, bool WQU = false>
 int launch_on(const Args &a, cudaStream_t s) {
     DeviceInfo *di;
     int rc = device_info(&di);
     if (rc) return rc;
     if (a.total_tiles == 0 && !a.one_scale_out) return FOCUS_OK;
-    const int occ = KIND == KIND_FWD ? di->occ_fwd : (KIND == KIND_BWD ? di->occ_bwd : di->occ_step);
+    const int occ = KIND == KIND_FWD ? di->occ_fwd
+                    : KIND == KIND_BWD ? di->occ_bwd
+                    : (WQU ? di->occ_step_wqu : di->occ_step);
     int64_t grid = grid_for(a.total_tiles, di->sms, occ);
     if (grid < 1) grid = 1;   // the pack of an empty tensor still writes its tensor scale
-    pipe_kernel<KIND><<<(unsigned)grid, CTA_THREADS, stage_smem_bytes<KIND>(), s>>>(a);
+    pipe_kernel<KIND, WQU><<<(unsigned)grid, CTA_THREADS, stage_smem_bytes<KIND>(), s>>>(a);
     return launch_status();
 }
 
@@ -336,7 +343,7 @@ int focus_adamw_step(float *p, const float *g, float *exp_avg, float *exp_avg_sq
 
 int focus_table_prepare(focus_tensor_desc *d, int n, int purpose, int64_t *total_tiles) {
     if (!d || !total_tiles) return FOCUS_ERR_NULL;
-    if (n < 0 || (purpose != 0 && purpose != 1)) return FOCUS_ERR_VALUE;
+    if (n < 0 || purpose < 0 || purpose > 2) return FOCUS_ERR_VALUE;
     int64_t tiles = 0, blocks = 0;
     for (int i = 0; i < n; ++i) {
         focus_tensor_desc &e = d[i];
@@ -354,6 +361,7 @@ int focus_table_prepare(focus_tensor_desc *d, int n, int purpose, int64_t *total
             if ((e.codes == nullptr) != (e.scales == nullptr)) return FOCUS_ERR_NULL;
             if (purpose == 1 && (!e.dWq || !e.m_exp_avg || !e.m_exp_avg_sq || !e.q_exp_avg || !e.q_exp_avg_sq))
                 return FOCUS_ERR_NULL;
+            if (purpose == 2 && (!e.dWq || !e.dm || !e.dq)) return FOCUS_ERR_NULL;
             if ((e.dm == nullptr) != (e.dq == nullptr)) return FOCUS_ERR_NULL;
         }
         e.block_begin = blocks;
@@ -390,7 +398,8 @@ int focus_step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_ti
     int rc = check_hyper(hp->lr_m, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
     if (rc) return rc;
     if ((rc = check_hyper(hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
-    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD | FOCUS_STEP_PACK_UPDATED))
+    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD | FOCUS_STEP_PACK_UPDATED |
+                            FOCUS_STEP_WQ_UPDATED))
         return FOCUS_ERR_VALUE;
     if (n == 0) return FOCUS_OK;
     if (!descs_dev) return FOCUS_ERR_NULL;
@@ -404,7 +413,36 @@ int focus_step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_ti
     a.write_grad = (flags & FOCUS_STEP_WRITE_GRAD) ? 1 : 0;
     a.pack_updated = (flags & FOCUS_STEP_PACK_UPDATED) ? 1 : 0;
     a.hp = make_hyper(hp->lr_m, hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
+    if (flags & FOCUS_STEP_WQ_UPDATED) return launch_on<KIND_STEP, true>(a, (cudaStream_t)stream);
     return launch_on<KIND_STEP>(a, (cudaStream_t)stream);
+}
+
+int focus_fwd_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {
+    if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
+    if (n == 0) return FOCUS_OK;
+    if (!descs_dev) return FOCUS_ERR_NULL;
+    if (!aligned16(descs_dev)) return FOCUS_ERR_ALIGN;
+    Args a{};
+    a.table = descs_dev;
+    a.n_tensors = n;
+    a.total_tiles = total_tiles;
+    a.write_wq = 1;
+    return launch_on<KIND_FWD>(a, (cudaStream_t)stream);
+}
+
+int focus_ste_bwd_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, int accumulate,
+                        focus_stream_t stream) {
+    if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
+    if (accumulate != 0 && accumulate != 1) return FOCUS_ERR_VALUE;
+    if (n == 0) return FOCUS_OK;
+    if (!descs_dev) return FOCUS_ERR_NULL;
+    if (!aligned16(descs_dev)) return FOCUS_ERR_ALIGN;
+    Args a{};
+    a.table = descs_dev;
+    a.n_tensors = n;
+    a.total_tiles = total_tiles;
+    a.accumulate = accumulate;
+    return launch_on<KIND_BWD>(a, (cudaStream_t)stream);
 }
 
 int focus_pack_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {

@@ -204,11 +204,31 @@ __device__ __forceinline__ void encode_block(const TV &T, const uint32_t *w, flo
     }
 }
 
+// w' = bf16(fl(fl(c*S)*s2)) of one block from its two code words and scale byte.
+template <class TV>
+__device__ __forceinline__ void store_wq_from_codes(const TV &T, uint32_t blk, const uint32_t codes[2], uint32_t sbyte) {
+    const uint16_t S_h = (uint16_t)e4m3_normal_f16_bits(sbyte);
+    const uint64_t s2_2 = f2_pack(T.s2, T.s2);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t h2 = e2m1_pair_f16x2((codes[k] >> (8 * j)) & 0xffu);
+            const uint64_t p = f2_mul(f2_pack(mul_f16_exact(lo16(h2), S_h), mul_f16_exact(hi16(h2), S_h)), s2_2);
+            o[j] = pack_bf16x2(f2_lo(p), f2_hi(p));
+        }
+        __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + (2u * blk + (uint32_t)k), make_uint4(o[0], o[1], o[2], o[3]));
+    }
+}
+
 // The forward, the straight-through gradients and the AdamW update of one block.
+// WQU (step only, FOCUS_STEP_WQ_UPDATED): W' is that of the updated m and q,
+// a compile-time choice so that the other step variants keep its registers.
 // TV is any view of a tensor with members d (descriptor), s2, den and nblk:
 // the consumer warps pass the stage record in shared memory, so the
 // descriptor's pointers are read where used instead of held in registers.
-template <int KIND, class TV>
+template <int KIND, bool WQU, class TV>
 __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block &B) {
     // A_b = max |w| over the block: max of the bf16 magnitude bit patterns (a NaN
     // or an infinity sorts above every finite magnitude, which is how it is found)
@@ -229,7 +249,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
     const uint16_t S_h = (uint16_t)e4m3_normal_f16_bits(sbyte);
     const uint64_t s2_2 = f2_pack(T.s2, T.s2);
 
-    const bool want_wq = KIND != KIND_BWD && a.write_wq && T.d.Wq != nullptr && B.valid;
+    const bool want_wq = KIND != KIND_BWD && !WQU && a.write_wq && T.d.Wq != nullptr && B.valid;
     float sig[2], sq[2];
     double et[2];                               // e^-q of the forward, reused by the export
     uint64_t sm2 = 0ull;                        // sum of g * (in ? c - y : c), pairwise
@@ -327,13 +347,19 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
                 reinterpret_cast<float2 *>(T.d.q_exp_avg)[B.blk] = make_float2(f2_lo(v1), f2_hi(v1));
                 reinterpret_cast<float2 *>(T.d.q_exp_avg_sq)[B.blk] = make_float2(f2_lo(v2), f2_hi(v2));
             }
-            // NVFP4 export of the updated m and q: what a pack after this step would write
-            if (a.pack_updated && B.valid && T.d.codes) {
+            // the forward of the updated m and q: NVFP4 export (what a pack after this
+            // step would write) and/or W' for the next step's forward
+            const bool exp_codes = a.pack_updated && T.d.codes != nullptr;
+            const bool exp_wq = WQU && T.d.Wq != nullptr;
+            if (B.valid && (exp_codes || exp_wq)) {
                 uint32_t sb2, codes2[2];
                 encode_block(T, B.w, A, B.m, f2_lo(qp), f2_hi(qp), et[0], et[1], q_old0, q_old1, sb2, codes2);
-                uint2 cc; cc.x = codes2[0]; cc.y = codes2[1];
-                reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
-                T.d.scales[B.blk] = (uint8_t)sb2;
+                if (exp_codes) {
+                    uint2 cc; cc.x = codes2[0]; cc.y = codes2[1];
+                    reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
+                    T.d.scales[B.blk] = (uint8_t)sb2;
+                }
+                if (exp_wq) store_wq_from_codes(T, B.blk, codes2, sb2);
             }
         }
     }
@@ -466,8 +492,17 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
         const uint32_t first = found ? (uint32_t)(tile - T.d.tile_begin) * TILE_BLOCKS : 0u;
         const int64_t left = T.nblk - (int64_t)first;
         const uint32_t nb = found ? (uint32_t)(left < TILE_BLOCKS ? left : TILE_BLOCKS) : 0u;
-        const uint32_t mode = (!found || !T.ok) ? MODE_SKIP : (nb == (uint32_t)TILE_BLOCKS ? MODE_BULK : MODE_DIRECT);
-        if (found && !T.ok) atomicOr(&g_error_flags, 2u);
+        // a descriptor without a pointer this kernel needs (a table prepared for
+        // another purpose) is skipped and reported, never dereferenced
+        bool complete = T.d.W != nullptr && T.d.m != nullptr && T.d.q != nullptr;
+        if (KIND != KIND_FWD) complete = complete && T.d.dWq != nullptr;
+        if (KIND == KIND_BWD || a.accumulate || a.write_grad) complete = complete && T.d.dm != nullptr && T.d.dq != nullptr;
+        if (KIND == KIND_STEP)
+            complete = complete && T.d.m_exp_avg && T.d.m_exp_avg_sq && T.d.q_exp_avg && T.d.q_exp_avg_sq;
+        if (KIND != KIND_BWD && T.d.codes != nullptr) complete = complete && T.d.scales != nullptr;
+        const bool usable = found && T.ok && (complete || T.nblk == 0);
+        const uint32_t mode = !usable ? MODE_SKIP : (nb == (uint32_t)TILE_BLOCKS ? MODE_BULK : MODE_DIRECT);
+        if (found && !(T.ok && complete)) atomicOr(&g_error_flags, 2u);
         inf.d = T.d;
         inf.nblk = T.nblk;
         inf.s2 = T.s2;
@@ -512,7 +547,7 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
 }
 
 // The consumers: NC_WARPS warps computing from the ring.
-template <int KIND>
+template <int KIND, bool WQU>
 __device__ __forceinline__ void consume(const Args &a, const unsigned char *smem, uint64_t *full, uint64_t *empty,
                                         const StageInfo *info) {
     using L = Layout<KIND>;
@@ -534,14 +569,14 @@ __device__ __forceinline__ void consume(const Args &a, const unsigned char *smem
             Block B;
             if (mode == MODE_BULK) load_block_smem<KIND>(a, stage, B, lb, inf.first + lb);
             else load_block_global<KIND>(inf, a, B, inf.first + lb);
-            compute_block<KIND>(inf, a, B);
+            compute_block<KIND, WQU>(inf, a, B);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
     }
 }
 
-template <int KIND>
+template <int KIND, bool WQU = false>
 __global__ void __launch_bounds__(CTA_THREADS, Depth<KIND>::MIN_CTAS) pipe_kernel(const Args a) {
     constexpr int S = Depth<KIND>::STAGES;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -561,7 +596,7 @@ __global__ void __launch_bounds__(CTA_THREADS, Depth<KIND>::MIN_CTAS) pipe_kerne
         if (threadIdx.x == CONSUMERS) produce<KIND>(a, smem, full, empty, info);
         return;
     }
-    consume<KIND>(a, smem, full, empty, info);
+    consume<KIND, WQU>(a, smem, full, empty, info);
 }
 
 // ---------------------------------------------------------------------------

@@ -28,6 +28,7 @@ FOCUS_OK = 0
 FOCUS_STEP_ACCUMULATE = 1
 FOCUS_STEP_WRITE_GRAD = 2
 FOCUS_STEP_PACK_UPDATED = 4
+FOCUS_STEP_WQ_UPDATED = 8
 
 
 class focus_tensor_desc(ctypes.Structure):
@@ -60,6 +61,8 @@ _SIGS = {
     "focus_s2_multi": ([_P, _I, _I64, _P, _SZ, _P], _I),
     "focus_step_fused": ([_P, _I, _I64, ctypes.POINTER(focus_hparams), _I64, ctypes.c_uint, _P], _I),
     "focus_pack_multi": ([_P, _I, _I64, _P], _I),
+    "focus_fwd_multi": ([_P, _I, _I64, _P], _I),
+    "focus_ste_bwd_multi": ([_P, _I, _I64, _I, _P], _I),
     "focus_get_error": ([_P], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -205,6 +208,15 @@ def focus_step_fused(table_dev, n: int, total_tiles: int, hp: focus_hparams, ste
                      stream=None):
     _check(_lib.focus_step_fused(_ptr(table_dev), int(n), int(total_tiles), ctypes.byref(hp), int(step),
                                  int(flags), _stream(stream)), "focus_step_fused")
+
+
+def focus_fwd_multi(table_dev, n: int, total_tiles: int, stream=None):
+    _check(_lib.focus_fwd_multi(_ptr(table_dev), int(n), int(total_tiles), _stream(stream)), "focus_fwd_multi")
+
+
+def focus_ste_bwd_multi(table_dev, n: int, total_tiles: int, accumulate: bool = False, stream=None):
+    _check(_lib.focus_ste_bwd_multi(_ptr(table_dev), int(n), int(total_tiles), 1 if accumulate else 0,
+                                    _stream(stream)), "focus_ste_bwd_multi")
 
 
 def focus_pack_multi(table_dev, n: int, total_tiles: int, stream=None):

@@ -213,11 +213,18 @@ typedef struct focus_hparams {
 #define FOCUS_STEP_PACK_UPDATED 4u /* codes/scales receive the NVFP4 export of the UPDATED m and q (what
                                       focus_pack_multi would write after this call) instead of the
                                       forward's; W is not read again */
+#define FOCUS_STEP_WQ_UPDATED 8u   /* W' receives the forward of the UPDATED m and q (what focus_fwd_multi
+                                      would write after this call: the next step's fake-quantized
+                                      weight) instead of the forward's */
 
-/* Checks every entry (pointers, alignment, shapes, which outputs are present
- * for `purpose`: 0 = s2/forward/pack only, 1 = also focus_step_fused) and
- * fills block_begin and tile_begin.  Host memory in, host memory out.
- * *total_tiles receives the number of work tiles, passed to the calls below. */
+/* Checks every entry (pointers, alignment, shapes, which inputs are present
+ * for `purpose`: 0 = s2/forward/pack, 1 = also focus_step_fused (dWq and the
+ * four moments), 2 = also focus_ste_bwd_multi (dWq, dm, dq)) and fills
+ * block_begin and tile_begin.  Host memory in, host memory out.
+ * *total_tiles receives the number of work tiles, passed to the calls below.
+ * A device-resident table cannot be checked again at call time: a kernel that
+ * meets an entry lacking a pointer it needs skips that entry and sets the
+ * device flag (FOCUS_ERR_NONFINITE_INPUT from focus_get_error). */
 int focus_table_prepare(focus_tensor_desc *descs_host, int n_tensors, int purpose, int64_t *total_tiles);
 
 /* Workspace bytes focus_s2_multi needs for a prepared table. */
@@ -231,11 +238,25 @@ int focus_s2_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t to
  * forward (W' when desc.Wq != NULL, codes/scales when present), straight-
  * through backward, AdamW on m and q (lr_m for m, lr_q for q) at step `step`.
  * hp is a host pointer.  flags: FOCUS_STEP_ACCUMULATE, FOCUS_STEP_WRITE_GRAD
- * (both need desc.dm and desc.dq), FOCUS_STEP_PACK_UPDATED.  W' is the
- * forward's, i.e. of m and q before the update; codes and scales are the
- * forward's too unless FOCUS_STEP_PACK_UPDATED is set. */
+ * (both need desc.dm and desc.dq), FOCUS_STEP_PACK_UPDATED,
+ * FOCUS_STEP_WQ_UPDATED.  W', codes and scales are the forward's, i.e. of m
+ * and q before the update, unless FOCUS_STEP_WQ_UPDATED / _PACK_UPDATED make
+ * them those of the updated m and q. */
 int focus_step_fused(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
                      const focus_hparams *hp, int64_t step, unsigned flags, focus_stream_t stream);
+
+/* Forward of every entry in one launch: W' (desc.Wq), and the codes and
+ * scales when present.  Card, "What this is": the S_b, c_i and w'_i
+ * equations. */
+int focus_fwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
+                    focus_stream_t stream);
+
+/* Straight-through backward of every entry in one launch (as focus_ste_bwd):
+ * desc.dm/dq receive the gradients, added to what they hold when
+ * accumulate = 1 -- the micro-batches of a step before the one that runs
+ * focus_step_fused with FOCUS_STEP_ACCUMULATE.  The table needs purpose 2. */
+int focus_ste_bwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles, int accumulate,
+                        focus_stream_t stream);
 
 /* NVFP4 pack of every entry with codes and scales present (desc.s2 holds the
  * tensor scale, which the caller exports). */

@@ -99,6 +99,17 @@ def test_table_prepare_on_host(F):
         F.focus_table_prepare(descs, 1)
     assert e.value.status == 1
     assert F.focus_table_prepare(descs, 0) == tiles
+    # a table backward needs dW', dm and dq; purposes beyond 2 do not exist
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, 2)
+    assert e.value.status == 1
+    for i in range(n):
+        descs[i].dm = P + 65536 * (i + 1)
+        descs[i].dq = P + 65536 * (i + 1) + 4096
+    assert F.focus_table_prepare(descs, 2) == tiles
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, 3)
+    assert e.value.status == 4
     descs[2].in_ = 40
     with pytest.raises(F.FocusError) as e:
         F.focus_table_prepare(descs, 0)
@@ -110,11 +121,20 @@ def test_table_prepare_on_host(F):
     assert e.value.status == 3
 
 
+def test_multi_entry_checks(F):
+    assert F.raw_call("focus_ste_bwd_multi", P, 1, 1, 2, None) == 4        # accumulate must be 0 or 1
+    assert F.raw_call("focus_ste_bwd_multi", None, 1, 1, 0, None) == 1
+    assert F.raw_call("focus_fwd_multi", U, 1, 1, None) == 3
+    assert F.raw_call("focus_fwd_multi", P, -1, 1, None) == 4
+    assert F.raw_call("focus_fwd_multi", P, 0, 0, None) == 0                  # empty table: nothing to do
+
+
 def test_step_hparam_checks(F):
     hp = F.focus_hparams(5e-3, 1e-3, 0.9, 0.999, 1e-8, 0.0)
     assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(hp), 0, 0, None) == 4
-    assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(hp), 1, 8, None) == 4
+    # unknown flag bits (every call here fails its host checks: nothing is launched)
     assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(hp), 1, 16, None) == 4
+    assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(hp), 1, 32 | 1, None) == 4
     assert F.raw_call("focus_step_fused", P, 1, 1, None, 1, 0, None) == 1
     bad = F.focus_hparams(5e-3, -1e-3, 0.9, 0.999, 1e-8, 0.0)
     assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(bad), 1, 0, None) == 4

@@ -311,3 +311,88 @@ def test_nonfinite_input_sets_flag(F):
     m[0, 0] = float("inf")
     F.focus_fwd(W, m, q, 1e-4, Wq)
     assert F.focus_get_error() == 7
+
+
+@pytest.mark.parametrize("accumulate", [False, True])
+def test_fwd_and_bwd_multi(F, accumulate):
+    """The one-launch forward and straight-through backward over a table."""
+    from fp4_post_weight_b200.table import FocusTable, PURPOSE_BACKWARD
+    shapes = SHAPES + [(0, 32)]
+    ents = _entries(shapes, 80)
+    g = torch.Generator(device="cuda").manual_seed(8)
+    if accumulate:
+        for e in ents:
+            e.dm.copy_(synth.normal(e.dm.shape, 0, 1e-5, g, "cuda"))
+            e.dq.copy_(synth.normal(e.dq.shape, 0, 1e-7, g, "cuda"))
+    host_in = [(host_bits(e.W), host_bits(e.dWq), host(e.m).copy(), host(e.q).copy(), host(e.dm).copy(),
+                host(e.dq).copy()) for e in ents]
+    tab = FocusTable(ents, PURPOSE_BACKWARD)
+    tab.s2()
+    tab.fwd()
+    tab.bwd(accumulate=accumulate)
+    assert F.focus_get_error() == 0
+    for e, (Wb, Gb, m, q, dm0, dq0) in zip(ents, host_in):
+        if Wb.size == 0:
+            continue
+        s2 = oracle.s2(Wb)
+        ref = oracle.fwd(Wb, m, q, s2)
+        mism = check_forward(ref, Wq=host_bits(e.Wq), codes=unpack_codes(host(e.codes)), scales=host(e.scales))
+        skip = block_mask(mism)
+        if accumulate:
+            rdm, rdq = oracle.ste_bwd(Wb, Gb, m, q, s2, dm=dm0, dq=dq0)
+        else:
+            rdm, rdq = oracle.ste_bwd(Wb, Gb, m, q, s2)
+        assert_close(host(e.dm), rdm, "dm", skip)
+        assert_close(host(e.dq), rdq, "dq", np.repeat(skip, 2, axis=1))
+        assert np.array_equal(host(e.m), m) and np.array_equal(host(e.q), q)
+
+
+def test_micro_batch_step(F):
+    """A calibration step over four micro-batches (gradient accumulation, as the
+    card's calibration runs it): W' of the current m and q from the table
+    forward, the straight-through gradients of micro-batches 1-3 summed into
+    dm/dq, then the fused step adds micro-batch 4, updates m and q, and with
+    FOCUS_STEP_WQ_UPDATED writes the next step's W' in the same pass."""
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    shapes = [(37, 1040), (64, 512), (128, 2048), (3, 48)]
+    ents = _entries(shapes, 90, with_pack=False)
+    g = torch.Generator(device="cuda").manual_seed(9)
+    grads = [[synth.normal_bf16(e.W.shape, 1e-3, g, "cuda") for _ in range(4)] for e in ents]
+    host_in = [(host_bits(e.W), host(e.m).copy(), host(e.q).copy(), [host_bits(x) for x in gs])
+               for e, gs in zip(ents, grads)]
+    tab = FocusTable(ents)
+    tab.s2()
+    tab.fwd()
+    torch.cuda.synchronize()
+    for e, (Wb, m, q, _) in zip(ents, host_in):
+        check_forward(oracle.fwd(Wb, m, q, oracle.s2(Wb)), Wq=host_bits(e.Wq))
+    for j in range(3):
+        for e, gs in zip(ents, grads):
+            e.dWq.copy_(gs[j])
+        tab.bwd(accumulate=j > 0)
+    for e, gs in zip(ents, grads):
+        e.dWq.copy_(gs[3])
+    tab.step(1, hparams(), flags=F.FOCUS_STEP_ACCUMULATE | F.FOCUS_STEP_WRITE_GRAD | F.FOCUS_STEP_WQ_UPDATED)
+    assert F.focus_get_error() == 0
+    wq_next = [e.Wq.clone() for e in ents]
+    for e, (Wb, m, q, Gs) in zip(ents, host_in):
+        s2 = oracle.s2(Wb)
+        skip = block_mask(check_forward(oracle.fwd(Wb, m, q, s2)))
+        dm, dq = oracle.ste_bwd(Wb, Gs[0], m, q, s2)
+        for j in (1, 2):
+            oracle.ste_bwd(Wb, Gs[j], m, q, s2, dm=dm, dq=dq)
+        z = [np.zeros_like(m), np.zeros_like(m), np.zeros_like(q), np.zeros_like(q)]
+        _, gm, gq = oracle.step(Wb, Gs[3], m, q, *z, s2, 1, want_wq=False, dm_acc=dm, dq_acc=dq)
+        skq = np.repeat(skip, 2, axis=1)
+        assert_close(host(e.dm), gm, "dm over four micro-batches", skip)
+        assert_close(host(e.dq), gq, "dq over four micro-batches", skq)
+        assert_close(host(e.m), m, "m", skip)
+        assert_close(host(e.q), q, "q", skq)
+        for name, want, sk in zip(("m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"), z,
+                                  (skip, skip, skq, skq)):
+            assert_close(host(getattr(e, name)), want, name, sk)
+    # the step's W' is bit for bit the table forward of the updated m and q
+    tab.fwd()
+    assert F.focus_get_error() == 0
+    for e, w in zip(ents, wq_next):
+        assert torch.equal(e.Wq.view(torch.int16), w.view(torch.int16))
