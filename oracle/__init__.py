@@ -76,6 +76,8 @@ def lib():
         L.fo_step.restype = ctypes.c_int
         L.fo_pack.argtypes = [_P, _P, _P, _F, _I64, _I64, _P, _P, _P]
         L.fo_pack.restype = ctypes.c_int
+        L.fo_f46.argtypes = [_P, _I64, _I64, _F, ctypes.c_int, _P, _P, _P, _P, _P, _P]
+        L.fo_f46.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -233,3 +235,31 @@ def pack(W, m, q, s2v):
     ts = np.zeros(1, np.float32)
     _chk(lib().fo_pack(_p(W), _p(m), _p(q), float(s2v), out, inn, _p(codes), _p(scales), _p(ts)))
     return codes, scales, ts[0]
+
+
+@dataclass
+class FourOverSix:
+    codes: np.ndarray       # uint8 [rows, cols], one E2M1 code per element
+    scales: np.ndarray      # uint8 [rows, cols/16], E4M3 byte of the chosen block scale
+    Xq: np.ndarray          # uint16 bf16 bits [rows, cols], dequantized values
+    four: np.ndarray        # uint8 [rows, cols/16], 1 where the target 4 was chosen
+    errs: np.ndarray        # float64 [rows, cols/16, 2], squared errors of the targets 6 and 4
+    row_scales: np.ndarray | None   # float32 [rows] with one scale per row, else None
+
+
+def fouroversix(X, s=None) -> FourOverSix:
+    """FourOverSix round to nearest.  s: the tensor scale (weights), or None for
+    one scale per row (per-token activations), computed from each row."""
+    X = _c(X, np.uint16)
+    rows, cols = X.shape
+    nb = cols // 16
+    codes = np.empty((rows, cols), np.uint8)
+    scales = np.empty((rows, nb), np.uint8)
+    Xq = np.empty((rows, cols), np.uint16)
+    four = np.empty((rows, nb), np.uint8)
+    errs = np.empty((rows, nb, 2), np.float64)
+    per_row = s is None
+    rs = np.empty(rows, np.float32) if per_row else None
+    _chk(lib().fo_f46(_p(X), rows, cols, 0.0 if per_row else float(s), 1 if per_row else 0, _p(codes),
+                      _p(scales), _p(Xq), _p(four), _p(errs), _p(rs)))
+    return FourOverSix(codes, scales, Xq, four, errs, rs)

@@ -505,3 +505,142 @@ int fo_pack(const uint16_t *W, const float *m, const float *q, float s2, int64_t
     *tensor_scale = s2;
     return FO_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* FourOverSix: round-to-nearest NVFP4 with a choice of two block targets    */
+/* ------------------------------------------------------------------------ */
+/*
+ * Sources: [card] section "Calibration", the activation bullet: every
+ * 16-element block's scale maps the block maximum to 6 or to 4, whichever
+ * has the lower error, with one FP32 scale per token; [card] section
+ * "Perplexity": round-to-nearest FourOverSix weights are the reference row;
+ * "Llama-3.1-8B-Instruct FlipQuant MixFP4 maps", section "What this is": the
+ * rest of the format is NVFP4 (16-element blocks, E4M3 scale, FP32 tensor
+ * scale).
+ *
+ * Readings (the pages give the rule in words only):
+ *  - The candidate for target T (6 or 4) is the card's block equations with
+ *    m = 1, sigmoid = 1 and T in place of 6: x_T = fl(A / fl(T*s)); scale 1
+ *    when x_T == 0; S_T = e4m3(clamp(x_T, 2^-6, 448)); D_T = fl(S_T*s);
+ *    c_i = E2M1(clamp(fl(w_i/D_T), -6, 6)).  With T = 6 this is plain NVFP4
+ *    round to nearest.
+ *  - "error" is the squared error of the dequantized block,
+ *    sum_i (w_i - c_i*S_T*s)^2, evaluated in binary64 with one rounding per
+ *    operation and the terms added in element order (c*S*s is exact there).
+ *  - The target 4 is taken only when its error is strictly lower; equal
+ *    errors keep 6.
+ *  - The dequantized value is bf16(fl(fl(c*S)*s)), as w' of the card.
+ *  - One scale per token: s_t = fl(A_row / 2688), the tensor scale's formula
+ *    over one row.  A row whose maximum is 0 has s_t = 0; its blocks get
+ *    scale byte 0x38 (1.0), codes 0 and values 0.
+ */
+
+typedef struct {
+    int sb[2];         /* E4M3 byte of S_T for T = 6 (index 0) and T = 4 (index 1) */
+    int code[2][16];   /* E2M1 codes under each target */
+    double err[2];     /* squared error under each target */
+    int four;          /* 1 when the target 4 is chosen */
+} fo_f46_block;
+
+static void f46_candidate(const float *w, float A, float s, float target, int *sb, int *code, double *err)
+{
+    float den = target * s;
+    float x = A / den;
+    if (x == 0.0f) x = 1.0f;
+    if (x < 0x1p-6f) x = 0x1p-6f;
+    if (x > 448.0f) x = 448.0f;
+    *sb = fo_e4m3_encode(x);
+    float S = (float)fo_e4m3_decode(*sb);
+    float D = S * s;
+    double e = 0.0;
+    for (int i = 0; i < 16; ++i) {
+        float u = w[i] / D;
+        if (u < -6.0f) u = -6.0f;
+        if (u > 6.0f) u = 6.0f;
+        code[i] = fo_e2m1_encode(u);
+        double v = fo_e2m1_decode(code[i]) * (double)S * (double)s;   /* exact */
+        double d = (double)w[i] - v;
+        e = e + d * d;
+    }
+    *err = e;
+}
+
+/* Both candidates of one block of 16 bf16 values with scale s > 0, and the choice. */
+static void f46_block(const uint16_t *w16, float s, fo_f46_block *B)
+{
+    float w[16];
+    float A = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        w[i] = fo_bf16_to_f32(w16[i]);
+        float a = fabsf(w[i]);
+        if (a > A) A = a;
+    }
+    f46_candidate(w, A, s, 6.0f, &B->sb[0], B->code[0], &B->err[0]);
+    f46_candidate(w, A, s, 4.0f, &B->sb[1], B->code[1], &B->err[1]);
+    B->four = B->err[1] < B->err[0];
+}
+
+/* FourOverSix over a row-major [rows, cols] bf16 tensor (cols % 16 == 0).
+ * per_row = 0: s is the tensor scale (s2 of the weights, > 0);
+ * per_row = 1: every row gets its own scale s_t, written to row_scales[r].
+ * Outputs (each may be NULL):
+ *   codes  u8 [rows, cols]        E2M1 code of the chosen target, one per element
+ *   scales u8 [rows, cols/16]     E4M3 byte of the chosen scale
+ *   Xq     bf16 bits [rows, cols] dequantized values
+ *   four   u8 [rows, cols/16]     1 where the target 4 was chosen
+ *   errs   f64 [rows, cols/16, 2] squared errors of the targets 6 and 4    */
+int fo_f46(const uint16_t *X, int64_t rows, int64_t cols, float s, int per_row, uint8_t *codes,
+           uint8_t *scales, uint16_t *Xq, uint8_t *four, double *errs, float *row_scales)
+{
+    int rc = check_shape(rows, cols);
+    if (rc) return rc;
+    if (!per_row && (rc = check_s2(s))) return rc;
+    if (per_row && !row_scales) return FO_ERR_VALUE;
+    const int64_t nb = cols / 16;
+    int bad = 0;
+#pragma omp parallel for reduction(| : bad) schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *xr = X + r * cols;
+        float sr = s;
+        for (int64_t i = 0; i < cols; ++i)
+            if (!isfinite(fo_bf16_to_f32(xr[i]))) bad = 1;
+        if (per_row) {
+            float A = 0.0f;
+            for (int64_t i = 0; i < cols; ++i) {
+                float a = fabsf(fo_bf16_to_f32(xr[i]));
+                if (a > A) A = a;
+            }
+            sr = A / 2688.0f;
+            row_scales[r] = sr;
+        }
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t blk = r * nb + b;
+            const int64_t e0 = r * cols + 16 * b;
+            if (sr == 0.0f) {           /* a row of zeros */
+                if (scales) scales[blk] = 0x38;
+                if (four) four[blk] = 0;
+                if (errs) { errs[2 * blk] = 0.0; errs[2 * blk + 1] = 0.0; }
+                for (int i = 0; i < 16; ++i) {
+                    if (codes) codes[e0 + i] = 0;
+                    if (Xq) Xq[e0 + i] = 0;
+                }
+                continue;
+            }
+            fo_f46_block B;
+            f46_block(xr + 16 * b, sr, &B);
+            const int t = B.four;
+            const float S = (float)fo_e4m3_decode(B.sb[t]);
+            if (scales) scales[blk] = (uint8_t)B.sb[t];
+            if (four) four[blk] = (uint8_t)t;
+            if (errs) { errs[2 * blk] = B.err[0]; errs[2 * blk + 1] = B.err[1]; }
+            for (int i = 0; i < 16; ++i) {
+                if (codes) codes[e0 + i] = (uint8_t)B.code[t][i];
+                if (Xq) {
+                    float cS = (float)fo_e2m1_decode(B.code[t][i]) * S;
+                    Xq[e0 + i] = fo_f32_to_bf16(cS * sr);
+                }
+            }
+        }
+    }
+    return bad ? FO_ERR_NONFINITE : FO_OK;
+}
