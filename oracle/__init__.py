@@ -243,7 +243,7 @@ class FourOverSix:
     scales: np.ndarray      # uint8 [rows, cols/16], E4M3 byte of the chosen block scale
     Xq: np.ndarray          # uint16 bf16 bits [rows, cols], dequantized values
     four: np.ndarray        # uint8 [rows, cols/16], 1 where the target 4 was chosen
-    errs: np.ndarray        # float64 [rows, cols/16, 2], squared errors of the targets 6 and 4
+    errs: np.ndarray        # float32 [rows, cols/16, 2], squared errors of the targets 6 and 4
     row_scales: np.ndarray | None   # float32 [rows] with one scale per row, else None
 
 
@@ -257,7 +257,7 @@ def fouroversix(X, s=None) -> FourOverSix:
     scales = np.empty((rows, nb), np.uint8)
     Xq = np.empty((rows, cols), np.uint16)
     four = np.empty((rows, nb), np.uint8)
-    errs = np.empty((rows, nb, 2), np.float64)
+    errs = np.empty((rows, nb, 2), np.float32)
     per_row = s is None
     rs = np.empty(rows, np.float32) if per_row else None
     _chk(lib().fo_f46(_p(X), rows, cols, 0.0 if per_row else float(s), 1 if per_row else 0, _p(codes),

@@ -525,8 +525,13 @@ int fo_pack(const uint16_t *W, const float *m, const float *q, float s2, int64_t
  *    c_i = E2M1(clamp(fl(w_i/D_T), -6, 6)).  With T = 6 this is plain NVFP4
  *    round to nearest.
  *  - "error" is the squared error of the dequantized block,
- *    sum_i (w_i - c_i*S_T*s)^2, evaluated in binary64 with one rounding per
- *    operation and the terms added in element order (c*S*s is exact there).
+ *    sum_i (w_i - c_i*S_T*s)^2.  The pages fix no precision for it; it
+ *    decides an integer (the target), so it is evaluated in the kernels'
+ *    precision, binary32, in this order: d_i = fl(w_i - (c_i*S_T)*s) with one
+ *    rounding (c_i*S_T is exact, so this is one fused multiply-add); the even
+ *    elements i = 0, 2, ..., 14 and the odd elements i = 1, 3, ..., 15 are
+ *    summed separately, each as E <- fl(d_i*d_i + E) in index order from 0;
+ *    the error is fl(E_even + E_odd).
  *  - The target 4 is taken only when its error is strictly lower; equal
  *    errors keep 6.
  *  - The dequantized value is bf16(fl(fl(c*S)*s)), as w' of the card.
@@ -538,11 +543,11 @@ int fo_pack(const uint16_t *W, const float *m, const float *q, float s2, int64_t
 typedef struct {
     int sb[2];         /* E4M3 byte of S_T for T = 6 (index 0) and T = 4 (index 1) */
     int code[2][16];   /* E2M1 codes under each target */
-    double err[2];     /* squared error under each target */
+    float err[2];      /* squared error under each target */
     int four;          /* 1 when the target 4 is chosen */
 } fo_f46_block;
 
-static void f46_candidate(const float *w, float A, float s, float target, int *sb, int *code, double *err)
+static void f46_candidate(const float *w, float A, float s, float target, int *sb, int *code, float *err)
 {
     float den = target * s;
     float x = A / den;
@@ -552,17 +557,17 @@ static void f46_candidate(const float *w, float A, float s, float target, int *s
     *sb = fo_e4m3_encode(x);
     float S = (float)fo_e4m3_decode(*sb);
     float D = S * s;
-    double e = 0.0;
+    float E[2] = {0.0f, 0.0f};      /* even and odd elements */
     for (int i = 0; i < 16; ++i) {
         float u = w[i] / D;
         if (u < -6.0f) u = -6.0f;
         if (u > 6.0f) u = 6.0f;
         code[i] = fo_e2m1_encode(u);
-        double v = fo_e2m1_decode(code[i]) * (double)S * (double)s;   /* exact */
-        double d = (double)w[i] - v;
-        e = e + d * d;
+        float cS = (float)fo_e2m1_decode(code[i]) * S;                 /* exact */
+        float d = fmaf(-cS, s, w[i]);
+        E[i & 1] = fmaf(d, d, E[i & 1]);
     }
-    *err = e;
+    *err = E[0] + E[1];
 }
 
 /* Both candidates of one block of 16 bf16 values with scale s > 0, and the choice. */
@@ -588,9 +593,9 @@ static void f46_block(const uint16_t *w16, float s, fo_f46_block *B)
  *   scales u8 [rows, cols/16]     E4M3 byte of the chosen scale
  *   Xq     bf16 bits [rows, cols] dequantized values
  *   four   u8 [rows, cols/16]     1 where the target 4 was chosen
- *   errs   f64 [rows, cols/16, 2] squared errors of the targets 6 and 4    */
+ *   errs   f32 [rows, cols/16, 2] squared errors of the targets 6 and 4    */
 int fo_f46(const uint16_t *X, int64_t rows, int64_t cols, float s, int per_row, uint8_t *codes,
-           uint8_t *scales, uint16_t *Xq, uint8_t *four, double *errs, float *row_scales)
+           uint8_t *scales, uint16_t *Xq, uint8_t *four, float *errs, float *row_scales)
 {
     int rc = check_shape(rows, cols);
     if (rc) return rc;
@@ -619,7 +624,7 @@ int fo_f46(const uint16_t *X, int64_t rows, int64_t cols, float s, int per_row, 
             if (sr == 0.0f) {           /* a row of zeros */
                 if (scales) scales[blk] = 0x38;
                 if (four) four[blk] = 0;
-                if (errs) { errs[2 * blk] = 0.0; errs[2 * blk + 1] = 0.0; }
+                if (errs) { errs[2 * blk] = 0.0f; errs[2 * blk + 1] = 0.0f; }
                 for (int i = 0; i < 16; ++i) {
                     if (codes) codes[e0 + i] = 0;
                     if (Xq) Xq[e0 + i] = 0;

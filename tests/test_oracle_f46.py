@@ -42,7 +42,7 @@ def test_worked_example_weights():
     np.testing.assert_array_equal(r.scales, np.array(ex["scales"], np.uint8))
     np.testing.assert_array_equal(r.four, np.array(ex["four"], np.uint8))
     np.testing.assert_array_equal(r.codes, np.array(ex["codes"], np.uint8))
-    np.testing.assert_array_equal(r.errs, np.array(ex["errs_over_u2"]) * u * u)
+    np.testing.assert_array_equal(r.errs, (np.array(ex["errs_over_u2"]) * u * u).astype(F))
     assert ex["Xq_equals_W"] and np.array_equal(r.Xq, W)
 
 
@@ -61,8 +61,21 @@ def test_worked_example_tokens():
     assert ex["Xq_equals_X"] and np.array_equal(r.Xq, X)
 
 
+LD = np.longdouble
+
+
+def fma32(a, b, c):
+    """fl32(a*b + c) with one rounding, for binary32 arrays: a*b is exact in the
+    64-bit significand of x87 extended precision, and so is the sum unless c
+    dwarfs a*b, where both roundings give c's neighbourhood alike."""
+    assert np.finfo(LD).nmant >= 63
+    return (a.astype(LD) * b.astype(LD) + c.astype(LD)).astype(F)
+
+
 def candidate(Wf, s, T):
-    """Independent numpy model of one target: scale bytes, codes, bf16 values, squared errors."""
+    """Independent numpy model of one target: scale bytes, codes, bf16 values, squared errors
+    (binary32: d = fl(w - c*S*s) in one rounding, even and odd elements summed apart by
+    fused multiply-adds in index order, then added)."""
     out, inn = Wf.shape
     b = Wf.reshape(-1, 16)
     A = np.abs(b).max(1)
@@ -75,11 +88,12 @@ def candidate(Wf, s, T):
     y = b / D[:, None]
     c8 = np.clip(y, F(-6), F(6)).astype(ml_dtypes.float4_e2m1fn)
     c = c8.astype(F)
-    v = c.astype(np.float64) * S.astype(np.float64)[:, None] * np.float64(s)
-    err = np.zeros(b.shape[0])
-    for i in range(16):                 # element order, one rounding per step
-        d = b[:, i].astype(np.float64) - v[:, i]
-        err = err + d * d
+    cS = c * S[:, None]                                       # exact
+    E = [np.zeros(b.shape[0], F), np.zeros(b.shape[0], F)]
+    for i in range(16):
+        d = fma32(-cS[:, i], np.full(b.shape[0], s, F), b[:, i])
+        E[i & 1] = fma32(d, d, E[i & 1])
+    err = (E[0] + E[1]).astype(F)
     wq = (c * S[:, None]) * s
     wq16 = torch.from_numpy(wq.astype(F)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     return (sb.view(np.uint8).reshape(out, inn // 16), (c8.view(np.uint8) & 0xF).reshape(out, inn),
