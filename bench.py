@@ -5,9 +5,8 @@ up, down: 224 tensors, 6,979,321,856 weights), synthetic: W ~ N(0, 0.02) bf16,
 m = 1, q = 6, dW' ~ N(0, 1e-3) bf16, zero AdamW moments at step 1.  One step
 is one pass of the whole hot path over all 224 tensors:
   s2 of every tensor (two launches),
-  the fused forward + straight-through backward + AdamW step (one launch,
-  W' written, W read once),
-  the NVFP4 export pack of the updated parameters (one launch).
+  the fused forward + straight-through backward + AdamW step with the NVFP4
+  export of the updated parameters (one launch, W' written, W read once).
 Metric: Gelem/s = weights per second of whole steps (all ranks).  The
 roofline object reports the fused step kernel against the measured HBM copy
 bandwidth.
@@ -250,6 +249,9 @@ def run_ours(args, world, rank, local):
             "peak": peaks["hbm_gbs"], "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)",
             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(),
             "bytes_per_elem": BYTES_STEP, "launch_ms": round(step_kernel_ms, 4)}
+    rows = None
+    if not args.no_rows:
+        rows = measure_next_rows(ents, dev, N, peaks, world)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_seconds)
@@ -264,7 +266,7 @@ def run_ours(args, world, rank, local):
                            "l2": f"inputs larger than L2 ({N * 8.25 / 1e9:.1f} GB resident per GPU vs 126 MB L2)",
                            "parallelism": f"dp{world} (one model per GPU, no collective)",
                            "bytes_per_elem_step": BYTES_S2 + BYTES_STEP},
-                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "next_rows": rows,
                 "gpu_launches": 3 * args.steps, "clocks": clk,
                 "kernel_ms": {"fused_step": round(step_kernel_ms, 4), "fused_step_min": round(min(kms), 4),
                               "fused_step_max": round(max(kms), 4)}}
@@ -272,6 +274,104 @@ def run_ours(args, world, rank, local):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def _timed(fn, stream, reps: int = 5, warm: int = 3):
+    """Mean device time (ms) of fn() over reps calls, each bracketed by events on stream."""
+    import torch
+    for _ in range(warm):
+        fn()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev) / reps
+
+
+def _roof(bytes_moved: float, ms: float, peak: float) -> dict:
+    gbs = bytes_moved / (ms * 1e-3) / 1e9
+    return {"ms": round(ms, 4), "achieved_gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+
+
+def measure_next_rows(ents, dev, N, peaks, world):
+    """The rows after the hot path, each timed per launch with CUDA events on the
+    launching stream, after the headline's timed region (inputs larger than L2):
+      * FourOverSix round to nearest over the same 224 weights (one launch; codes
+        and scales, and codes, scales and W');
+      * FourOverSix with one scale per token over one decoder layer's linear
+        inputs for a micro-batch of 4096 tokens (q/k/v, o and gate/up inputs
+        [4096, 4096], the down input [4096, 14336]: 208 MB);
+      * a calibration step over four micro-batches: three table backward passes
+        (the first overwriting dm/dq, then accumulating) and the fused step
+        with FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WQ_UPDATED."""
+    import torch
+
+    import synth
+    from fp4_post_weight_b200 import focus as F
+    from fp4_post_weight_b200.table import Entry, FocusTable, PURPOSE_FOUROVERSIX, hparams
+    from fp4_post_weight_b200 import dist as D
+    stream = torch.cuda.current_stream(dev)
+    peak = peaks["hbm_gbs"]
+    out = {}
+    # FourOverSix weights
+    t_cs = FocusTable([Entry(W=e.W, m=None, q=None, s2=e.s2, codes=e.codes, scales=e.scales) for e in ents],
+                      PURPOSE_FOUROVERSIX)
+    t_all = FocusTable([Entry(W=e.W, m=None, q=None, s2=e.s2, codes=e.codes, scales=e.scales, Wq=e.Wq)
+                        for e in ents], PURPOSE_FOUROVERSIX)
+    ms = _timed(t_cs.fouroversix, stream)
+    r = {"kernel": "pipe_kernel<KIND_F46>", "bytes_per_weight": 2.5625, **_roof(2.5625 * N, ms, peak)}
+    ms = _timed(t_all.fouroversix, stream)
+    r["with_Wq"] = {"bytes_per_weight": 4.5625, **_roof(4.5625 * N, ms, peak)}
+    r["Gelem_s"] = round(N * world / (r["ms"] * 1e-3) / 1e9, 2)
+    out["fouroversix_weights_llama8b"] = r
+    # FourOverSix activations, one scale per token
+    Xs = [synth.activations(4096, h, dev, seed=50 + j) for j, h in enumerate((4096, 4096, 4096, 14336))]
+    bufs = [(torch.empty(X.shape[0], device=dev), torch.empty((X.shape[0], X.shape[1] // 2), dtype=torch.uint8,
+                                                                device=dev),
+             torch.empty((X.shape[0], X.shape[1] // 16), dtype=torch.uint8, device=dev)) for X in Xs]
+    n_act = sum(X.numel() for X in Xs)
+    b_act = sum(X.numel() * (2 + 0.5 + 0.0625) + 4 * X.shape[0] for X in Xs)
+
+    def act():
+        for X, (ts, c, sc) in zip(Xs, bufs):
+            F.focus_fouroversix_act(X, ts, c, sc)
+    ms = _timed(act, stream)
+    out["fouroversix_act_4096_tokens_one_layer"] = {"kernel": "f46_rows_kernel", "launches": 4,
+                                                     "elements": n_act, "bytes_per_elem": 2.5625,
+                                                     "Gelem_s": round(n_act / (ms * 1e-3) / 1e9, 2),
+                                                     **_roof(b_act, ms, peak)}
+    del Xs, bufs
+    # the calibration step over four micro-batches
+    for e in ents:
+        e.dm = torch.zeros_like(e.m)
+        e.dq = torch.zeros_like(e.q)
+    tab = FocusTable(ents)
+    hp = hparams()
+    t_b0 = _timed(lambda: tab.bwd(accumulate=False), stream)
+    t_b1 = _timed(lambda: tab.bwd(accumulate=True), stream)
+    cnt = [100]
+
+    def last():
+        cnt[0] += 1
+        tab.step(cnt[0], hp, F.FOCUS_STEP_ACCUMULATE | F.FOCUS_STEP_WQ_UPDATED)
+    t_st = _timed(last, stream)
+    tot = t_b0 + 2 * t_b1 + t_st
+    out["micro_batch_step_llama8b"] = {
+        "micro_batches": 4, "ms": round(tot, 3), "Gelem_s": round(N * world / (tot * 1e-3) / 1e9, 2),
+        "bwd_first": {"kernel": "pipe_kernel<KIND_BWD>", "bytes_per_weight": 5.5, **_roof(5.5 * N, t_b0, peak)},
+        "bwd_accumulate": {"kernel": "pipe_kernel<KIND_BWD>", "bytes_per_weight": 6.25,
+                           **_roof(6.25 * N, t_b1, peak)},
+        "step_accumulate_wq_updated": {"kernel": "pipe_kernel<KIND_STEP, true>", "bytes_per_weight": 11.25,
+                                       **_roof(11.25 * N, t_st, peak)}}
+    if F.focus_get_error() != 0:
+        raise SystemExit("device status after the next-row measurements is not OK")
+    for e in ents:
+        e.dm = e.dq = None
+    D.barrier()
+    return out
 
 
 def run_e2e(args, ents, N, world, dev):
@@ -445,6 +545,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the next-row measurements")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--reference-seconds", type=float, default=4.0)
     args = ap.parse_args()

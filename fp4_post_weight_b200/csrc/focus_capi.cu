@@ -24,7 +24,7 @@ constexpr int MAX_DEVICES = 64;
 
 struct DeviceInfo {
     int sms = 0;
-    int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_amax = 0, occ_adam = 0;
+    int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_f46 = 0, occ_rows = 0, occ_amax = 0, occ_adam = 0;
 };
 
 std::once_flag g_once[MAX_DEVICES];
@@ -52,12 +52,17 @@ int device_info(DeviceInfo **out) {
                                                       stage_smem_bytes<KIND_STEP>());
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_step_wqu, pipe_kernel<KIND_STEP, true>, CTA_THREADS,
                                                       stage_smem_bytes<KIND_STEP>());
+        cudaFuncSetAttribute(pipe_kernel<KIND_F46>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)stage_smem_bytes<KIND_F46>());
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_f46, pipe_kernel<KIND_F46>, CTA_THREADS,
+                                                      stage_smem_bytes<KIND_F46>());
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows, f46_rows_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_amax, amax_tiles_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_adam, adamw_kernel, THREADS, 0);
     });
     DeviceInfo &d = g_info[dev];
-    if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_step_wqu <= 0 || d.occ_amax <= 0 ||
-        d.occ_adam <= 0)
+    if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_step_wqu <= 0 || d.occ_f46 <= 0 ||
+        d.occ_rows <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0)
         return FOCUS_ERR_CUDA;
     *out = &d;
     return FOCUS_OK;
@@ -146,6 +151,7 @@ int launch_on(const Args &a, cudaStream_t s) {
     if (a.total_tiles == 0 && !a.one_scale_out) return FOCUS_OK;
     const int occ = KIND == KIND_FWD ? di->occ_fwd
                     : KIND == KIND_BWD ? di->occ_bwd
+                    : KIND == KIND_F46 ? di->occ_f46
                     : (WQU ? di->occ_step_wqu : di->occ_step);
     int64_t grid = grid_for(a.total_tiles, di->sms, occ);
     if (grid < 1) grid = 1;   // the pack of an empty tensor still writes its tensor scale
@@ -343,7 +349,7 @@ int focus_adamw_step(float *p, const float *g, float *exp_avg, float *exp_avg_sq
 
 int focus_table_prepare(focus_tensor_desc *d, int n, int purpose, int64_t *total_tiles) {
     if (!d || !total_tiles) return FOCUS_ERR_NULL;
-    if (n < 0 || purpose < 0 || purpose > 2) return FOCUS_ERR_VALUE;
+    if (n < 0 || purpose < 0 || purpose > 3) return FOCUS_ERR_VALUE;
     int64_t tiles = 0, blocks = 0;
     for (int i = 0; i < n; ++i) {
         focus_tensor_desc &e = d[i];
@@ -353,7 +359,9 @@ int focus_table_prepare(focus_tensor_desc *d, int n, int purpose, int64_t *total
         if (!aligned16(e.s2)) return FOCUS_ERR_ALIGN;
         const int64_t nblk = e.out * (e.in / 16);
         if (nblk > 0) {
-            if (!e.W || !e.m || !e.q) return FOCUS_ERR_NULL;
+            if (!e.W) return FOCUS_ERR_NULL;
+            if (purpose != 3 && (!e.m || !e.q)) return FOCUS_ERR_NULL;
+            if (purpose == 3 && !e.codes && !e.Wq) return FOCUS_ERR_NULL;     // FourOverSix writes something
             const void *ptrs[] = {e.W, e.m, e.q, e.Wq, e.codes, e.scales, e.dm, e.dq, e.dWq,
                                   e.m_exp_avg, e.m_exp_avg_sq, e.q_exp_avg, e.q_exp_avg_sq};
             for (const void *p : ptrs)
@@ -455,6 +463,54 @@ int focus_pack_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_ti
     a.n_tensors = n;
     a.total_tiles = total_tiles;
     return launch_on<KIND_FWD>(a, (cudaStream_t)stream);
+}
+
+int focus_fouroversix_weight(const uint16_t *W, int64_t out, int64_t in, float s2, uint8_t *codes, uint8_t *scales,
+                             uint16_t *Wq, focus_stream_t stream) {
+    int rc = check_shape(out, in);
+    if (rc) return rc;
+    if ((rc = check_s2(s2))) return rc;
+    if ((codes == nullptr) != (scales == nullptr)) return FOCUS_ERR_NULL;
+    if (!codes && !Wq) return FOCUS_ERR_NULL;
+    if (out * in == 0) return FOCUS_OK;
+    if (!W) return FOCUS_ERR_NULL;
+    if (!aligned16(W) || !aligned16(codes) || !aligned16(scales) || !aligned16(Wq)) return FOCUS_ERR_ALIGN;
+    Args a{};
+    a.one = one_desc(W, nullptr, Wq, nullptr, nullptr, out, in);
+    a.one.codes = codes;
+    a.one.scales = scales;
+    a.one_s2 = s2;
+    a.n_tensors = 1;
+    a.total_tiles = tiles_of(out, in);
+    return launch_on<KIND_F46>(a, (cudaStream_t)stream);
+}
+
+int focus_fouroversix_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {
+    if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
+    if (n == 0) return FOCUS_OK;
+    if (!descs_dev) return FOCUS_ERR_NULL;
+    if (!aligned16(descs_dev)) return FOCUS_ERR_ALIGN;
+    Args a{};
+    a.table = descs_dev;
+    a.n_tensors = n;
+    a.total_tiles = total_tiles;
+    return launch_on<KIND_F46>(a, (cudaStream_t)stream);
+}
+
+int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
+                          uint8_t *scales, uint16_t *Xq, focus_stream_t stream) {
+    int rc = check_shape(tokens, hidden);
+    if (rc) return rc;
+    if (tokens * hidden == 0) return FOCUS_OK;
+    if (!X || !token_scales || !codes || !scales) return FOCUS_ERR_NULL;
+    if (!aligned16(X) || !aligned16(token_scales) || !aligned16(codes) || !aligned16(scales) || !aligned16(Xq))
+        return FOCUS_ERR_ALIGN;
+    DeviceInfo *di;
+    if ((rc = device_info(&di))) return rc;
+    const int64_t grid = grid_for(tokens, di->sms, di->occ_rows);
+    f46_rows_kernel<<<(unsigned)grid, THREADS, 0, (cudaStream_t)stream>>>(X, tokens, hidden, token_scales, codes,
+                                                                         scales, Xq);
+    return launch_status();
 }
 
 int focus_get_error(focus_stream_t stream) {

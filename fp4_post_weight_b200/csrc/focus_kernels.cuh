@@ -55,7 +55,12 @@ constexpr unsigned FULL = 0xffffffffu;
 // (This header is compiled into exactly one translation unit.)
 __device__ unsigned int g_error_flags = 0;
 
-enum Kind : int { KIND_FWD = 0, KIND_BWD = 1, KIND_STEP = 2 };
+enum Kind : int { KIND_FWD = 0, KIND_BWD = 1, KIND_STEP = 2, KIND_F46 = 3 };
+
+// Which inputs a kind reads besides W: dW' (and the gradient accumulators),
+// and the scale parameters m and q.  FourOverSix reads W alone.
+__host__ __device__ constexpr bool has_grad(int kind) { return kind == KIND_BWD || kind == KIND_STEP; }
+__host__ __device__ constexpr bool has_mq(int kind) { return kind != KIND_F46; }
 
 struct Args {
     const focus_tensor_desc *table;  // device table, or nullptr: use `one`
@@ -134,15 +139,17 @@ __device__ __forceinline__ void load_block_global(const TV &T, const Args &a, Bl
     const uint4 w0 = __ldcs(W), w1 = __ldcs(W + 1);
     B.w[0] = w0.x; B.w[1] = w0.y; B.w[2] = w0.z; B.w[3] = w0.w;
     B.w[4] = w1.x; B.w[5] = w1.y; B.w[6] = w1.z; B.w[7] = w1.w;
-    if (KIND != KIND_FWD) {
+    if (has_grad(KIND)) {
         const uint4 *G = reinterpret_cast<const uint4 *>(T.d.dWq) + 2u * blk;
         const uint4 g0 = __ldcs(G), g1 = __ldcs(G + 1);
         B.g[0] = g0.x; B.g[1] = g0.y; B.g[2] = g0.z; B.g[3] = g0.w;
         B.g[4] = g1.x; B.g[5] = g1.y; B.g[6] = g1.z; B.g[7] = g1.w;
     }
-    B.m = T.d.m[blk];
-    const float2 q = reinterpret_cast<const float2 *>(T.d.q)[blk];
-    B.q[0] = q.x; B.q[1] = q.y;
+    if (has_mq(KIND)) {
+        B.m = T.d.m[blk];
+        const float2 q = reinterpret_cast<const float2 *>(T.d.q)[blk];
+        B.q[0] = q.x; B.q[1] = q.y;
+    }
     if (KIND == KIND_STEP) {
         B.mv1 = T.d.m_exp_avg[blk];
         B.mv2 = T.d.m_exp_avg_sq[blk];
@@ -150,7 +157,7 @@ __device__ __forceinline__ void load_block_global(const TV &T, const Args &a, Bl
         const float2 v2 = reinterpret_cast<const float2 *>(T.d.q_exp_avg_sq)[blk];
         B.qv1[0] = v1.x; B.qv1[1] = v1.y; B.qv2[0] = v2.x; B.qv2[1] = v2.y;
     }
-    if (KIND != KIND_FWD && a.accumulate) {
+    if (has_grad(KIND) && a.accumulate) {
         B.gm_in = T.d.dm[blk];
         const float2 gq = reinterpret_cast<const float2 *>(T.d.dq)[blk];
         B.gq_in[0] = gq.x; B.gq_in[1] = gq.y;
@@ -222,6 +229,109 @@ __device__ __forceinline__ void store_wq_from_codes(const TV &T, uint32_t blk, c
     }
 }
 
+// ---------------------------------------------------------------------------
+// FourOverSix round to nearest (model card, section "Calibration": each
+// 16-element block's scale maps the block maximum to 6 or to 4, whichever has
+// the lower error; section "Perplexity": round-to-nearest FourOverSix weights)
+// ---------------------------------------------------------------------------
+
+// One target T of a block: x = fl(A / fl(T*s)), scale 1 when x == 0,
+// S = e4m3(clamp(x, 2^-6, 448)), D = fl(S*s), c = E2M1(clamp(fl(w/D), -6, 6)).
+// Returns the block's squared error in binary32: d = fl(w - (c*S)*s) in one
+// rounding, the even and the odd elements summed apart by fused multiply-adds
+// (one packed lane each, in element order), then added.
+__device__ __forceinline__ float f46_target(const uint32_t *w, float A, float s, float Ts, uint32_t &sb,
+                                            uint32_t codes[2]) {
+    float x = __fdiv_rn(A, Ts);
+    x = (x == 0.0f) ? 1.0f : x;
+    x = fminf(fmaxf(x, 0x1p-6f), 448.0f);
+    sb = e4m3_byte(x);
+    const float S = e4m3_normal_f32(sb);
+    const uint16_t S_h = (uint16_t)e4m3_normal_f16_bits(sb);
+    const float D = __fmul_rn(S, s);
+    const bool fast = D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f;
+    const float nr = fast ? -rcp_rn(D) : 0.0f;
+    const uint64_t D2 = f2_pack(D, D), nr2 = f2_pack(nr, nr), ns2 = f2_pack(-s, -s);
+    uint64_t E2 = 0ull;                         // (even, odd) partial sums
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        uint32_t code = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t wv = w[4 * k + j];
+            const uint64_t y2 = fast ? div_by_f2(bf16x2_neg_f2(wv), D2, nr2)
+                                     : f2_pack(__fdiv_rn(bf16_lo(wv), D), __fdiv_rn(bf16_hi(wv), D));
+            const uint32_t byte = e2m1_pair(f2_lo(y2), f2_hi(y2));
+            code |= byte << (8 * j);
+            const uint32_t h2 = e2m1_pair_f16x2(byte);
+            const uint64_t cs2 = f2_pack(mul_f16_exact(lo16(h2), S_h), mul_f16_exact(hi16(h2), S_h));
+            const uint64_t d2 = f2_fma(cs2, ns2, bf16x2_f2(wv));
+            E2 = f2_fma(d2, d2, E2);
+        }
+        codes[k] = code;
+    }
+    return __fadd_rn(f2_lo(E2), f2_hi(E2));
+}
+
+// FourOverSix of one block with scale s > 0 (den6 = fl(6*s), den4 = fl(4*s)):
+// the chosen scale byte and codes; the target 4 only when its error is lower.
+__device__ __forceinline__ bool f46_block(const uint32_t *w, float s, float den6, float den4, uint32_t &sb,
+                                          uint32_t codes[2]) {
+    uint32_t am = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) am = __vmaxu2(am, w[j] & 0x7fff7fffu);
+    const float A = __uint_as_float(max(am & 0xffffu, am >> 16) << 16);
+    uint32_t sb4, c4[2];
+    const float e6 = f46_target(w, A, s, den6, sb, codes);
+    const float e4 = f46_target(w, A, s, den4, sb4, c4);
+    const bool four = e4 < e6;
+    if (four) { sb = sb4; codes[0] = c4[0]; codes[1] = c4[1]; }
+    return four;
+}
+
+// The bf16 bits of w' = bf16(fl(fl(c*S)*s)) for the 16 codes of a block, as
+// four 16-byte words.
+__device__ __forceinline__ void wq_words(const uint32_t codes[2], uint32_t sbyte, float s, uint4 out[2]) {
+    const uint16_t S_h = (uint16_t)e4m3_normal_f16_bits(sbyte);
+    const uint64_t s_2 = f2_pack(s, s);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t h2 = e2m1_pair_f16x2((codes[k] >> (8 * j)) & 0xffu);
+            const uint64_t p = f2_mul(f2_pack(mul_f16_exact(lo16(h2), S_h), mul_f16_exact(hi16(h2), S_h)), s_2);
+            o[j] = pack_bf16x2(f2_lo(p), f2_hi(p));
+        }
+        out[k] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// FourOverSix of one block of a weight tensor (tensor scale s2 = T.s2).
+template <class TV>
+__device__ __forceinline__ void compute_block_f46(const TV &T, Block &B) {
+    uint32_t am = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) am = __vmaxu2(am, B.w[j] & 0x7fff7fffu);
+    const bool bad = B.valid && max(am & 0xffffu, am >> 16) >= 0x7f80u;
+    if (B.valid) {
+        const float s = T.s2;
+        uint32_t sb, codes[2];
+        f46_block(B.w, s, __fmul_rn(6.0f, s), __fmul_rn(4.0f, s), sb, codes);
+        if (T.d.codes) {
+            reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = make_uint2(codes[0], codes[1]);
+            T.d.scales[B.blk] = (uint8_t)sb;
+        }
+        if (T.d.Wq) {
+            uint4 o[2];
+            wq_words(codes, sb, s, o);
+            __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + 2u * B.blk, o[0]);
+            __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + 2u * B.blk + 1u, o[1]);
+        }
+    }
+    if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_error_flags, 1u);
+}
+
 // The forward, the straight-through gradients and the AdamW update of one block.
 // WQU (step only, FOCUS_STEP_WQ_UPDATED): W' is that of the updated m and q,
 // a compile-time choice so that the other step variants keep its registers.
@@ -230,6 +340,10 @@ __device__ __forceinline__ void store_wq_from_codes(const TV &T, uint32_t blk, c
 // descriptor's pointers are read where used instead of held in registers.
 template <int KIND, bool WQU, class TV>
 __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block &B) {
+    if constexpr (KIND == KIND_F46) {
+        compute_block_f46(T, B);
+        return;
+    }
     // A_b = max |w| over the block: max of the bf16 magnitude bit patterns (a NaN
     // or an infinity sorts above every finite magnitude, which is how it is found)
     uint32_t am = 0u;
@@ -292,7 +406,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
             __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + (2u * B.blk + (uint32_t)k), o);
         }
         sq[k] = 0.0f;
-        if (KIND != KIND_FWD) {
+        if (has_grad(KIND)) {
             // straight-through sums, element by element: g*t with t = c - y inside the
             // clamp and c outside (c - y is exact near the code, so the sum is well
             // conditioned), and g*y inside the clamp, per sub-block
@@ -318,7 +432,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
         if (T.d.scales) T.d.scales[B.blk] = (uint8_t)sbyte;
     }
 
-    if (KIND != KIND_FWD) {
+    if (has_grad(KIND)) {
         // dL/dm = inS*(A/6)*sum g*t;  dL/dq_k = -(1 - sigma_k)*S*s2*sum_k g*y_in
         float gm = inS ? (A * (1.0f / 6.0f)) * (f2_lo(sm2) + f2_hi(sm2)) : 0.0f;
         float gq0 = -((((1.0f - sig[0]) * S) * T.s2) * sq[0]);
@@ -372,13 +486,14 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
 
 template <int KIND>
 struct Layout {
-    static constexpr bool G_ = KIND != KIND_FWD;         // dW' and the gradient accumulators
+    static constexpr bool G_ = has_grad(KIND);           // dW' and the gradient accumulators
+    static constexpr bool MQ = has_mq(KIND);             // m and q
     static constexpr bool ST = KIND == KIND_STEP;        // AdamW moments
     static constexpr uint32_t W = 0;
     static constexpr uint32_t G = W + TILE_BLOCKS * 32;
     static constexpr uint32_t M = G + (G_ ? TILE_BLOCKS * 32 : 0);
-    static constexpr uint32_t Q = M + TILE_BLOCKS * 4;
-    static constexpr uint32_t MV1 = Q + TILE_BLOCKS * 8;
+    static constexpr uint32_t Q = M + (MQ ? TILE_BLOCKS * 4 : 0);
+    static constexpr uint32_t MV1 = Q + (MQ ? TILE_BLOCKS * 8 : 0);
     static constexpr uint32_t MV2 = MV1 + (ST ? TILE_BLOCKS * 4 : 0);
     static constexpr uint32_t QV1 = MV2 + (ST ? TILE_BLOCKS * 4 : 0);
     static constexpr uint32_t QV2 = QV1 + (ST ? TILE_BLOCKS * 8 : 0);
@@ -395,6 +510,7 @@ template <int KIND> struct Depth;
 template <> struct Depth<KIND_FWD> { static constexpr int STAGES = 6, MIN_CTAS = 3; };
 template <> struct Depth<KIND_BWD> { static constexpr int STAGES = 4, MIN_CTAS = 2; };
 template <> struct Depth<KIND_STEP> { static constexpr int STAGES = 2, MIN_CTAS = 3; };
+template <> struct Depth<KIND_F46> { static constexpr int STAGES = 8, MIN_CTAS = 3; };
 
 template <int KIND>
 constexpr uint32_t stage_smem_bytes() { return Depth<KIND>::STAGES * Layout<KIND>::BYTES; }
@@ -427,15 +543,17 @@ __device__ __forceinline__ void load_block_smem(const Args &a, const unsigned ch
     const uint4 w0 = W[0], w1 = W[1];
     B.w[0] = w0.x; B.w[1] = w0.y; B.w[2] = w0.z; B.w[3] = w0.w;
     B.w[4] = w1.x; B.w[5] = w1.y; B.w[6] = w1.z; B.w[7] = w1.w;
-    if (KIND != KIND_FWD) {
+    if (has_grad(KIND)) {
         const uint4 *G = reinterpret_cast<const uint4 *>(stage + L::G) + 2u * lb;
         const uint4 g0 = G[0], g1 = G[1];
         B.g[0] = g0.x; B.g[1] = g0.y; B.g[2] = g0.z; B.g[3] = g0.w;
         B.g[4] = g1.x; B.g[5] = g1.y; B.g[6] = g1.z; B.g[7] = g1.w;
     }
-    B.m = reinterpret_cast<const float *>(stage + L::M)[lb];
-    const float2 q = reinterpret_cast<const float2 *>(stage + L::Q)[lb];
-    B.q[0] = q.x; B.q[1] = q.y;
+    if (has_mq(KIND)) {
+        B.m = reinterpret_cast<const float *>(stage + L::M)[lb];
+        const float2 q = reinterpret_cast<const float2 *>(stage + L::Q)[lb];
+        B.q[0] = q.x; B.q[1] = q.y;
+    }
     if (KIND == KIND_STEP) {
         B.mv1 = reinterpret_cast<const float *>(stage + L::MV1)[lb];
         B.mv2 = reinterpret_cast<const float *>(stage + L::MV2)[lb];
@@ -443,7 +561,7 @@ __device__ __forceinline__ void load_block_smem(const Args &a, const unsigned ch
         const float2 v2 = reinterpret_cast<const float2 *>(stage + L::QV2)[lb];
         B.qv1[0] = v1.x; B.qv1[1] = v1.y; B.qv2[0] = v2.x; B.qv2[1] = v2.y;
     }
-    if (KIND != KIND_FWD && a.accumulate) {
+    if (has_grad(KIND) && a.accumulate) {
         B.gm_in = reinterpret_cast<const float *>(stage + L::GM)[lb];
         const float2 gq = reinterpret_cast<const float2 *>(stage + L::GQ)[lb];
         B.gq_in[0] = gq.x; B.gq_in[1] = gq.y;
@@ -494,8 +612,8 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
         const uint32_t nb = found ? (uint32_t)(left < TILE_BLOCKS ? left : TILE_BLOCKS) : 0u;
         // a descriptor without a pointer this kernel needs (a table prepared for
         // another purpose) is skipped and reported, never dereferenced
-        bool complete = T.d.W != nullptr && T.d.m != nullptr && T.d.q != nullptr;
-        if (KIND != KIND_FWD) complete = complete && T.d.dWq != nullptr;
+        bool complete = T.d.W != nullptr && (!has_mq(KIND) || (T.d.m != nullptr && T.d.q != nullptr));
+        if (has_grad(KIND)) complete = complete && T.d.dWq != nullptr;
         if (KIND == KIND_BWD || a.accumulate || a.write_grad) complete = complete && T.d.dm != nullptr && T.d.dq != nullptr;
         if (KIND == KIND_STEP)
             complete = complete && T.d.m_exp_avg && T.d.m_exp_avg_sq && T.d.q_exp_avg && T.d.q_exp_avg_sq;
@@ -518,18 +636,20 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
             const uint32_t f = first;
             mbar_arrive_expect_tx(bar, L::tx_bytes(a.accumulate != 0));
             bulk_g2s(smem_u32(stage + L::W), reinterpret_cast<const uint4 *>(T.d.W) + 2u * f, TILE_BLOCKS * 32, bar);
-            if (KIND != KIND_FWD)
+            if (has_grad(KIND))
                 bulk_g2s(smem_u32(stage + L::G), reinterpret_cast<const uint4 *>(T.d.dWq) + 2u * f, TILE_BLOCKS * 32,
                          bar);
-            bulk_g2s(smem_u32(stage + L::M), T.d.m + f, TILE_BLOCKS * 4, bar);
-            bulk_g2s(smem_u32(stage + L::Q), T.d.q + 2u * f, TILE_BLOCKS * 8, bar);
+            if (has_mq(KIND)) {
+                bulk_g2s(smem_u32(stage + L::M), T.d.m + f, TILE_BLOCKS * 4, bar);
+                bulk_g2s(smem_u32(stage + L::Q), T.d.q + 2u * f, TILE_BLOCKS * 8, bar);
+            }
             if (KIND == KIND_STEP) {
                 bulk_g2s(smem_u32(stage + L::MV1), T.d.m_exp_avg + f, TILE_BLOCKS * 4, bar);
                 bulk_g2s(smem_u32(stage + L::MV2), T.d.m_exp_avg_sq + f, TILE_BLOCKS * 4, bar);
                 bulk_g2s(smem_u32(stage + L::QV1), T.d.q_exp_avg + 2u * f, TILE_BLOCKS * 8, bar);
                 bulk_g2s(smem_u32(stage + L::QV2), T.d.q_exp_avg_sq + 2u * f, TILE_BLOCKS * 8, bar);
             }
-            if (KIND != KIND_FWD && a.accumulate) {
+            if (has_grad(KIND) && a.accumulate) {
                 bulk_g2s(smem_u32(stage + L::GM), T.d.dm + f, TILE_BLOCKS * 4, bar);
                 bulk_g2s(smem_u32(stage + L::GQ), T.d.dq + 2u * f, TILE_BLOCKS * 8, bar);
             }
@@ -672,6 +792,65 @@ __global__ void __launch_bounds__(THREADS) s2_finish_kernel(const Args a, const 
             const float s2 = __fdiv_rn(A, 2688.0f);
             if (a.table) *d.s2 = s2;
             else *one_out = s2;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// FourOverSix with one scale per token (model card, section "Calibration",
+// activation bullet): s_t = fl(max_row |x| / 2688), then every block of the
+// row as for the weights.  One CTA per row and loop: the first pass reads the
+// row from HBM for its maximum, the second reads it again (from L2) and
+// writes codes, scales and, when asked, the dequantized row.  A row whose
+// maximum is 0 has s_t = 0: block scales 0x38 (1.0), codes 0, values 0.
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(THREADS) f46_rows_kernel(const uint16_t *__restrict__ X, int64_t rows, int64_t cols,
+                                                           float *__restrict__ row_scales, uint8_t *__restrict__ codes,
+                                                           uint8_t *__restrict__ scales, uint16_t *__restrict__ Xq) {
+    __shared__ uint32_t red[THREADS / 32];
+    const int64_t chunks = cols / 8;          // 16-byte words of a row
+    const int64_t nb = cols / 16;
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(X + r * cols);
+        uint32_t mx = 0u;
+        for (int64_t c = threadIdx.x; c < chunks; c += THREADS) {
+            const uint4 v = xr[c];
+            const uint32_t m2 = __vmaxu2(__vmaxu2(v.x & 0x7fff7fffu, v.y & 0x7fff7fffu),
+                                         __vmaxu2(v.z & 0x7fff7fffu, v.w & 0x7fff7fffu));
+            mx = max(mx, max(m2 & 0xffffu, m2 >> 16));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(FULL, mx, o));
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+        __syncthreads();
+        uint32_t amax = 0u;
+#pragma unroll
+        for (int w = 0; w < THREADS / 32; ++w) amax = max(amax, red[w]);
+        __syncthreads();                       // red is rewritten by the next row
+        if (amax >= 0x7f80u) {                 // a non-finite value: flag it, write nothing of the row
+            if (threadIdx.x == 0) atomicOr(&g_error_flags, 1u);
+            continue;
+        }
+        const float s = __fdiv_rn(__uint_as_float(amax << 16), 2688.0f);
+        if (threadIdx.x == 0) row_scales[r] = s;
+        const float den6 = __fmul_rn(6.0f, s), den4 = __fmul_rn(4.0f, s);
+        for (int64_t b = threadIdx.x; b < nb; b += THREADS) {
+            const int64_t blk = r * nb + b;
+            uint32_t sb = 0x38u, cw[2] = {0u, 0u};
+            uint4 o[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+            if (s != 0.0f) {
+                const uint4 v0 = xr[2 * b], v1 = xr[2 * b + 1];
+                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                f46_block(w, s, den6, den4, sb, cw);
+                if (Xq) wq_words(cw, sb, s, o);
+            }
+            reinterpret_cast<uint2 *>(codes)[blk] = make_uint2(cw[0], cw[1]);
+            scales[blk] = (uint8_t)sb;
+            if (Xq) {
+                __stcs(reinterpret_cast<uint4 *>(Xq) + 2 * blk, o[0]);
+                __stcs(reinterpret_cast<uint4 *>(Xq) + 2 * blk + 1, o[1]);
+            }
         }
     }
 }

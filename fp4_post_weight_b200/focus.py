@@ -63,6 +63,9 @@ _SIGS = {
     "focus_pack_multi": ([_P, _I, _I64, _P], _I),
     "focus_fwd_multi": ([_P, _I, _I64, _P], _I),
     "focus_ste_bwd_multi": ([_P, _I, _I64, _I, _P], _I),
+    "focus_fouroversix_weight": ([_P, _I64, _I64, _F, _P, _P, _P, _P], _I),
+    "focus_fouroversix_multi": ([_P, _I, _I64, _P], _I),
+    "focus_fouroversix_act": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _I),
     "focus_get_error": ([_P], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -221,6 +224,29 @@ def focus_ste_bwd_multi(table_dev, n: int, total_tiles: int, accumulate: bool = 
 
 def focus_pack_multi(table_dev, n: int, total_tiles: int, stream=None):
     _check(_lib.focus_pack_multi(_ptr(table_dev), int(n), int(total_tiles), _stream(stream)), "focus_pack_multi")
+
+
+def focus_fouroversix_weight(W, s2: float, codes, scales, Wq=None, stream=None, out=None, in_=None):
+    """FourOverSix round to nearest of a weight with tensor scale s2: codes
+    [out, in/2] u8, scales [out, in/16] u8 (both or neither), Wq bf16 (optional)."""
+    _bf16(W, "W"); _bf16(Wq, "Wq")
+    o, i = _shape(W, out, in_)
+    _check(_lib.focus_fouroversix_weight(_ptr(W), o, i, float(s2), _ptr(codes), _ptr(scales), _ptr(Wq),
+                                         _stream(stream)), "focus_fouroversix_weight")
+
+
+def focus_fouroversix_multi(table_dev, n: int, total_tiles: int, stream=None):
+    _check(_lib.focus_fouroversix_multi(_ptr(table_dev), int(n), int(total_tiles), _stream(stream)),
+           "focus_fouroversix_multi")
+
+
+def focus_fouroversix_act(X, token_scales, codes, scales, Xq=None, stream=None, tokens=None, hidden=None):
+    """FourOverSix with one scale per token: token_scales [tokens] f32, codes
+    [tokens, hidden/2] u8, scales [tokens, hidden/16] u8, Xq bf16 (optional)."""
+    _bf16(X, "X"); _bf16(Xq, "Xq"); _f32(token_scales, "token_scales")
+    t, h = _shape(X, tokens, hidden)
+    _check(_lib.focus_fouroversix_act(_ptr(X), t, h, _ptr(token_scales), _ptr(codes), _ptr(scales), _ptr(Xq),
+                                      _stream(stream)), "focus_fouroversix_act")
 
 
 def focus_get_error(stream=None) -> int:

@@ -19,6 +19,7 @@ _FIELDS = ("W", "dWq", "Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg",
 PURPOSE_FORWARD = 0
 PURPOSE_STEP = 1
 PURPOSE_BACKWARD = 2
+PURPOSE_FOUROVERSIX = 3
 
 
 @dataclass
@@ -78,6 +79,9 @@ class FocusTable:
 
     def bwd(self, accumulate: bool = False, stream=None):
         F.focus_ste_bwd_multi(self.dev, self.n, self.total_tiles, accumulate, stream)
+
+    def fouroversix(self, stream=None):
+        F.focus_fouroversix_multi(self.dev, self.n, self.total_tiles, stream)
 
 
 def hparams(lr_m=5e-3, lr_q=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0) -> F.focus_hparams:

@@ -219,8 +219,9 @@ typedef struct focus_hparams {
 
 /* Checks every entry (pointers, alignment, shapes, which inputs are present
  * for `purpose`: 0 = s2/forward/pack, 1 = also focus_step_fused (dWq and the
- * four moments), 2 = also focus_ste_bwd_multi (dWq, dm, dq)) and fills
- * block_begin and tile_begin.  Host memory in, host memory out.
+ * four moments), 2 = also focus_ste_bwd_multi (dWq, dm, dq), 3 = s2 and
+ * FourOverSix only (W and s2; m and q may be NULL; codes+scales or Wq)) and
+ * fills block_begin and tile_begin.  Host memory in, host memory out.
  * *total_tiles receives the number of work tiles, passed to the calls below.
  * A device-resident table cannot be checked again at call time: a kernel that
  * meets an entry lacking a pointer it needs skips that entry and sets the
@@ -262,6 +263,47 @@ int focus_ste_bwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64
  * tensor scale, which the caller exports). */
 int focus_pack_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
                      focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * FourOverSix round to nearest: plain NVFP4 (E2M1 codes, one E4M3 scale per
+ * 16 elements, an FP32 scale per tensor or per token) in which every block's
+ * scale maps the block maximum to 6 or to 4, whichever gives the lower
+ * squared error.  Model card "FOCUS NVFP4 scales for Llama-3.2-1B-Instruct",
+ * section "Calibration" (activation bullet: one scale per token) and section
+ * "Perplexity" (round-to-nearest FourOverSix weights, the reference row);
+ * "Llama-3.1-8B-Instruct FlipQuant MixFP4 maps", section "What this is".
+ * Per block, for the targets T = 6 and T = 4 (s the tensor or token scale):
+ *   x_T = fl(A_b / fl(T*s));  x_T == 0 -> 1;  S_T = e4m3_rne(clamp(x_T, 2^-6, 448))
+ *   c_i = E2M1_rne(clamp(fl(w_i / fl(S_T*s)), -6, 6))
+ *   err_T = fl(E_even + E_odd), E over the even / odd elements in index
+ *           order, E <- fma(d_i, d_i, E), d_i = fma(-(c_i*S_T), s, w_i)
+ * The target 4 is taken when err_4 < err_6 (a tie keeps 6); the dequantized
+ * value is bf16(fl(fl(c_i*S)*s)).  Outputs use the focus_pack_nvfp4 layout
+ * (codes [rows][cols/2], element 2j in the low nibble; scales [rows][cols/16]).
+ * ------------------------------------------------------------------------- */
+
+/* Weights with the tensor scale s2 (by value: finite and > 0, else
+ * FOCUS_ERR_VALUE).  W [out, in] bf16, device; codes/scales (both or
+ * neither) and Wq [out, in] bf16 (nullable) are device outputs; at least one
+ * of codes or Wq is required.  Non-finite weights set the device flag. */
+int focus_fouroversix_weight(const uint16_t *W, int64_t out, int64_t in, float s2, uint8_t *codes,
+                             uint8_t *scales, uint16_t *Wq, focus_stream_t stream);
+
+/* The same over every entry of a table (purpose 3, or any purpose whose
+ * entries carry codes+scales or Wq) in one launch: desc.W, desc.s2 (device,
+ * as focus_s2_multi writes it), desc.codes/scales and desc.Wq. */
+int focus_fouroversix_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
+                            focus_stream_t stream);
+
+/* Activations with one scale per token: X [tokens, hidden] bf16, device
+ * (hidden % 16 == 0); token_scales [tokens] float, device, receives
+ * s_t = fl(max_row |x| / 2688); codes [tokens][hidden/2], scales
+ * [tokens][hidden/16] and Xq [tokens, hidden] bf16 (nullable) are device
+ * outputs.  A row whose maximum is 0 gets s_t = 0, scale bytes 0x38, codes 0
+ * and values 0.  A row holding a non-finite value sets the device flag and
+ * its outputs are left unwritten.  One launch, X read once from HBM. */
+int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales,
+                          uint8_t *codes, uint8_t *scales, uint16_t *Xq, focus_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Synchronizes `stream`, then reports and clears the sticky device flag:

@@ -252,3 +252,21 @@ def bits(t: torch.Tensor):
 def from_bits(a, device="cpu") -> torch.Tensor:
     import numpy as np
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def activations(tokens: int, hidden: int, device, seed: int = 5, outlier_channels: float = 0.005,
+                outlier_factor: float = 30.0, zero_tokens: int = 1) -> torch.Tensor:
+    """Activations X [tokens, hidden] bf16 with the structure of a decoder's
+    linear inputs: N(0, 1) per element, a fixed set of outlier channels
+    (``outlier_channels`` of the columns, scaled by ``outlier_factor``, as
+    hidden states of large language models show) and ``zero_tokens`` all-zero
+    rows at the end (padding).  The card's calibration runs micro-batches of
+    8 windows of 512 tokens (4096 tokens per forward pass)."""
+    g = _gen(seed, device)
+    X = torch.randn((tokens, hidden), generator=g, device=device, dtype=torch.float32)
+    n_out = max(1, int(round(outlier_channels * hidden)))
+    cols = torch.randperm(hidden, generator=g, device=device)[:n_out]
+    X[:, cols] *= outlier_factor
+    if zero_tokens:
+        X[tokens - zero_tokens:] = 0.0
+    return X.to(torch.bfloat16)

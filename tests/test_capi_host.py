@@ -99,7 +99,7 @@ def test_table_prepare_on_host(F):
         F.focus_table_prepare(descs, 1)
     assert e.value.status == 1
     assert F.focus_table_prepare(descs, 0) == tiles
-    # a table backward needs dW', dm and dq; purposes beyond 2 do not exist
+    # a table backward needs dW', dm and dq; purposes beyond 3 do not exist
     with pytest.raises(F.FocusError) as e:
         F.focus_table_prepare(descs, 2)
     assert e.value.status == 1
@@ -108,7 +108,7 @@ def test_table_prepare_on_host(F):
         descs[i].dq = P + 65536 * (i + 1) + 4096
     assert F.focus_table_prepare(descs, 2) == tiles
     with pytest.raises(F.FocusError) as e:
-        F.focus_table_prepare(descs, 3)
+        F.focus_table_prepare(descs, 4)
     assert e.value.status == 4
     descs[2].in_ = 40
     with pytest.raises(F.FocusError) as e:
@@ -138,3 +138,43 @@ def test_step_hparam_checks(F):
     assert F.raw_call("focus_step_fused", P, 1, 1, None, 1, 0, None) == 1
     bad = F.focus_hparams(5e-3, -1e-3, 0.9, 0.999, 1e-8, 0.0)
     assert F.raw_call("focus_step_fused", P, 1, 1, ctypes.byref(bad), 1, 0, None) == 4
+
+
+def test_fouroversix_checks(F):
+    f32 = ctypes.c_float
+    # weights: shape, tensor scale, outputs (codes and scales together; codes or Wq), alignment
+    assert F.raw_call("focus_fouroversix_weight", P, 4, 24, f32(1.0), P, P, None, None) == 2
+    assert F.raw_call("focus_fouroversix_weight", P, 4, 16, f32(0.0), P, P, None, None) == 4
+    assert F.raw_call("focus_fouroversix_weight", P, 4, 16, f32(float("nan")), P, P, None, None) == 4
+    assert F.raw_call("focus_fouroversix_weight", P, 4, 16, f32(1.0), P, None, None, None) == 1
+    assert F.raw_call("focus_fouroversix_weight", P, 4, 16, f32(1.0), None, None, None, None) == 1
+    assert F.raw_call("focus_fouroversix_weight", None, 4, 16, f32(1.0), P, P, None, None) == 1
+    assert F.raw_call("focus_fouroversix_weight", U, 4, 16, f32(1.0), P, P, None, None) == 3
+    assert F.raw_call("focus_fouroversix_weight", P, 4, 16, f32(1.0), None, None, U, None) == 3
+    assert F.raw_call("focus_fouroversix_weight", P, 0, 16, f32(1.0), P, P, None, None) == 0   # empty
+    assert F.raw_call("focus_fouroversix_multi", P, -1, 1, None) == 4
+    assert F.raw_call("focus_fouroversix_multi", None, 1, 1, None) == 1
+    assert F.raw_call("focus_fouroversix_multi", U, 1, 1, None) == 3
+    # activations: per-token scales, codes and scales are required
+    assert F.raw_call("focus_fouroversix_act", P, 4, 40, P, P, P, None, None) == 2
+    assert F.raw_call("focus_fouroversix_act", P, 4, 32, None, P, P, None, None) == 1
+    assert F.raw_call("focus_fouroversix_act", P, 4, 32, P, None, P, None, None) == 1
+    assert F.raw_call("focus_fouroversix_act", P, 4, 32, P, P, P, U, None) == 3
+    assert F.raw_call("focus_fouroversix_act", P, 0, 32, P, P, P, None, None) == 0             # no tokens
+
+
+def test_table_prepare_fouroversix(F):
+    descs = (F.focus_tensor_desc * 2)()
+    for i, (o, k) in enumerate([(8, 64), (3, 32)]):
+        d = descs[i]
+        d.W = P + 4096 * i; d.s2 = P + 65536 + 16 * i
+        d.out, d.in_ = o, k
+    with pytest.raises(F.FocusError) as e:          # nothing to write
+        F.focus_table_prepare(descs, 3)
+    assert e.value.status == 1
+    for i in range(2):
+        descs[i].Wq = P + 131072 + 4096 * i
+    assert F.focus_table_prepare(descs, 3) == 2     # m and q are not needed
+    with pytest.raises(F.FocusError) as e:          # the FOCUS purposes still need m and q
+        F.focus_table_prepare(descs, 0)
+    assert e.value.status == 1

@@ -1,0 +1,149 @@
+"""GPU parity of the FourOverSix quantizer against the oracle, bit for bit:
+weights with a tensor scale (single tensor and multi-tensor table, shapes
+spanning several 4096-weight tiles and ragged tails), activations with one
+scale per token (rows of one and of several blocks per thread, a zero row),
+the hand-derived worked example, and the non-finite flag.  The E4M3 and E2M1
+decisions and the target choice are all taken in binary32 on both sides, so
+every output must match exactly."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.parity import host, host_bits, unpack_codes
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 16), (3, 48), (2, 4096), (37, 1040), (7, 4112), (128, 2048), (257, 160)]
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+@pytest.fixture(scope="module")
+def F():
+    from fp4_post_weight_b200 import focus
+    return focus
+
+
+def weights(shape, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    W = synth.add_outliers(synth.normal_bf16(shape, 0.02, g, "cuda"), 2e-3, 20.0, g)
+    if W.numel() >= 64:
+        W.view(-1)[:16] = 0
+    return W
+
+
+def outputs(o, i, dev="cuda"):
+    return (torch.empty((o, i // 2), dtype=torch.uint8, device=dev),
+            torch.empty((o, i // 16), dtype=torch.uint8, device=dev),
+            torch.empty((o, i), dtype=torch.bfloat16, device=dev))
+
+
+def assert_same(ref, codes, scales, Xq):
+    np.testing.assert_array_equal(host(scales), ref.scales)
+    np.testing.assert_array_equal(unpack_codes(host(codes)), ref.codes)
+    np.testing.assert_array_equal(host_bits(Xq), ref.Xq)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_weight(F, shape):
+    W = weights(shape, 20 + shape[0])
+    Wb = host_bits(W)
+    s2 = oracle.s2(Wb)
+    codes, scales, Wq = outputs(*shape)
+    F.focus_fouroversix_weight(W, float(s2), codes, scales, Wq)
+    assert F.focus_get_error() == 0
+    ref = oracle.fouroversix(Wb, s2)
+    assert_same(ref, codes, scales, Wq)
+    if W.numel() >= 4096:
+        assert 0 < ref.four.mean() < 1
+
+
+def test_weight_outputs_optional(F):
+    W = weights((64, 512), 3)
+    Wb = host_bits(W)
+    s2 = oracle.s2(Wb)
+    ref = oracle.fouroversix(Wb, s2)
+    codes, scales, Wq = outputs(64, 512)
+    F.focus_fouroversix_weight(W, float(s2), codes, scales, None)
+    Wq.fill_(7.0)
+    F.focus_fouroversix_weight(W, float(s2), None, None, Wq)
+    assert F.focus_get_error() == 0
+    np.testing.assert_array_equal(host(scales), ref.scales)
+    np.testing.assert_array_equal(unpack_codes(host(codes)), ref.codes)
+    np.testing.assert_array_equal(host_bits(Wq), ref.Xq)
+
+
+def test_weight_table(F):
+    from fp4_post_weight_b200.table import Entry, FocusTable, PURPOSE_FOUROVERSIX
+    shapes = SHAPES + [(0, 32)]
+    ents = []
+    for j, sh in enumerate(shapes):
+        W = weights(sh, 40 + j) if sh[0] * sh[1] else torch.zeros(sh, dtype=torch.bfloat16, device="cuda")
+        c, s, q = outputs(*sh)
+        ents.append(Entry(W=W, m=None, q=None, s2=torch.zeros(1, device="cuda"), codes=c, scales=s, Wq=q))
+    tab = FocusTable(ents, PURPOSE_FOUROVERSIX)
+    tab.s2()
+    tab.fouroversix()
+    assert F.focus_get_error() == 0
+    for e in ents:
+        if e.W.numel() == 0:
+            continue
+        Wb = host_bits(e.W)
+        s2 = oracle.s2(Wb)
+        assert host(e.s2)[0] == s2
+        assert_same(oracle.fouroversix(Wb, s2), e.codes, e.scales, e.Wq)
+
+
+@pytest.mark.parametrize("tokens,hidden", [(1, 16), (5, 48), (33, 4096), (17, 14336), (300, 1040), (3, 64)])
+def test_activations(F, tokens, hidden):
+    X = synth.activations(tokens, hidden, "cuda", seed=tokens + hidden, zero_tokens=1 if tokens > 2 else 0)
+    ts = torch.full((tokens,), -1.0, device="cuda")
+    codes, scales, Xq = outputs(tokens, hidden)
+    F.focus_fouroversix_act(X, ts, codes, scales, Xq)
+    assert F.focus_get_error() == 0
+    ref = oracle.fouroversix(host_bits(X))
+    np.testing.assert_array_equal(host(ts), ref.row_scales)
+    assert_same(ref, codes, scales, Xq)
+    if tokens > 2:
+        assert host(ts)[-1] == 0 and np.all(host(scales)[-1] == 0x38)
+
+
+def test_worked_example_on_gpu(F):
+    gold = json.load(open(os.path.join(HERE, "golden", "fouroversix_worked.json")))
+    u = gold["unit"]
+    W = torch.tensor(np.array(gold["weights"]["W_over_u"]) * u, dtype=torch.float32).to(torch.bfloat16).cuda()
+    codes, scales, Wq = outputs(*W.shape)
+    F.focus_fouroversix_weight(W, u * gold["weights"]["s_over_u"], codes, scales, Wq)
+    ex = gold["weights"]["expected"]
+    np.testing.assert_array_equal(host(scales), np.array(ex["scales"], np.uint8))
+    np.testing.assert_array_equal(unpack_codes(host(codes)), np.array(ex["codes"], np.uint8))
+    assert torch.equal(Wq.view(torch.int16), W.view(torch.int16))
+    X = torch.tensor(np.array(gold["tokens"]["X_over_u"]) * u, dtype=torch.float32).to(torch.bfloat16).cuda()
+    ts = torch.empty(X.shape[0], device="cuda")
+    codes, scales, Xq = outputs(*X.shape)
+    F.focus_fouroversix_act(X, ts, codes, scales, Xq)
+    ex = gold["tokens"]["expected"]
+    np.testing.assert_array_equal(host(ts), np.array(ex["row_scales_over_u"], np.float32) * np.float32(u))
+    np.testing.assert_array_equal(host(scales), np.array(ex["scales"], np.uint8))
+    np.testing.assert_array_equal(unpack_codes(host(codes))[0], np.array(ex["codes_row0"], np.uint8))
+    assert torch.equal(Xq.view(torch.int16), X.view(torch.int16))
+    assert F.focus_get_error() == 0
+
+
+def test_nonfinite_sets_flag(F):
+    X = synth.activations(8, 64, "cuda", zero_tokens=0)
+    X[3, 5] = float("inf")
+    ts = torch.zeros(8, device="cuda")
+    codes, scales, Xq = outputs(8, 64)
+    assert F.focus_get_error() == 0
+    F.focus_fouroversix_act(X, ts, codes, scales, Xq)
+    assert F.focus_get_error() == 7
+    W = weights((4, 64), 1)
+    W[2, 9] = float("nan")
+    F.focus_fouroversix_weight(W, 1e-4, codes[:4], scales[:4], None)
+    assert F.focus_get_error() == 7
+    assert F.focus_get_error() == 0
