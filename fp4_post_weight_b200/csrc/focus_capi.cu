@@ -513,6 +513,29 @@ int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, flo
     return launch_status();
 }
 
+size_t focus_scales_swizzled_bytes(int64_t rows, int64_t cols) {
+    if (rows < 0 || cols < 0) return 0;
+    return (size_t)(((rows + 127) / 128) * 128) * (size_t)(((cols + 3) / 4) * 4);
+}
+
+int focus_scales_swizzle(const uint8_t *scales, int64_t rows, int64_t cols, uint8_t *out, size_t out_bytes,
+                         focus_stream_t stream) {
+    if (rows < 0 || cols < 0) return FOCUS_ERR_SHAPE;
+    const size_t need = focus_scales_swizzled_bytes(rows, cols);
+    if (need == 0) return FOCUS_OK;
+    if (!out || (!scales && rows * cols > 0)) return FOCUS_ERR_NULL;
+    if (!aligned16(out) || !aligned16(scales)) return FOCUS_ERR_ALIGN;
+    if (out_bytes < need) return FOCUS_ERR_WORKSPACE;
+    DeviceInfo *di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    const int64_t words = (int64_t)(need / 4);
+    const int64_t grid = grid_for((words + THREADS - 1) / THREADS, di->sms, 8);
+    scales_swizzle_kernel<<<(unsigned)grid, THREADS, 0, (cudaStream_t)stream>>>(scales, rows, cols,
+                                                                               reinterpret_cast<uint32_t *>(out), words);
+    return launch_status();
+}
+
 int focus_get_error(focus_stream_t stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FOCUS_ERR_CUDA;
     unsigned int flags = 0;

@@ -87,7 +87,10 @@ struct TensorRef {
     float s2;
     float den;      // fl(6 * s2)
     float rden;     // fl(1 / den)
+    float den4;     // fl(4 * s2) (FourOverSix)
+    float rden4;    // fl(1 / den4)
     bool den_ok;    // den inside the range where the quotient by rden is exact
+    bool den46_ok;  // den and den4 both inside it
     bool ok;        // s2 usable
 };
 
@@ -105,6 +108,9 @@ __device__ __forceinline__ void load_tensor(const Args &a, int t, TensorRef &r) 
     r.den = __fmul_rn(6.0f, r.s2);
     r.den_ok = r.ok && r.den >= 0x1p-60f && r.den <= 0x1p60f;
     r.rden = r.den_ok ? rcp_rn(r.den) : 0.0f;
+    r.den4 = __fmul_rn(4.0f, r.s2);
+    r.den46_ok = r.den_ok && r.den4 >= 0x1p-60f && r.den4 <= 0x1p60f;
+    r.rden4 = r.den46_ok ? rcp_rn(r.den4) : 0.0f;
 }
 
 // ---------------------------------------------------------------------------
@@ -235,58 +241,123 @@ __device__ __forceinline__ void store_wq_from_codes(const TV &T, uint32_t blk, c
 // the lower error; section "Perplexity": round-to-nearest FourOverSix weights)
 // ---------------------------------------------------------------------------
 
-// One target T of a block: x = fl(A / fl(T*s)), scale 1 when x == 0,
-// S = e4m3(clamp(x, 2^-6, 448)), D = fl(S*s), c = E2M1(clamp(fl(w/D), -6, 6)).
-// Returns the block's squared error in binary32: d = fl(w - (c*S)*s) in one
-// rounding, the even and the odd elements summed apart by fused multiply-adds
-// (one packed lane each, in element order), then added.
-__device__ __forceinline__ float f46_target(const uint32_t *w, float A, float s, float Ts, uint32_t &sb,
-                                            uint32_t codes[2]) {
-    float x = __fdiv_rn(A, Ts);
+// The scales a FourOverSix block needs from its tensor (or token) scale s:
+// the quotient denominators fl(6*s), fl(4*s), their correctly rounded
+// reciprocals, and whether both lie in [2^-60, 2^60], where the quotient by
+// the reciprocal (div_full) is exact.
+struct F46Scale {
+    float s, den6, rden6, den4, rden4;
+    bool den_ok;
+};
+
+__device__ __forceinline__ F46Scale f46_scale(float s) {
+    F46Scale c;
+    c.s = s;
+    c.den6 = __fmul_rn(6.0f, s);
+    c.den4 = __fmul_rn(4.0f, s);
+    c.den_ok = c.den6 >= 0x1p-60f && c.den6 <= 0x1p60f && c.den4 >= 0x1p-60f && c.den4 <= 0x1p60f;
+    c.rden6 = c.den_ok ? rcp_rn(c.den6) : 0.0f;
+    c.rden4 = c.den_ok ? rcp_rn(c.den4) : 0.0f;
+    return c;
+}
+
+// x_T = fl(A / den) for A >= 0: the Markstein quotient where it is exact,
+// the IEEE division elsewhere.
+__device__ __forceinline__ float f46_x(float A, float den, float rden, bool den_ok) {
+    if (den_ok && A <= 0x1p60f && (A >= 0x1p-60f || A == 0.0f)) return div_full(A, den, rden);
+    return __fdiv_rn(A, den);
+}
+
+// Scale byte, its value, its binary16 bits and D = fl(S*s) of target x.
+struct F46Target {
+    uint32_t sb;
+    float D, nr;          // D and -fl(1/D) (0 when D is outside the fast range)
+    uint16_t S_h;
+    bool fast;
+};
+
+__device__ __forceinline__ F46Target f46_target(float x, float s, float A) {
+    F46Target t;
     x = (x == 0.0f) ? 1.0f : x;
     x = fminf(fmaxf(x, 0x1p-6f), 448.0f);
-    sb = e4m3_byte(x);
-    const float S = e4m3_normal_f32(sb);
-    const uint16_t S_h = (uint16_t)e4m3_normal_f16_bits(sb);
-    const float D = __fmul_rn(S, s);
-    const bool fast = D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f;
-    const float nr = fast ? -rcp_rn(D) : 0.0f;
-    const uint64_t D2 = f2_pack(D, D), nr2 = f2_pack(nr, nr), ns2 = f2_pack(-s, -s);
-    uint64_t E2 = 0ull;                         // (even, odd) partial sums
+    t.sb = e4m3_byte(x);
+    t.S_h = (uint16_t)e4m3_normal_f16_bits(t.sb);
+    t.D = __fmul_rn(e4m3_normal_f32(t.sb), s);
+    t.fast = t.D >= 0x1p-60f && t.D <= 0x1p60f && A <= 0x1p60f;
+    t.nr = t.fast ? -rcp_rn(t.D) : 0.0f;
+    return t;
+}
+
+// Codes of one pair of weights (negated, as a packed pair) under a target, and
+// the pair's contribution to the target's squared error: d' = fl(c*S*s - w)
+// = -fl(w - c*S*s) in one rounding (c*S is exact), E <- fma(d', d', E), one
+// packed lane for the even element and one for the odd.  FAST: the quotient
+// from the reciprocal (D2, nr2 = (D, D), (-fl(1/D), ...)); else IEEE division.
+template <bool FAST>
+__device__ __forceinline__ uint32_t f46_pair(uint64_t nw, uint32_t wv, float D, uint64_t D2, uint64_t nr2,
+                                             uint16_t S_h, uint64_t s_2, uint64_t &E2) {
+    uint64_t y2;
+    if (FAST) y2 = div_by_f2(nw, D2, nr2);
+    else y2 = f2_pack(__fdiv_rn(bf16_lo(wv), D), __fdiv_rn(bf16_hi(wv), D));
+    const uint32_t byte = e2m1_pair(f2_lo(y2), f2_hi(y2));
+    const uint32_t h2 = e2m1_pair_f16x2(byte);
+    const uint64_t cs2 = f2_pack(mul_f16_exact(lo16(h2), S_h), mul_f16_exact(hi16(h2), S_h));
+    const uint64_t d2 = f2_fma(cs2, s_2, nw);
+    E2 = f2_fma(d2, d2, E2);
+    return byte;
+}
+
+// Both targets side by side over the block's pairs: code words and errors.
+template <bool FAST>
+__device__ __forceinline__ void f46_both(const uint32_t *w, const F46Target &t6, const F46Target &t4, float s,
+                                         uint32_t c6[2], uint32_t c4[2], float &e6, float &e4) {
+    const uint64_t s_2 = f2_pack(s, s);
+    const uint64_t D6 = f2_pack(t6.D, t6.D), n6 = f2_pack(t6.nr, t6.nr);
+    const uint64_t D4 = f2_pack(t4.D, t4.D), n4 = f2_pack(t4.nr, t4.nr);
+    uint64_t E6 = 0ull, E4 = 0ull;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-        uint32_t code = 0u;
+        uint32_t a6 = 0u, a4 = 0u;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint32_t wv = w[4 * k + j];
-            const uint64_t y2 = fast ? div_by_f2(bf16x2_neg_f2(wv), D2, nr2)
-                                     : f2_pack(__fdiv_rn(bf16_lo(wv), D), __fdiv_rn(bf16_hi(wv), D));
-            const uint32_t byte = e2m1_pair(f2_lo(y2), f2_hi(y2));
-            code |= byte << (8 * j);
-            const uint32_t h2 = e2m1_pair_f16x2(byte);
-            const uint64_t cs2 = f2_pack(mul_f16_exact(lo16(h2), S_h), mul_f16_exact(hi16(h2), S_h));
-            const uint64_t d2 = f2_fma(cs2, ns2, bf16x2_f2(wv));
-            E2 = f2_fma(d2, d2, E2);
+            const uint64_t nw = bf16x2_neg_f2(wv);
+            a6 |= f46_pair<FAST>(nw, wv, t6.D, D6, n6, t6.S_h, s_2, E6) << (8 * j);
+            a4 |= f46_pair<FAST>(nw, wv, t4.D, D4, n4, t4.S_h, s_2, E4) << (8 * j);
         }
-        codes[k] = code;
+        c6[k] = a6;
+        c4[k] = a4;
     }
-    return __fadd_rn(f2_lo(E2), f2_hi(E2));
+    e6 = __fadd_rn(f2_lo(E6), f2_hi(E6));
+    e4 = __fadd_rn(f2_lo(E4), f2_hi(E4));
 }
 
-// FourOverSix of one block with scale s > 0 (den6 = fl(6*s), den4 = fl(4*s)):
-// the chosen scale byte and codes; the target 4 only when its error is lower.
-__device__ __forceinline__ bool f46_block(const uint32_t *w, float s, float den6, float den4, uint32_t &sb,
+// FourOverSix of one block with block maximum A (bf16 magnitude, exact) and
+// scale sc.s > 0.  The error of each target is fl(E_even + E_odd).  Returns
+// true when the target 4 is chosen (its error strictly lower); sb and codes
+// receive the choice.
+__device__ __forceinline__ bool f46_block(const uint32_t *w, float A, const F46Scale &sc, uint32_t &sb,
                                           uint32_t codes[2]) {
+    const F46Target t6 = f46_target(f46_x(A, sc.den6, sc.rden6, sc.den_ok), sc.s, A);
+    const F46Target t4 = f46_target(f46_x(A, sc.den4, sc.rden4, sc.den_ok), sc.s, A);
+    uint32_t c6[2], c4[2];
+    float e6, e4;
+    if (t6.fast && t4.fast) f46_both<true>(w, t6, t4, sc.s, c6, c4, e6, e4);
+    else f46_both<false>(w, t6, t4, sc.s, c6, c4, e6, e4);
+    const bool four = e4 < e6;
+    sb = four ? t4.sb : t6.sb;
+    codes[0] = four ? c4[0] : c6[0];
+    codes[1] = four ? c4[1] : c6[1];
+    return four;
+}
+
+// Block maximum |w| of 16 bf16 values as bf16 magnitude bits (exact; NaN and
+// infinity sort above every finite magnitude).
+__device__ __forceinline__ uint32_t block_amax_bits(const uint32_t *w) {
     uint32_t am = 0u;
 #pragma unroll
     for (int j = 0; j < 8; ++j) am = __vmaxu2(am, w[j] & 0x7fff7fffu);
-    const float A = __uint_as_float(max(am & 0xffffu, am >> 16) << 16);
-    uint32_t sb4, c4[2];
-    const float e6 = f46_target(w, A, s, den6, sb, codes);
-    const float e4 = f46_target(w, A, s, den4, sb4, c4);
-    const bool four = e4 < e6;
-    if (four) { sb = sb4; codes[0] = c4[0]; codes[1] = c4[1]; }
-    return four;
+    return max(am & 0xffffu, am >> 16);
 }
 
 // The bf16 bits of w' = bf16(fl(fl(c*S)*s)) for the 16 codes of a block, as
@@ -310,21 +381,21 @@ __device__ __forceinline__ void wq_words(const uint32_t codes[2], uint32_t sbyte
 // FourOverSix of one block of a weight tensor (tensor scale s2 = T.s2).
 template <class TV>
 __device__ __forceinline__ void compute_block_f46(const TV &T, Block &B) {
-    uint32_t am = 0u;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) am = __vmaxu2(am, B.w[j] & 0x7fff7fffu);
-    const bool bad = B.valid && max(am & 0xffffu, am >> 16) >= 0x7f80u;
+    const uint32_t abits = block_amax_bits(B.w);
+    const bool bad = B.valid && abits >= 0x7f80u;
     if (B.valid) {
-        const float s = T.s2;
+        F46Scale sc;
+        sc.s = T.s2; sc.den6 = T.den; sc.rden6 = T.rden; sc.den4 = T.den4; sc.rden4 = T.rden4;
+        sc.den_ok = T.den46_ok;
         uint32_t sb, codes[2];
-        f46_block(B.w, s, __fmul_rn(6.0f, s), __fmul_rn(4.0f, s), sb, codes);
+        f46_block(B.w, __uint_as_float(abits << 16), sc, sb, codes);
         if (T.d.codes) {
             reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = make_uint2(codes[0], codes[1]);
             T.d.scales[B.blk] = (uint8_t)sb;
         }
         if (T.d.Wq) {
             uint4 o[2];
-            wq_words(codes, sb, s, o);
+            wq_words(codes, sb, T.s2, o);
             __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + 2u * B.blk, o[0]);
             __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + 2u * B.blk + 1u, o[1]);
         }
@@ -529,7 +600,9 @@ struct StageInfo {
     uint32_t first;    // first block of the tile within the tensor
     uint32_t nb;       // blocks in the tile
     uint32_t mode;     // MODE_*
-    uint32_t pad[3];
+    float den4;        // FourOverSix: fl(4*s2), its reciprocal, both quotients exact by reciprocal
+    float rden4;
+    uint32_t den46_ok;
 };
 
 // A block's inputs from a staged tile (local block lb of the tile).
@@ -627,6 +700,9 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
         inf.den = T.den;
         inf.rden = T.rden;
         inf.den_ok = T.den_ok ? 1u : 0u;
+        inf.den4 = T.den4;
+        inf.rden4 = T.rden4;
+        inf.den46_ok = T.den46_ok ? 1u : 0u;
         inf.first = first;
         inf.nb = nb;
         inf.mode = mode;
@@ -834,7 +910,7 @@ __global__ void __launch_bounds__(THREADS) f46_rows_kernel(const uint16_t *__res
         }
         const float s = __fdiv_rn(__uint_as_float(amax << 16), 2688.0f);
         if (threadIdx.x == 0) row_scales[r] = s;
-        const float den6 = __fmul_rn(6.0f, s), den4 = __fmul_rn(4.0f, s);
+        const F46Scale sc = f46_scale(s);
         for (int64_t b = threadIdx.x; b < nb; b += THREADS) {
             const int64_t blk = r * nb + b;
             uint32_t sb = 0x38u, cw[2] = {0u, 0u};
@@ -842,7 +918,7 @@ __global__ void __launch_bounds__(THREADS) f46_rows_kernel(const uint16_t *__res
             if (s != 0.0f) {
                 const uint4 v0 = xr[2 * b], v1 = xr[2 * b + 1];
                 const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                f46_block(w, s, den6, den4, sb, cw);
+                f46_block(w, __uint_as_float(block_amax_bits(w) << 16), sc, sb, cw);
                 if (Xq) wq_words(cw, sb, s, o);
             }
             reinterpret_cast<uint2 *>(codes)[blk] = make_uint2(cw[0], cw[1]);
@@ -852,6 +928,36 @@ __global__ void __launch_bounds__(THREADS) f46_rows_kernel(const uint16_t *__res
                 __stcs(reinterpret_cast<uint4 *>(Xq) + 2 * blk + 1, o[1]);
             }
         }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 scale factors [rows][cols] (row-major, one byte per 16-element block)
+// -> the 128x4-atom layout the sm_100 block-scaled tensor-core GEMM reads:
+// rows padded to 128 and columns to 4, atoms of 128 rows x 4 columns (512
+// bytes) stored band by band (column groups inner), scale (r, c) of an atom
+// at byte 16*(r mod 32) + 4*(r div 32) + c.  One thread per 4-byte output
+// word (one row's 4 scales): the writes are coalesced; padding is written 0.
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(THREADS) scales_swizzle_kernel(const uint8_t *__restrict__ lin, int64_t rows,
+                                                                 int64_t cols, uint32_t *__restrict__ out,
+                                                                 int64_t words) {
+    const int64_t groups = (cols + 3) / 4;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t wi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; wi < words; wi += stride) {
+        const int64_t atom = wi >> 7;                       // 128 words per atom
+        const uint32_t in = (uint32_t)wi & 127u;            // word 4*(r mod 32) + (r div 32) of the atom
+        const int64_t r = (atom / groups) * 128 + 32 * (in & 3u) + (in >> 2);
+        const int64_t c0 = (atom % groups) * 4;
+        uint32_t v = 0u;
+        if (r < rows) {
+            const uint8_t *src = lin + r * cols + c0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (c0 + c < cols) v |= (uint32_t)src[c] << (8 * c);
+        }
+        out[wi] = v;
     }
 }
 

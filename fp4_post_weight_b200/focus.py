@@ -66,6 +66,8 @@ _SIGS = {
     "focus_fouroversix_weight": ([_P, _I64, _I64, _F, _P, _P, _P, _P], _I),
     "focus_fouroversix_multi": ([_P, _I, _I64, _P], _I),
     "focus_fouroversix_act": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _I),
+    "focus_scales_swizzled_bytes": ([_I64, _I64], _SZ),
+    "focus_scales_swizzle": ([_P, _I64, _I64, _P, _SZ, _P], _I),
     "focus_get_error": ([_P], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -247,6 +249,17 @@ def focus_fouroversix_act(X, token_scales, codes, scales, Xq=None, stream=None, 
     t, h = _shape(X, tokens, hidden)
     _check(_lib.focus_fouroversix_act(_ptr(X), t, h, _ptr(token_scales), _ptr(codes), _ptr(scales), _ptr(Xq),
                                       _stream(stream)), "focus_fouroversix_act")
+
+
+def focus_scales_swizzled_bytes(rows: int, cols: int) -> int:
+    return int(_lib.focus_scales_swizzled_bytes(int(rows), int(cols)))
+
+
+def focus_scales_swizzle(scales, out, stream=None, rows=None, cols=None):
+    """E4M3 scales [rows, cols] -> the 128x4-atom layout of sm_100 block-scaled GEMMs (into out)."""
+    r, c = _shape(scales, rows, cols)
+    nbytes = out.numel() * out.element_size() if isinstance(out, torch.Tensor) else 1 << 62
+    _check(_lib.focus_scales_swizzle(_ptr(scales), r, c, _ptr(out), nbytes, _stream(stream)), "focus_scales_swizzle")
 
 
 def focus_get_error(stream=None) -> int:

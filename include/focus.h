@@ -306,6 +306,23 @@ int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, flo
                           uint8_t *codes, uint8_t *scales, uint16_t *Xq, focus_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Scale factors for sm_100 block-scaled GEMMs.  The pages deploy the export
+ * as plain NVFP4 for standard NVFP4 kernels (card, "What this is"); on sm_100
+ * those kernels (cuBLASLt's NVFP4 GEMM, the tcgen05 block-scaled MMA; PyTorch
+ * calls the layout SWIZZLE_32_4_4) read an operand's E4M3 scales [rows][K/16]
+ * in NVIDIA's 128x4 layout: rows padded to 128 and columns to 4, atoms of 128
+ * rows x 4 columns (512 bytes) stored band by band with the column groups
+ * inner, scale (r, c) of an atom at byte 16*(r mod 32) + 4*(r div 32) + c.
+ *   scales  [rows][cols] u8, device, as focus_pack_nvfp4 / the FourOverSix
+ *           calls write them (cols = K/16)
+ *   out     device, at least focus_scales_swizzled_bytes(rows, cols) bytes
+ *           (else FOCUS_ERR_WORKSPACE); every byte is written, padding 0
+ * ------------------------------------------------------------------------- */
+size_t focus_scales_swizzled_bytes(int64_t rows, int64_t cols);
+int focus_scales_swizzle(const uint8_t *scales, int64_t rows, int64_t cols, uint8_t *out, size_t out_bytes,
+                         focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Synchronizes `stream`, then reports and clears the sticky device flag:
  * FOCUS_ERR_DEVICE_TIMEOUT when a kernel's pipeline wait ran out,
  * FOCUS_ERR_NONFINITE_INPUT when any kernel since the last call met a

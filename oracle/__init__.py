@@ -78,6 +78,8 @@ def lib():
         L.fo_pack.restype = ctypes.c_int
         L.fo_f46.argtypes = [_P, _I64, _I64, _F, ctypes.c_int, _P, _P, _P, _P, _P, _P]
         L.fo_f46.restype = ctypes.c_int
+        L.fo_swizzled_bytes.argtypes = [_I64, _I64]; L.fo_swizzled_bytes.restype = _I64
+        L.fo_scales_swizzle.argtypes = [_P, _I64, _I64, _P]; L.fo_scales_swizzle.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -263,3 +265,13 @@ def fouroversix(X, s=None) -> FourOverSix:
     _chk(lib().fo_f46(_p(X), rows, cols, 0.0 if per_row else float(s), 1 if per_row else 0, _p(codes),
                       _p(scales), _p(Xq), _p(four), _p(errs), _p(rs)))
     return FourOverSix(codes, scales, Xq, four, errs, rs)
+
+
+def scales_swizzle(scales: np.ndarray) -> np.ndarray:
+    """E4M3 scale bytes [rows, cols] -> the 128x4-atom layout of the sm_100
+    block-scaled GEMM (flat uint8, rows padded to 128 and cols to 4, zeros)."""
+    scales = _c(scales, np.uint8)
+    rows, cols = scales.shape
+    out = np.empty(int(lib().fo_swizzled_bytes(rows, cols)), np.uint8)
+    _chk(lib().fo_scales_swizzle(_p(scales), rows, cols, _p(out)))
+    return out

@@ -649,3 +649,38 @@ int fo_f46(const uint16_t *X, int64_t rows, int64_t cols, float s, int per_row, 
     }
     return bad ? FO_ERR_NONFINITE : FO_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* scale factors in the layout of the sm_100 block-scaled tensor-core GEMM   */
+/* ------------------------------------------------------------------------ */
+/*
+ * Not on the pages: the card deploys the export as plain NVFP4 for standard
+ * NVFP4 kernels ("What this is"), and on sm_100 those kernels (cuBLASLt's
+ * block-scaled GEMM, the tcgen05 block-scaled MMA) read the E4M3 scale
+ * factors of an operand [rows][K/16] in NVIDIA's published 128x4 layout:
+ * the scale matrix is padded to a multiple of 128 rows and of 4 columns and
+ * cut into atoms of 128 rows x 4 columns (512 bytes), stored atom by atom,
+ * the atoms of one 128-row band first (row-major over bands and column
+ * groups); inside an atom, scale (r, c) is byte 16*(r mod 32) + 4*(r div 32)
+ * + c.  Padding bytes are 0.
+ */
+int64_t fo_swizzled_bytes(int64_t rows, int64_t cols)
+{
+    if (rows < 0 || cols < 0) return -1;
+    return ((rows + 127) / 128 * 128) * ((cols + 3) / 4 * 4);
+}
+
+int fo_scales_swizzle(const uint8_t *lin, int64_t rows, int64_t cols, uint8_t *out)
+{
+    if (rows < 0 || cols < 0) return FO_ERR_SHAPE;
+    const int64_t C = (cols + 3) / 4 * 4;
+    memset(out, 0, (size_t)fo_swizzled_bytes(rows, cols));
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c = 0; c < cols; ++c) {
+            const int64_t atom = (r / 128) * (C / 4) + c / 4;
+            const int64_t rr = r % 128;
+            out[atom * 512 + 16 * (rr % 32) + 4 * (rr / 32) + c % 4] = lin[r * cols + c];
+        }
+    }
+    return FO_OK;
+}

@@ -178,3 +178,15 @@ def test_table_prepare_fouroversix(F):
     with pytest.raises(F.FocusError) as e:          # the FOCUS purposes still need m and q
         F.focus_table_prepare(descs, 0)
     assert e.value.status == 1
+
+
+def test_swizzle_checks(F):
+    assert F.focus_scales_swizzled_bytes(1, 1) == 512
+    assert F.focus_scales_swizzled_bytes(130, 6) == 256 * 8
+    assert F.focus_scales_swizzled_bytes(0, 7) == 0
+    assert F.raw_call("focus_scales_swizzle", P, -1, 4, P, 4096, None) == 2
+    assert F.raw_call("focus_scales_swizzle", P, 0, 4, P, 0, None) == 0          # nothing to write
+    assert F.raw_call("focus_scales_swizzle", P, 4, 4, None, 4096, None) == 1
+    assert F.raw_call("focus_scales_swizzle", None, 4, 4, P, 4096, None) == 1
+    assert F.raw_call("focus_scales_swizzle", P, 4, 4, U, 4096, None) == 3
+    assert F.raw_call("focus_scales_swizzle", P, 4, 4, P, 511, None) == 5        # output too small
