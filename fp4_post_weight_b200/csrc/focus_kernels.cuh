@@ -184,11 +184,12 @@ __device__ __forceinline__ float scaled_max(const TV &T, float A, float m) {
 
 // NVFP4 codes and E4M3 scale byte of one block for block factor m and
 // sub-block logits q0, q1 (the forward's decisions only).
-// The sub-block sigmoids come from sigmoid_near with the forward's e^-q (t0, t1
-// at the logits q0_old, q1_old), bit-identical to evaluating them afresh.
+// The sub-block sigmoids come from sigmoid_step with the forward's binary64
+// sigmoids (s0, s1 at the logits q0_old, q1_old), bit-identical to evaluating
+// them afresh.
 template <class TV>
 __device__ __forceinline__ void encode_block(const TV &T, const uint32_t *w, float A, float m, float q0, float q1,
-                                             double t0, double t1, float q0_old, float q1_old, uint32_t &sbyte,
+                                             double s0, double s1, float q0_old, float q1_old, uint32_t &sbyte,
                                              uint32_t codes[2]) {
     const float x = scaled_max(T, A, m);
     float xc = (x == 0.0f) ? 1.0f : x;
@@ -197,7 +198,7 @@ __device__ __forceinline__ void encode_block(const TV &T, const uint32_t *w, flo
     const float S = e4m3_normal_f32(sbyte);
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-        const float sig = k ? sigmoid_near(t1, q1_old, q1) : sigmoid_near(t0, q0_old, q0);
+        const float sig = k ? sigmoid_step(s1, q1_old, q1) : sigmoid_step(s0, q0_old, q0);
         const float D = __fmul_rn(__fmul_rn(S, sig), T.s2);
         uint32_t code = 0u;
         if (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f) {
@@ -436,13 +437,13 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
 
     const bool want_wq = KIND != KIND_BWD && !WQU && a.write_wq && T.d.Wq != nullptr && B.valid;
     float sig[2], sq[2];
-    double et[2];                               // e^-q of the forward, reused by the export
+    double s64[2];                              // the forward's binary64 sigmoids, reused by the export
     uint64_t sm2 = 0ull;                        // sum of g * (in ? c - y : c), pairwise
     uint32_t codes[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
         // D_k = fl(fl(S*sigmoid(q_k))*s2); y_i = fl(w_i/D_k); c_i = E2M1(clamp(y_i, -6, 6))
-        sig[k] = sigmoid_rn_t(B.q[k], et[k]);
+        sig[k] = sigmoid_fast(B.q[k], s64[k]);
         const float D = __fmul_rn(__fmul_rn(S, sig[k]), T.s2);
         uint64_t y2[4];
         if (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f) {
@@ -538,7 +539,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
             const bool exp_wq = WQU && T.d.Wq != nullptr;
             if (B.valid && (exp_codes || exp_wq)) {
                 uint32_t sb2, codes2[2];
-                encode_block(T, B.w, A, B.m, f2_lo(qp), f2_hi(qp), et[0], et[1], q_old0, q_old1, sb2, codes2);
+                encode_block(T, B.w, A, B.m, f2_lo(qp), f2_hi(qp), s64[0], s64[1], q_old0, q_old1, sb2, codes2);
                 if (exp_codes) {
                     uint2 cc; cc.x = codes2[0]; cc.y = codes2[1];
                     reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;

@@ -13,9 +13,12 @@
 * The reciprocal from the hardware approximation and one Newton step equals
   __frcp_rn for every significand; the twice-corrected quotient used for the
   scaled block maximum equals __fdiv_rn (every divisor significand for 1024
-  pseudo-random numerators, and 2^30 pseudo-random pairs); the sigmoid of an
-  updated logit computed from the old e^-q equals sigmoid_rn (2^28 pairs,
-  logits up to +-100).
+  pseudo-random numerators, and 2^30 pseudo-random pairs).
+* The forward's sigmoid (own e^x, a rounding-certainty test, sigmoid_rn where
+  it cannot decide) equals sigmoid_rn for EVERY binary32 logit with
+  |q| <= 100; the export's sigmoid of an updated logit (a Taylor step from the
+  forward's binary64 sigmoid) equals sigmoid_rn on 2^29 pairs with steps of
+  every magnitude.
 """
 import ctypes
 import os
@@ -44,9 +47,10 @@ def lib():
     L.check_rcp.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_ulonglong)]
     L.check_div_full.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong),
                                  ctypes.POINTER(ctypes.c_float)]
-    L.check_sigmoid_near.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong),
-                                     ctypes.POINTER(ctypes.c_float)]
     L.e2m1_raw_bytes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    L.check_sigmoid_fast.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_float)]
+    L.check_sigmoid_step.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong),
+                                     ctypes.POINTER(ctypes.c_float)]
     return L
 
 
@@ -92,9 +96,24 @@ def test_full_quotient(lib, mode, seed):
     assert n.value == 0, f"{n.value} quotients differ, e.g. a={ex[0]!r} b={ex[1]!r} got {ex[2]!r} want {ex[3]!r}"
 
 
-@pytest.mark.parametrize("seed", [11, 12])
-def test_sigmoid_of_updated_logit(lib, seed):
-    n = ctypes.c_ulonglong(0)
+def test_sigmoid_fast_every_logit(lib):
+    """Every binary32 logit with |q| <= 100: the forward's sigmoid equals sigmoid_rn
+    bit for bit, its binary64 value is within 2^-49, and the fast path decides
+    the rounding for nearly every logit."""
+    c = (ctypes.c_ulonglong * 4)()
     ex = (ctypes.c_float * 4)()
-    assert lib.check_sigmoid_near(seed, ctypes.byref(n), ex) == 0
-    assert n.value == 0, f"{n.value} differ, e.g. q0={ex[0]!r} q1={ex[1]!r} got {ex[2]!r} want {ex[3]!r}"
+    assert lib.check_sigmoid_fast(c, ex) == 0
+    assert c[2] > 2_000_000_000
+    assert c[0] == 0, f"{c[0]} sigmoids differ, e.g. q={ex[0]!r} got {ex[1]!r} want {ex[2]!r}"
+    assert c[1] == 0, f"{c[1]} binary64 values outside 2^-49"
+    assert c[3] > 0.999 * c[2] * 0.8
+
+
+@pytest.mark.parametrize("seed", [21, 22])
+def test_sigmoid_step_of_updated_logit(lib, seed):
+    c = (ctypes.c_ulonglong * 4)()
+    ex = (ctypes.c_float * 4)()
+    assert lib.check_sigmoid_step(seed, c, ex) == 0
+    assert c[1] == 1 << 28
+    assert c[0] == 0, f"{c[0]} differ, e.g. q0={ex[0]!r} q1={ex[1]!r} got {ex[2]!r} want {ex[3]!r}"
+    assert c[2] > 0.5 * c[1]            # the Taylor step decides most roundings
