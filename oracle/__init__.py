@@ -78,6 +78,9 @@ def lib():
         L.fo_pack.restype = ctypes.c_int
         L.fo_f46.argtypes = [_P, _I64, _I64, _F, ctypes.c_int, _P, _P, _P, _P, _P, _P]
         L.fo_f46.restype = ctypes.c_int
+        L.fo_mx_fwd.argtypes = [_P, _P, _P, _I64, _I64, _P, _P, _P]; L.fo_mx_fwd.restype = ctypes.c_int
+        L.fo_mx_ste_bwd.argtypes = [_P, _P, _P, _P, _I64, _I64, _P, _P, ctypes.c_int]
+        L.fo_mx_ste_bwd.restype = ctypes.c_int
         L.fo_swizzled_bytes.argtypes = [_I64, _I64]; L.fo_swizzled_bytes.restype = _I64
         L.fo_scales_swizzle.argtypes = [_P, _I64, _I64, _P]; L.fo_scales_swizzle.restype = ctypes.c_int
         _lib = L
@@ -275,3 +278,38 @@ def scales_swizzle(scales: np.ndarray) -> np.ndarray:
     out = np.empty(int(lib().fo_swizzled_bytes(rows, cols)), np.uint8)
     _chk(lib().fo_scales_swizzle(_p(scales), rows, cols, _p(out)))
     return out
+
+
+@dataclass
+class MXForward:
+    Wq: np.ndarray       # uint16 bf16 bits [out, in]
+    codes: np.ndarray    # uint8 [out, in], one E2M1 code per element
+    scales: np.ndarray   # uint8 [out, in/32], E8M0 bytes
+
+
+def mx_fwd(W, m, q) -> MXForward:
+    """MXFP4 variant: m [out, in/32], q [out, in/8]."""
+    W = _c(W, np.uint16); m = _c(m, np.float32); q = _c(q, np.float32)
+    out, inn = W.shape
+    if m.size != out * (inn // 32) or q.size != out * (inn // 8):
+        raise ValueError("m/q size does not match W")
+    Wq = np.empty((out, inn), np.uint16)
+    codes = np.empty((out, inn), np.uint8)
+    scales = np.empty((out, inn // 32), np.uint8)
+    _chk(lib().fo_mx_fwd(_p(W), _p(m), _p(q), out, inn, _p(Wq), _p(codes), _p(scales)))
+    return MXForward(Wq, codes, scales)
+
+
+def mx_ste_bwd(W, dWq, m, q, dm=None, dq=None):
+    """MXFP4 straight-through gradients (added to dm/dq in place when given)."""
+    W = _c(W, np.uint16); dWq = _c(dWq, np.uint16)
+    m = _c(m, np.float32); q = _c(q, np.float32)
+    out, inn = W.shape
+    acc = dm is not None
+    if acc:
+        dm = _c(dm, np.float32); dq = _c(dq, np.float32)
+    else:
+        dm = np.empty((out, inn // 32), np.float32)
+        dq = np.empty((out, inn // 8), np.float32)
+    _chk(lib().fo_mx_ste_bwd(_p(W), _p(dWq), _p(m), _p(q), out, inn, _p(dm), _p(dq), 1 if acc else 0))
+    return dm, dq

@@ -684,3 +684,166 @@ int fo_scales_swizzle(const uint8_t *lin, int64_t rows, int64_t cols, uint8_t *o
     }
     return FO_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4 variant: 32-element blocks, E8M0 scale, four sub-blocks of 8        */
+/* ------------------------------------------------------------------------ */
+/*
+ * Sources: "Technische Samenvatting: FOCUS ...", section "Probleemstelling"
+ * (MXFP4 shares one E8M0 scale per 32 values) and section "Methodologie",
+ * items 2 and 3 (the quantization scale is the hardware scale times a
+ * learnable coefficient; each hardware block -- 32 values for MXFP4 -- is cut
+ * into sub-blocks of 8 with a coefficient each, the dequantization scale
+ * stays shared); the card's equations ("What this is") for the structure.
+ *
+ * Readings (the pages give no MXFP4 formula):
+ *  - MXFP4 has no tensor scale.  The block scale follows the format's own
+ *    conversion rule (the OCP Microscaling specification: a shared exponent
+ *    of floor(log2(max|v|)) minus 2, the largest E2M1 exponent) applied to
+ *    the scaled maximum: x_b = fl(A_b * m_b); S_b = 2^(floor(log2 x_b) - 2),
+ *    the exponent clamped to E8M0's [-127, 127]; x_b == 0 gives scale 1 (as
+ *    the card's zero-block rule); x_b < 0 gives 2^-127.
+ *  - c_i = E2M1(clamp(fl(w_i / D_k), -6, 6)) with D_k = fl(S_b * sigmoid(q_k))
+ *    for sub-block k = 0..3; w'_i = bf16(fl(c_i * S_b)).
+ *  - Straight-through backward as for NVFP4 with s2 = 1 and the power-of-two
+ *    rounding passed straight through (S_b = x_b/4 for the gradient):
+ *    dm_b = inS * (A_b/4) * sum_i g_i*(in_i ? c_i - y_i : c_i), inS = [x_b >=
+ *    2^-125] (inside the exponent clamp; x_b < 2^128 always), and
+ *    dq_k = -(1 - sigma_k) * S_b * sum_{i in k} in_i*g_i*y_i.
+ *  - Layout: m [out][in/32], q [out][in/8] (q[r][4b+k] for sub-block k of
+ *    block b), codes as the NVFP4 pack, E8M0 bytes [out][in/32] (exponent
+ *    + 127).
+ */
+
+typedef struct {
+    float A, x;
+    int inS;
+    int sb;           /* E8M0 byte */
+    float S;
+    float sigma[4];
+    float y[32];
+    int in[32];
+    int code[32];
+    float c[32];
+    float wq[32];     /* fl(c*S) before the bf16 cast */
+} fo_mx_block;
+
+/* floor(log2 x) of a positive finite binary32 (exact, from frexp). */
+static int floor_log2f(float x)
+{
+    int e;
+    frexpf(x, &e);            /* x = f * 2^e, f in [0.5, 1) */
+    return e - 1;
+}
+
+static void mx_quantize_block(const uint16_t *w16, float m_b, const float *q4, fo_mx_block *B)
+{
+    float w[32];
+    float A = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+        w[i] = fo_bf16_to_f32(w16[i]);
+        float a = fabsf(w[i]);
+        if (a > A) A = a;
+    }
+    B->A = A;
+    float x = A * m_b;
+    B->x = x;
+    int e;
+    if (x == 0.0f) e = 0;
+    else if (x < 0.0f) e = -127;
+    else {
+        e = floor_log2f(x) - 2;
+        if (e < -127) e = -127;
+        if (e > 127) e = 127;
+    }
+    B->inS = x >= 0x1p-125f;      /* the exponent clamp: floor(log2 x) >= -125 (x < 2^128 < 2^130 always) */
+    B->sb = e + 127;
+    B->S = ldexpf(1.0f, e);
+    for (int k = 0; k < 4; ++k) {
+        float sig = fo_sigmoid(q4[k]);
+        float D = B->S * sig;
+        B->sigma[k] = sig;
+        for (int j = 0; j < 8; ++j) {
+            int i = 8 * k + j;
+            float y = w[i] / D;
+            float u = y;
+            if (u < -6.0f) u = -6.0f;
+            if (u > 6.0f) u = 6.0f;
+            B->y[i] = y;
+            B->in[i] = (y >= -6.0f) && (y <= 6.0f);
+            B->code[i] = fo_e2m1_encode(u);
+            B->c[i] = (float)fo_e2m1_decode(B->code[i]);
+            B->wq[i] = B->c[i] * B->S;
+        }
+    }
+}
+
+static int check_shape_mx(int64_t out, int64_t in)
+{
+    if (out < 0 || in < 0 || (in % 32) != 0) return FO_ERR_SHAPE;
+    return FO_OK;
+}
+
+/* MXFP4 forward.  Outputs may be NULL: Wq bf16 [out, in]; codes u8 [out, in]
+ * (one per element); scales u8 [out, in/32] (E8M0). */
+int fo_mx_fwd(const uint16_t *W, const float *m, const float *q, int64_t out, int64_t in, uint16_t *Wq,
+              uint8_t *codes, uint8_t *scales)
+{
+    int rc = check_shape_mx(out, in);
+    if (rc) return rc;
+    const int64_t nb = in / 32;
+    int bad = 0;
+#pragma omp parallel for reduction(| : bad) schedule(static)
+    for (int64_t r = 0; r < out; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t blk = r * nb + b;
+            const int64_t e0 = r * in + 32 * b;
+            if (!isfinite(m[blk])) bad = 1;
+            for (int k = 0; k < 4; ++k)
+                if (!isfinite(q[4 * blk + k])) bad = 1;
+            for (int i = 0; i < 32; ++i)
+                if (!isfinite(fo_bf16_to_f32(W[e0 + i]))) bad = 1;
+            fo_mx_block B;
+            mx_quantize_block(W + e0, m[blk], q + 4 * blk, &B);
+            if (scales) scales[blk] = (uint8_t)B.sb;
+            for (int i = 0; i < 32; ++i) {
+                if (Wq) Wq[e0 + i] = fo_f32_to_bf16(B.wq[i]);
+                if (codes) codes[e0 + i] = (uint8_t)B.code[i];
+            }
+        }
+    }
+    return bad ? FO_ERR_NONFINITE : FO_OK;
+}
+
+/* MXFP4 straight-through backward: dm [out, in/32], dq [out, in/8] as
+ * binary32 (sums in binary64, rounded once; accumulate = 1 adds to them). */
+int fo_mx_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, const float *q, int64_t out, int64_t in,
+                  float *dm, float *dq, int accumulate)
+{
+    int rc = check_shape_mx(out, in);
+    if (rc) return rc;
+    const int64_t nb = in / 32;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < out; ++r) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t blk = r * nb + b;
+            const int64_t e0 = r * in + 32 * b;
+            fo_mx_block B;
+            mx_quantize_block(W + e0, m[blk], q + 4 * blk, &B);
+            double sm = 0.0, sq[4] = {0.0, 0.0, 0.0, 0.0};
+            for (int i = 0; i < 32; ++i) {
+                double g = (double)fo_bf16_to_f32(dWq[e0 + i]);
+                double t = B.in[i] ? ((double)B.c[i] - (double)B.y[i]) : (double)B.c[i];
+                sm += g * t;
+                if (B.in[i]) sq[i / 8] += g * (double)B.y[i];
+            }
+            double gm = B.inS ? ((double)B.A / 4.0) * sm : 0.0;
+            dm[blk] = (float)(accumulate ? (double)dm[blk] + gm : gm);
+            for (int k = 0; k < 4; ++k) {
+                double gq = -(1.0 - (double)B.sigma[k]) * (double)B.S * sq[k];
+                dq[4 * blk + k] = (float)(accumulate ? (double)dq[4 * blk + k] + gq : gq);
+            }
+        }
+    }
+    return FO_OK;
+}
