@@ -306,7 +306,10 @@ def measure_next_rows(ents, dev, N, peaks, world):
         [4096, 4096], the down input [4096, 14336]: 208 MB);
       * a calibration step over four micro-batches: three table backward passes
         (the first overwriting dm/dq, then accumulating) and the fused step
-        with FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WQ_UPDATED."""
+        with FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WQ_UPDATED;
+      * the MXFP4 variant's fused step over the same 224 weights (one launch per
+        tensor; reads W, dW', m, q and moments, writes W', m, q and moments:
+        9.75 B per weight)."""
     import torch
 
     import synth
@@ -366,10 +369,28 @@ def measure_next_rows(ents, dev, N, peaks, world):
                            **_roof(6.25 * N, t_b1, peak)},
         "step_accumulate_wq_updated": {"kernel": "pipe_kernel<KIND_STEP, true>", "bytes_per_weight": 11.25,
                                        **_roof(11.25 * N, t_st, peak)}}
-    if F.focus_get_error() != 0:
-        raise SystemExit("device status after the next-row measurements is not OK")
     for e in ents:
         e.dm = e.dq = None
+    del tab
+    # the MXFP4 variant: one fused step per tensor (224 launches), m = 1, q = 6, zero moments
+    mx = []
+    for e in ents:
+        o, i = e.W.shape
+        mx.append((torch.ones((o, i // 32), device=dev), torch.full((o, i // 8), 6.0, device=dev),
+                   torch.zeros((o, i // 32), device=dev), torch.zeros((o, i // 32), device=dev),
+                   torch.zeros((o, i // 8), device=dev), torch.zeros((o, i // 8), device=dev)))
+    cnt_mx = [0]
+
+    def mx_step():
+        cnt_mx[0] += 1
+        for e, (m, q, a1, a2, b1, b2) in zip(ents, mx):
+            F.focus_mx_step(e.W, e.dWq, m, q, a1, a2, b1, b2, hp, cnt_mx[0], 0, e.Wq)
+    ms = _timed(mx_step, stream)
+    out["mxfp4_step_llama8b"] = {"kernel": "mx_kernel<KIND_STEP>", "launches": len(ents), "bytes_per_weight": 9.75,
+                                 "Gelem_s": round(N * world / (ms * 1e-3) / 1e9, 2), **_roof(9.75 * N, ms, peak)}
+    del mx
+    if F.focus_get_error() != 0:
+        raise SystemExit("device status after the next-row measurements is not OK")
     D.barrier()
     return out
 

@@ -13,6 +13,7 @@
 
 #include "focus.h"
 #include "focus_kernels.cuh"
+#include "focus_mx.cuh"
 
 namespace focus {
 
@@ -25,6 +26,7 @@ constexpr int MAX_DEVICES = 64;
 struct DeviceInfo {
     int sms = 0;
     int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_f46 = 0, occ_rows = 0, occ_amax = 0, occ_adam = 0;
+    int occ_mx[3] = {0, 0, 0};
 };
 
 std::once_flag g_once[MAX_DEVICES];
@@ -59,10 +61,14 @@ int device_info(DeviceInfo **out) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows, f46_rows_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_amax, amax_tiles_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_adam, adamw_kernel, THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[0], mx_kernel<KIND_FWD>, THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[1], mx_kernel<KIND_BWD>, THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[2], mx_kernel<KIND_STEP>, THREADS, 0);
     });
     DeviceInfo &d = g_info[dev];
     if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_step_wqu <= 0 || d.occ_f46 <= 0 ||
-        d.occ_rows <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0)
+        d.occ_rows <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 || d.occ_mx[1] <= 0 ||
+        d.occ_mx[2] <= 0)
         return FOCUS_ERR_CUDA;
     *out = &d;
     return FOCUS_OK;
@@ -156,6 +162,23 @@ int launch_on(const Args &a, cudaStream_t s) {
     int64_t grid = grid_for(a.total_tiles, di->sms, occ);
     if (grid < 1) grid = 1;   // the pack of an empty tensor still writes its tensor scale
     pipe_kernel<KIND, WQU><<<(unsigned)grid, CTA_THREADS, stage_smem_bytes<KIND>(), s>>>(a);
+    return launch_status();
+}
+
+int check_shape_mx(int64_t out, int64_t in) {
+    if (out < 0 || in < 0 || (in % 32) != 0) return FOCUS_ERR_SHAPE;
+    if (in > 0 && out > MAX_BLOCKS / (in / 32 > 0 ? in / 32 : 1)) return FOCUS_ERR_SHAPE;
+    return FOCUS_OK;
+}
+
+template <int KIND>
+int launch_mx(const MxArgs &a, cudaStream_t s) {
+    DeviceInfo *di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    if (a.nblk == 0) return FOCUS_OK;
+    const int64_t grid = grid_for((a.nblk + THREADS - 1) / THREADS, di->sms, di->occ_mx[KIND]);
+    mx_kernel<KIND><<<(unsigned)grid, THREADS, 0, s>>>(a);
     return launch_status();
 }
 
@@ -511,6 +534,65 @@ int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, flo
     f46_rows_kernel<<<(unsigned)grid, THREADS, 0, (cudaStream_t)stream>>>(X, tokens, hidden, token_scales, codes,
                                                                          scales, Xq);
     return launch_status();
+}
+
+int focus_mx_fwd(const uint16_t *W, const float *m, const float *q, int64_t out, int64_t in, uint16_t *Wq,
+                 uint8_t *codes, uint8_t *scales, focus_stream_t stream) {
+    int rc = check_shape_mx(out, in);
+    if (rc) return rc;
+    if ((codes == nullptr) != (scales == nullptr)) return FOCUS_ERR_NULL;
+    if (!Wq && !codes) return FOCUS_ERR_NULL;
+    if (out * in == 0) return FOCUS_OK;
+    if (!W || !m || !q) return FOCUS_ERR_NULL;
+    if (!aligned16(W) || !aligned16(m) || !aligned16(q) || !aligned16(Wq) || !aligned16(codes) || !aligned16(scales))
+        return FOCUS_ERR_ALIGN;
+    MxArgs a{};
+    a.W = W; a.m = const_cast<float *>(m); a.q = const_cast<float *>(q);
+    a.Wq = Wq; a.codes = codes; a.scales = scales;
+    a.nblk = out * (in / 32);
+    return launch_mx<KIND_FWD>(a, (cudaStream_t)stream);
+}
+
+int focus_mx_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, const float *q, int64_t out, int64_t in,
+                     float *dm, float *dq, int accumulate, focus_stream_t stream) {
+    int rc = check_shape_mx(out, in);
+    if (rc) return rc;
+    if (accumulate != 0 && accumulate != 1) return FOCUS_ERR_VALUE;
+    if (out * in == 0) return FOCUS_OK;
+    if (!W || !dWq || !m || !q || !dm || !dq) return FOCUS_ERR_NULL;
+    if (!aligned16(W) || !aligned16(dWq) || !aligned16(m) || !aligned16(q) || !aligned16(dm) || !aligned16(dq))
+        return FOCUS_ERR_ALIGN;
+    MxArgs a{};
+    a.W = W; a.dWq = dWq; a.m = const_cast<float *>(m); a.q = const_cast<float *>(q);
+    a.dm = dm; a.dq = dq; a.accumulate = accumulate;
+    a.nblk = out * (in / 32);
+    return launch_mx<KIND_BWD>(a, (cudaStream_t)stream);
+}
+
+int focus_mx_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, float *m_exp_avg, float *m_exp_avg_sq,
+                  float *q_exp_avg, float *q_exp_avg_sq, int64_t out, int64_t in, const focus_hparams *hp,
+                  int64_t step, unsigned flags, uint16_t *Wq, float *dm, float *dq, focus_stream_t stream) {
+    int rc = check_shape_mx(out, in);
+    if (rc) return rc;
+    if (!hp) return FOCUS_ERR_NULL;
+    if ((rc = check_hyper(hp->lr_m, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
+    if ((rc = check_hyper(hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
+    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD)) return FOCUS_ERR_VALUE;
+    if (out * in == 0) return FOCUS_OK;
+    if (!W || !dWq || !m || !q || !m_exp_avg || !m_exp_avg_sq || !q_exp_avg || !q_exp_avg_sq) return FOCUS_ERR_NULL;
+    if (flags && (!dm || !dq)) return FOCUS_ERR_NULL;
+    const void *ptrs[] = {W, dWq, m, q, m_exp_avg, m_exp_avg_sq, q_exp_avg, q_exp_avg_sq, Wq, dm, dq};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return FOCUS_ERR_ALIGN;
+    MxArgs a{};
+    a.W = W; a.dWq = dWq; a.Wq = Wq; a.m = m; a.q = q;
+    a.m_ea = m_exp_avg; a.m_eas = m_exp_avg_sq; a.q_ea = q_exp_avg; a.q_eas = q_exp_avg_sq;
+    a.dm = dm; a.dq = dq;
+    a.accumulate = (flags & FOCUS_STEP_ACCUMULATE) ? 1 : 0;
+    a.write_grad = (flags & FOCUS_STEP_WRITE_GRAD) ? 1 : 0;
+    a.hp = make_hyper(hp->lr_m, hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
+    a.nblk = out * (in / 32);
+    return launch_mx<KIND_STEP>(a, (cudaStream_t)stream);
 }
 
 size_t focus_scales_swizzled_bytes(int64_t rows, int64_t cols) {

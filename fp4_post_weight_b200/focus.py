@@ -66,6 +66,10 @@ _SIGS = {
     "focus_fouroversix_weight": ([_P, _I64, _I64, _F, _P, _P, _P, _P], _I),
     "focus_fouroversix_multi": ([_P, _I, _I64, _P], _I),
     "focus_fouroversix_act": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _I),
+    "focus_mx_fwd": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _P], _I),
+    "focus_mx_ste_bwd": ([_P, _P, _P, _P, _I64, _I64, _P, _P, _I, _P], _I),
+    "focus_mx_step": ([_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, ctypes.POINTER(focus_hparams), _I64,
+                       ctypes.c_uint, _P, _P, _P, _P], _I),
     "focus_scales_swizzled_bytes": ([_I64, _I64], _SZ),
     "focus_scales_swizzle": ([_P, _I64, _I64, _P, _SZ, _P], _I),
     "focus_get_error": ([_P], _I),
@@ -249,6 +253,33 @@ def focus_fouroversix_act(X, token_scales, codes, scales, Xq=None, stream=None, 
     t, h = _shape(X, tokens, hidden)
     _check(_lib.focus_fouroversix_act(_ptr(X), t, h, _ptr(token_scales), _ptr(codes), _ptr(scales), _ptr(Xq),
                                       _stream(stream)), "focus_fouroversix_act")
+
+
+def focus_mx_fwd(W, m, q, Wq=None, codes=None, scales=None, stream=None, out=None, in_=None):
+    """MXFP4 variant forward: m [out, in/32], q [out, in/8]; Wq bf16 and/or codes+scales."""
+    _bf16(W, "W"); _bf16(Wq, "Wq"); _f32(m, "m"); _f32(q, "q")
+    o, i = _shape(W, out, in_)
+    _check(_lib.focus_mx_fwd(_ptr(W), _ptr(m), _ptr(q), o, i, _ptr(Wq), _ptr(codes), _ptr(scales),
+                             _stream(stream)), "focus_mx_fwd")
+
+
+def focus_mx_ste_bwd(W, dWq, m, q, dm, dq, accumulate: bool = False, stream=None, out=None, in_=None):
+    _bf16(W, "W"); _bf16(dWq, "dWq"); _f32(m, "m"); _f32(q, "q"); _f32(dm, "dm"); _f32(dq, "dq")
+    o, i = _shape(W, out, in_)
+    _check(_lib.focus_mx_ste_bwd(_ptr(W), _ptr(dWq), _ptr(m), _ptr(q), o, i, _ptr(dm), _ptr(dq),
+                                 1 if accumulate else 0, _stream(stream)), "focus_mx_ste_bwd")
+
+
+def focus_mx_step(W, dWq, m, q, m_exp_avg, m_exp_avg_sq, q_exp_avg, q_exp_avg_sq, hp: focus_hparams, step: int,
+                  flags: int = 0, Wq=None, dm=None, dq=None, stream=None, out=None, in_=None):
+    _bf16(W, "W"); _bf16(dWq, "dWq"); _bf16(Wq, "Wq")
+    for t, nm in ((m, "m"), (q, "q"), (m_exp_avg, "m_exp_avg"), (m_exp_avg_sq, "m_exp_avg_sq"),
+                  (q_exp_avg, "q_exp_avg"), (q_exp_avg_sq, "q_exp_avg_sq"), (dm, "dm"), (dq, "dq")):
+        _f32(t, nm)
+    o, i = _shape(W, out, in_)
+    _check(_lib.focus_mx_step(_ptr(W), _ptr(dWq), _ptr(m), _ptr(q), _ptr(m_exp_avg), _ptr(m_exp_avg_sq),
+                              _ptr(q_exp_avg), _ptr(q_exp_avg_sq), o, i, ctypes.byref(hp), int(step), int(flags),
+                              _ptr(Wq), _ptr(dm), _ptr(dq), _stream(stream)), "focus_mx_step")
 
 
 def focus_scales_swizzled_bytes(rows: int, cols: int) -> int:

@@ -306,6 +306,46 @@ int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, flo
                           uint8_t *codes, uint8_t *scales, uint16_t *Xq, focus_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * MXFP4 variant: 32-element blocks with an E8M0 scale and four sub-blocks of
+ * 8, no tensor scale.  "Technische Samenvatting: FOCUS ...", sections
+ * "Probleemstelling" (MXFP4 shares an E8M0 scale per 32 values) and
+ * "Methodologie" items 2-3 (hardware scale x learnable coefficient; sub-blocks
+ * of 8 inside each hardware block of 32); the card's equations give the
+ * structure.  The pages give no MXFP4 formula; the scale follows the OCP
+ * Microscaling rule on the scaled maximum.  Per block b, sub-blocks k = 0..3:
+ *   x_b = fl(A_b * m_b);  S_b = 2^(floor(log2 x_b) - 2), exponent clamped to
+ *   [-127, 127]; S_b = 1 when x_b == 0
+ *   D_k = fl(S_b * sigmoid(q_k));  c_i = E2M1_rne(clamp(fl(w_i/D_k), -6, 6))
+ *   w'_i = bf16(fl(c_i * S_b))
+ *   dm_b = [x_b >= 2^-125] (A_b/4) sum_i g_i (in_i ? c_i - y_i : c_i)
+ *   dq_k = -(1 - sigma_k) S_b sum_{i in k} in_i g_i y_i
+ * Layout: W, dW', W' bf16 [out][in] with in % 32 == 0 (else FOCUS_ERR_SHAPE);
+ * m and its moments float [out][in/32]; q and its moments float [out][in/8]
+ * (q[r][4b+k]); codes [out][in/2] (element 2j in the low nibble); scales
+ * [out][in/32] E8M0 bytes (exponent + 127).  All device pointers, 16-byte
+ * aligned; one tensor per call.
+ * ------------------------------------------------------------------------- */
+
+/* Forward: Wq (nullable) and codes+scales (both or neither; at least one
+ * output). */
+int focus_mx_fwd(const uint16_t *W, const float *m, const float *q, int64_t out, int64_t in, uint16_t *Wq,
+                 uint8_t *codes, uint8_t *scales, focus_stream_t stream);
+
+/* Straight-through backward into dm [out][in/32], dq [out][in/8] (added to
+ * what they hold when accumulate = 1). */
+int focus_mx_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, const float *q, int64_t out,
+                     int64_t in, float *dm, float *dq, int accumulate, focus_stream_t stream);
+
+/* One fused step of one tensor: forward (W' when Wq != NULL), straight-through
+ * backward, AdamW on m (lr_m) and q (lr_q) in place.  flags:
+ * FOCUS_STEP_ACCUMULATE, FOCUS_STEP_WRITE_GRAD (both need dm and dq); other
+ * bits give FOCUS_ERR_VALUE. */
+int focus_mx_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, float *m_exp_avg,
+                  float *m_exp_avg_sq, float *q_exp_avg, float *q_exp_avg_sq, int64_t out, int64_t in,
+                  const focus_hparams *hp, int64_t step, unsigned flags, uint16_t *Wq, float *dm, float *dq,
+                  focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Scale factors for sm_100 block-scaled GEMMs.  The pages deploy the export
  * as plain NVFP4 for standard NVFP4 kernels (card, "What this is"); on sm_100
  * those kernels (cuBLASLt's NVFP4 GEMM, the tcgen05 block-scaled MMA; PyTorch

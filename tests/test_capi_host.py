@@ -190,3 +190,20 @@ def test_swizzle_checks(F):
     assert F.raw_call("focus_scales_swizzle", None, 4, 4, P, 4096, None) == 1
     assert F.raw_call("focus_scales_swizzle", P, 4, 4, U, 4096, None) == 3
     assert F.raw_call("focus_scales_swizzle", P, 4, 4, P, 511, None) == 5        # output too small
+
+
+def test_mx_checks(F):
+    f32 = ctypes.c_float
+    hp = F.focus_hparams(5e-3, 1e-3, 0.9, 0.999, 1e-8, 0.0)
+    assert F.raw_call("focus_mx_fwd", P, P, P, 4, 48, P, None, None, None) == 2      # in % 32
+    assert F.raw_call("focus_mx_fwd", P, P, P, 4, 32, None, None, None, None) == 1   # no output
+    assert F.raw_call("focus_mx_fwd", P, P, P, 4, 32, None, P, None, None) == 1      # codes without scales
+    assert F.raw_call("focus_mx_fwd", U, P, P, 4, 32, P, None, None, None) == 3
+    assert F.raw_call("focus_mx_fwd", P, P, P, 0, 32, P, None, None, None) == 0      # empty
+    assert F.raw_call("focus_mx_ste_bwd", P, P, P, P, 4, 32, P, P, 2, None) == 4     # accumulate flag
+    assert F.raw_call("focus_mx_ste_bwd", P, None, P, P, 4, 32, P, P, 0, None) == 1
+    args = lambda step, flags, dm: (P, P, P, P, P, P, P, P, 4, 32, ctypes.byref(hp), step, flags, None, dm, dm, None)
+    assert F.raw_call("focus_mx_step", *args(0, 0, None)) == 4                       # step < 1
+    assert F.raw_call("focus_mx_step", *args(1, 4, None)) == 4                       # no export flags for MXFP4
+    assert F.raw_call("focus_mx_step", *args(1, 1, None)) == 1                       # accumulate needs dm, dq
+    assert F.raw_call("focus_mx_step", P, P, P, P, P, P, P, P, 4, 32, None, 1, 0, None, None, None, None) == 1

@@ -114,8 +114,11 @@ def _entries(shapes, seed, with_pack=True, warm=False):
         e = Entry(W=W, m=m, q=q, s2=torch.zeros(1, device="cuda"), dWq=dW, Wq=torch.empty_like(W))
         g = torch.Generator(device="cuda").manual_seed(100 + j)
         if warm:
-            e.m_exp_avg = synth.normal(m.shape, 0, 1e-4, g, "cuda"); e.m_exp_avg_sq = synth.normal(m.shape, 0, 1e-4, g, "cuda") ** 2
-            e.q_exp_avg = synth.normal(q.shape, 0, 1e-6, g, "cuda"); e.q_exp_avg_sq = synth.normal(q.shape, 0, 1e-6, g, "cuda") ** 2
+            # moments as a run leaves them: exp_avg_sq >= exp_avg^2
+            e.m_exp_avg = synth.normal(m.shape, 0, 1e-4, g, "cuda")
+            e.m_exp_avg_sq = e.m_exp_avg ** 2 + synth.normal(m.shape, 0, 1e-4, g, "cuda") ** 2
+            e.q_exp_avg = synth.normal(q.shape, 0, 1e-6, g, "cuda")
+            e.q_exp_avg_sq = e.q_exp_avg ** 2 + synth.normal(q.shape, 0, 1e-6, g, "cuda") ** 2
         else:
             e.m_exp_avg = torch.zeros_like(m); e.m_exp_avg_sq = torch.zeros_like(m)
             e.q_exp_avg = torch.zeros_like(q); e.q_exp_avg_sq = torch.zeros_like(q)

@@ -1,0 +1,113 @@
+"""GPU parity of the MXFP4 variant (32-element blocks, E8M0 scale, four
+sub-blocks of 8) against the oracle: forward (W', codes, E8M0 scales) bit for
+bit, straight-through gradients and the fused step (m, q, moments) within
+|gpu - ref| <= 1e-7 + 1e-5 |ref|, on shapes spanning many blocks with ragged
+grid tails, a Llama-sized tensor, and the non-finite flag."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.parity import assert_close, host, host_bits, unpack_codes
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 32), (3, 96), (37, 1056), (128, 2048), (7, 4128), (257, 160)]
+
+
+@pytest.fixture(scope="module")
+def F():
+    from fp4_post_weight_b200 import focus
+    return focus
+
+
+def make(shape, seed, dev="cuda"):
+    g = torch.Generator(device=dev).manual_seed(seed)
+    o, i = shape
+    W = synth.add_outliers(synth.normal_bf16(shape, 0.02, g, dev), 2e-3, 20.0, g)
+    if o * i >= 128:
+        W.view(-1)[:32] = 0                     # a zero block
+        W.view(-1)[32:64] *= 1e-30              # a tiny block: x near the E8M0 clamp
+    m = synth.uniform((o, i // 32), 0.3, 2.5, g, dev)
+    q = synth.normal((o, i // 8), 3.0, 3.0, g, dev)
+    dW = synth.normal_bf16(shape, 1e-3, g, dev)
+    return W, m, q, dW
+
+
+def forward(F, W, m, q):
+    o, i = W.shape
+    Wq = torch.empty_like(W)
+    codes = torch.empty((o, i // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((o, i // 32), dtype=torch.uint8, device="cuda")
+    F.focus_mx_fwd(W, m, q, Wq, codes, scales)
+    return Wq, codes, scales
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_mx_forward(F, shape):
+    W, m, q, _ = make(shape, 30 + shape[0])
+    Wq, codes, scales = forward(F, W, m, q)
+    assert F.focus_get_error() == 0
+    ref = oracle.mx_fwd(host_bits(W), host(m), host(q))
+    np.testing.assert_array_equal(host(scales), ref.scales)
+    np.testing.assert_array_equal(unpack_codes(host(codes)), ref.codes)
+    np.testing.assert_array_equal(host_bits(Wq), ref.Wq)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_mx_backward(F, shape):
+    W, m, q, dW = make(shape, 50 + shape[0])
+    o, i = shape
+    dm = torch.empty((o, i // 32), device="cuda")
+    dq = torch.empty((o, i // 8), device="cuda")
+    F.focus_mx_ste_bwd(W, dW, m, q, dm, dq)
+    rdm, rdq = oracle.mx_ste_bwd(host_bits(W), host_bits(dW), host(m), host(q))
+    assert_close(host(dm), rdm, "dm")
+    assert_close(host(dq), rdq, "dq")
+    F.focus_mx_ste_bwd(W, dW, m, q, dm, dq, accumulate=True)
+    oracle.mx_ste_bwd(host_bits(W), host_bits(dW), host(m), host(q), dm=rdm, dq=rdq)
+    assert_close(host(dm), rdm, "dm (accumulated)")
+    assert_close(host(dq), rdq, "dq (accumulated)")
+    assert F.focus_get_error() == 0
+
+
+@pytest.mark.parametrize("shape,step,warm", [((37, 1056), 1, False), ((128, 2048), 5, True), ((1024, 14336), 1, False)])
+def test_mx_step(F, shape, step, warm):
+    from fp4_post_weight_b200.table import hparams
+    W, m, q, dW = make(shape, 70 + step)
+    g = torch.Generator(device="cuda").manual_seed(9)
+    if warm:
+        # moments as a run leaves them: exp_avg_sq >= exp_avg^2 (else the update is not bounded by ~lr
+        # and amplifies rounding differences in the gradient)
+        v1m, v1q = synth.normal(m.shape, 0, 1e-4, g, "cuda"), synth.normal(q.shape, 0, 1e-6, g, "cuda")
+        mo = [v1m, v1m ** 2 + synth.normal(m.shape, 0, 1e-4, g, "cuda") ** 2,
+              v1q, v1q ** 2 + synth.normal(q.shape, 0, 1e-6, g, "cuda") ** 2]
+    else:
+        mo = [torch.zeros_like(m), torch.zeros_like(m), torch.zeros_like(q), torch.zeros_like(q)]
+    hm, hq, hmo = host(m).copy(), host(q).copy(), [host(x).copy() for x in mo]
+    Wb, Gb = host_bits(W), host_bits(dW)
+    Wq = torch.empty_like(W)
+    dm, dq = torch.empty_like(m), torch.empty_like(q)
+    F.focus_mx_step(W, dW, m, q, *mo, hparams(), step, F.FOCUS_STEP_WRITE_GRAD, Wq, dm, dq)
+    assert F.focus_get_error() == 0
+    ref = oracle.mx_fwd(Wb, hm, hq)
+    np.testing.assert_array_equal(host_bits(Wq), ref.Wq)               # W' of the parameters before the update
+    gm, gq = oracle.mx_ste_bwd(Wb, Gb, hm, hq)
+    assert_close(host(dm), gm, "dm")
+    assert_close(host(dq), gq, "dq")
+    oracle.adamw(hm, gm, hmo[0], hmo[1], 5e-3, step)
+    oracle.adamw(hq, gq, hmo[2], hmo[3], 1e-3, step)
+    assert_close(host(m), hm, "m")
+    assert_close(host(q), hq, "q")
+    for name, t, r in zip(("m exp_avg", "m exp_avg_sq", "q exp_avg", "q exp_avg_sq"), mo, hmo):
+        assert_close(host(t), r, name)
+
+
+def test_mx_nonfinite_sets_flag(F):
+    W, m, q, _ = make((4, 64), 3)
+    W[2, 5] = float("nan")
+    assert F.focus_get_error() == 0
+    forward(F, W, m, q)
+    assert F.focus_get_error() == 7
+    assert F.focus_get_error() == 0
