@@ -580,7 +580,7 @@ struct Layout {
 
 template <int KIND> struct Depth;
 template <> struct Depth<KIND_FWD> { static constexpr int STAGES = 6, MIN_CTAS = 3; };
-template <> struct Depth<KIND_BWD> { static constexpr int STAGES = 4, MIN_CTAS = 2; };
+template <> struct Depth<KIND_BWD> { static constexpr int STAGES = 3, MIN_CTAS = 3; };
 template <> struct Depth<KIND_STEP> { static constexpr int STAGES = 2, MIN_CTAS = 3; };
 template <> struct Depth<KIND_F46> { static constexpr int STAGES = 8, MIN_CTAS = 3; };
 
