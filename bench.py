@@ -48,10 +48,16 @@ TRAFFIC_RECORD = "profiles/focus_step_fused_export_llama8b_2layers.md"
 
 
 def kernel_source_hash() -> str:
+    """Hash of the code (comments and whitespace removed) of the kernel sources:
+    the recorded DRAM traffic is valid while it is unchanged."""
+    import re
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p)) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        h.update(re.sub(r"\s+", "", src).encode())
     return h.hexdigest()[:16]
 
 

@@ -18,19 +18,25 @@
 // end of a tensor) is read by the consumers straight from global memory.  The
 // prefetch depth is therefore set by the number of stages, not by registers.
 //
-// Inside a tile each 16-block is owned by a pair of adjacent consumer lanes,
-// lane parity k = sub-block k: a lane takes its 8 weights (16 bytes) of W and
-// of dW', its q and q moments, and (with its partner) the block's m.  The block
-// maximum and the m-gradient are combined across the pair with one shuffle
-// each.  Outputs go from registers straight to global memory, coalesced: a warp
-// writes 512 contiguous bytes of W', 128 of q.
+// Inside a tile each 16-block is owned by one consumer thread: it takes the
+// block's 32 bytes of W (and of dW') from the stage, its m, its two q and
+// their moments, and does the block's work (A_b, x_b, S_b, the m-gradient and
+// its AdamW update) once.  Outputs go from registers straight to global
+// memory: W' as two 16-byte streaming stores per block, the codes as 8 bytes.
+//
+// Besides the FOCUS kinds (forward, backward, fused step) the same pipeline
+// runs FourOverSix round to nearest (KIND_F46, W alone is staged); the
+// per-token FourOverSix kernel, the scale relayout and the standalone AdamW
+// below are plain grid-stride kernels.
 //
 // Exactness.  Forward decisions (S_b, codes, w') are taken in binary32 with
 // explicit round-to-nearest intrinsics (__fmul_rn / __fdiv_rn cannot be fused
 // or reassociated by the compiler); sigmoid is evaluated in binary64 and
 // rounded once.  The hardware conversions cvt.rn.satfinite.{e4m3x2,e2m1x2}.f32
 // round to nearest even; the E4M3 input is always inside [2^-6, 448], where
-// every E4M3 value is normal.
+// every E4M3 value is normal.  The sigmoid is evaluated with few binary64
+// operations and rounded only when the rounding is certain (focus_device.cuh);
+// the result equals the direct evaluation bit for bit.
 #pragma once
 
 #include <cstdint>
