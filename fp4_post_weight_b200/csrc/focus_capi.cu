@@ -58,7 +58,7 @@ int device_info(DeviceInfo **out) {
                              (int)stage_smem_bytes<KIND_F46>());
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_f46, pipe_kernel<KIND_F46>, CTA_THREADS,
                                                       stage_smem_bytes<KIND_F46>());
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows, f46_rows_kernel, THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows, f46_rows_kernel, ROW_THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_amax, amax_tiles_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_adam, adamw_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[0], mx_kernel<KIND_FWD>, THREADS, 0);
@@ -531,7 +531,7 @@ int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, flo
     DeviceInfo *di;
     if ((rc = device_info(&di))) return rc;
     const int64_t grid = grid_for(tokens, di->sms, di->occ_rows);
-    f46_rows_kernel<<<(unsigned)grid, THREADS, 0, (cudaStream_t)stream>>>(X, tokens, hidden, token_scales, codes,
+    f46_rows_kernel<<<(unsigned)grid, ROW_THREADS, 0, (cudaStream_t)stream>>>(X, tokens, hidden, token_scales, codes,
                                                                          scales, Xq);
     return launch_status();
 }
