@@ -207,3 +207,26 @@ def test_mx_checks(F):
     assert F.raw_call("focus_mx_step", *args(1, 4, None)) == 4                       # no export flags for MXFP4
     assert F.raw_call("focus_mx_step", *args(1, 1, None)) == 1                       # accumulate needs dm, dq
     assert F.raw_call("focus_mx_step", P, P, P, P, P, P, P, P, 4, 32, None, 1, 0, None, None, None, None) == 1
+
+
+def test_maximum_tensor_size(F):
+    """A tensor of more than 2^31 - 2^16 blocks is rejected on the host (block
+    indices inside a tensor stay 32-bit in the kernels); nothing is launched."""
+    f32 = ctypes.c_float
+    rows = 32768
+    in16 = 16 * 65536                 # 65,536 16-blocks per row: 2^31 blocks in all
+    assert _c(F, "focus_fwd", P, P, P, f32(1.0), rows, in16, P, None) == 2
+    assert _c(F, "focus_ste_bwd", P, P, P, P, f32(1.0), rows, in16, P, P, 0, None) == 2
+    assert _c(F, "focus_pack_nvfp4", P, P, P, f32(1.0), rows, in16, P, P, P, None) == 2
+    assert _c(F, "focus_s2", P, rows, in16, P, P, 1 << 40, None) == 2
+    assert F.focus_s2_workspace_bytes(rows, in16) == 0
+    assert F.raw_call("focus_fouroversix_weight", P, rows, in16, f32(1.0), P, P, None, None) == 2
+    assert F.raw_call("focus_fouroversix_act", P, rows, in16, P, P, P, None, None) == 2
+    in32 = 32 * 65536                 # MXFP4: 65,536 32-blocks per row
+    assert F.raw_call("focus_mx_fwd", P, P, P, rows, in32, P, None, None, None) == 2
+    descs = (F.focus_tensor_desc * 1)()
+    descs[0].W = descs[0].m = descs[0].q = descs[0].s2 = P
+    descs[0].out, descs[0].in_ = rows, in16
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, 0)
+    assert e.value.status == 2
