@@ -401,11 +401,25 @@ def measure_next_rows(ents, dev, N, peaks, world):
     return out
 
 
+def host_budget_bytes(world: int) -> int:
+    """Pinned host memory one rank may take for the e2e leg: 60% of the memory
+    the host has available, shared by the ranks."""
+    try:
+        with open("/proc/meminfo") as f:
+            kb = next(int(l.split()[1]) for l in f if l.startswith("MemAvailable:"))
+        avail = kb * 1024
+    except Exception:
+        avail = 64 << 30
+    return int(0.6 * avail / max(world, 1))
+
+
 def run_e2e(args, ents, N, world, dev):
     """The same step through the C ABI with host buffers: per step every input
     (W, dW', m, q, moments) is copied from pinned host memory and every output
     (W', m, q, moments, codes, scales, s2) is copied back, tensor by tensor on
-    two copy streams overlapping the compute stream."""
+    two copy streams overlapping the compute stream.  It runs on as many whole
+    decoder layers as the host's memory holds for every rank (all 32 on one
+    B200 machine: 77 GB pinned); the rate is per weight, so it is the same metric."""
     import torch
 
     from fp4_post_weight_b200 import dist as D
@@ -413,6 +427,12 @@ def run_e2e(args, ents, N, world, dev):
     from fp4_post_weight_b200.table import FocusTable, hparams
     ins = ("W", "dWq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq")
     outs = ("Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq", "codes", "scales", "s2")
+    names = set(ins) | set(outs)
+    per_layer = sum(getattr(e, n).numel() * getattr(e, n).element_size() for e in ents[:7] for n in names)
+    layers = max(1, min(len(ents) // 7, host_budget_bytes(world) // per_layer))
+    layers = int(D.min_over_ranks(layers)) if world > 1 else layers
+    ents = ents[:7 * layers]
+    N = sum(e.W.numel() for e in ents)
     hosts = []
     for e in ents:
         h = {}
@@ -461,7 +481,8 @@ def run_e2e(args, ents, N, world, dev):
     ms = D.max_over_ranks(s.elapsed_time(e)) / steps
     del hosts
     return {"value": round(N * world / (ms * 1e-3) / 1e9, 3), "unit": "Gelem/s", "h2d_bytes_per_step": bi,
-            "d2h_bytes_per_step": bo, "ms_per_step": round(ms, 2), "steps": steps}
+            "d2h_bytes_per_step": bo, "ms_per_step": round(ms, 2), "steps": steps, "layers": layers,
+            "weights_per_rank": N}
 
 
 # ---------------------------------------------------------------------------

@@ -47,6 +47,17 @@ def max_over_ranks(x: float) -> float:
     return float(t.item())
 
 
+def min_over_ranks(x: float) -> float:
+    """The min of a per-rank number over all ranks (a size every rank can afford)."""
+    d = _dist()
+    if d is None or d.get_world_size() == 1:
+        return float(x)
+    dev = torch.device("cuda", torch.cuda.current_device()) if d.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    d.all_reduce(t, op=d.ReduceOp.MIN)
+    return float(t.item())
+
+
 def shard(sizes, world: int, rank: int):
     """Indices of the tensors rank `rank` owns when one model is split over
     `world` GPUs: greedy by size (largest first onto the least loaded rank),

@@ -29,6 +29,8 @@ def _worker(rank, world, port, q):
         assert (w, r) == (world, rank)
         D.barrier()
         t = D.max_over_ranks(10.0 + rank * 3.5)
+        lo = D.min_over_ranks(10.0 + rank * 3.5)
+        assert lo == 10.0                          # the size every rank can afford
         # each rank's model is seeded apart from the others'
         seeds = [D.seed_base(r) + j for j in range(224)]
         g = synth.llama_8b_tensor(0, (16, 64), "cpu", seed_base=D.seed_base(r))
@@ -70,5 +72,6 @@ def test_two_gloo_ranks():
 
 def test_single_process_defaults():
     assert D.max_over_ranks(3.0) == 3.0
+    assert D.min_over_ranks(3.0) == 3.0
     D.barrier()
     assert D.shard([5, 1, 1], 1, 0) == [0, 1, 2]
