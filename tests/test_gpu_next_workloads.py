@@ -1,0 +1,102 @@
+"""GPU parity of the later rows at the benchmark's sizes, in the launch
+configurations bench.py times:
+
+* FourOverSix weights over all 224 Llama-3.1-8B linears in one multi-tensor
+  launch (codes, scales and W'), layer 0 in full and a 1/64 row sample of
+  every other tensor, bit for bit against the oracle with each tensor's s2;
+* FourOverSix with one scale per token over one decoder layer's linear inputs
+  for a micro-batch of 4096 tokens (four launches), in full;
+* the MXFP4 fused step, one launch per tensor, on layer 0 of the 8B shapes
+  with the benchmark's parameters (m = 1, q = 6, zero moments), a 1/16 row
+  sample against the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.parity import assert_close, host, host_bits, unpack_codes
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def F():
+    from fp4_post_weight_b200 import focus
+    return focus
+
+
+def _rows(out, stride):
+    r = list(range(0, out, stride))
+    if r[-1] != out - 1:
+        r.append(out - 1)
+    return torch.tensor(r, device="cuda")
+
+
+def test_fouroversix_weights_llama_8b_one_launch(F):
+    from fp4_post_weight_b200.table import Entry, FocusTable, PURPOSE_FOUROVERSIX
+    ents, samples = [], []
+    for j, (_, (o, i)) in enumerate(synth.LLAMA_8B.tensors()):
+        t = synth.llama_8b_tensor(j, (o, i), "cuda", with_grad=False)
+        ents.append(Entry(W=t.W, m=None, q=None, s2=torch.zeros(1, device="cuda"),
+                          codes=torch.empty((o, i // 2), dtype=torch.uint8, device="cuda"),
+                          scales=torch.empty((o, i // 16), dtype=torch.uint8, device="cuda"),
+                          Wq=torch.empty_like(t.W)))
+        samples.append(None if j < 7 else _rows(o, 64))
+    tab = FocusTable(ents, PURPOSE_FOUROVERSIX)
+    tab.s2()
+    tab.fouroversix()
+    assert F.focus_get_error() == 0
+    checked = four = 0
+    for e, rows in zip(ents, samples):
+        s2 = oracle.s2(host_bits(e.W))
+        assert host(e.s2)[0] == s2
+        sel = (lambda x: x) if rows is None else (lambda x: x[rows])
+        ref = oracle.fouroversix(host_bits(sel(e.W)), s2)
+        np.testing.assert_array_equal(host(sel(e.scales)), ref.scales)
+        np.testing.assert_array_equal(unpack_codes(host(sel(e.codes))), ref.codes)
+        np.testing.assert_array_equal(host_bits(sel(e.Wq)), ref.Xq)
+        checked += ref.codes.size
+        four += int(ref.four.sum())
+    print(f"FourOverSix 8B: {checked} weights checked, target 4 in {four} blocks")
+
+
+def test_fouroversix_activations_one_layer_4096_tokens(F):
+    for j, h in enumerate((4096, 4096, 4096, 14336)):
+        X = synth.activations(4096, h, "cuda", seed=50 + j)
+        ts = torch.empty(4096, device="cuda")
+        codes = torch.empty((4096, h // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((4096, h // 16), dtype=torch.uint8, device="cuda")
+        Xq = torch.empty_like(X)
+        F.focus_fouroversix_act(X, ts, codes, scales, Xq)
+        assert F.focus_get_error() == 0
+        ref = oracle.fouroversix(host_bits(X))
+        np.testing.assert_array_equal(host(ts), ref.row_scales)
+        np.testing.assert_array_equal(host(scales), ref.scales)
+        np.testing.assert_array_equal(unpack_codes(host(codes)), ref.codes)
+        np.testing.assert_array_equal(host_bits(Xq), ref.Xq)
+
+
+def test_mx_step_llama_8b_layer0_sampled(F):
+    from fp4_post_weight_b200.table import hparams
+    for j, (_, (o, i)) in enumerate(synth.LLAMA_8B.tensors()[:7]):
+        t = synth.llama_8b_tensor(j, (o, i), "cuda")
+        m = torch.ones((o, i // 32), device="cuda")
+        q = torch.full((o, i // 8), 6.0, device="cuda")
+        mo = [torch.zeros_like(m), torch.zeros_like(m), torch.zeros_like(q), torch.zeros_like(q)]
+        rows = _rows(o, 16)
+        Wb, Gb = host_bits(t.W[rows]), host_bits(t.dWq[rows])
+        hm, hq = host(m[rows]).copy(), host(q[rows]).copy()
+        hmo = [host(x[rows]).copy() for x in mo]
+        Wq = torch.empty_like(t.W)
+        F.focus_mx_step(t.W, t.dWq, m, q, *mo, hparams(), 1, 0, Wq)
+        assert F.focus_get_error() == 0
+        np.testing.assert_array_equal(host_bits(Wq[rows]), oracle.mx_fwd(Wb, hm, hq).Wq)
+        gm, gq = oracle.mx_ste_bwd(Wb, Gb, hm, hq)
+        oracle.adamw(hm, gm, hmo[0], hmo[1], 5e-3, 1)
+        oracle.adamw(hq, gq, hmo[2], hmo[3], 1e-3, 1)
+        assert_close(host(m[rows]), hm, "m")
+        assert_close(host(q[rows]), hq, "q")
+        for name, x, r in zip(("m exp_avg", "m exp_avg_sq", "q exp_avg", "q exp_avg_sq"), mo, hmo):
+            assert_close(host(x[rows]), r, name)
