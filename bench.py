@@ -275,7 +275,7 @@ def run_ours(args, world, rank, local):
                 "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "next_rows": rows,
                 "gpu_launches": 3 * args.steps, "clocks": clk,
                 "kernel_ms": {"fused_step": round(step_kernel_ms, 4), "fused_step_min": round(min(kms), 4),
-                              "fused_step_max": round(max(kms), 4)}}
+                              "fused_step_max": round(max(kms), 4), "fused_step_each": [round(x, 3) for x in kms]}}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -313,6 +313,8 @@ def measure_next_rows(ents, dev, N, peaks, world):
       * a calibration step over four micro-batches: three table backward passes
         (the first overwriting dm/dq, then accumulating) and the fused step
         with FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WQ_UPDATED;
+      * the same step unfused (forward, backward, standalone AdamW: 15.5 B per
+        weight in 450 launches), for what the fusion buys;
       * the MXFP4 variant's fused step over the same 224 weights (one launch per
         tensor; reads W, dW', m, q and moments, writes W', m, q and moments:
         9.75 B per weight)."""
@@ -375,6 +377,26 @@ def measure_next_rows(ents, dev, N, peaks, world):
                            **_roof(6.25 * N, t_b1, peak)},
         "step_accumulate_wq_updated": {"kernel": "pipe_kernel<KIND_STEP, true>", "bytes_per_weight": 11.25,
                                        **_roof(11.25 * N, t_st, peak)}}
+    # the same step unfused: table forward (W'), table backward, then the
+    # standalone AdamW on every tensor's m and q (448 launches)
+    for e in ents:
+        e.dm.zero_(); e.dq.zero_()
+    cnt_u = [200]
+
+    def unfused():
+        cnt_u[0] += 1
+        tab.fwd()
+        tab.bwd(accumulate=False)
+        for e in ents:
+            F.focus_adamw_step(e.m, e.dm, e.m_exp_avg, e.m_exp_avg_sq, hp.lr_m, cnt_u[0])
+            F.focus_adamw_step(e.q, e.dq, e.q_exp_avg, e.q_exp_avg_sq, hp.lr_q, cnt_u[0])
+    t_f = _timed(tab.fwd, stream)
+    t_u = _timed(unfused, stream)
+    out["unfused_step_llama8b"] = {
+        "kernels": "pipe_kernel<KIND_FWD> + pipe_kernel<KIND_BWD> + adamw_kernel x448", "bytes_per_weight": 15.5,
+        "ms": round(t_u, 3), "Gelem_s": round(N * world / (t_u * 1e-3) / 1e9, 2),
+        "fwd": {"kernel": "pipe_kernel<KIND_FWD>", "bytes_per_weight": 4.75, **_roof(4.75 * N, t_f, peak)},
+        "vs_fused_step_without_export": "the fused step moves 10.5 B per weight in one launch"}
     for e in ents:
         e.dm = e.dq = None
     del tab
