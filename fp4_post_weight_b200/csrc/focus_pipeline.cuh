@@ -61,13 +61,14 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Waits until the phase of parity `parity` of the barrier has completed.
-// Returns false if that does not happen within the limits.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Returns false if that does not happen within `limit_ns` of wall time (or
+// WAIT_MAX_ITERS polls).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = WAIT_LIMIT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1; i < WAIT_MAX_ITERS; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0 && global_ns() - t0 > WAIT_LIMIT_NS) return false;
+        if ((i & 63u) == 0 && global_ns() - t0 > limit_ns) return false;
     }
     return false;
 }

@@ -14,6 +14,8 @@
   __frcp_rn for every significand; the twice-corrected quotient used for the
   scaled block maximum equals __fdiv_rn (every divisor significand for 1024
   pseudo-random numerators, and 2^30 pseudo-random pairs).
+* The pipeline's bounded wait gives up (and reports) on a barrier nothing
+  completes, and succeeds on one that is completed.
 * The forward's sigmoid (own e^x, a rounding-certainty test, sigmoid_rn where
   it cannot decide) equals sigmoid_rn for EVERY binary32 logit with
   |q| <= 100; the export's sigmoid of an updated logit (a Taylor step from the
@@ -48,6 +50,7 @@ def lib():
     L.check_div_full.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong),
                                  ctypes.POINTER(ctypes.c_float)]
     L.e2m1_raw_bytes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    L.check_wait.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
     L.check_sigmoid_fast.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_float)]
     L.check_sigmoid_step.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong),
                                      ctypes.POINTER(ctypes.c_float)]
@@ -117,3 +120,16 @@ def test_sigmoid_step_of_updated_logit(lib, seed):
     assert c[1] == 1 << 28
     assert c[0] == 0, f"{c[0]} differ, e.g. q0={ex[0]!r} q1={ex[1]!r} got {ex[2]!r} want {ex[3]!r}"
     assert c[2] > 0.5 * c[1]            # the Taylor step decides most roundings
+
+
+def test_bounded_wait_runs_out_and_reports(lib):
+    """Failure detection without a GPU fault: a pipeline wait on a barrier that
+    nothing completes gives up after its limit (2 ms here; 2 s in the kernels)
+    and returns false -- the kernels then set the timeout flag, which
+    focus_get_error reports as FOCUS_ERR_DEVICE_TIMEOUT -- while a wait on a
+    completed barrier returns true.  Nothing hangs or traps."""
+    res = (ctypes.c_ulonglong * 3)()
+    assert lib.check_wait(2_000_000, res) == 0
+    assert res[0] == 0, "the wait on a barrier nothing completes did not give up"
+    assert 2_000_000 <= res[1] < 1_000_000_000, f"gave up after {res[1]} ns"
+    assert res[2] == 1, "the wait on a completed barrier failed"
