@@ -422,8 +422,8 @@ int focus_s2_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tile
     return launch_s2(a, static_cast<uint32_t *>(ws_dev), nullptr, n, (cudaStream_t)stream);
 }
 
-int focus_step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, const focus_hparams *hp,
-                     int64_t step, unsigned flags, focus_stream_t stream) {
+static int step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, const focus_hparams *hp,
+                      int64_t step, unsigned flags, uint32_t *amax_ws, focus_stream_t stream) {
     if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
     if (!hp) return FOCUS_ERR_NULL;
     int rc = check_hyper(hp->lr_m, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
@@ -443,9 +443,32 @@ int focus_step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_ti
     a.accumulate = (flags & FOCUS_STEP_ACCUMULATE) ? 1 : 0;
     a.write_grad = (flags & FOCUS_STEP_WRITE_GRAD) ? 1 : 0;
     a.pack_updated = (flags & FOCUS_STEP_PACK_UPDATED) ? 1 : 0;
+    a.amax_ws = amax_ws;
     a.hp = make_hyper(hp->lr_m, hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
     if (flags & FOCUS_STEP_WQ_UPDATED) return launch_on<KIND_STEP, true>(a, (cudaStream_t)stream);
     return launch_on<KIND_STEP>(a, (cudaStream_t)stream);
+}
+
+int focus_step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, const focus_hparams *hp,
+                     int64_t step, unsigned flags, focus_stream_t stream) {
+    return step_fused(descs_dev, n, total_tiles, hp, step, flags, nullptr, stream);
+}
+
+int focus_step_fused_amax(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, const focus_hparams *hp,
+                          int64_t step, unsigned flags, uint32_t *amax_ws, focus_stream_t stream) {
+    if (n > 0 && !amax_ws) return FOCUS_ERR_NULL;
+    if (!aligned16(amax_ws)) return FOCUS_ERR_ALIGN;
+    return step_fused(descs_dev, n, total_tiles, hp, step, flags, amax_ws, stream);
+}
+
+int focus_s2_from_amax(const focus_tensor_desc *descs_dev, int n, uint32_t *amax_ws, focus_stream_t stream) {
+    if (n < 0) return FOCUS_ERR_VALUE;
+    if (n == 0) return FOCUS_OK;
+    if (!descs_dev || !amax_ws) return FOCUS_ERR_NULL;
+    if (!aligned16(descs_dev) || !aligned16(amax_ws)) return FOCUS_ERR_ALIGN;
+    s2_from_amax_kernel<<<(unsigned)((n + THREADS - 1) / THREADS), THREADS, 0, (cudaStream_t)stream>>>(descs_dev, n,
+                                                                                                      amax_ws);
+    return launch_status();
 }
 
 int focus_fwd_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {

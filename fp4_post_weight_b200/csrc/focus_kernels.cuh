@@ -79,6 +79,7 @@ struct Args {
     int accumulate;                  // bwd: add into dm/dq; step: FOCUS_STEP_ACCUMULATE
     int write_grad;                  // step: FOCUS_STEP_WRITE_GRAD
     int pack_updated;                // step: FOCUS_STEP_PACK_UPDATED
+    uint32_t *amax_ws;               // step: per-tensor max |w| (bf16 magnitude bits) for the next s2, or nullptr
     Hyper hp;
 };
 
@@ -430,6 +431,14 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
     const uint32_t abits = max(am & 0xffffu, am >> 16);
     const float A = __uint_as_float(abits << 16);
     const bool bad = B.valid && (abits >= 0x7f80u || !finitef(B.m) || !finitef(B.q[0]) || !finitef(B.q[1]));
+    // The tensor maximum for the next step's s2 (focus_step_fused_amax): the warp's
+    // maximum of the block maxima (the blocks past a ragged end have w = 0) into the
+    // stage record in shared memory; the producer folds the stage maxima of a tensor
+    // and writes them out (T is the stage record here).
+    if (KIND == KIND_STEP && a.amax_ws != nullptr) {
+        const uint32_t wm = __reduce_max_sync(FULL, abits);
+        if ((threadIdx.x & 31) == 0 && wm != 0u) atomicMax(const_cast<uint32_t *>(&T.amax), wm);
+    }
 
     // S_b = e4m3(clamp(fl(fl(A*m)/fl(6*s2)), 2^-6, 448)), scale 1 when the scaled max is 0
     const float x = scaled_max(T, A, B.m);
@@ -610,6 +619,28 @@ struct StageInfo {
     float den4;        // FourOverSix: fl(4*s2), its reciprocal, both quotients exact by reciprocal
     float rden4;
     uint32_t den46_ok;
+    uint32_t tensor;   // index of the tile's tensor in the table
+    uint32_t amax;     // fused step with s2 for the next step: max |w| bits of the tile (consumers' smem atomics)
+};
+
+// The running tensor maximum the producer keeps for focus_step_fused_amax: the
+// stage maxima of consecutive tiles of one tensor are folded in a register and
+// written with one global atomic when the tensor changes (about one atomic per
+// CTA and tensor, instead of one per warp and tile, which contended at L2).
+struct AmaxFold {
+    uint32_t tensor = 0xffffffffu;
+    uint32_t v = 0u;
+    __device__ __forceinline__ void add(uint32_t *ws, uint32_t t, uint32_t x) {
+        if (t != tensor) {
+            flush(ws);
+            tensor = t;
+            v = 0u;
+        }
+        v = max(v, x);
+    }
+    __device__ __forceinline__ void flush(uint32_t *ws) {
+        if (tensor != 0xffffffffu && v != 0u) atomicMax(ws + tensor, v);
+    }
 };
 
 // A block's inputs from a staged tile (local block lb of the tile).
@@ -677,15 +708,22 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
     uint32_t pending = 0;             // stages whose last use was filled by bulk copies
     uint32_t pending_parity = 0;      // and the parity of that use
     uint32_t it = 0;
+    bool timed_out = false;
+    AmaxFold fold;
     for (int64_t tile = blockIdx.x; tile < a.total_tiles; tile += gridDim.x, ++it) {
         const uint32_t st = it % S;
         const uint32_t ph = (it / S) & 1u;
         if (!mbar_wait(smem_u32(&empty[st]), ph ^ 1u)) {
             atomicOr(&g_error_flags, 8u);
+            timed_out = true;
             break;
         }
         pending &= ~(1u << st);       // the consumers released it: its copies have landed
         StageInfo &inf = info[st];
+        if (KIND == KIND_STEP && a.amax_ws != nullptr) {
+            if (it >= (uint32_t)S) fold.add(a.amax_ws, inf.tensor, inf.amax);   // the stage's previous tile
+            inf.amax = 0u;
+        }
         const bool found = seek_tensor(a, tile, t, T, have);
         const uint32_t first = found ? (uint32_t)(tile - T.d.tile_begin) * TILE_BLOCKS : 0u;
         const int64_t left = T.nblk - (int64_t)first;
@@ -710,6 +748,7 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
         inf.den4 = T.den4;
         inf.rden4 = T.rden4;
         inf.den46_ok = T.den46_ok ? 1u : 0u;
+        inf.tensor = (uint32_t)t;
         inf.first = first;
         inf.nb = nb;
         inf.mode = mode;
@@ -741,6 +780,19 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
         } else {
             mbar_arrive(bar);
         }
+    }
+    // The tensor maxima of the last uses of the stages: wait (bounded) until the
+    // consumers have released them, fold them in and write the running maximum.
+    if (KIND == KIND_STEP && a.amax_ws != nullptr && !timed_out) {
+        for (uint32_t j = it > (uint32_t)S ? it - (uint32_t)S : 0u; j < it; ++j) {
+            const uint32_t st = j % S;
+            if (!mbar_wait(smem_u32(&empty[st]), (j / S) & 1u)) {
+                atomicOr(&g_error_flags, 8u);
+                break;
+            }
+            fold.add(a.amax_ws, info[st].tensor, info[st].amax);
+        }
+        fold.flush(a.amax_ws);
     }
     // Before the CTA may exit, every bulk copy it issued must have landed (normally
     // the consumers already waited for all of them; this matters after a timeout).
@@ -968,6 +1020,19 @@ __global__ void __launch_bounds__(THREADS) scales_swizzle_kernel(const uint8_t *
         }
         out[wi] = v;
     }
+}
+
+// s2 = fl(A / 2688) of every tensor from the maxima a step accumulated
+// (focus_step_fused_amax), one thread per tensor; the workspace word is
+// cleared for the next step.
+__global__ void __launch_bounds__(THREADS) s2_from_amax_kernel(const focus_tensor_desc *table, int n,
+                                                               uint32_t *amax_ws) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n) return;
+    const uint32_t v = amax_ws[t];
+    if (v >= 0x7f80u) atomicOr(&g_error_flags, 1u);
+    *table[t].s2 = __fdiv_rn(__uint_as_float(v << 16), 2688.0f);
+    amax_ws[t] = 0u;
 }
 
 // ---------------------------------------------------------------------------

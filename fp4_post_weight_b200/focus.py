@@ -61,6 +61,8 @@ _SIGS = {
     "focus_s2_multi": ([_P, _I, _I64, _P, _SZ, _P], _I),
     "focus_step_fused": ([_P, _I, _I64, ctypes.POINTER(focus_hparams), _I64, ctypes.c_uint, _P], _I),
     "focus_pack_multi": ([_P, _I, _I64, _P], _I),
+    "focus_step_fused_amax": ([_P, _I, _I64, ctypes.POINTER(focus_hparams), _I64, ctypes.c_uint, _P, _P], _I),
+    "focus_s2_from_amax": ([_P, _I, _P, _P], _I),
     "focus_fwd_multi": ([_P, _I, _I64, _P], _I),
     "focus_ste_bwd_multi": ([_P, _I, _I64, _I, _P], _I),
     "focus_fouroversix_weight": ([_P, _I64, _I64, _F, _P, _P, _P, _P], _I),
@@ -217,6 +219,18 @@ def focus_step_fused(table_dev, n: int, total_tiles: int, hp: focus_hparams, ste
                      stream=None):
     _check(_lib.focus_step_fused(_ptr(table_dev), int(n), int(total_tiles), ctypes.byref(hp), int(step),
                                  int(flags), _stream(stream)), "focus_step_fused")
+
+
+def focus_step_fused_amax(table_dev, n: int, total_tiles: int, hp: focus_hparams, step: int, amax_ws, flags: int = 0,
+                          stream=None):
+    """focus_step_fused that also accumulates every tensor's max |w| into amax_ws (n int32 words)."""
+    _check(_lib.focus_step_fused_amax(_ptr(table_dev), int(n), int(total_tiles), ctypes.byref(hp), int(step),
+                                      int(flags), _ptr(amax_ws), _stream(stream)), "focus_step_fused_amax")
+
+
+def focus_s2_from_amax(table_dev, n: int, amax_ws, stream=None):
+    """desc.s2 = fl(max|w| / 2688) from a step's accumulated maxima; clears amax_ws."""
+    _check(_lib.focus_s2_from_amax(_ptr(table_dev), int(n), _ptr(amax_ws), _stream(stream)), "focus_s2_from_amax")
 
 
 def focus_fwd_multi(table_dev, n: int, total_tiles: int, stream=None):

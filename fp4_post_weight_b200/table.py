@@ -60,6 +60,7 @@ class FocusTable:
         raw = torch.frombuffer(bytearray(bytes(descs)), dtype=torch.uint8)
         self.dev = raw.to(dev)                  # 256-byte aligned device copy
         self._ws = None
+        self._amax = None
 
     def s2(self, stream=None):
         need = F.focus_s2_multi_workspace_bytes(self.total_tiles)
@@ -70,6 +71,16 @@ class FocusTable:
     def step(self, step: int, hp: F.focus_hparams | None = None, flags: int = 0, stream=None):
         hp = hp or hparams()
         F.focus_step_fused(self.dev, self.n, self.total_tiles, hp, step, flags, stream)
+
+    def step_s2(self, step: int, hp: F.focus_hparams | None = None, flags: int = 0, stream=None):
+        """The fused step that also leaves each tensor's s2 for the next step (two launches:
+        the step, which reduces the block maxima it computes into the tensor maxima, and
+        the one that turns them into s2).  The step reads the current desc.s2."""
+        hp = hp or hparams()
+        if self._amax is None:
+            self._amax = torch.zeros(max(self.n, 4), dtype=torch.int32, device=self.dev.device)
+        F.focus_step_fused_amax(self.dev, self.n, self.total_tiles, hp, step, self._amax, flags, stream)
+        F.focus_s2_from_amax(self.dev, self.n, self._amax, stream)
 
     def pack(self, stream=None):
         F.focus_pack_multi(self.dev, self.n, self.total_tiles, stream)

@@ -246,6 +246,21 @@ int focus_s2_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t to
 int focus_step_fused(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
                      const focus_hparams *hp, int64_t step, unsigned flags, focus_stream_t stream);
 
+/* The same step, also computing each entry's s2 for the next step: the step
+ * reduces the block maxima it computes anyway into the tensor's max |w|
+ * (bf16 magnitude bits, atomically maximised into amax_ws[i] for entry i), and
+ * focus_s2_from_amax then writes desc.s2 = fl(max / 2688) -- card, field
+ * table, row s2 -- and clears amax_ws.  W is frozen, so this is the s2 a
+ * separate focus_s2_multi pass would compute, without a second read of W.
+ *   amax_ws  n_tensors uint32 words, device, 16-byte aligned; zero before the
+ *            first step (focus_s2_from_amax leaves it zero for the next one).
+ * The step itself reads desc.s2 as focus_step_fused does (the previous value,
+ * or one from focus_s2_multi before the first step). */
+int focus_step_fused_amax(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
+                          const focus_hparams *hp, int64_t step, unsigned flags, uint32_t *amax_ws,
+                          focus_stream_t stream);
+int focus_s2_from_amax(const focus_tensor_desc *descs_dev, int n_tensors, uint32_t *amax_ws, focus_stream_t stream);
+
 /* Forward of every entry in one launch: W' (desc.Wq), and the codes and
  * scales when present.  Card, "What this is": the S_b, c_i and w'_i
  * equations. */

@@ -230,3 +230,14 @@ def test_maximum_tensor_size(F):
     with pytest.raises(F.FocusError) as e:
         F.focus_table_prepare(descs, 0)
     assert e.value.status == 2
+
+
+def test_step_amax_checks(F):
+    hp = F.focus_hparams(5e-3, 1e-3, 0.9, 0.999, 1e-8, 0.0)
+    assert F.raw_call("focus_step_fused_amax", P, 1, 1, ctypes.byref(hp), 1, 0, None, None) == 1   # no workspace
+    assert F.raw_call("focus_step_fused_amax", P, 1, 1, ctypes.byref(hp), 1, 0, U, None) == 3
+    assert F.raw_call("focus_step_fused_amax", P, 1, 1, ctypes.byref(hp), 0, 0, P, None) == 4      # step < 1
+    assert F.raw_call("focus_s2_from_amax", P, -1, P, None) == 4
+    assert F.raw_call("focus_s2_from_amax", P, 1, None, None) == 1
+    assert F.raw_call("focus_s2_from_amax", U, 1, P, None) == 3
+    assert F.raw_call("focus_s2_from_amax", P, 0, P, None) == 0

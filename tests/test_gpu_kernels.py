@@ -399,3 +399,27 @@ def test_micro_batch_step(F):
     assert F.focus_get_error() == 0
     for e, w in zip(ents, wq_next):
         assert torch.equal(e.Wq.view(torch.int16), w.view(torch.int16))
+
+
+def test_step_with_s2_for_the_next_step(F):
+    """focus_step_fused_amax + focus_s2_from_amax: the step's outputs are bit for
+    bit those of focus_step_fused, and afterwards every desc.s2 equals the oracle's
+    s2 of its W (W is frozen), so the next step reads the same s2 a separate
+    focus_s2_multi pass would give; two steps in a row agree with the plain path."""
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    shapes = SHAPES + [(0, 32)]
+    ea, eb = _entries(shapes, 95), _entries(shapes, 95)
+    ta, tb = FocusTable(ea), FocusTable(eb)
+    ta.s2(); tb.s2()
+    for t in (1, 2):
+        ta.step_s2(t, hparams(), flags=F.FOCUS_STEP_PACK_UPDATED)
+        tb.s2()
+        tb.step(t, hparams(), flags=F.FOCUS_STEP_PACK_UPDATED)
+        assert F.focus_get_error() == 0
+        for a, b in zip(ea, eb):
+            for name in ("Wq", "codes", "scales", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"):
+                x, y = getattr(a, name), getattr(b, name)
+                assert torch.equal(x.view(torch.uint8), y.view(torch.uint8)), (t, name)
+            want = oracle.s2(host_bits(a.W)) if a.W.numel() else np.float32(0)
+            assert host(a.s2)[0] == want and host(b.s2)[0] == want
+    assert int(ta._amax.abs().sum()) == 0          # cleared for the next step
