@@ -262,7 +262,7 @@ def run_ours(args, world, rank, local):
 
     peaks = measured_peaks()
     achieved = N * BYTES_STEP / (step_kernel_ms * 1e-3) / 1e9
-    roof = {"bound": "hbm", "kernel": "pipe_kernel<KIND_STEP> (focus_step_fused with the export pack)", "achieved": round(achieved, 1),
+    roof = {"bound": "hbm", "kernel": "pipe_kernel<KIND_STEP> (focus_step_fused_amax: step, export pack, tensor maxima)", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)",
             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(),
             "bytes_per_elem": BYTES_STEP, "launch_ms": round(step_kernel_ms, 4)}
