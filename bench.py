@@ -326,6 +326,8 @@ def measure_next_rows(ents, dev, N, peaks, world):
         with FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WQ_UPDATED;
       * the same step unfused (forward, backward, standalone AdamW: 15.5 B per
         weight in 450 launches), for what the fusion buys;
+      * Llama-3.1-70B generated on the device and stepped one layer at a time
+        (layers 0, 40, 79: s2, then the fused step with the export), per layer;
       * the MXFP4 variant's fused step over the same 224 weights (one launch per
         tensor; reads W, dW', m, q and moments, writes W', m, q and moments:
         9.75 B per weight)."""
@@ -428,6 +430,37 @@ def measure_next_rows(ents, dev, N, peaks, world):
     out["mxfp4_step_llama8b"] = {"kernel": "mx_kernel<KIND_STEP>", "launches": len(ents), "bytes_per_weight": 9.75,
                                  "Gelem_s": round(N * world / (ms * 1e-3) / 1e9, 2), **_roof(9.75 * N, ms, peak)}
     del mx
+    # Llama-3.1-70B, generated on the device one layer at a time and stepped there:
+    # s2 of the layer, then the fused step with the export of the updated parameters
+    # (timed per layer), layers 0, 40 and 79
+
+    per_layer = []
+    for layer in (0, 40, 79):
+        lts = synth.llama_70b_layer(layer, dev)
+        lents = []
+        for t in lts:
+            o, i = t.W.shape
+            lents.append(Entry(W=t.W, m=t.m, q=t.q, s2=torch.zeros(1, device=dev), dWq=t.dWq, Wq=torch.empty_like(t.W),
+                               m_exp_avg=torch.zeros_like(t.m), m_exp_avg_sq=torch.zeros_like(t.m),
+                               q_exp_avg=torch.zeros_like(t.q), q_exp_avg_sq=torch.zeros_like(t.q),
+                               codes=torch.empty((o, i // 2), dtype=torch.uint8, device=dev),
+                               scales=torch.empty((o, i // 16), dtype=torch.uint8, device=dev)))
+        ltab = FocusTable(lents)
+        ltab.s2()
+        cl = [0]
+
+        def lstep():
+            cl[0] += 1
+            ltab.step_s2(cl[0], hp, F.FOCUS_STEP_PACK_UPDATED)
+        per_layer.append(_timed(lstep, stream))
+        del ltab, lents, lts
+    n70 = sum(o * i for _, (o, i) in synth.LLAMA_70B.layer_shapes())
+    t70 = sum(per_layer) / len(per_layer)
+    out["llama70b_per_layer_step"] = {"kernel": "pipe_kernel<KIND_STEP> + s2_from_amax_kernel", "layers": [0, 40, 79],
+                                      "weights_per_layer": n70, "bytes_per_weight": 11.0625,
+                                      "Gelem_s": round(n70 * world / (t70 * 1e-3) / 1e9, 2),
+                                      "ms_per_layer": [round(x, 3) for x in per_layer],
+                                      **_roof(11.0625 * n70, t70, peak)}
     if F.focus_get_error() != 0:
         raise SystemExit("device status after the next-row measurements is not OK")
     D.barrier()
