@@ -265,6 +265,7 @@ def run_ours(args, world, rank, local):
     roof = {"bound": "hbm", "kernel": "pipe_kernel<KIND_STEP> (focus_step_fused_amax: step, export pack, tensor maxima)", "achieved": round(achieved, 1),
             "peak": peaks["hbm_gbs"], "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)",
             "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(),
+            "nominal_gbs": 8000.0, "frac_of_nominal": round(achieved / 8000.0, 4),
             "bytes_per_elem": BYTES_STEP, "launch_ms": round(step_kernel_ms, 4)}
     rows = None
     if not args.no_rows:
