@@ -368,7 +368,18 @@ def measure_next_rows(ents, dev, N, peaks, world):
                                                      "elements": n_act, "bytes_per_elem": 2.5625,
                                                      "Gelem_s": round(n_act / (ms * 1e-3) / 1e9, 2),
                                                      **_roof(b_act, ms, peak)}
-    del Xs, bufs
+    # the same writing the scales in the 128x4 layout of sm_100 block-scaled GEMMs
+    # (4096 tokens and hidden/16 columns: no padding, the same bytes)
+    swz = [torch.empty(F.focus_scales_swizzled_bytes(X.shape[0], X.shape[1] // 16), dtype=torch.uint8, device=dev)
+           for X in Xs]
+
+    def act_swz():
+        for X, (ts, c, _), sw in zip(Xs, bufs, swz):
+            F.focus_fouroversix_act_swizzled(X, ts, c, sw)
+    ms = _timed(act_swz, stream)
+    out["fouroversix_act_4096_tokens_one_layer"]["scales_128x4"] = {
+        "kernel": "f46_rows_kernel<SWZ>", "Gelem_s": round(n_act / (ms * 1e-3) / 1e9, 2), **_roof(b_act, ms, peak)}
+    del Xs, bufs, swz
     # the calibration step over four micro-batches
     for e in ents:
         e.dm = torch.zeros_like(e.m)
@@ -514,9 +525,16 @@ def run_e2e(args, ents, N, world, dev):
     bi = sum(h[n].numel() * h[n].element_size() for h in hosts for n in ins)
     bo = sum(h[n].numel() * h[n].element_size() for h in hosts for n in outs)
 
+    done_out = [None] * len(ents)     # per tensor: its read-back of the previous step
+
     def step(t):
         done_in, done_c = [], []
-        for e, h in zip(ents, hosts):
+        for j, (e, h) in enumerate(zip(ents, hosts)):
+            # a tensor's upload must not overwrite it while its previous read-back
+            # runs (and reads the host copy that read-back writes): wait for that
+            # tensor only, so the next step's uploads overlap this step's read-backs
+            if done_out[j] is not None:
+                h2d.wait_event(done_out[j])
             with torch.cuda.stream(h2d):
                 for n in ins:
                     getattr(e, n).copy_(h[n], non_blocking=True)
@@ -525,13 +543,12 @@ def run_e2e(args, ents, N, world, dev):
             comp.wait_event(ev)
             tab.step_s2(t, hp, F.FOCUS_STEP_PACK_UPDATED, stream=comp)
             ec = torch.cuda.Event(); ec.record(comp); done_c.append(ec)
-        for e, h, ec in zip(ents, hosts, done_c):
+        for j, (e, h, ec) in enumerate(zip(ents, hosts, done_c)):
             d2h.wait_event(ec)
             with torch.cuda.stream(d2h):
                 for n in outs:
                     h[n].copy_(getattr(e, n), non_blocking=True)
-        # the next step's uploads must not overwrite tensors still being read back
-        h2d.wait_stream(d2h)
+            eo = torch.cuda.Event(); eo.record(d2h); done_out[j] = eo
 
     for tab in tabs:
         tab.s2(stream=comp)                           # s2 before the first step

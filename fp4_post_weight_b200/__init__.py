@@ -13,6 +13,7 @@ _BINDING_NAMES = {"focus_s2", "focus_fwd", "focus_ste_bwd", "focus_adamw_step", 
                   "focus_table_prepare", "focus_s2_multi", "focus_step_fused", "focus_pack_multi",
                   "focus_fwd_multi", "focus_ste_bwd_multi", "focus_s2_noalloc",
                   "focus_fouroversix_weight", "focus_fouroversix_multi", "focus_fouroversix_act",
+                  "focus_fouroversix_act_swizzled",
                   "focus_scales_swizzle", "focus_scales_swizzled_bytes", "focus_mx_fwd", "focus_mx_ste_bwd",
                   "focus_mx_step", "focus_step_fused_amax", "focus_s2_from_amax",
                   "focus_get_error", "focus_s2_workspace_bytes", "focus_s2_multi_workspace_bytes",

@@ -25,7 +25,7 @@ constexpr int MAX_DEVICES = 64;
 
 struct DeviceInfo {
     int sms = 0;
-    int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_f46 = 0, occ_rows = 0, occ_amax = 0, occ_adam = 0;
+    int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_f46 = 0, occ_rows = 0, occ_rows_swz = 0, occ_amax = 0, occ_adam = 0;
     int occ_mx[3] = {0, 0, 0};
 };
 
@@ -58,7 +58,8 @@ int device_info(DeviceInfo **out) {
                              (int)stage_smem_bytes<KIND_F46>());
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_f46, pipe_kernel<KIND_F46>, CTA_THREADS,
                                                       stage_smem_bytes<KIND_F46>());
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows, f46_rows_kernel, ROW_THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows, f46_rows_kernel<false>, ROW_THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows_swz, f46_rows_kernel<true>, ROW_THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_amax, amax_tiles_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_adam, adamw_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[0], mx_kernel<KIND_FWD>, THREADS, 0);
@@ -67,7 +68,7 @@ int device_info(DeviceInfo **out) {
     });
     DeviceInfo &d = g_info[dev];
     if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_step_wqu <= 0 || d.occ_f46 <= 0 ||
-        d.occ_rows <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 || d.occ_mx[1] <= 0 ||
+        d.occ_rows <= 0 || d.occ_rows_swz <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 || d.occ_mx[1] <= 0 ||
         d.occ_mx[2] <= 0)
         return FOCUS_ERR_CUDA;
     *out = &d;
@@ -554,8 +555,27 @@ int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, flo
     DeviceInfo *di;
     if ((rc = device_info(&di))) return rc;
     const int64_t grid = grid_for(tokens, di->sms, di->occ_rows);
-    f46_rows_kernel<<<(unsigned)grid, ROW_THREADS, 0, (cudaStream_t)stream>>>(X, tokens, hidden, token_scales, codes,
-                                                                         scales, Xq);
+    f46_rows_kernel<false><<<(unsigned)grid, ROW_THREADS, 0, (cudaStream_t)stream>>>(X, tokens, hidden, token_scales,
+                                                                                codes, scales, Xq);
+    return launch_status();
+}
+
+int focus_fouroversix_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales,
+                                   uint8_t *codes, uint8_t *scales_swz, size_t scales_bytes, uint16_t *Xq,
+                                   focus_stream_t stream) {
+    int rc = check_shape(tokens, hidden);
+    if (rc) return rc;
+    if (tokens * hidden == 0) return FOCUS_OK;
+    if (!X || !token_scales || !codes || !scales_swz) return FOCUS_ERR_NULL;
+    if (!aligned16(X) || !aligned16(token_scales) || !aligned16(codes) || !aligned16(scales_swz) || !aligned16(Xq))
+        return FOCUS_ERR_ALIGN;
+    if (scales_bytes < focus_scales_swizzled_bytes(tokens, hidden / 16)) return FOCUS_ERR_WORKSPACE;
+    DeviceInfo *di;
+    if ((rc = device_info(&di))) return rc;
+    const int64_t rows_out = (tokens + 127) / 128 * 128;
+    const int64_t grid = grid_for(rows_out, di->sms, di->occ_rows_swz);
+    f46_rows_kernel<true><<<(unsigned)grid, ROW_THREADS, 0, (cudaStream_t)stream>>>(X, tokens, hidden, token_scales,
+                                                                               codes, scales_swz, Xq);
     return launch_status();
 }
 

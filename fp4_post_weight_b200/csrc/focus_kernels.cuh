@@ -942,13 +942,32 @@ __global__ void __launch_bounds__(THREADS) s2_finish_kernel(const Args a, const 
 
 constexpr int ROW_THREADS = 128;               // threads of the per-token kernel: 8 rows in flight per SM (12% faster than 256)
 
+// Byte of scale (r, c) in the 128x4-atom layout of sm_100 block-scaled GEMMs
+// (rows padded to 128, columns to 4; `groups` = column groups of 4): atoms of
+// 128 rows x 4 columns, 512 bytes, stored band by band with the column groups
+// inner; inside an atom, byte 16*(r mod 32) + 4*((r div 32) mod 4) + (c mod 4).
+__device__ __forceinline__ int64_t swizzled_offset(int64_t r, int64_t c, int64_t groups) {
+    return (((r >> 7) * groups + (c >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (c & 3);
+}
+
+// SWZ: the block scales go straight into the 128x4-atom layout (`scales` holds
+// the padded buffer), and the CTAs that draw a padding row, or a row's padding
+// columns, write them 0.
+template <bool SWZ>
 __global__ void __launch_bounds__(ROW_THREADS) f46_rows_kernel(const uint16_t *__restrict__ X, int64_t rows, int64_t cols,
                                                            float *__restrict__ row_scales, uint8_t *__restrict__ codes,
                                                            uint8_t *__restrict__ scales, uint16_t *__restrict__ Xq) {
     __shared__ uint32_t red[ROW_THREADS / 32];
     const int64_t chunks = cols / 8;          // 16-byte words of a row
     const int64_t nb = cols / 16;
-    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int64_t groups = (nb + 3) / 4;      // SWZ: column groups of the padded layout
+    const int64_t rows_out = SWZ ? (rows + 127) / 128 * 128 : rows;
+    for (int64_t r = blockIdx.x; r < rows_out; r += gridDim.x) {
+        if (SWZ && r >= rows) {                // a padding row: its words of every column group are 0
+            for (int64_t g = threadIdx.x; g < groups; g += ROW_THREADS)
+                *reinterpret_cast<uint32_t *>(scales + swizzled_offset(r, 4 * g, groups)) = 0u;
+            continue;
+        }
         const uint4 *xr = reinterpret_cast<const uint4 *>(X + r * cols);
         uint32_t mx = 0u;
         for (int64_t c = threadIdx.x; c < chunks; c += ROW_THREADS) {
@@ -983,12 +1002,14 @@ __global__ void __launch_bounds__(ROW_THREADS) f46_rows_kernel(const uint16_t *_
                 if (Xq) wq_words(cw, sb, s, o);
             }
             reinterpret_cast<uint2 *>(codes)[blk] = make_uint2(cw[0], cw[1]);
-            scales[blk] = (uint8_t)sb;
+            scales[SWZ ? swizzled_offset(r, b, groups) : blk] = (uint8_t)sb;
             if (Xq) {
                 __stcs(reinterpret_cast<uint4 *>(Xq) + 2 * blk, o[0]);
                 __stcs(reinterpret_cast<uint4 *>(Xq) + 2 * blk + 1, o[1]);
             }
         }
+        if (SWZ)                               // the row's padding columns (at most 3)
+            for (int64_t c = nb + threadIdx.x; c < 4 * groups; c += ROW_THREADS) scales[swizzled_offset(r, c, groups)] = 0u;
     }
 }
 

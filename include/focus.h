@@ -320,6 +320,18 @@ int focus_fouroversix_multi(const focus_tensor_desc *descs_dev, int n_tensors, i
 int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales,
                           uint8_t *codes, uint8_t *scales, uint16_t *Xq, focus_stream_t stream);
 
+/* The same, with the block scales written straight into the 128x4-atom layout
+ * that focus_scales_swizzle produces (declared below), the layout an sm_100
+ * block-scaled GEMM reads for its activation operand: scales_swz (device, at
+ * least focus_scales_swizzled_bytes(tokens, hidden/16) bytes, else
+ * FOCUS_ERR_WORKSPACE) receives every byte, padding rows and columns 0.  The
+ * result equals focus_fouroversix_act followed by focus_scales_swizzle, in one
+ * launch.  A row holding a non-finite value sets the device flag and leaves
+ * its outputs, padding columns included, unwritten. */
+int focus_fouroversix_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales,
+                                   uint8_t *codes, uint8_t *scales_swz, size_t scales_bytes, uint16_t *Xq,
+                                   focus_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * MXFP4 variant: 32-element blocks with an E8M0 scale and four sub-blocks of
  * 8, no tensor scale.  "Technische Samenvatting: FOCUS ...", sections

@@ -38,6 +38,59 @@ def test_swizzle_matches_oracle(F, rows, cols):
     np.testing.assert_array_equal(host(out), oracle.scales_swizzle(host(sc)))
 
 
+@pytest.mark.parametrize("tokens,hidden", [(1, 16), (5, 96), (128, 64), (130, 1040), (300, 4096), (33, 14336)])
+def test_fouroversix_act_swizzled_matches_oracle(F, tokens, hidden):
+    """Per-token FourOverSix writing its scales straight into the 128x4 layout: the
+    oracle's quantization followed by the oracle's relayout, bit for bit, padding
+    included (the buffer starts filled with 0xAB)."""
+    X = synth.activations(tokens, hidden, "cuda", seed=7 * tokens + hidden, zero_tokens=1 if tokens > 2 else 0)
+    ts = torch.full((tokens,), -1.0, device="cuda")
+    codes = torch.empty((tokens, hidden // 2), dtype=torch.uint8, device="cuda")
+    Xq = torch.empty_like(X)
+    sw = torch.full((F.focus_scales_swizzled_bytes(tokens, hidden // 16),), 0xAB, dtype=torch.uint8, device="cuda")
+    F.focus_fouroversix_act_swizzled(X, ts, codes, sw, Xq)
+    assert F.focus_get_error() == 0
+    ref = oracle.fouroversix(host_bits(X))
+    np.testing.assert_array_equal(host(ts), ref.row_scales)
+    np.testing.assert_array_equal(unpack_codes(host(codes)), ref.codes)
+    np.testing.assert_array_equal(host_bits(Xq), ref.Xq)
+    np.testing.assert_array_equal(host(sw), oracle.scales_swizzle(ref.scales))
+
+
+def test_fouroversix_act_swizzled_nonfinite_row(F):
+    """A row holding infinity sets the device flag and leaves its outputs unwritten
+    (its scale bytes, padding columns included, keep the fill); the other rows match
+    the oracle."""
+    tokens, hidden = 6, 96                                 # 6 scale columns: 2 padding columns per row
+    X = synth.activations(tokens, hidden, "cuda", seed=3, zero_tokens=0)
+    X[2, 17] = float("inf")
+    ts = torch.zeros(tokens, device="cuda")
+    codes = torch.zeros((tokens, hidden // 2), dtype=torch.uint8, device="cuda")
+    sw = torch.full((F.focus_scales_swizzled_bytes(tokens, hidden // 16),), 0xAB, dtype=torch.uint8, device="cuda")
+    assert F.focus_get_error() == 0
+    F.focus_fouroversix_act_swizzled(X, ts, codes, sw)
+    assert F.focus_get_error() == 7
+    Xh = host_bits(X)
+    good = [r for r in range(tokens) if r != 2]
+    ref = oracle.fouroversix(Xh[good])
+    lin = np.zeros((tokens, hidden // 16), np.uint8)
+    lin[good] = ref.scales
+    want = oracle.scales_swizzle(lin)
+    got = host(sw)
+    # the bytes of row 2 in the layout: a 1-row marker pushed through the oracle's relayout
+    mark = np.zeros((tokens, hidden // 16), np.uint8)
+    mark[2] = 1
+    row2 = oracle.scales_swizzle(mark) == 1
+    mark_pad = np.zeros((tokens, 8), np.uint8)
+    mark_pad[2, 6:] = 1
+    row2_pad = oracle.scales_swizzle(mark_pad) == 1
+    assert np.all(got[row2] == 0xAB) and np.all(got[row2_pad] == 0xAB)
+    rest = ~(row2 | row2_pad)
+    np.testing.assert_array_equal(got[rest], want[rest])
+    np.testing.assert_array_equal(unpack_codes(host(codes))[good], ref.codes)
+    assert np.all(host(codes)[2] == 0)
+
+
 E2M1 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6], np.float64)
 
 
@@ -94,7 +147,12 @@ def test_export_feeds_sm100_block_scaled_gemm(F):
     wsc = torch.empty((N, K // 16), dtype=torch.uint8, device="cuda")
     F.focus_pack_nvfp4(W, m, q, s2, wc, wsc, torch.zeros(1, device="cuda"))
     xs_sw, ws_sw = swizzle_gpu(F, xs), swizzle_gpu(F, wsc)
+    # the per-token quantizer that writes the 128x4 layout itself gives the same bytes
+    xs_fused = torch.empty_like(xs_sw)
+    xc_fused = torch.empty_like(xc)
+    F.focus_fouroversix_act_swizzled(X, torch.empty_like(ts), xc_fused, xs_fused)
     assert F.focus_get_error() == 0
+    assert torch.equal(xs_fused, xs_sw) and torch.equal(xc_fused, xc)
 
     Xd, Wd = dequant(host(xc), host(xs)), dequant(host(wc), host(wsc))
     tsh = host(ts).astype(np.float64)[:, None]
