@@ -336,7 +336,7 @@ def measure_next_rows(ents, dev, N, peaks, world):
 
     import synth
     from fp4_post_weight_b200 import focus as F
-    from fp4_post_weight_b200.table import Entry, FocusTable, PURPOSE_FOUROVERSIX, hparams
+    from fp4_post_weight_b200.table import PURPOSE_FOUROVERSIX, PURPOSE_MX, Entry, FocusTable, hparams
     from fp4_post_weight_b200 import dist as D
     stream = torch.cuda.current_stream(dev)
     peak = peaks["hbm_gbs"]
@@ -425,7 +425,8 @@ def measure_next_rows(ents, dev, N, peaks, world):
     for e in ents:
         e.dm = e.dq = None
     del tab
-    # the MXFP4 variant: one fused step per tensor (224 launches), m = 1, q = 6, zero moments
+    # the MXFP4 variant: one fused step per tensor (224 launches), m = 1, q = 6, zero moments,
+    # then the same as one launch over a table
     mx = []
     for e in ents:
         o, i = e.W.shape
@@ -439,9 +440,21 @@ def measure_next_rows(ents, dev, N, peaks, world):
         for e, (m, q, a1, a2, b1, b2) in zip(ents, mx):
             F.focus_mx_step(e.W, e.dWq, m, q, a1, a2, b1, b2, hp, cnt_mx[0], 0, e.Wq)
     ms = _timed(mx_step, stream)
-    out["mxfp4_step_llama8b"] = {"kernel": "mx_kernel<KIND_STEP>", "launches": len(ents), "bytes_per_weight": 9.75,
-                                 "Gelem_s": round(N * world / (ms * 1e-3) / 1e9, 2), **_roof(9.75 * N, ms, peak)}
-    del mx
+    r = {"kernel": "mx_kernel<KIND_STEP>", "launches": len(ents), "bytes_per_weight": 9.75,
+         "Gelem_s": round(N * world / (ms * 1e-3) / 1e9, 2), **_roof(9.75 * N, ms, peak)}
+    # the same over a table of all the tensors: one launch
+    mx_tab = FocusTable([Entry(W=e.W, m=m, q=q, s2=None, dWq=e.dWq, Wq=e.Wq, m_exp_avg=a1, m_exp_avg_sq=a2,
+                               q_exp_avg=b1, q_exp_avg_sq=b2) for e, (m, q, a1, a2, b1, b2) in zip(ents, mx)],
+                        PURPOSE_MX)
+
+    def mx_step_table():
+        cnt_mx[0] += 1
+        mx_tab.mx_step(cnt_mx[0], hp)
+    ms = _timed(mx_step_table, stream)
+    r["one_launch"] = {"kernel": "mx_multi_kernel<KIND_STEP>", "launches": 1,
+                       "Gelem_s": round(N * world / (ms * 1e-3) / 1e9, 2), **_roof(9.75 * N, ms, peak)}
+    out["mxfp4_step_llama8b"] = r
+    del mx, mx_tab
     # Llama-3.1-70B, generated on the device one layer at a time and stepped there:
     # s2 of the layer, then the fused step with the export of the updated parameters
     # (timed per layer), layers 0, 40 and 79

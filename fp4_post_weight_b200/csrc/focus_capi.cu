@@ -26,7 +26,7 @@ constexpr int MAX_DEVICES = 64;
 struct DeviceInfo {
     int sms = 0;
     int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_f46 = 0, occ_rows = 0, occ_rows_swz = 0, occ_amax = 0, occ_adam = 0;
-    int occ_mx[3] = {0, 0, 0};
+    int occ_mx[3] = {0, 0, 0}, occ_mx_multi[3] = {0, 0, 0};
 };
 
 std::once_flag g_once[MAX_DEVICES];
@@ -65,11 +65,15 @@ int device_info(DeviceInfo **out) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[0], mx_kernel<KIND_FWD>, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[1], mx_kernel<KIND_BWD>, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[2], mx_kernel<KIND_STEP>, THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[0], mx_multi_kernel<KIND_FWD>, MX_TILE_BLOCKS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[1], mx_multi_kernel<KIND_BWD>, MX_TILE_BLOCKS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[2], mx_multi_kernel<KIND_STEP>, MX_TILE_BLOCKS,
+                                                      0);
     });
     DeviceInfo &d = g_info[dev];
     if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_step_wqu <= 0 || d.occ_f46 <= 0 ||
         d.occ_rows <= 0 || d.occ_rows_swz <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 || d.occ_mx[1] <= 0 ||
-        d.occ_mx[2] <= 0)
+        d.occ_mx[2] <= 0 || d.occ_mx_multi[0] <= 0 || d.occ_mx_multi[1] <= 0 || d.occ_mx_multi[2] <= 0)
         return FOCUS_ERR_CUDA;
     *out = &d;
     return FOCUS_OK;
@@ -180,6 +184,28 @@ int launch_mx(const MxArgs &a, cudaStream_t s) {
     if (a.nblk == 0) return FOCUS_OK;
     const int64_t grid = grid_for((a.nblk + THREADS - 1) / THREADS, di->sms, di->occ_mx[KIND]);
     mx_kernel<KIND><<<(unsigned)grid, THREADS, 0, s>>>(a);
+    return launch_status();
+}
+
+template <int KIND>
+int launch_mx_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, int accumulate, int write_grad,
+                    const Hyper &hp, cudaStream_t s) {
+    if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
+    if (n == 0 || total_tiles == 0) return FOCUS_OK;
+    if (!descs_dev) return FOCUS_ERR_NULL;
+    if (!aligned16(descs_dev)) return FOCUS_ERR_ALIGN;
+    DeviceInfo *di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    MxMultiArgs a{};
+    a.table = descs_dev;
+    a.n_tensors = n;
+    a.total_tiles = total_tiles;
+    a.accumulate = accumulate;
+    a.write_grad = write_grad;
+    a.hp = hp;
+    const int64_t grid = grid_for(total_tiles, di->sms, di->occ_mx_multi[KIND]);
+    mx_multi_kernel<KIND><<<(unsigned)grid, MX_TILE_BLOCKS, 0, s>>>(a);
     return launch_status();
 }
 
@@ -373,8 +399,31 @@ int focus_adamw_step(float *p, const float *g, float *exp_avg, float *exp_avg_sq
 
 int focus_table_prepare(focus_tensor_desc *d, int n, int purpose, int64_t *total_tiles) {
     if (!d || !total_tiles) return FOCUS_ERR_NULL;
-    if (n < 0 || purpose < 0 || purpose > 3) return FOCUS_ERR_VALUE;
+    if (n < 0 || purpose < 0 || purpose > FOCUS_PURPOSE_MX) return FOCUS_ERR_VALUE;
     int64_t tiles = 0, blocks = 0;
+    if (purpose == FOCUS_PURPOSE_MX) {
+        for (int i = 0; i < n; ++i) {
+            focus_tensor_desc &e = d[i];
+            int rc = check_shape_mx(e.out, e.in);
+            if (rc) return rc;
+            const int64_t nblk = e.out * (e.in / 32);
+            if (nblk > 0) {
+                if (!e.W || !e.m || !e.q) return FOCUS_ERR_NULL;
+                const void *ptrs[] = {e.W, e.m, e.q, e.Wq, e.codes, e.scales, e.dm, e.dq, e.dWq,
+                                      e.m_exp_avg, e.m_exp_avg_sq, e.q_exp_avg, e.q_exp_avg_sq};
+                for (const void *p : ptrs)
+                    if (p && !aligned16(p)) return FOCUS_ERR_ALIGN;
+                if ((e.codes == nullptr) != (e.scales == nullptr)) return FOCUS_ERR_NULL;
+                if ((e.dm == nullptr) != (e.dq == nullptr)) return FOCUS_ERR_NULL;
+            }
+            e.block_begin = blocks;
+            e.tile_begin = tiles;
+            blocks += nblk;
+            tiles += (nblk + MX_TILE_BLOCKS - 1) / MX_TILE_BLOCKS;
+        }
+        *total_tiles = tiles;
+        return FOCUS_OK;
+    }
     for (int i = 0; i < n; ++i) {
         focus_tensor_desc &e = d[i];
         int rc = check_shape(e.out, e.in);
@@ -636,6 +685,33 @@ int focus_mx_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, fl
     a.hp = make_hyper(hp->lr_m, hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
     a.nblk = out * (in / 32);
     return launch_mx<KIND_STEP>(a, (cudaStream_t)stream);
+}
+
+
+int focus_mx_fwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
+                       focus_stream_t stream) {
+    return launch_mx_multi<KIND_FWD>(descs_dev, n_tensors, total_tiles, 0, 0, Hyper{}, (cudaStream_t)stream);
+}
+
+int focus_mx_ste_bwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles, int accumulate,
+                           focus_stream_t stream) {
+    if (accumulate != 0 && accumulate != 1) return FOCUS_ERR_VALUE;
+    return launch_mx_multi<KIND_BWD>(descs_dev, n_tensors, total_tiles, accumulate, 0, Hyper{},
+                                     (cudaStream_t)stream);
+}
+
+int focus_mx_step_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
+                        const focus_hparams *hp, int64_t step, unsigned flags, focus_stream_t stream) {
+    if (!hp) return FOCUS_ERR_NULL;
+    int rc;
+    if ((rc = check_hyper(hp->lr_m, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
+    if ((rc = check_hyper(hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
+    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD)) return FOCUS_ERR_VALUE;
+    return launch_mx_multi<KIND_STEP>(descs_dev, n_tensors, total_tiles, (flags & FOCUS_STEP_ACCUMULATE) ? 1 : 0,
+                                      (flags & FOCUS_STEP_WRITE_GRAD) ? 1 : 0,
+                                      make_hyper(hp->lr_m, hp->lr_q, hp->beta1, hp->beta2, hp->eps,
+                                                 hp->weight_decay, step),
+                                      (cudaStream_t)stream);
 }
 
 size_t focus_scales_swizzled_bytes(int64_t rows, int64_t cols) {

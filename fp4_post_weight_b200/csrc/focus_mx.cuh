@@ -16,10 +16,12 @@
 // (32 exact products summed in binary64, rounded once), dq_k = -(1 - sigma_k)
 // S_b sum_k in g y (binary32).
 //
-// Work decomposition: one thread per 32-block, grid-stride over the blocks of
-// one tensor; W and dW' arrive as four 16-byte loads each, m as one float, q
-// and its moments as one float4 each.  No shared-memory staging: a thread has
-// 128 bytes of loads in flight, enough at full occupancy.
+// Work decomposition: one thread per 32-block; W and dW' arrive as four
+// 16-byte loads each, m as one float, q and its moments as one float4 each.
+// No shared-memory staging: a thread has 128 bytes of loads in flight, enough
+// at full occupancy.  mx_kernel strides over the blocks of one tensor;
+// mx_multi_kernel walks the tiles (4096 weights, 128 blocks) of a table of
+// tensors, one launch for a whole model.
 #pragma once
 
 #include <cstdint>
@@ -56,10 +58,10 @@ __device__ __forceinline__ float pow2f(int e) {           // 2^e for e in [-127,
     return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : 0x1p-127f;
 }
 
+// One 32-block of the tensor `a` describes.
 template <int KIND>
-__global__ void __launch_bounds__(THREADS) mx_kernel(const MxArgs a) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < a.nblk; blk += stride) {
+__device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
+    {
         uint32_t w[16], g[16];
         const uint4 *Wp = reinterpret_cast<const uint4 *>(a.W) + 4 * blk;
 #pragma unroll
@@ -176,6 +178,82 @@ __global__ void __launch_bounds__(THREADS) mx_kernel(const MxArgs a) {
             }
         }
         if (bad) atomicOr(&g_error_flags, 1u);
+    }
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(THREADS) mx_kernel(const MxArgs a) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < a.nblk; blk += stride)
+        mx_block<KIND>(a, blk);
+}
+
+// ---------------------------------------------------------------------------
+// Many tensors in one launch.  The table uses focus_tensor_desc with the
+// MXFP4 shapes (m [out][in/32], q [out][in/8], scales [out][in/32]); its
+// tile_begin fields count tiles of MX_TILE_BLOCKS 32-blocks (4096 weights).
+// Each CTA keeps the descriptor of its current tensor in shared memory as an
+// MxArgs, refreshed by thread 0 when the CTA's next tile lies past it (a
+// CTA-uniform test, so the barriers around it are reached by every thread).
+// ---------------------------------------------------------------------------
+
+constexpr int MX_TILE_BLOCKS = 128;        // 32-blocks per tile, one per thread
+
+struct MxMultiArgs {
+    const focus_tensor_desc *table;
+    int n_tensors;
+    int64_t total_tiles;
+    int accumulate;
+    int write_grad;
+    Hyper hp;
+};
+
+template <int KIND>
+__global__ void __launch_bounds__(MX_TILE_BLOCKS) mx_multi_kernel(const MxMultiArgs g) {
+    __shared__ MxArgs sa;
+    __shared__ int64_t s_range[2];          // tiles [first, end) of the current tensor
+    int t = 0;                              // thread 0's table cursor
+    int64_t first = 0, end = 0;
+    for (int64_t tile = blockIdx.x; tile < g.total_tiles; tile += gridDim.x) {
+        if (tile >= end) {
+            __syncthreads();                // every thread is done with the previous descriptor
+            if (threadIdx.x == 0) {
+                focus_tensor_desc d;
+                int64_t nb = 0, e = 0;
+                for (;;) {
+                    d = g.table[t];
+                    nb = d.out * (d.in / 32);
+                    e = d.tile_begin + (nb + MX_TILE_BLOCKS - 1) / MX_TILE_BLOCKS;
+                    if (tile < e || t + 1 >= g.n_tensors) break;
+                    ++t;
+                }
+                // a descriptor without a pointer the call needs is skipped and reported
+                bool ok = d.W != nullptr && d.m != nullptr && d.q != nullptr;
+                if (KIND != KIND_FWD) ok = ok && d.dWq != nullptr;
+                if (KIND == KIND_STEP)
+                    ok = ok && d.m_exp_avg && d.m_exp_avg_sq && d.q_exp_avg && d.q_exp_avg_sq;
+                if (KIND == KIND_BWD || g.accumulate || g.write_grad) ok = ok && d.dm && d.dq;
+                if ((d.codes == nullptr) != (d.scales == nullptr)) ok = false;
+                if (!ok && nb > 0) atomicOr(&g_error_flags, 2u);
+                sa.W = d.W; sa.dWq = d.dWq; sa.Wq = d.Wq;
+                sa.m = d.m; sa.q = d.q;
+                sa.m_ea = d.m_exp_avg; sa.m_eas = d.m_exp_avg_sq; sa.q_ea = d.q_exp_avg; sa.q_eas = d.q_exp_avg_sq;
+                sa.codes = d.codes; sa.scales = d.scales;
+                sa.dm = d.dm; sa.dq = d.dq;
+                sa.nblk = ok ? nb : 0;
+                sa.accumulate = g.accumulate;
+                sa.write_grad = g.write_grad;
+                sa.hp = g.hp;
+                s_range[0] = d.tile_begin;
+                s_range[1] = e;
+            }
+            __syncthreads();
+            first = s_range[0];
+            end = s_range[1];
+            if (tile >= end) break;         // past the last tensor (uniform): nothing left
+        }
+        const int64_t blk = (tile - first) * MX_TILE_BLOCKS + threadIdx.x;
+        if (tile >= first && blk < sa.nblk) mx_block<KIND>(sa, blk);
     }
 }
 

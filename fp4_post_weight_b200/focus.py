@@ -29,6 +29,7 @@ FOCUS_STEP_ACCUMULATE = 1
 FOCUS_STEP_WRITE_GRAD = 2
 FOCUS_STEP_PACK_UPDATED = 4
 FOCUS_STEP_WQ_UPDATED = 8
+FOCUS_PURPOSE_MX = 4
 
 
 class focus_tensor_desc(ctypes.Structure):
@@ -73,6 +74,9 @@ _SIGS = {
     "focus_mx_ste_bwd": ([_P, _P, _P, _P, _I64, _I64, _P, _P, _I, _P], _I),
     "focus_mx_step": ([_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, ctypes.POINTER(focus_hparams), _I64,
                        ctypes.c_uint, _P, _P, _P, _P], _I),
+    "focus_mx_fwd_multi": ([_P, _I, _I64, _P], _I),
+    "focus_mx_ste_bwd_multi": ([_P, _I, _I64, _I, _P], _I),
+    "focus_mx_step_multi": ([_P, _I, _I64, ctypes.POINTER(focus_hparams), _I64, ctypes.c_uint, _P], _I),
     "focus_scales_swizzled_bytes": ([_I64, _I64], _SZ),
     "focus_scales_swizzle": ([_P, _I64, _I64, _P, _SZ, _P], _I),
     "focus_get_error": ([_P], _I),
@@ -307,6 +311,22 @@ def focus_mx_step(W, dWq, m, q, m_exp_avg, m_exp_avg_sq, q_exp_avg, q_exp_avg_sq
     _check(_lib.focus_mx_step(_ptr(W), _ptr(dWq), _ptr(m), _ptr(q), _ptr(m_exp_avg), _ptr(m_exp_avg_sq),
                               _ptr(q_exp_avg), _ptr(q_exp_avg_sq), o, i, ctypes.byref(hp), int(step), int(flags),
                               _ptr(Wq), _ptr(dm), _ptr(dq), _stream(stream)), "focus_mx_step")
+
+
+def focus_mx_fwd_multi(table_dev, n: int, total_tiles: int, stream=None):
+    """MXFP4 forward over a table prepared with FOCUS_PURPOSE_MX, one launch."""
+    _check(_lib.focus_mx_fwd_multi(_ptr(table_dev), int(n), int(total_tiles), _stream(stream)), "focus_mx_fwd_multi")
+
+
+def focus_mx_ste_bwd_multi(table_dev, n: int, total_tiles: int, accumulate: bool = False, stream=None):
+    _check(_lib.focus_mx_ste_bwd_multi(_ptr(table_dev), int(n), int(total_tiles), 1 if accumulate else 0,
+                                       _stream(stream)), "focus_mx_ste_bwd_multi")
+
+
+def focus_mx_step_multi(table_dev, n: int, total_tiles: int, hp: focus_hparams, step: int, flags: int = 0,
+                        stream=None):
+    _check(_lib.focus_mx_step_multi(_ptr(table_dev), int(n), int(total_tiles), ctypes.byref(hp), int(step),
+                                    int(flags), _stream(stream)), "focus_mx_step_multi")
 
 
 def focus_scales_swizzled_bytes(rows: int, cols: int) -> int:

@@ -20,6 +20,7 @@ PURPOSE_FORWARD = 0
 PURPOSE_STEP = 1
 PURPOSE_BACKWARD = 2
 PURPOSE_FOUROVERSIX = 3
+PURPOSE_MX = 4                                # the MXFP4 calls (focus_mx_*_multi): in % 32 == 0, no s2
 
 
 @dataclass
@@ -28,7 +29,7 @@ class Entry:
     W: torch.Tensor
     m: torch.Tensor
     q: torch.Tensor
-    s2: torch.Tensor                          # one float32 on the device
+    s2: torch.Tensor | None                   # one float32 on the device (None for an MXFP4 table)
     dWq: torch.Tensor | None = None
     Wq: torch.Tensor | None = None
     m_exp_avg: torch.Tensor | None = None
@@ -93,6 +94,16 @@ class FocusTable:
 
     def fouroversix(self, stream=None):
         F.focus_fouroversix_multi(self.dev, self.n, self.total_tiles, stream)
+
+    # MXFP4 (a table built with PURPOSE_MX)
+    def mx_fwd(self, stream=None):
+        F.focus_mx_fwd_multi(self.dev, self.n, self.total_tiles, stream)
+
+    def mx_bwd(self, accumulate: bool = False, stream=None):
+        F.focus_mx_ste_bwd_multi(self.dev, self.n, self.total_tiles, accumulate, stream)
+
+    def mx_step(self, step: int, hp: F.focus_hparams | None = None, flags: int = 0, stream=None):
+        F.focus_mx_step_multi(self.dev, self.n, self.total_tiles, hp or hparams(), step, flags, stream)
 
 
 def hparams(lr_m=5e-3, lr_q=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0) -> F.focus_hparams:

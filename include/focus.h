@@ -207,6 +207,9 @@ typedef struct focus_hparams {
     float weight_decay;    /* 0 */
 } focus_hparams;
 
+/* focus_table_prepare purpose of a table for the MXFP4 multi-tensor calls. */
+#define FOCUS_PURPOSE_MX 4
+
 /* Flags of focus_step_fused. */
 #define FOCUS_STEP_ACCUMULATE 1u  /* add dm/dq (earlier micro-batches) to this step's gradients */
 #define FOCUS_STEP_WRITE_GRAD 2u  /* write the gradients used by the update into dm/dq */
@@ -220,8 +223,13 @@ typedef struct focus_hparams {
 /* Checks every entry (pointers, alignment, shapes, which inputs are present
  * for `purpose`: 0 = s2/forward/pack, 1 = also focus_step_fused (dWq and the
  * four moments), 2 = also focus_ste_bwd_multi (dWq, dm, dq), 3 = s2 and
- * FourOverSix only (W and s2; m and q may be NULL; codes+scales or Wq)) and
- * fills block_begin and tile_begin.  Host memory in, host memory out.
+ * FourOverSix only (W and s2; m and q may be NULL; codes+scales or Wq),
+ * FOCUS_PURPOSE_MX (4) = the MXFP4 calls focus_mx_*_multi (in % 32 == 0; W,
+ * m and q present; s2 unused; the other pointers optional here and checked by
+ * the kernels: an entry lacking one its call needs is skipped and flagged))
+ * and fills block_begin and tile_begin (for purpose 4 in 32-blocks and tiles
+ * of 128 of them: 4096 weights, as for the other purposes).  Host memory in,
+ * host memory out.
  * *total_tiles receives the number of work tiles, passed to the calls below.
  * A device-resident table cannot be checked again at call time: a kernel that
  * meets an entry lacking a pointer it needs skips that entry and sets the
@@ -371,6 +379,19 @@ int focus_mx_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, fl
                   float *m_exp_avg_sq, float *q_exp_avg, float *q_exp_avg_sq, int64_t out, int64_t in,
                   const focus_hparams *hp, int64_t step, unsigned flags, uint16_t *Wq, float *dm, float *dq,
                   focus_stream_t stream);
+
+/* The same three over every entry of a table prepared with FOCUS_PURPOSE_MX,
+ * in one launch each (per entry: W, m, q; the forward writes Wq and/or
+ * codes+scales, whichever the entry has; the backward needs dWq, dm, dq; the
+ * step needs dWq and the four moments, writes Wq when present, and needs dm,
+ * dq under FOCUS_STEP_ACCUMULATE / FOCUS_STEP_WRITE_GRAD).  An entry lacking a
+ * pointer its call needs is skipped and sets the device flag. */
+int focus_mx_fwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
+                       focus_stream_t stream);
+int focus_mx_ste_bwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles, int accumulate,
+                           focus_stream_t stream);
+int focus_mx_step_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
+                        const focus_hparams *hp, int64_t step, unsigned flags, focus_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Scale factors for sm_100 block-scaled GEMMs.  The pages deploy the export

@@ -108,8 +108,11 @@ def test_table_prepare_on_host(F):
         descs[i].dq = P + 65536 * (i + 1) + 4096
     assert F.focus_table_prepare(descs, 2) == tiles
     with pytest.raises(F.FocusError) as e:
-        F.focus_table_prepare(descs, 4)
+        F.focus_table_prepare(descs, 5)
     assert e.value.status == 4
+    with pytest.raises(F.FocusError) as e:      # MXFP4: in must be a multiple of 32
+        F.focus_table_prepare(descs, F.FOCUS_PURPOSE_MX)
+    assert e.value.status == 2
     descs[2].in_ = 40
     with pytest.raises(F.FocusError) as e:
         F.focus_table_prepare(descs, 0)
@@ -119,6 +122,62 @@ def test_table_prepare_on_host(F):
     with pytest.raises(F.FocusError) as e:
         F.focus_table_prepare(descs, 0)
     assert e.value.status == 3
+
+
+def test_table_prepare_mx(F):
+    """A table for the MXFP4 calls: 32-blocks, tiles of 128 of them (4096 weights),
+    W, m and q required, s2 not needed, pointers both-or-neither as elsewhere."""
+    shapes = [(4, 32), (3, 96), (300, 4096), (0, 64)]
+    n = len(shapes)
+    descs = (F.focus_tensor_desc * n)()
+    for i, (o, k) in enumerate(shapes):
+        d = descs[i]
+        for name in ("W", "m", "q"):
+            setattr(d, name, P + 4096 * (i + 1))
+        d.out, d.in_ = o, k
+    tiles = F.focus_table_prepare(descs, F.FOCUS_PURPOSE_MX)
+    nblk = [o * k // 32 for o, k in shapes]
+    t = [(b + 127) // 128 for b in nblk]
+    assert [descs[i].block_begin for i in range(n)] == [sum(nblk[:i]) for i in range(n)]
+    assert [descs[i].tile_begin for i in range(n)] == [sum(t[:i]) for i in range(n)]
+    assert tiles == sum(t) == 1 + 1 + 300 + 0
+    descs[1].codes = P                          # codes without scales
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, F.FOCUS_PURPOSE_MX)
+    assert e.value.status == 1
+    descs[1].scales = P
+    descs[1].dm = P                             # dm without dq
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, F.FOCUS_PURPOSE_MX)
+    assert e.value.status == 1
+    descs[1].dq = U                             # misaligned
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, F.FOCUS_PURPOSE_MX)
+    assert e.value.status == 3
+    descs[1].dm = descs[1].dq = None
+    descs[2].q = None
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, F.FOCUS_PURPOSE_MX)
+    assert e.value.status == 1
+    descs[2].q = P
+    descs[0].in_ = 48
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, F.FOCUS_PURPOSE_MX)
+    assert e.value.status == 2
+
+
+def test_mx_multi_checks(F):
+    hp = F.focus_hparams(5e-3, 1e-3, 0.9, 0.999, 1e-8, 0.0)
+    assert F.raw_call("focus_mx_fwd_multi", P, -1, 1, None) == 4
+    assert F.raw_call("focus_mx_fwd_multi", None, 1, 1, None) == 1
+    assert F.raw_call("focus_mx_fwd_multi", U, 1, 1, None) == 3
+    assert F.raw_call("focus_mx_fwd_multi", None, 0, 0, None) == 0            # nothing to do
+    assert F.raw_call("focus_mx_ste_bwd_multi", P, 1, 1, 2, None) == 4        # accumulate must be 0 or 1
+    assert F.raw_call("focus_mx_ste_bwd_multi", None, 1, 1, 0, None) == 1
+    assert F.raw_call("focus_mx_step_multi", P, 1, 1, None, 1, 0, None) == 1
+    assert F.raw_call("focus_mx_step_multi", P, 1, 1, ctypes.byref(hp), 0, 0, None) == 4    # step >= 1
+    assert F.raw_call("focus_mx_step_multi", P, 1, 1, ctypes.byref(hp), 1, 4, None) == 4    # no export flag
+    assert F.raw_call("focus_mx_step_multi", U, 1, 1, ctypes.byref(hp), 1, 0, None) == 3
 
 
 def test_multi_entry_checks(F):

@@ -2,7 +2,9 @@
 sub-blocks of 8) against the oracle: forward (W', codes, E8M0 scales) bit for
 bit, straight-through gradients and the fused step (m, q, moments) within
 |gpu - ref| <= 1e-7 + 1e-5 |ref|, on shapes spanning many blocks with ragged
-grid tails, a Llama-sized tensor, and the non-finite flag."""
+grid tails, a Llama-sized tensor, and the non-finite flag; then the same three
+over a table of tensors, one launch each (an empty entry, ragged tiles, an
+incomplete entry skipped and flagged)."""
 import numpy as np
 import pytest
 import torch
@@ -111,3 +113,114 @@ def test_mx_nonfinite_sets_flag(F):
     forward(F, W, m, q)
     assert F.focus_get_error() == 7
     assert F.focus_get_error() == 0
+
+
+# ---------------------------------------------------------------------------
+# many tensors in one launch (a table prepared for the MXFP4 calls)
+# ---------------------------------------------------------------------------
+
+MULTI_SHAPES = [(1, 32), (3, 96), (37, 1056), (0, 64), (128, 2048), (7, 4128), (257, 160)]
+
+
+def mx_table(F, seed, moments="zero", missing=None):
+    """A table over MULTI_SHAPES (an empty tensor in the middle; 4096-weight tiles with
+    ragged ends) with every output present, except the fields named in `missing` on
+    entry 2."""
+    from fp4_post_weight_b200.table import PURPOSE_MX, Entry, FocusTable
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    ents, hosts = [], []
+    for j, shape in enumerate(MULTI_SHAPES):
+        o, i = shape
+        if o * i:
+            W, m, q, dW = make(shape, seed + 10 * j)
+        else:
+            W, dW = torch.empty(shape, dtype=torch.bfloat16, device="cuda"), torch.empty(shape, dtype=torch.bfloat16,
+                                                                                         device="cuda")
+            m, q = torch.empty((o, i // 32), device="cuda"), torch.empty((o, i // 8), device="cuda")
+        if moments == "warm":
+            v1m, v1q = synth.normal(m.shape, 0, 1e-4, g, "cuda"), synth.normal(q.shape, 0, 1e-6, g, "cuda")
+            mo = [v1m, v1m ** 2 + synth.normal(m.shape, 0, 1e-4, g, "cuda") ** 2,
+                  v1q, v1q ** 2 + synth.normal(q.shape, 0, 1e-6, g, "cuda") ** 2]
+        else:
+            mo = [torch.zeros_like(m), torch.zeros_like(m), torch.zeros_like(q), torch.zeros_like(q)]
+        e = Entry(W=W, m=m, q=q, s2=None, dWq=dW, Wq=torch.empty_like(W), m_exp_avg=mo[0], m_exp_avg_sq=mo[1],
+                  q_exp_avg=mo[2], q_exp_avg_sq=mo[3],
+                  codes=torch.empty((o, i // 2), dtype=torch.uint8, device="cuda"),
+                  scales=torch.empty((o, i // 32), dtype=torch.uint8, device="cuda"),
+                  dm=torch.zeros_like(m), dq=torch.zeros_like(q))
+        if j == 2 and missing:
+            for name in missing:
+                setattr(e, name, None)
+        ents.append(e)
+        hosts.append((host_bits(W), host_bits(dW), host(m).copy(), host(q).copy(), [host(x).copy() for x in mo]))
+    return FocusTable(ents, PURPOSE_MX), hosts
+
+
+def test_mx_multi_forward(F):
+    tab, hosts = mx_table(F, 300)
+    tab.mx_fwd()
+    assert F.focus_get_error() == 0
+    for e, (Wb, _, hm, hq, _) in zip(tab.entries, hosts):
+        if e.W.numel() == 0:
+            continue
+        ref = oracle.mx_fwd(Wb, hm, hq)
+        np.testing.assert_array_equal(host(e.scales), ref.scales)
+        np.testing.assert_array_equal(unpack_codes(host(e.codes)), ref.codes)
+        np.testing.assert_array_equal(host_bits(e.Wq), ref.Wq)
+
+
+def test_mx_multi_backward(F):
+    tab, hosts = mx_table(F, 400)
+    tab.mx_bwd()
+    tab.mx_bwd(accumulate=True)
+    assert F.focus_get_error() == 0
+    for e, (Wb, Gb, hm, hq, _) in zip(tab.entries, hosts):
+        if e.W.numel() == 0:
+            continue
+        rdm, rdq = oracle.mx_ste_bwd(Wb, Gb, hm, hq)
+        oracle.mx_ste_bwd(Wb, Gb, hm, hq, dm=rdm, dq=rdq)
+        assert_close(host(e.dm), rdm, "dm (two micro-batches)")
+        assert_close(host(e.dq), rdq, "dq (two micro-batches)")
+
+
+@pytest.mark.parametrize("step,moments", [(1, "zero"), (5, "warm")])
+def test_mx_multi_step(F, step, moments):
+    from fp4_post_weight_b200.table import hparams
+    tab, hosts = mx_table(F, 500 + step, moments)
+    tab.mx_step(step, hparams(), F.FOCUS_STEP_WRITE_GRAD)
+    assert F.focus_get_error() == 0
+    for e, (Wb, Gb, hm, hq, hmo) in zip(tab.entries, hosts):
+        if e.W.numel() == 0:
+            continue
+        ref = oracle.mx_fwd(Wb, hm, hq)
+        np.testing.assert_array_equal(host_bits(e.Wq), ref.Wq)          # W' of the parameters before the update
+        gm, gq = oracle.mx_ste_bwd(Wb, Gb, hm, hq)
+        assert_close(host(e.dm), gm, "dm")
+        assert_close(host(e.dq), gq, "dq")
+        oracle.adamw(hm, gm, hmo[0], hmo[1], 5e-3, step)
+        oracle.adamw(hq, gq, hmo[2], hmo[3], 1e-3, step)
+        assert_close(host(e.m), hm, "m")
+        assert_close(host(e.q), hq, "q")
+        for name, t, r in zip(("m exp_avg", "m exp_avg_sq", "q exp_avg", "q exp_avg_sq"),
+                              (e.m_exp_avg, e.m_exp_avg_sq, e.q_exp_avg, e.q_exp_avg_sq), hmo):
+            assert_close(host(t), r, name)
+
+
+def test_mx_multi_step_skips_an_incomplete_entry(F):
+    """An entry without a pointer the step needs (its second moment of q) is skipped
+    and flagged; the other entries are stepped as usual."""
+    from fp4_post_weight_b200.table import hparams
+    tab, hosts = mx_table(F, 600, missing=("q_exp_avg_sq",))
+    m2 = host(tab.entries[2].m).copy()
+    assert F.focus_get_error() == 0
+    tab.mx_step(1, hparams())
+    assert F.focus_get_error() == 7
+    np.testing.assert_array_equal(host(tab.entries[2].m), m2)          # untouched
+    Wb, Gb, hm, hq, hmo = hosts[1]
+    gm, gq = oracle.mx_ste_bwd(Wb, Gb, hm, hq)
+    oracle.adamw(hm, gm, hmo[0], hmo[1], 5e-3, 1)
+    assert_close(host(tab.entries[1].m), hm, "m of the entry before")
+    Wb, Gb, hm, hq, hmo = hosts[4]
+    gm, gq = oracle.mx_ste_bwd(Wb, Gb, hm, hq)
+    oracle.adamw(hq, gq, hmo[2], hmo[3], 1e-3, 1)
+    assert_close(host(tab.entries[4].q), hq, "q of an entry after")

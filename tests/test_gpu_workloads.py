@@ -8,9 +8,10 @@
 * C2: all 112 Llama-3.2-1B linears, one fused step as one multi-tensor launch:
   full parity of W', gradients, m, q and moments.
 * C3: all 224 Llama-3.1-8B linears in exactly the launch configuration the
-  benchmark times (s2, then the fused step with W' and the export of the
-  updated parameters): full parity on one tensor of each shape, a 1/64 row
-  sample of every other tensor.
+  benchmark times (the fused step with W', the export of the updated
+  parameters and the tensor maxima, then s2 from those maxima): full parity on
+  one tensor of each shape, a 1/64 row sample of every other tensor, every
+  tensor's maximum and its s2 after the step.
 * C5: Llama-3.1-70B layers 0, 40 and 79, one layer at a time: a 1/256 row
   sample.
 
@@ -220,8 +221,9 @@ def _rows(out, stride):
 
 
 def test_c3_llama_8b_bench_configuration(F):
-    """The benchmark's launch: s2 over all 224 tensors, then one fused step with W'
-    and the NVFP4 export of the updated parameters."""
+    """The benchmark's launch: s2 over all 224 tensors, then the fused step with W',
+    the NVFP4 export of the updated parameters and the tensor maxima, then s2 of
+    every tensor from those maxima (equal to the first s2: W is frozen)."""
     from fp4_post_weight_b200.table import FocusTable, hparams
     tensors = []
     for j, (_, sh) in enumerate(synth.LLAMA_8B.tensors()):
@@ -231,12 +233,22 @@ def test_c3_llama_8b_bench_configuration(F):
     full_idx = {j for j in range(7)}                  # layer 0: one tensor of each shape, in full
     samples = [None if j in full_idx else _rows(t.W.shape[0], 64) for j, t in enumerate(tensors)]
     snaps = [_snapshot(t, rows) for t, rows in zip(tensors, samples)]
-    s2s = [oracle.s2(host_bits(t.W)) for t in tensors]          # over every row, from the generated W
+    s2s, amax_bits = [], []
+    for t in tensors:                                 # over every row, from the generated W
+        wb = host_bits(t.W)
+        s2s.append(oracle.s2(wb))
+        amax_bits.append(int(np.max(wb & 0x7FFF)))    # max |w| as bf16 magnitude bits
+        del wb
     ents = _table_entries(tensors, want_grad=False, export=True)
     tab = FocusTable(ents)
     tab.s2()
-    tab.step(1, hparams(), flags=F.FOCUS_STEP_PACK_UPDATED)
+    ws = torch.zeros(max(tab.n, 4), dtype=torch.int32, device="cuda")
+    F.focus_step_fused_amax(tab.dev, tab.n, tab.total_tiles, hparams(), 1, ws, F.FOCUS_STEP_PACK_UPDATED)
     assert F.focus_get_error() == 0
+    assert host(ws)[:tab.n].tolist() == amax_bits    # the maxima the step reduced, every tensor
+    F.focus_s2_from_amax(tab.dev, tab.n, ws)
+    assert F.focus_get_error() == 0
+    assert not host(ws).any()                         # cleared for the next step
     tot = {}
     checked = 0
     for e, snap, rows, s2 in zip(ents, snaps, samples, s2s):
