@@ -296,26 +296,27 @@ __device__ __forceinline__ F46Target f46_target(float x, float s, float A) {
     return t;
 }
 
-// Codes of one pair of weights (negated, as a packed pair) under a target, and
-// the pair's contribution to the target's squared error: d' = fl(c*S*s - w)
-// = -fl(w - c*S*s) in one rounding (c*S is exact), E <- fma(d', d', E), one
-// packed lane for the even element and one for the odd.  FAST: the quotient
-// from the reciprocal (D2, nr2 = (D, D), (-fl(1/D), ...)); else IEEE division.
+// The quotient pair y = w / D of one pair of weights under a target.  FAST:
+// from the reciprocal (nw the negated pair, D2, nr2 = (D, D), (-fl(1/D), ...));
+// else IEEE division.
 template <bool FAST>
-__device__ __forceinline__ uint32_t f46_pair(uint64_t nw, uint32_t wv, float D, uint64_t D2, uint64_t nr2,
-                                             uint16_t S_h, uint64_t s_2, uint64_t &E2) {
-    uint64_t y2;
-    if (FAST) y2 = div_by_f2(nw, D2, nr2);
-    else y2 = f2_pack(__fdiv_rn(bf16_lo(wv), D), __fdiv_rn(bf16_hi(wv), D));
-    const uint32_t byte = e2m1_pair(f2_lo(y2), f2_hi(y2));
-    const uint32_t h2 = e2m1_pair_f16x2(byte);
+__device__ __forceinline__ uint64_t f46_quot(uint64_t nw, uint32_t wv, float D, uint64_t D2, uint64_t nr2) {
+    if (FAST) return div_by_f2(nw, D2, nr2);
+    return f2_pack(__fdiv_rn(bf16_lo(wv), D), __fdiv_rn(bf16_hi(wv), D));
+}
+
+// A pair's contribution to a target's squared error from its code values h2
+// (binary16 pair): d' = fl(c*S*s - w) = -fl(w - c*S*s) in one rounding (c*S
+// is exact), E <- fma(d', d', E), one packed lane for the even element and one
+// for the odd.
+__device__ __forceinline__ void f46_err(uint32_t h2, uint64_t nw, uint16_t S_h, uint64_t s_2, uint64_t &E2) {
     const uint64_t cs2 = f2_pack(mul_f16_exact(lo16(h2), S_h), mul_f16_exact(hi16(h2), S_h));
     const uint64_t d2 = f2_fma(cs2, s_2, nw);
     E2 = f2_fma(d2, d2, E2);
-    return byte;
 }
 
 // Both targets side by side over the block's pairs: code words and errors.
+// Each 8-element half is converted four pairs at a time (e2m1_quad).
 template <bool FAST>
 __device__ __forceinline__ void f46_both(const uint32_t *w, const F46Target &t6, const F46Target &t4, float s,
                                          uint32_t c6[2], uint32_t c4[2], float &e6, float &e4) {
@@ -325,16 +326,21 @@ __device__ __forceinline__ void f46_both(const uint32_t *w, const F46Target &t6,
     uint64_t E6 = 0ull, E4 = 0ull;
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
-        uint32_t a6 = 0u, a4 = 0u;
+        uint64_t nw[4], y[4];
+        uint32_t h[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint32_t wv = w[4 * k + j];
-            const uint64_t nw = bf16x2_neg_f2(wv);
-            a6 |= f46_pair<FAST>(nw, wv, t6.D, D6, n6, t6.S_h, s_2, E6) << (8 * j);
-            a4 |= f46_pair<FAST>(nw, wv, t4.D, D4, n4, t4.S_h, s_2, E4) << (8 * j);
+            nw[j] = bf16x2_neg_f2(w[4 * k + j]);
+            y[j] = f46_quot<FAST>(nw[j], w[4 * k + j], t6.D, D6, n6);
         }
-        c6[k] = a6;
-        c4[k] = a4;
+        c6[k] = e2m1_quad(y, h);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) f46_err(h[j], nw[j], t6.S_h, s_2, E6);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) y[j] = f46_quot<FAST>(nw[j], w[4 * k + j], t4.D, D4, n4);
+        c4[k] = e2m1_quad(y, h);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) f46_err(h[j], nw[j], t4.S_h, s_2, E4);
     }
     e6 = __fadd_rn(f2_lo(E6), f2_hi(E6));
     e4 = __fadd_rn(f2_lo(E4), f2_hi(E4));

@@ -8,7 +8,8 @@ configurations bench.py times:
   for a micro-batch of 4096 tokens (four launches), in full;
 * the MXFP4 fused step, one launch per tensor, on layer 0 of the 8B shapes
   with the benchmark's parameters (m = 1, q = 6, zero moments), a 1/16 row
-  sample against the oracle.
+  sample against the oracle, and the same step as one launch over a table of
+  all 224 tensors (layer 0 at 1/16, the rest at 1/128 of the rows).
 """
 import numpy as np
 import pytest
@@ -100,3 +101,41 @@ def test_mx_step_llama_8b_layer0_sampled(F):
         assert_close(host(q[rows]), hq, "q")
         for name, x, r in zip(("m exp_avg", "m exp_avg_sq", "q exp_avg", "q exp_avg_sq"), mo, hmo):
             assert_close(host(x[rows]), r, name)
+
+
+def test_mx_step_table_llama_8b_sampled(F):
+    """The MXFP4 step as one launch over a table of all 224 8B linears (the bench's
+    one-launch line): a 1/16 row sample of layer 0 and a 1/128 row sample of every
+    other tensor against the oracle."""
+    from fp4_post_weight_b200.table import PURPOSE_MX, Entry, FocusTable, hparams
+    ents, checks = [], []
+    for j, (_, (o, i)) in enumerate(synth.LLAMA_8B.tensors()):
+        t = synth.llama_8b_tensor(j, (o, i), "cuda")
+        m = torch.ones((o, i // 32), device="cuda")
+        q = torch.full((o, i // 8), 6.0, device="cuda")
+        e = Entry(W=t.W, m=m, q=q, s2=None, dWq=t.dWq, Wq=torch.empty_like(t.W),
+                  m_exp_avg=torch.zeros_like(m), m_exp_avg_sq=torch.zeros_like(m),
+                  q_exp_avg=torch.zeros_like(q), q_exp_avg_sq=torch.zeros_like(q))
+        ents.append(e)
+        rows = _rows(o, 16 if j < 7 else 128)
+        checks.append((rows, host_bits(t.W[rows]), host_bits(t.dWq[rows])))
+    tab = FocusTable(ents, PURPOSE_MX)
+    tab.mx_step(1, hparams())
+    assert F.focus_get_error() == 0
+    checked = 0
+    for e, (rows, Wb, Gb) in zip(ents, checks):
+        o, i = e.W.shape
+        hm = np.ones((len(rows), i // 32), np.float32)
+        hq = np.full((len(rows), i // 8), 6.0, np.float32)
+        hmo = [np.zeros_like(hm), np.zeros_like(hm), np.zeros_like(hq), np.zeros_like(hq)]
+        np.testing.assert_array_equal(host_bits(e.Wq[rows]), oracle.mx_fwd(Wb, hm, hq).Wq)
+        gm, gq = oracle.mx_ste_bwd(Wb, Gb, hm, hq)
+        oracle.adamw(hm, gm, hmo[0], hmo[1], 5e-3, 1)
+        oracle.adamw(hq, gq, hmo[2], hmo[3], 1e-3, 1)
+        assert_close(host(e.m[rows]), hm, "m")
+        assert_close(host(e.q[rows]), hq, "q")
+        for name, x, r in zip(("m exp_avg", "m exp_avg_sq", "q exp_avg", "q exp_avg_sq"),
+                              (e.m_exp_avg, e.m_exp_avg_sq, e.q_exp_avg, e.q_exp_avg_sq), hmo):
+            assert_close(host(x[rows]), r, name)
+        checked += Wb.size
+    print(f"MXFP4 table step: {checked} weights checked over {len(ents)} tensors")
