@@ -505,18 +505,20 @@ def host_budget_bytes(world: int) -> int:
 
 
 def run_e2e(args, ents, N, world, dev):
-    """The same step through the C ABI with host buffers: per step every input
-    (W, dW', m, q, moments) is copied from pinned host memory and every output
-    (W', m, q, moments, codes, scales, s2) is copied back, tensor by tensor on
-    two copy streams overlapping the compute stream.  It runs on as many whole
-    decoder layers as the host's memory holds for every rank (all 32 on one
-    B200 machine: 77 GB pinned); the rate is per weight, so it is the same metric."""
+    """The same step through the C ABI with HOST buffers: focus_step_host, the
+    library's host-buffer executor, uploads every input (W, dW', m, q, moments,
+    s2) from pinned host memory, steps each tensor and reads every output (W',
+    m, q, moments, codes, scales, s2) back, overlapping the uploads and
+    read-backs of neighbouring tensors with the step; one blocking call per
+    step.  It runs on as many whole decoder layers as the host's memory holds
+    for every rank (all 32 on one B200 machine: 77 GB pinned); the rate is per
+    weight, so it is the same metric."""
     import torch
 
     from fp4_post_weight_b200 import dist as D
     from fp4_post_weight_b200 import focus as F
-    from fp4_post_weight_b200.table import FocusTable, hparams
-    ins = ("W", "dWq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq")
+    from fp4_post_weight_b200.table import Entry, HostTable, hparams
+    ins = ("W", "dWq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq", "s2")
     outs = ("Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq", "codes", "scales", "s2")
     names = set(ins) | set(outs)
     per_layer = sum(getattr(e, n).numel() * getattr(e, n).element_size() for e in ents[:7] for n in names)
@@ -527,60 +529,36 @@ def run_e2e(args, ents, N, world, dev):
     hosts = []
     for e in ents:
         h = {}
-        for n in set(ins) | set(outs):
+        for n in names:
             t = getattr(e, n)
             h[n] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
             h[n].copy_(t)
-        hosts.append(h)
-    tabs = [FocusTable([e]) for e in ents]
-    h2d, comp, d2h = torch.cuda.Stream(dev), torch.cuda.current_stream(dev), torch.cuda.Stream(dev)
+        hosts.append(Entry(W=h["W"], m=h["m"], q=h["q"], s2=h["s2"], dWq=h["dWq"], Wq=h["Wq"],
+                           m_exp_avg=h["m_exp_avg"], m_exp_avg_sq=h["m_exp_avg_sq"], q_exp_avg=h["q_exp_avg"],
+                           q_exp_avg_sq=h["q_exp_avg_sq"], codes=h["codes"], scales=h["scales"]))
+    htab = HostTable(hosts, dev)
     hp = hparams()
-    bi = sum(h[n].numel() * h[n].element_size() for h in hosts for n in ins)
-    bo = sum(h[n].numel() * h[n].element_size() for h in hosts for n in outs)
-
-    done_out = [None] * len(ents)     # per tensor: its read-back of the previous step
-
-    def step(t):
-        done_in, done_c = [], []
-        for j, (e, h) in enumerate(zip(ents, hosts)):
-            # a tensor's upload must not overwrite it while its previous read-back
-            # runs (and reads the host copy that read-back writes): wait for that
-            # tensor only, so the next step's uploads overlap this step's read-backs
-            if done_out[j] is not None:
-                h2d.wait_event(done_out[j])
-            with torch.cuda.stream(h2d):
-                for n in ins:
-                    getattr(e, n).copy_(h[n], non_blocking=True)
-                ev = torch.cuda.Event(); ev.record(h2d); done_in.append(ev)
-        for e, tab, ev in zip(ents, tabs, done_in):
-            comp.wait_event(ev)
-            tab.step_s2(t, hp, F.FOCUS_STEP_PACK_UPDATED, stream=comp)
-            ec = torch.cuda.Event(); ec.record(comp); done_c.append(ec)
-        for j, (e, h, ec) in enumerate(zip(ents, hosts, done_c)):
-            d2h.wait_event(ec)
-            with torch.cuda.stream(d2h):
-                for n in outs:
-                    h[n].copy_(getattr(e, n), non_blocking=True)
-            eo = torch.cuda.Event(); eo.record(d2h); done_out[j] = eo
-
-    for tab in tabs:
-        tab.s2(stream=comp)                           # s2 before the first step
+    bi = sum(getattr(h, n).numel() * getattr(h, n).element_size() for h in hosts for n in ins)
+    bo = sum(getattr(h, n).numel() * getattr(h, n).element_size() for h in hosts for n in outs)
+    stream = torch.cuda.current_stream(dev)
     steps = max(1, args.e2e_steps)
-    step(1)
+    htab.step(1, hp, F.FOCUS_STEP_PACK_UPDATED, stream)          # warm-up (s2 is in the host copies)
     torch.cuda.synchronize()
     D.barrier()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(h2d)
+    s.record(stream)
     for k in range(steps):
-        step(2 + k)
-    d2h.synchronize()
-    e.record(d2h)
+        htab.step(2 + k, hp, F.FOCUS_STEP_PACK_UPDATED, stream)  # blocking: results are in host memory
+    e.record(stream)
     torch.cuda.synchronize()
     ms = D.max_over_ranks(s.elapsed_time(e)) / steps
-    del hosts
+    st = F.focus_get_error()
+    if st != 0:
+        raise SystemExit(f"device status after the host-buffer steps: {F.focus_status_string(st)}")
+    del hosts, htab
     return {"value": round(N * world / (ms * 1e-3) / 1e9, 3), "unit": "Gelem/s", "h2d_bytes_per_step": bi,
             "d2h_bytes_per_step": bo, "ms_per_step": round(ms, 2), "steps": steps, "layers": layers,
-            "weights_per_rank": N}
+            "weights_per_rank": N, "api": "focus_step_host (one blocking call per step)"}
 
 
 # ---------------------------------------------------------------------------

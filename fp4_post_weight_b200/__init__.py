@@ -16,6 +16,7 @@ _BINDING_NAMES = {"focus_s2", "focus_fwd", "focus_ste_bwd", "focus_adamw_step", 
                   "focus_fouroversix_act_swizzled",
                   "focus_scales_swizzle", "focus_scales_swizzled_bytes", "focus_mx_fwd", "focus_mx_ste_bwd",
                   "focus_mx_step", "focus_mx_fwd_multi", "focus_mx_ste_bwd_multi", "focus_mx_step_multi",
+                  "focus_step_host", "focus_step_host_workspace_bytes",
                   "focus_step_fused_amax", "focus_s2_from_amax",
                   "focus_get_error", "focus_s2_workspace_bytes", "focus_s2_multi_workspace_bytes",
                   "focus_status_string", "focus_version", "FocusError", "focus_tensor_desc", "focus_hparams"}

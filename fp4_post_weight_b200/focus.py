@@ -30,6 +30,7 @@ FOCUS_STEP_WRITE_GRAD = 2
 FOCUS_STEP_PACK_UPDATED = 4
 FOCUS_STEP_WQ_UPDATED = 8
 FOCUS_PURPOSE_MX = 4
+FOCUS_HOST_S2_FIRST = 16
 
 
 class focus_tensor_desc(ctypes.Structure):
@@ -79,6 +80,8 @@ _SIGS = {
     "focus_mx_step_multi": ([_P, _I, _I64, ctypes.POINTER(focus_hparams), _I64, ctypes.c_uint, _P], _I),
     "focus_scales_swizzled_bytes": ([_I64, _I64], _SZ),
     "focus_scales_swizzle": ([_P, _I64, _I64, _P, _SZ, _P], _I),
+    "focus_step_host_workspace_bytes": ([_P, _I], _SZ),
+    "focus_step_host": ([_P, _I, ctypes.POINTER(focus_hparams), _I64, ctypes.c_uint, _P, _SZ, _P], _I),
     "focus_get_error": ([_P], _I),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -338,6 +341,29 @@ def focus_scales_swizzle(scales, out, stream=None, rows=None, cols=None):
     r, c = _shape(scales, rows, cols)
     nbytes = out.numel() * out.element_size() if isinstance(out, torch.Tensor) else 1 << 62
     _check(_lib.focus_scales_swizzle(_ptr(scales), r, c, _ptr(out), nbytes, _stream(stream)), "focus_scales_swizzle")
+
+
+def host_ptr(x):
+    """Address of a contiguous CPU tensor (for focus_step_host), or None."""
+    if x is None:
+        return None
+    if not isinstance(x, torch.Tensor) or x.is_cuda:
+        raise ValueError("host tensors only")
+    if not x.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return x.data_ptr() if x.numel() else None
+
+
+def focus_step_host_workspace_bytes(descs_host, n: int) -> int:
+    return int(_lib.focus_step_host_workspace_bytes(descs_host, int(n)))
+
+
+def focus_step_host(descs_host, n: int, hp: focus_hparams, step: int, flags: int, ws, stream=None):
+    """The fused step over tensors in host memory (descs_host: a focus_tensor_desc array
+    holding host pointers); blocks until every result is back in host memory."""
+    nbytes = ws.numel() * ws.element_size() if isinstance(ws, torch.Tensor) else 1 << 62
+    _check(_lib.focus_step_host(descs_host, int(n), ctypes.byref(hp), int(step), int(flags), _ptr(ws), nbytes,
+                                _stream(stream)), "focus_step_host")
 
 
 def focus_get_error(stream=None) -> int:

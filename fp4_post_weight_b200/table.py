@@ -109,3 +109,27 @@ class FocusTable:
 def hparams(lr_m=5e-3, lr_q=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0) -> F.focus_hparams:
     """The card's calibration setting: AdamW, lr 5e-3 for m and 1e-3 for q, betas 0.9/0.999, wd 0."""
     return F.focus_hparams(lr_m, lr_q, beta1, beta2, eps, weight_decay)
+
+
+class HostTable:
+    """Tensors held in host memory, stepped through focus_step_host: every call uploads
+    the step's inputs, steps each tensor on the device and reads the updated parameters
+    and outputs back (blocking).  Entries use host tensors (pinned for overlap): W,
+    dWq, m, q, the moments, s2 (one float32) and optionally Wq, codes, scales."""
+
+    def __init__(self, entries: list[Entry], device=None):
+        self.entries = list(entries)
+        n = len(self.entries)
+        self.n = n
+        descs = (F.focus_tensor_desc * max(n, 1))()
+        for i, e in enumerate(self.entries):
+            d = descs[i]
+            for name in _FIELDS:
+                setattr(d, name, F.host_ptr(getattr(e, name)))
+            d.out, d.in_ = int(e.W.shape[0]), int(e.W.shape[1])
+        self.descs = descs
+        need = F.focus_step_host_workspace_bytes(descs, n) if n else 0
+        self.ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device or "cuda")
+
+    def step(self, step: int, hp: F.focus_hparams | None = None, flags: int = 0, stream=None):
+        F.focus_step_host(self.descs, self.n, hp or hparams(), step, flags, self.ws, stream)

@@ -411,6 +411,44 @@ int focus_scales_swizzle(const uint8_t *scales, int64_t rows, int64_t cols, uint
                          focus_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * The fused step over tensors held in HOST memory (the same computation as
+ * focus_step_fused_amax + focus_s2_from_amax on device-resident tensors).
+ *
+ * host_descs: n_tensors focus_tensor_desc in host memory whose pointers are
+ * HOST pointers: W, dWq (read), m, q and the four moments (read, then
+ * overwritten with the updated values), s2 (one float: read unless
+ * FOCUS_HOST_S2_FIRST, then overwritten with s2 for the next step), Wq and
+ * codes+scales (optional outputs, written); dm and dq must be NULL
+ * (FOCUS_ERR_VALUE); block_begin and tile_begin are ignored.  Shapes as in
+ * focus_table_prepare (in % 16 == 0); empty tensors are skipped.
+ *
+ * Per tensor, in three device slots carved from the caller's workspace: the
+ * inputs are uploaded, the step (with s2 first under FOCUS_HOST_S2_FIRST, and
+ * the tensor maximum) runs on `stream`, and the outputs are read back; the
+ * upload and read-back of neighbouring tensors run on two streams of the call
+ * while a tensor is stepped.  Host buffers should be pinned (page-locked):
+ * pageable buffers give the same results, with the copies serialised by the
+ * host.
+ *
+ * ws_dev: device memory, 256-byte aligned, at least
+ * focus_step_host_workspace_bytes(host_descs, n_tensors) bytes (three slots
+ * of 8.81 bytes per weight of the largest tensor plus small fields), else
+ * FOCUS_ERR_WORKSPACE.  flags: FOCUS_STEP_PACK_UPDATED, FOCUS_STEP_WQ_UPDATED,
+ * FOCUS_HOST_S2_FIRST; others give FOCUS_ERR_VALUE.  Every entry is checked on
+ * the host before anything is enqueued (a missing pointer: FOCUS_ERR_NULL; a
+ * stored s2 that is not finite and > 0 without FOCUS_HOST_S2_FIRST:
+ * FOCUS_ERR_VALUE).
+ *
+ * BLOCKING: the call returns when every result is in host memory (it creates
+ * and releases its two copy streams and its events).  The device flag is
+ * reported by focus_get_error as for the other calls.
+ * ------------------------------------------------------------------------- */
+#define FOCUS_HOST_S2_FIRST 16u   /* compute s2 from W in the slot before the step (first step) */
+size_t focus_step_host_workspace_bytes(const focus_tensor_desc *host_descs, int n_tensors);
+int focus_step_host(const focus_tensor_desc *host_descs, int n_tensors, const focus_hparams *hp, int64_t step,
+                    unsigned flags, void *ws_dev, size_t ws_bytes, focus_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Synchronizes `stream`, then reports and clears the sticky device flag:
  * FOCUS_ERR_DEVICE_TIMEOUT when a kernel's pipeline wait ran out,
  * FOCUS_ERR_NONFINITE_INPUT when any kernel since the last call met a

@@ -180,6 +180,47 @@ def test_mx_multi_checks(F):
     assert F.raw_call("focus_mx_step_multi", U, 1, 1, ctypes.byref(hp), 1, 0, None) == 3
 
 
+def test_step_host_checks(F):
+    """focus_step_host checks every entry on the host before it enqueues anything."""
+    hp = F.focus_hparams(5e-3, 1e-3, 0.9, 0.999, 1e-8, 0.0)
+    S = ctypes.c_size_t
+    s2 = (ctypes.c_float * 2)(0.01, 0.0)
+    descs = (F.focus_tensor_desc * 2)()
+    for i, (o, k) in enumerate([(4, 32), (3, 16)]):
+        d = descs[i]
+        for name in ("W", "dWq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"):
+            setattr(d, name, P)
+        d.s2 = ctypes.addressof(s2) + 4 * i
+        d.out, d.in_ = o, k
+    need = F.focus_step_host_workspace_bytes(descs, 2)
+    # three slots of the largest tensor (128 weights): about 8.8 bytes per weight plus fields
+    assert 3 * 8.8125 * 128 <= need <= 3 * (8.8125 * 128 + 16 * 256)
+    W = 1 << 40                                   # a 256-byte aligned address, never dereferenced
+    call = lambda *a: F.raw_call("focus_step_host", *a)
+    assert call(descs, -1, ctypes.byref(hp), 1, 0, W, S(need), None) == 4
+    assert call(descs, 2, None, 1, 0, W, S(need), None) == 1
+    assert call(descs, 2, ctypes.byref(hp), 1, 1, W, S(need), None) == 4          # ACCUMULATE: not on this path
+    assert call(descs, 0, ctypes.byref(hp), 1, 0, None, S(0), None) == 0
+    assert call(None, 2, ctypes.byref(hp), 1, 0, W, S(need), None) == 1
+    assert call(descs, 2, ctypes.byref(hp), 1, 0, W, S(need), None) == 4          # entry 1: s2 = 0
+    assert call(descs, 1, ctypes.byref(hp), 1, 0, None, S(need), None) == 1       # no workspace
+    assert call(descs, 1, ctypes.byref(hp), 1, 0, W + 16, S(need), None) == 3     # not 256-byte aligned
+    assert call(descs, 1, ctypes.byref(hp), 1, 0, W, S(need - 1), None) == 5
+    s2[1] = 0.02
+    descs[1].in_ = 24
+    assert call(descs, 2, ctypes.byref(hp), 1, 0, W, S(need), None) == 2
+    assert F.focus_step_host_workspace_bytes(descs, 2) == 0
+    descs[1].in_ = 16
+    descs[1].q_exp_avg = None
+    assert call(descs, 2, ctypes.byref(hp), 1, 0, W, S(need), None) == 1
+    descs[1].q_exp_avg = P
+    descs[1].dm = P
+    assert call(descs, 2, ctypes.byref(hp), 1, 0, W, S(need), None) == 4          # no gradient buffers
+    descs[1].dm = None
+    descs[1].codes = P                                                             # codes without scales
+    assert call(descs, 2, ctypes.byref(hp), 1, 0, W, S(need), None) == 1
+
+
 def test_multi_entry_checks(F):
     assert F.raw_call("focus_ste_bwd_multi", P, 1, 1, 2, None) == 4        # accumulate must be 0 or 1
     assert F.raw_call("focus_ste_bwd_multi", None, 1, 1, 0, None) == 1
