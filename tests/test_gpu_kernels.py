@@ -423,3 +423,48 @@ def test_step_with_s2_for_the_next_step(F):
             want = oracle.s2(host_bits(a.W)) if a.W.numel() else np.float32(0)
             assert host(a.s2)[0] == want and host(b.s2)[0] == want
     assert int(ta._amax.abs().sum()) == 0          # cleared for the next step
+
+
+def test_step_skips_an_all_zero_tensor_and_reports_it(F):
+    """A tensor whose W is all zero has s2 = 0, which the method cannot divide by:
+    the table step leaves that entry untouched and sets the device flag
+    (FOCUS_ERR_NONFINITE_INPUT); the other entries are stepped exactly as in a
+    table without it, and the tensor maximum leaves s2 = 0 for the zero tensor."""
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    shapes = [(37, 1040), (64, 256), (7, 4112)]
+    ea, eb = _entries(shapes, 120), _entries(shapes, 120)
+    ea[1].W.zero_()
+    m_before = ea[1].m.clone()
+    q_before = ea[1].q.clone()
+    ta, tb = FocusTable(ea), FocusTable([eb[0], eb[2]])
+    ta.s2(); tb.s2()
+    assert F.focus_get_error() == 0
+    assert host(ea[1].s2)[0] == 0.0
+    ta.step_s2(1, hparams(), flags=F.FOCUS_STEP_PACK_UPDATED)
+    assert F.focus_get_error() == 7
+    assert F.focus_get_error() == 0                 # cleared
+    tb.step_s2(1, hparams(), flags=F.FOCUS_STEP_PACK_UPDATED)
+    assert F.focus_get_error() == 0
+    assert torch.equal(ea[1].m, m_before) and torch.equal(ea[1].q, q_before)
+    assert host(ea[1].s2)[0] == 0.0
+    for a, b in ((ea[0], eb[0]), (ea[2], eb[2])):
+        for name in ("Wq", "codes", "scales", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq", "s2"):
+            x, y = getattr(a, name), getattr(b, name)
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8)), name
+
+
+def test_step_on_a_table_without_moments_is_skipped_and_reported(F):
+    """A table prepared for the forward (purpose 0: no AdamW moments) handed to the
+    step: the kernel meets entries lacking pointers it needs, skips them without
+    dereferencing anything and sets the device flag; nothing is written."""
+    from fp4_post_weight_b200.table import PURPOSE_FORWARD, Entry, FocusTable, hparams
+    W, m, q, dW = make((37, 1040), 130)
+    e = Entry(W=W, m=m, q=q, s2=torch.zeros(1, device="cuda"), dWq=dW, Wq=torch.zeros_like(W))
+    tab = FocusTable([e], PURPOSE_FORWARD)
+    tab.s2()
+    assert F.focus_get_error() == 0
+    m0, q0 = m.clone(), q.clone()
+    tab.step(1, hparams())
+    assert F.focus_get_error() == 7
+    assert torch.equal(m, m0) and torch.equal(q, q0)
+    assert not e.Wq.view(torch.int16).any()
