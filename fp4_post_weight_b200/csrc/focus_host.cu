@@ -140,7 +140,6 @@ int focus_step_host(const focus_tensor_desc *h, int n, const focus_hparams *hp, 
     if (!R.ok) return FOCUS_ERR_CUDA;
     std::vector<focus_tensor_desc> dd(n);     // the device descriptors (host copies, uploaded per tensor)
     std::vector<int> slot_of(n, -1);
-    std::vector<int64_t> tiles_of(n, 0);
     const unsigned step_flags = flags & (FOCUS_STEP_PACK_UPDATED | FOCUS_STEP_WQ_UPDATED);
     int rc = FOCUS_OK;
     bool cuda_ok = cudaEventRecord(R.entry, comp) == cudaSuccess && cudaStreamWaitEvent(R.up, R.entry, 0) == cudaSuccess;
@@ -173,7 +172,6 @@ int focus_step_host(const focus_tensor_desc *h, int n, const focus_hparams *hp, 
         d.in = e.in;
         int64_t tiles = 0;
         if (rc == FOCUS_OK) rc = focus_table_prepare(&d, 1, 1, &tiles);
-        tiles_of[i] = tiles;
         slot_of[i] = s;
         if (rc != FOCUS_OK) return;
         // upload: after the slot's previous read-back
