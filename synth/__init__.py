@@ -98,17 +98,19 @@ class Tensors:
 
 
 def adam_states(t: Tensors, g: torch.Generator | None = None, warm: bool = False) -> Tensors:
-    """Zero AdamW moments (step 1), or warm ones: first moments N(0, 1e-4),
-    second moments |N(0, 1e-6)|^2-like non-negative values (a later step)."""
+    """Zero AdamW moments (step 1), or warm ones as a run leaves them (a later
+    step): first moments v1 ~ N(0, sigma), second moments v2 = v1^2 + N(0, sigma)^2,
+    random, non-negative and at least v1^2 (an EMA of squares bounds the EMA of
+    the values), with sigma = 1e-4 for m and 1e-6 for q."""
     dev = t.m.device
     if not warm:
         t.m_v1 = torch.zeros_like(t.m); t.m_v2 = torch.zeros_like(t.m)
         t.q_v1 = torch.zeros_like(t.q); t.q_v2 = torch.zeros_like(t.q)
     else:
         t.m_v1 = normal(t.m.shape, 0.0, 1e-4, g, dev)
-        t.m_v2 = normal(t.m.shape, 0.0, 1e-4, g, dev) ** 2
+        t.m_v2 = t.m_v1 ** 2 + normal(t.m.shape, 0.0, 1e-4, g, dev) ** 2
         t.q_v1 = normal(t.q.shape, 0.0, 1e-6, g, dev)
-        t.q_v2 = normal(t.q.shape, 0.0, 1e-6, g, dev) ** 2
+        t.q_v2 = t.q_v1 ** 2 + normal(t.q.shape, 0.0, 1e-6, g, dev) ** 2
     return t
 
 

@@ -5,7 +5,8 @@
 * C4: the stress tensor W[8192, 8192] (Student-t, planted zero, tie and clamp
   blocks): forward, pack and straight-through backward, full parity, and the
   counts of the planted cases.
-* C2: all 112 Llama-3.2-1B linears, one fused step as one multi-tensor launch:
+* C2: all 112 Llama-3.2-1B linears, one fused step as one multi-tensor launch
+  (step 1 with zero AdamW moments, and step 5 with warm ones):
   full parity of W', gradients, m, q and moments.
 * C3: all 224 Llama-3.1-8B linears in exactly the launch configuration the
   benchmark times (the fused step with W', the export of the updated
@@ -188,24 +189,28 @@ def _compare_step(e, snap, s2, step, rows=None, export=False):
     return out
 
 
-def test_c2_llama_1b_fused_step_full(F):
+@pytest.mark.parametrize("step,warm", [(1, False), (5, True)])
+def test_c2_llama_1b_fused_step_full(F, step, warm):
+    """All 112 Llama-3.2-1B linears in one fused step: at step 1 with zero AdamW
+    moments, and at step 5 with warm ones (random, non-negative second moments)."""
     from fp4_post_weight_b200.table import FocusTable, hparams
     tensors = []
+    g = torch.Generator(device="cuda").manual_seed(77)
     for j, (_, sh) in enumerate(synth.LLAMA_1B.tensors()):
         t = synth.llama_1b_tensor(j, sh, "cuda")
-        synth.adam_states(t)
+        synth.adam_states(t, g, warm=warm)
         tensors.append(t)
     snaps = [_snapshot(t) for t in tensors]
     ents = _table_entries(tensors)
     tab = FocusTable(ents)
     tab.s2()
-    tab.step(1, hparams(), flags=F.FOCUS_STEP_WRITE_GRAD)
+    tab.step(step, hparams(), flags=F.FOCUS_STEP_WRITE_GRAD)
     assert F.focus_get_error() == 0
     tot = {"code_mismatch": 0, "band": 0}
     for e, snap in zip(ents, snaps):
         s2 = oracle.s2(snap[0])
         assert host(e.s2)[0] == s2
-        r = _compare_step(e, snap, s2, 1)
+        r = _compare_step(e, snap, s2, step)
         for k in tot:
             tot[k] += r[k]
     n = synth.LLAMA_1B.n_elements()
