@@ -25,7 +25,8 @@ constexpr int MAX_DEVICES = 64;
 
 struct DeviceInfo {
     int sms = 0;
-    int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_f46 = 0, occ_rows = 0, occ_rows_swz = 0, occ_amax = 0, occ_adam = 0;
+    int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_f46 = 0,
+        occ_rows = 0, occ_rows_swz = 0, occ_amax = 0, occ_adam = 0;
     int occ_mx[3] = {0, 0, 0}, occ_mx_multi[3] = {0, 0, 0};
 };
 
@@ -65,15 +66,18 @@ int device_info(DeviceInfo **out) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[0], mx_kernel<KIND_FWD>, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[1], mx_kernel<KIND_BWD>, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[2], mx_kernel<KIND_STEP>, THREADS, 0);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[0], mx_multi_kernel<KIND_FWD>, MX_TILE_BLOCKS, 0);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[1], mx_multi_kernel<KIND_BWD>, MX_TILE_BLOCKS, 0);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[2], mx_multi_kernel<KIND_STEP>, MX_TILE_BLOCKS,
-                                                      0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[0], mx_multi_kernel<KIND_FWD>,
+                                                      MX_TILE_BLOCKS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[1], mx_multi_kernel<KIND_BWD>,
+                                                      MX_TILE_BLOCKS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[2], mx_multi_kernel<KIND_STEP>,
+                                                      MX_TILE_BLOCKS, 0);
     });
     DeviceInfo &d = g_info[dev];
     if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_step_wqu <= 0 || d.occ_f46 <= 0 ||
-        d.occ_rows <= 0 || d.occ_rows_swz <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 || d.occ_mx[1] <= 0 ||
-        d.occ_mx[2] <= 0 || d.occ_mx_multi[0] <= 0 || d.occ_mx_multi[1] <= 0 || d.occ_mx_multi[2] <= 0)
+        d.occ_rows <= 0 || d.occ_rows_swz <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 ||
+        d.occ_mx[1] <= 0 || d.occ_mx[2] <= 0 || d.occ_mx_multi[0] <= 0 || d.occ_mx_multi[1] <= 0 ||
+        d.occ_mx_multi[2] <= 0)
         return FOCUS_ERR_CUDA;
     *out = &d;
     return FOCUS_OK;
