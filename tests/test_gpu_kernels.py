@@ -213,6 +213,27 @@ def test_step_pack_updated_equals_pack_after_step(F):
         assert np.array_equal(host_bits(a.Wq), host_bits(b.Wq))
 
 
+def test_step_with_both_updated_outputs(F):
+    """FOCUS_STEP_PACK_UPDATED | FOCUS_STEP_WQ_UPDATED together (the next step's W'
+    and the export of the updated parameters from one pass): codes and scales are
+    bit for bit focus_pack_multi after the step, W' is bit for bit focus_fwd_multi
+    after the step, and m, q and the moments are those of the plain step."""
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    shapes = [(37, 1040), (64, 512), (128, 2048), (3, 48), (0, 32)]
+    ea, eb = _entries(shapes, 140, warm=True), _entries(shapes, 140, warm=True)
+    ta, tb = FocusTable(ea), FocusTable(eb)
+    ta.s2(); tb.s2()
+    ta.step(3, hparams(), flags=F.FOCUS_STEP_PACK_UPDATED | F.FOCUS_STEP_WQ_UPDATED)
+    tb.step(3, hparams())
+    tb.pack()
+    tb.fwd()
+    assert F.focus_get_error() == 0
+    for a, b in zip(ea, eb):
+        for name in ("codes", "scales", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"):
+            assert torch.equal(getattr(a, name), getattr(b, name)), name
+        assert np.array_equal(host_bits(a.Wq), host_bits(b.Wq))
+
+
 def test_pack_multi_leaves_wq_alone(F):
     from fp4_post_weight_b200.table import FocusTable
     ents = _entries([(16, 256)], 60)
