@@ -453,8 +453,21 @@ def measure_next_rows(ents, dev, N, peaks, world):
     ms = _timed(mx_step_table, stream)
     r["one_launch"] = {"kernel": "mx_multi_kernel<KIND_STEP>", "launches": 1,
                        "Gelem_s": round(N * world / (ms * 1e-3) / 1e9, 2), **_roof(9.75 * N, ms, peak)}
+    # the same with the MXFP4 export of the updated parameters (codes + E8M0 scales)
+    mx_exp = FocusTable([Entry(W=e.W, m=m, q=q, s2=None, dWq=e.dWq, Wq=e.Wq, m_exp_avg=a1, m_exp_avg_sq=a2,
+                               q_exp_avg=b1, q_exp_avg_sq=b2,
+                               codes=torch.empty((e.W.shape[0], e.W.shape[1] // 2), dtype=torch.uint8, device=dev),
+                               scales=torch.empty((e.W.shape[0], e.W.shape[1] // 32), dtype=torch.uint8, device=dev))
+                         for e, (m, q, a1, a2, b1, b2) in zip(ents, mx)], PURPOSE_MX)
+
+    def mx_step_export():
+        cnt_mx[0] += 1
+        mx_exp.mx_step(cnt_mx[0], hp, F.FOCUS_STEP_PACK_UPDATED)
+    ms = _timed(mx_step_export, stream)
+    r["one_launch_export"] = {"kernel": "mx_multi_kernel<KIND_STEP, EXPORT>", "launches": 1, "bytes_per_weight": 10.28125,
+                              "Gelem_s": round(N * world / (ms * 1e-3) / 1e9, 2), **_roof(10.28125 * N, ms, peak)}
     out["mxfp4_step_llama8b"] = r
-    del mx, mx_tab
+    del mx, mx_tab, mx_exp
     # Llama-3.1-70B, generated on the device one layer at a time and stepped there:
     # s2 of the layer, then the fused step with the export of the updated parameters
     # (timed per layer), layers 0, 40 and 79

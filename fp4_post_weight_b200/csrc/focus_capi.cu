@@ -27,7 +27,7 @@ struct DeviceInfo {
     int sms = 0;
     int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_f46 = 0,
         occ_rows = 0, occ_rows_swz = 0, occ_amax = 0, occ_adam = 0;
-    int occ_mx[3] = {0, 0, 0}, occ_mx_multi[3] = {0, 0, 0};
+    int occ_mx[3] = {0, 0, 0}, occ_mx_multi[3] = {0, 0, 0}, occ_mx_export = 0, occ_mx_multi_export = 0;
 };
 
 std::once_flag g_once[MAX_DEVICES];
@@ -72,12 +72,15 @@ int device_info(DeviceInfo **out) {
                                                       MX_TILE_BLOCKS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[2], mx_multi_kernel<KIND_STEP>,
                                                       MX_TILE_BLOCKS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_export, mx_kernel<KIND_STEP, true>, THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi_export, mx_multi_kernel<KIND_STEP, true>,
+                                                      MX_TILE_BLOCKS, 0);
     });
     DeviceInfo &d = g_info[dev];
     if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_step_wqu <= 0 || d.occ_f46 <= 0 ||
         d.occ_rows <= 0 || d.occ_rows_swz <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 ||
         d.occ_mx[1] <= 0 || d.occ_mx[2] <= 0 || d.occ_mx_multi[0] <= 0 || d.occ_mx_multi[1] <= 0 ||
-        d.occ_mx_multi[2] <= 0)
+        d.occ_mx_multi[2] <= 0 || d.occ_mx_export <= 0 || d.occ_mx_multi_export <= 0)
         return FOCUS_ERR_CUDA;
     *out = &d;
     return FOCUS_OK;
@@ -180,20 +183,21 @@ int check_shape_mx(int64_t out, int64_t in) {
     return FOCUS_OK;
 }
 
-template <int KIND>
+template <int KIND, bool EXPORT = false>
 int launch_mx(const MxArgs &a, cudaStream_t s) {
     DeviceInfo *di;
     int rc = device_info(&di);
     if (rc) return rc;
     if (a.nblk == 0) return FOCUS_OK;
-    const int64_t grid = grid_for((a.nblk + THREADS - 1) / THREADS, di->sms, di->occ_mx[KIND]);
-    mx_kernel<KIND><<<(unsigned)grid, THREADS, 0, s>>>(a);
+    const int occ = EXPORT ? di->occ_mx_export : di->occ_mx[KIND];
+    const int64_t grid = grid_for((a.nblk + THREADS - 1) / THREADS, di->sms, occ);
+    mx_kernel<KIND, EXPORT><<<(unsigned)grid, THREADS, 0, s>>>(a);
     return launch_status();
 }
 
 template <int KIND>
 int launch_mx_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, int accumulate, int write_grad,
-                    const Hyper &hp, cudaStream_t s) {
+                    const Hyper &hp, cudaStream_t s, int pack_updated = 0, int wq_updated = 0) {
     if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
     if (n == 0 || total_tiles == 0) return FOCUS_OK;
     if (!descs_dev) return FOCUS_ERR_NULL;
@@ -207,7 +211,16 @@ int launch_mx_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_til
     a.total_tiles = total_tiles;
     a.accumulate = accumulate;
     a.write_grad = write_grad;
+    a.pack_updated = pack_updated;
+    a.wq_updated = wq_updated;
     a.hp = hp;
+    if constexpr (KIND == KIND_STEP) {
+        if (pack_updated || wq_updated) {
+            const int64_t grid = grid_for(total_tiles, di->sms, di->occ_mx_multi_export);
+            mx_multi_kernel<KIND, true><<<(unsigned)grid, MX_TILE_BLOCKS, 0, s>>>(a);
+            return launch_status();
+        }
+    }
     const int64_t grid = grid_for(total_tiles, di->sms, di->occ_mx_multi[KIND]);
     mx_multi_kernel<KIND><<<(unsigned)grid, MX_TILE_BLOCKS, 0, s>>>(a);
     return launch_status();
@@ -673,10 +686,11 @@ int focus_mx_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, fl
     if (!hp) return FOCUS_ERR_NULL;
     if ((rc = check_hyper(hp->lr_m, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
     if ((rc = check_hyper(hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
-    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD)) return FOCUS_ERR_VALUE;
+    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD | FOCUS_STEP_WQ_UPDATED))
+        return FOCUS_ERR_VALUE;
     if (out * in == 0) return FOCUS_OK;
     if (!W || !dWq || !m || !q || !m_exp_avg || !m_exp_avg_sq || !q_exp_avg || !q_exp_avg_sq) return FOCUS_ERR_NULL;
-    if (flags && (!dm || !dq)) return FOCUS_ERR_NULL;
+    if ((flags & (FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD)) && (!dm || !dq)) return FOCUS_ERR_NULL;
     const void *ptrs[] = {W, dWq, m, q, m_exp_avg, m_exp_avg_sq, q_exp_avg, q_exp_avg_sq, Wq, dm, dq};
     for (const void *p : ptrs)
         if (!aligned16(p)) return FOCUS_ERR_ALIGN;
@@ -686,8 +700,10 @@ int focus_mx_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, fl
     a.dm = dm; a.dq = dq;
     a.accumulate = (flags & FOCUS_STEP_ACCUMULATE) ? 1 : 0;
     a.write_grad = (flags & FOCUS_STEP_WRITE_GRAD) ? 1 : 0;
+    a.wq_updated = (flags & FOCUS_STEP_WQ_UPDATED) ? 1 : 0;
     a.hp = make_hyper(hp->lr_m, hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
     a.nblk = out * (in / 32);
+    if (a.wq_updated) return launch_mx<KIND_STEP, true>(a, (cudaStream_t)stream);
     return launch_mx<KIND_STEP>(a, (cudaStream_t)stream);
 }
 
@@ -710,12 +726,15 @@ int focus_mx_step_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64
     int rc;
     if ((rc = check_hyper(hp->lr_m, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
     if ((rc = check_hyper(hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
-    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD)) return FOCUS_ERR_VALUE;
+    if (flags & ~(unsigned)(FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD | FOCUS_STEP_PACK_UPDATED |
+                            FOCUS_STEP_WQ_UPDATED))
+        return FOCUS_ERR_VALUE;
     return launch_mx_multi<KIND_STEP>(descs_dev, n_tensors, total_tiles, (flags & FOCUS_STEP_ACCUMULATE) ? 1 : 0,
                                       (flags & FOCUS_STEP_WRITE_GRAD) ? 1 : 0,
                                       make_hyper(hp->lr_m, hp->lr_q, hp->beta1, hp->beta2, hp->eps,
                                                  hp->weight_decay, step),
-                                      (cudaStream_t)stream);
+                                      (cudaStream_t)stream, (flags & FOCUS_STEP_PACK_UPDATED) ? 1 : 0,
+                                      (flags & FOCUS_STEP_WQ_UPDATED) ? 1 : 0);
 }
 
 size_t focus_scales_swizzled_bytes(int64_t rows, int64_t cols) {

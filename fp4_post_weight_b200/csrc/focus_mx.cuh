@@ -44,6 +44,8 @@ struct MxArgs {
     int64_t nblk;
     int accumulate;
     int write_grad;
+    int pack_updated;          // step, export build: codes+scales of the UPDATED m and q
+    int wq_updated;            // step, export build: W' of the UPDATED m and q
     Hyper hp;
 };
 
@@ -58,8 +60,62 @@ __device__ __forceinline__ float pow2f(int e) {           // 2^e for e in [-127,
     return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : 0x1p-127f;
 }
 
-// One 32-block of the tensor `a` describes.
-template <int KIND>
+// The export of one 32-block from the UPDATED m and q (qn): the same
+// arithmetic as the forward below, so the result is bit for bit what the
+// forward writes when run after the step.  Codes and scale when pack_updated,
+// W' when wq_updated.
+__device__ __forceinline__ void mx_encode(const MxArgs &a, int64_t blk, const uint32_t *w, float A, float m,
+                                          const float *qn) {
+    const bool want_codes = a.pack_updated && a.codes != nullptr;
+    const bool want_wq = a.wq_updated && a.Wq != nullptr;
+    if (!want_codes && !want_wq) return;
+    if (!finitef(m) || !finitef(qn[0]) || !finitef(qn[1]) || !finitef(qn[2]) || !finitef(qn[3]))
+        atomicOr(&g_error_flags, 1u);
+    const float x = __fmul_rn(A, m);
+    const int e = mx_exponent(x);
+    const float S = pow2f(e);
+    const uint64_t S2 = f2_pack(S, S);
+    uint32_t codes[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float D = __fmul_rn(S, sigmoid_rn(qn[k]));
+        uint64_t y2[4];
+        if (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f) {
+            const float nr = -rcp_rn(D);
+            const uint64_t D2 = f2_pack(D, D), nr2 = f2_pack(nr, nr);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) y2[j] = div_by_f2(bf16x2_neg_f2(w[4 * k + j]), D2, nr2);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                y2[j] = f2_pack(__fdiv_rn(bf16_lo(w[4 * k + j]), D), __fdiv_rn(bf16_hi(w[4 * k + j]), D));
+        }
+        uint32_t code = 0u, o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t byte = e2m1_pair(f2_lo(y2[j]), f2_hi(y2[j]));
+            code |= byte << (8 * j);
+            if (want_wq) {
+                const uint32_t h2 = e2m1_pair_f16x2(byte);
+                const float c0 = __half2float(__ushort_as_half(lo16(h2)));
+                const float c1 = __half2float(__ushort_as_half(hi16(h2)));
+                const uint64_t p = f2_mul(f2_pack(c0, c1), S2);
+                o[j] = pack_bf16x2(f2_lo(p), f2_hi(p));
+            }
+        }
+        codes[k] = code;
+        if (want_wq) __stcs(reinterpret_cast<uint4 *>(a.Wq) + 4 * blk + k, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+    if (want_codes) {
+        reinterpret_cast<uint4 *>(a.codes)[blk] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+        a.scales[blk] = (uint8_t)(e + 127);
+    }
+}
+
+// One 32-block of the tensor `a` describes.  EXPORT (step only): the codes,
+// scale and/or W' are those of the updated m and q (mx_encode) instead of the
+// forward's, a compile-time choice so that the plain step keeps its registers.
+template <int KIND, bool EXPORT = false>
 __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
     {
         uint32_t w[16], g[16];
@@ -137,11 +193,11 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
                 }
             }
             codes[k] = code;
-            if (KIND != KIND_BWD && a.Wq)
+            if (KIND != KIND_BWD && a.Wq && !(EXPORT && a.wq_updated))
                 __stcs(reinterpret_cast<uint4 *>(a.Wq) + 4 * blk + k, make_uint4(o[0], o[1], o[2], o[3]));
             sq[k] = (KIND != KIND_FWD) ? f2_lo(sq2) + f2_hi(sq2) : 0.0f;
         }
-        if (KIND != KIND_BWD && a.codes) {
+        if (KIND != KIND_BWD && a.codes && !(EXPORT && a.pack_updated)) {
             reinterpret_cast<uint4 *>(a.codes)[blk] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
             a.scales[blk] = (uint8_t)(e + 127);
         }
@@ -175,17 +231,21 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
                 reinterpret_cast<float4 *>(a.q)[blk] = make_float4(f2_lo(p01), f2_hi(p01), f2_lo(p23), f2_hi(p23));
                 reinterpret_cast<float4 *>(a.q_ea)[blk] = make_float4(f2_lo(a01), f2_hi(a01), f2_lo(a23), f2_hi(a23));
                 reinterpret_cast<float4 *>(a.q_eas)[blk] = make_float4(f2_lo(b01), f2_hi(b01), f2_lo(b23), f2_hi(b23));
+                if (EXPORT) {
+                    const float qn[4] = {f2_lo(p01), f2_hi(p01), f2_lo(p23), f2_hi(p23)};
+                    mx_encode(a, blk, w, A, m, qn);
+                }
             }
         }
         if (bad) atomicOr(&g_error_flags, 1u);
     }
 }
 
-template <int KIND>
+template <int KIND, bool EXPORT = false>
 __global__ void __launch_bounds__(THREADS) mx_kernel(const MxArgs a) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < a.nblk; blk += stride)
-        mx_block<KIND>(a, blk);
+        mx_block<KIND, EXPORT>(a, blk);
 }
 
 // ---------------------------------------------------------------------------
@@ -205,10 +265,12 @@ struct MxMultiArgs {
     int64_t total_tiles;
     int accumulate;
     int write_grad;
+    int pack_updated;
+    int wq_updated;
     Hyper hp;
 };
 
-template <int KIND>
+template <int KIND, bool EXPORT = false>
 __global__ void __launch_bounds__(MX_TILE_BLOCKS) mx_multi_kernel(const MxMultiArgs g) {
     __shared__ MxArgs sa;
     __shared__ int64_t s_range[2];          // tiles [first, end) of the current tensor
@@ -243,6 +305,8 @@ __global__ void __launch_bounds__(MX_TILE_BLOCKS) mx_multi_kernel(const MxMultiA
                 sa.nblk = ok ? nb : 0;
                 sa.accumulate = g.accumulate;
                 sa.write_grad = g.write_grad;
+                sa.pack_updated = g.pack_updated;
+                sa.wq_updated = g.wq_updated;
                 sa.hp = g.hp;
                 s_range[0] = d.tile_begin;
                 s_range[1] = e;
@@ -253,7 +317,7 @@ __global__ void __launch_bounds__(MX_TILE_BLOCKS) mx_multi_kernel(const MxMultiA
             if (tile >= end) break;         // past the last tensor (uniform): nothing left
         }
         const int64_t blk = (tile - first) * MX_TILE_BLOCKS + threadIdx.x;
-        if (tile >= first && blk < sa.nblk) mx_block<KIND>(sa, blk);
+        if (tile >= first && blk < sa.nblk) mx_block<KIND, EXPORT>(sa, blk);
     }
 }
 

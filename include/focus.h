@@ -373,8 +373,9 @@ int focus_mx_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, con
 
 /* One fused step of one tensor: forward (W' when Wq != NULL), straight-through
  * backward, AdamW on m (lr_m) and q (lr_q) in place.  flags:
- * FOCUS_STEP_ACCUMULATE, FOCUS_STEP_WRITE_GRAD (both need dm and dq); other
- * bits give FOCUS_ERR_VALUE. */
+ * FOCUS_STEP_ACCUMULATE, FOCUS_STEP_WRITE_GRAD (both need dm and dq),
+ * FOCUS_STEP_WQ_UPDATED (Wq receives the forward of the UPDATED m and q: what
+ * focus_mx_fwd would write after the call); other bits give FOCUS_ERR_VALUE. */
 int focus_mx_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, float *m_exp_avg,
                   float *m_exp_avg_sq, float *q_exp_avg, float *q_exp_avg_sq, int64_t out, int64_t in,
                   const focus_hparams *hp, int64_t step, unsigned flags, uint16_t *Wq, float *dm, float *dq,
@@ -383,9 +384,13 @@ int focus_mx_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, fl
 /* The same three over every entry of a table prepared with FOCUS_PURPOSE_MX,
  * in one launch each (per entry: W, m, q; the forward writes Wq and/or
  * codes+scales, whichever the entry has; the backward needs dWq, dm, dq; the
- * step needs dWq and the four moments, writes Wq when present, and needs dm,
- * dq under FOCUS_STEP_ACCUMULATE / FOCUS_STEP_WRITE_GRAD).  An entry lacking a
- * pointer its call needs is skipped and sets the device flag. */
+ * step needs dWq and the four moments, writes Wq and codes+scales when
+ * present, and needs dm, dq under FOCUS_STEP_ACCUMULATE /
+ * FOCUS_STEP_WRITE_GRAD).  The step's flags also take FOCUS_STEP_PACK_UPDATED
+ * (codes+scales of the UPDATED m and q: what focus_mx_fwd_multi would write
+ * after the call; W is not read again) and FOCUS_STEP_WQ_UPDATED (W' of the
+ * updated m and q); without them the step writes the forward's.  An entry
+ * lacking a pointer its call needs is skipped and sets the device flag. */
 int focus_mx_fwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
                        focus_stream_t stream);
 int focus_mx_ste_bwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles, int accumulate,

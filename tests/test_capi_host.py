@@ -176,7 +176,7 @@ def test_mx_multi_checks(F):
     assert F.raw_call("focus_mx_ste_bwd_multi", None, 1, 1, 0, None) == 1
     assert F.raw_call("focus_mx_step_multi", P, 1, 1, None, 1, 0, None) == 1
     assert F.raw_call("focus_mx_step_multi", P, 1, 1, ctypes.byref(hp), 0, 0, None) == 4    # step >= 1
-    assert F.raw_call("focus_mx_step_multi", P, 1, 1, ctypes.byref(hp), 1, 4, None) == 4    # no export flag
+    assert F.raw_call("focus_mx_step_multi", P, 1, 1, ctypes.byref(hp), 1, 16, None) == 4   # not a step flag
     assert F.raw_call("focus_mx_step_multi", U, 1, 1, ctypes.byref(hp), 1, 0, None) == 3
 
 
@@ -317,7 +317,8 @@ def test_mx_checks(F):
     assert F.raw_call("focus_mx_ste_bwd", P, None, P, P, 4, 32, P, P, 0, None) == 1
     args = lambda step, flags, dm: (P, P, P, P, P, P, P, P, 4, 32, ctypes.byref(hp), step, flags, None, dm, dm, None)
     assert F.raw_call("focus_mx_step", *args(0, 0, None)) == 4                       # step < 1
-    assert F.raw_call("focus_mx_step", *args(1, 4, None)) == 4                       # no export flags for MXFP4
+    assert F.raw_call("focus_mx_step", *args(1, 4, None)) == 4                       # no codes buffer: no pack flag
+    assert F.raw_call("focus_mx_step", *args(1, 16, None)) == 4                      # not a step flag
     assert F.raw_call("focus_mx_step", *args(1, 1, None)) == 1                       # accumulate needs dm, dq
     assert F.raw_call("focus_mx_step", P, P, P, P, P, P, P, P, 4, 32, None, 1, 0, None, None, None, None) == 1
 

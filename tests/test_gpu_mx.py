@@ -224,3 +224,36 @@ def test_mx_multi_step_skips_an_incomplete_entry(F):
     gm, gq = oracle.mx_ste_bwd(Wb, Gb, hm, hq)
     oracle.adamw(hq, gq, hmo[2], hmo[3], 1e-3, 1)
     assert_close(host(tab.entries[4].q), hq, "q of an entry after")
+
+
+def test_mx_multi_step_exports_the_update(F):
+    """FOCUS_STEP_PACK_UPDATED | FOCUS_STEP_WQ_UPDATED on the table step: codes, E8M0
+    scales and W' are bit for bit what focus_mx_fwd_multi writes after a plain step,
+    and m, q and the moments are those of the plain step."""
+    from fp4_post_weight_b200.table import hparams
+    ta, _ = mx_table(F, 700, "warm")
+    tb, _ = mx_table(F, 700, "warm")
+    ta.mx_step(4, hparams(), F.FOCUS_STEP_PACK_UPDATED | F.FOCUS_STEP_WQ_UPDATED)
+    tb.mx_step(4, hparams())
+    tb.mx_fwd()
+    assert F.focus_get_error() == 0
+    for a, b in zip(ta.entries, tb.entries):
+        for name in ("codes", "scales", "Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"):
+            x, y = getattr(a, name), getattr(b, name)
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8)), name
+
+
+def test_mx_step_wq_of_the_update(F):
+    """FOCUS_STEP_WQ_UPDATED on the single-tensor step: W' is bit for bit what
+    focus_mx_fwd writes after a plain step."""
+    from fp4_post_weight_b200.table import hparams
+    W, m, q, dW = make((37, 1056), 710)
+    mo = [torch.zeros_like(m), torch.zeros_like(m), torch.zeros_like(q), torch.zeros_like(q)]
+    m2, q2, mo2 = m.clone(), q.clone(), [x.clone() for x in mo]
+    Wq_a = torch.empty_like(W)
+    F.focus_mx_step(W, dW, m, q, *mo, hparams(), 1, F.FOCUS_STEP_WQ_UPDATED, Wq_a)
+    F.focus_mx_step(W, dW, m2, q2, *mo2, hparams(), 1, 0, torch.empty_like(W))
+    Wq_b, _, _ = forward(F, W, m2, q2)
+    assert F.focus_get_error() == 0
+    assert torch.equal(m, m2) and torch.equal(q, q2)
+    assert torch.equal(Wq_a.view(torch.int16), Wq_b.view(torch.int16))
