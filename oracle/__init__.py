@@ -78,6 +78,7 @@ def lib():
         L.fo_pack.restype = ctypes.c_int
         L.fo_f46.argtypes = [_P, _I64, _I64, _F, ctypes.c_int, _P, _P, _P, _P, _P, _P]
         L.fo_f46.restype = ctypes.c_int
+        L.fo_nvfp4_rows.argtypes = [_P, _I64, _I64, _P, _P, _P, _P]; L.fo_nvfp4_rows.restype = ctypes.c_int
         L.fo_mx_fwd.argtypes = [_P, _P, _P, _I64, _I64, _P, _P, _P]; L.fo_mx_fwd.restype = ctypes.c_int
         L.fo_mx_ste_bwd.argtypes = [_P, _P, _P, _P, _I64, _I64, _P, _P, ctypes.c_int]
         L.fo_mx_ste_bwd.restype = ctypes.c_int
@@ -268,6 +269,20 @@ def fouroversix(X, s=None) -> FourOverSix:
     _chk(lib().fo_f46(_p(X), rows, cols, 0.0 if per_row else float(s), 1 if per_row else 0, _p(codes),
                       _p(scales), _p(Xq), _p(four), _p(errs), _p(rs)))
     return FourOverSix(codes, scales, Xq, four, errs, rs)
+
+
+def nvfp4_rows(X) -> FourOverSix:
+    """NVFP4 round to nearest with one scale per row (per-token activations): the
+    card's block equations with m = 1, sigmoid = 1 and s_t = max_row|x|/2688.
+    Returns the FourOverSix record with four = 0 and errs = None."""
+    X = _c(X, np.uint16)
+    rows, cols = X.shape
+    codes = np.empty((rows, cols), np.uint8)
+    scales = np.empty((rows, cols // 16), np.uint8)
+    Xq = np.empty((rows, cols), np.uint16)
+    rs = np.empty(rows, np.float32)
+    _chk(lib().fo_nvfp4_rows(_p(X), rows, cols, _p(codes), _p(scales), _p(Xq), _p(rs)))
+    return FourOverSix(codes, scales, Xq, np.zeros((rows, cols // 16), np.uint8), None, rs)
 
 
 def scales_swizzle(scales: np.ndarray) -> np.ndarray:

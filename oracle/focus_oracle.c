@@ -651,6 +651,78 @@ int fo_f46(const uint16_t *X, int64_t rows, int64_t cols, float s, int per_row, 
 }
 
 /* ------------------------------------------------------------------------ */
+/* NVFP4 round to nearest with one scale per row (per-token activations)     */
+/* ------------------------------------------------------------------------ */
+/*
+ * [card] section "Perplexity", method list: the NVFP4 baseline quantizes
+ * activations to NVFP4 with one scale per token.  Read as the card's block
+ * equations ("What this is") with m = 1 and sigmoid = 1, applied to each row
+ * with its own scale s_t = fl(max_row |x| / 2688) in place of s2:
+ *   x_b = fl(A_b / fl(6*s_t)); x_b == 0 -> 1; S_b = e4m3(clamp(x_b, 2^-6, 448))
+ *   c_i = E2M1(clamp(fl(x_i / fl(S_b*s_t)), -6, 6));  x'_i = bf16(fl(fl(c_i*S_b)*s_t))
+ * A row of zeros gets s_t = 0, scale bytes 0x38 (the zero-block rule), codes 0
+ * and values 0.  Outputs as fo_f46 (codes one per element).
+ */
+int fo_nvfp4_rows(const uint16_t *X, int64_t rows, int64_t cols, uint8_t *codes, uint8_t *scales, uint16_t *Xq,
+                  float *row_scales)
+{
+    int rc = check_shape(rows, cols);
+    if (rc) return rc;
+    if (!row_scales) return FO_ERR_VALUE;
+    const int64_t nb = cols / 16;
+    int bad = 0;
+#pragma omp parallel for reduction(| : bad) schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *xr = X + r * cols;
+        float A_row = 0.0f;
+        for (int64_t i = 0; i < cols; ++i) {
+            float v = fo_bf16_to_f32(xr[i]);
+            if (!isfinite(v)) bad = 1;
+            if (fabsf(v) > A_row) A_row = fabsf(v);
+        }
+        const float st = A_row / 2688.0f;
+        row_scales[r] = st;
+        for (int64_t b = 0; b < nb; ++b) {
+            const int64_t blk = r * nb + b;
+            const int64_t e0 = r * cols + 16 * b;
+            if (st == 0.0f) {
+                if (scales) scales[blk] = 0x38;
+                for (int i = 0; i < 16; ++i) {
+                    if (codes) codes[e0 + i] = 0;
+                    if (Xq) Xq[e0 + i] = 0;
+                }
+                continue;
+            }
+            float w[16], A = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                w[i] = fo_bf16_to_f32(xr[16 * b + i]);
+                if (fabsf(w[i]) > A) A = fabsf(w[i]);
+            }
+            float x = A / (6.0f * st);
+            if (x == 0.0f) x = 1.0f;
+            if (x < 0x1p-6f) x = 0x1p-6f;
+            if (x > 448.0f) x = 448.0f;
+            const int sb = fo_e4m3_encode(x);
+            const float S = (float)fo_e4m3_decode(sb);
+            const float D = S * st;
+            if (scales) scales[blk] = (uint8_t)sb;
+            for (int i = 0; i < 16; ++i) {
+                float u = w[i] / D;
+                if (u < -6.0f) u = -6.0f;
+                if (u > 6.0f) u = 6.0f;
+                const int c = fo_e2m1_encode(u);
+                if (codes) codes[e0 + i] = (uint8_t)c;
+                if (Xq) {
+                    float cS = (float)fo_e2m1_decode(c) * S;                  /* exact */
+                    Xq[e0 + i] = fo_f32_to_bf16(cS * st);
+                }
+            }
+        }
+    }
+    return bad ? FO_ERR_NONFINITE : FO_OK;
+}
+
+/* ------------------------------------------------------------------------ */
 /* scale factors in the layout of the sm_100 block-scaled tensor-core GEMM   */
 /* ------------------------------------------------------------------------ */
 /*
