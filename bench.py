@@ -379,6 +379,16 @@ def measure_next_rows(ents, dev, N, peaks, world):
     ms = _timed(act_swz, stream)
     out["fouroversix_act_4096_tokens_one_layer"]["scales_128x4"] = {
         "kernel": "f46_rows_kernel<SWZ>", "Gelem_s": round(n_act / (ms * 1e-3) / 1e9, 2), **_roof(b_act, ms, peak)}
+    # plain NVFP4 round to nearest per token (the target 6 alone), same inputs and bytes
+
+    def act_rtn():
+        for X, (ts, c, sc) in zip(Xs, bufs):
+            F.focus_nvfp4_act(X, ts, c, sc)
+    ms = _timed(act_rtn, stream)
+    out["nvfp4_act_4096_tokens_one_layer"] = {"kernel": "f46_rows_kernel<RTN>", "launches": 4, "elements": n_act,
+                                               "bytes_per_elem": 2.5625,
+                                               "Gelem_s": round(n_act / (ms * 1e-3) / 1e9, 2),
+                                               **_roof(b_act, ms, peak)}
     del Xs, bufs, swz
     # the calibration step over four micro-batches
     for e in ents:

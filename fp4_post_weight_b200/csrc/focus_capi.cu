@@ -27,6 +27,7 @@ struct DeviceInfo {
     int sms = 0;
     int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_f46 = 0,
         occ_rows = 0, occ_rows_swz = 0, occ_amax = 0, occ_adam = 0;
+    int occ_rows_rtn[2] = {0, 0};   // per-token NVFP4: row-major scales, 128x4 layout
     int occ_mx[3] = {0, 0, 0}, occ_mx_multi[3] = {0, 0, 0}, occ_mx_export = 0, occ_mx_multi_export = 0;
 };
 
@@ -61,6 +62,8 @@ int device_info(DeviceInfo **out) {
                                                       stage_smem_bytes<KIND_F46>());
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows, f46_rows_kernel<false>, ROW_THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows_swz, f46_rows_kernel<true>, ROW_THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows_rtn[0], f46_rows_kernel<false, true>, ROW_THREADS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows_rtn[1], f46_rows_kernel<true, true>, ROW_THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_amax, amax_tiles_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_adam, adamw_kernel, THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx[0], mx_kernel<KIND_FWD>, THREADS, 0);
@@ -78,7 +81,7 @@ int device_info(DeviceInfo **out) {
     });
     DeviceInfo &d = g_info[dev];
     if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_step_wqu <= 0 || d.occ_f46 <= 0 ||
-        d.occ_rows <= 0 || d.occ_rows_swz <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 ||
+        d.occ_rows <= 0 || d.occ_rows_swz <= 0 || d.occ_rows_rtn[0] <= 0 || d.occ_rows_rtn[1] <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 ||
         d.occ_mx[1] <= 0 || d.occ_mx[2] <= 0 || d.occ_mx_multi[0] <= 0 || d.occ_mx_multi[1] <= 0 ||
         d.occ_mx_multi[2] <= 0 || d.occ_mx_export <= 0 || d.occ_mx_multi_export <= 0)
         return FOCUS_ERR_CUDA;
@@ -610,39 +613,61 @@ int focus_fouroversix_multi(const focus_tensor_desc *descs_dev, int n, int64_t t
     return launch_on<KIND_F46>(a, (cudaStream_t)stream);
 }
 
-int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
-                          uint8_t *scales, uint16_t *Xq, focus_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// The per-token quantizers: FourOverSix or NVFP4 round to nearest (rtn), the
+// block scales row-major or in the 128x4-atom layout (swz: scales_bytes is
+// the caller's buffer size).
+int act_rows(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
+             uint8_t *scales, size_t scales_bytes, uint16_t *Xq, bool rtn, bool swz, cudaStream_t stream) {
     int rc = check_shape(tokens, hidden);
     if (rc) return rc;
     if (tokens * hidden == 0) return FOCUS_OK;
     if (!X || !token_scales || !codes || !scales) return FOCUS_ERR_NULL;
     if (!aligned16(X) || !aligned16(token_scales) || !aligned16(codes) || !aligned16(scales) || !aligned16(Xq))
         return FOCUS_ERR_ALIGN;
+    if (swz && scales_bytes < focus_scales_swizzled_bytes(tokens, hidden / 16)) return FOCUS_ERR_WORKSPACE;
     DeviceInfo *di;
     if ((rc = device_info(&di))) return rc;
-    const int64_t grid = grid_for(tokens, di->sms, di->occ_rows);
-    f46_rows_kernel<false><<<(unsigned)grid, ROW_THREADS, 0, (cudaStream_t)stream>>>(X, tokens, hidden, token_scales,
-                                                                                codes, scales, Xq);
+    const int64_t rows_out = swz ? (tokens + 127) / 128 * 128 : tokens;
+    const int occ = rtn ? di->occ_rows_rtn[swz ? 1 : 0] : (swz ? di->occ_rows_swz : di->occ_rows);
+    const int64_t grid = grid_for(rows_out, di->sms, occ);
+    const unsigned g = (unsigned)grid;
+    if (swz && rtn) f46_rows_kernel<true, true><<<g, ROW_THREADS, 0, stream>>>(X, tokens, hidden, token_scales, codes,
+                                                                            scales, Xq);
+    else if (swz) f46_rows_kernel<true><<<g, ROW_THREADS, 0, stream>>>(X, tokens, hidden, token_scales, codes,
+                                                                      scales, Xq);
+    else if (rtn) f46_rows_kernel<false, true><<<g, ROW_THREADS, 0, stream>>>(X, tokens, hidden, token_scales, codes,
+                                                                             scales, Xq);
+    else f46_rows_kernel<false><<<g, ROW_THREADS, 0, stream>>>(X, tokens, hidden, token_scales, codes, scales, Xq);
     return launch_status();
+}
+}  // namespace
+
+extern "C" {
+
+int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
+                          uint8_t *scales, uint16_t *Xq, focus_stream_t stream) {
+    return act_rows(X, tokens, hidden, token_scales, codes, scales, 0, Xq, false, false, (cudaStream_t)stream);
 }
 
 int focus_fouroversix_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales,
                                    uint8_t *codes, uint8_t *scales_swz, size_t scales_bytes, uint16_t *Xq,
                                    focus_stream_t stream) {
-    int rc = check_shape(tokens, hidden);
-    if (rc) return rc;
-    if (tokens * hidden == 0) return FOCUS_OK;
-    if (!X || !token_scales || !codes || !scales_swz) return FOCUS_ERR_NULL;
-    if (!aligned16(X) || !aligned16(token_scales) || !aligned16(codes) || !aligned16(scales_swz) || !aligned16(Xq))
-        return FOCUS_ERR_ALIGN;
-    if (scales_bytes < focus_scales_swizzled_bytes(tokens, hidden / 16)) return FOCUS_ERR_WORKSPACE;
-    DeviceInfo *di;
-    if ((rc = device_info(&di))) return rc;
-    const int64_t rows_out = (tokens + 127) / 128 * 128;
-    const int64_t grid = grid_for(rows_out, di->sms, di->occ_rows_swz);
-    f46_rows_kernel<true><<<(unsigned)grid, ROW_THREADS, 0, (cudaStream_t)stream>>>(X, tokens, hidden, token_scales,
-                                                                               codes, scales_swz, Xq);
-    return launch_status();
+    return act_rows(X, tokens, hidden, token_scales, codes, scales_swz, scales_bytes, Xq, false, true,
+                    (cudaStream_t)stream);
+}
+
+int focus_nvfp4_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
+                    uint8_t *scales, uint16_t *Xq, focus_stream_t stream) {
+    return act_rows(X, tokens, hidden, token_scales, codes, scales, 0, Xq, true, false, (cudaStream_t)stream);
+}
+
+int focus_nvfp4_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
+                             uint8_t *scales_swz, size_t scales_bytes, uint16_t *Xq, focus_stream_t stream) {
+    return act_rows(X, tokens, hidden, token_scales, codes, scales_swz, scales_bytes, Xq, true, true,
+                    (cudaStream_t)stream);
 }
 
 int focus_mx_fwd(const uint16_t *W, const float *m, const float *q, int64_t out, int64_t in, uint16_t *Wq,

@@ -365,6 +365,27 @@ __device__ __forceinline__ bool f46_block(const uint32_t *w, float A, const F46S
     return four;
 }
 
+// NVFP4 round to nearest of one block (the target 6 alone: the card's block
+// equations with m = 1 and sigmoid = 1) with block maximum A and scale sc.s > 0.
+__device__ __forceinline__ void rtn_block(const uint32_t *w, float A, const F46Scale &sc, uint32_t &sb,
+                                          uint32_t codes[2]) {
+    const F46Target t6 = f46_target(f46_x(A, sc.den6, sc.rden6, sc.den_ok), sc.s, A);
+    sb = t6.sb;
+    const uint64_t D6 = f2_pack(t6.D, t6.D), n6 = f2_pack(t6.nr, t6.nr);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        uint64_t y[4];
+        uint32_t h[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t wv = w[4 * k + j];
+            y[j] = t6.fast ? f46_quot<true>(bf16x2_neg_f2(wv), wv, t6.D, D6, n6)
+                           : f46_quot<false>(bf16x2_neg_f2(wv), wv, t6.D, D6, n6);
+        }
+        codes[k] = e2m1_quad(y, h);
+    }
+}
+
 // Block maximum |w| of 16 bf16 values as bf16 magnitude bits (exact; NaN and
 // infinity sort above every finite magnitude).
 __device__ __forceinline__ uint32_t block_amax_bits(const uint32_t *w) {
@@ -958,8 +979,9 @@ __device__ __forceinline__ int64_t swizzled_offset(int64_t r, int64_t c, int64_t
 
 // SWZ: the block scales go straight into the 128x4-atom layout (`scales` holds
 // the padded buffer), and the CTAs that draw a padding row, or a row's padding
-// columns, write them 0.
-template <bool SWZ>
+// columns, write them 0.  RTN: plain NVFP4 round to nearest (the target 6
+// alone) instead of FourOverSix.
+template <bool SWZ, bool RTN = false>
 __global__ void __launch_bounds__(ROW_THREADS) f46_rows_kernel(const uint16_t *__restrict__ X, int64_t rows, int64_t cols,
                                                            float *__restrict__ row_scales, uint8_t *__restrict__ codes,
                                                            uint8_t *__restrict__ scales, uint16_t *__restrict__ Xq) {
@@ -1004,7 +1026,8 @@ __global__ void __launch_bounds__(ROW_THREADS) f46_rows_kernel(const uint16_t *_
             if (s != 0.0f) {
                 const uint4 v0 = xr[2 * b], v1 = xr[2 * b + 1];
                 const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                f46_block(w, __uint_as_float(block_amax_bits(w) << 16), sc, sb, cw);
+                if (RTN) rtn_block(w, __uint_as_float(block_amax_bits(w) << 16), sc, sb, cw);
+                else f46_block(w, __uint_as_float(block_amax_bits(w) << 16), sc, sb, cw);
                 if (Xq) wq_words(cw, sb, s, o);
             }
             reinterpret_cast<uint2 *>(codes)[blk] = make_uint2(cw[0], cw[1]);

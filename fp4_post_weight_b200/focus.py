@@ -71,6 +71,8 @@ _SIGS = {
     "focus_fouroversix_multi": ([_P, _I, _I64, _P], _I),
     "focus_fouroversix_act": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _I),
     "focus_fouroversix_act_swizzled": ([_P, _I64, _I64, _P, _P, _P, _SZ, _P, _P], _I),
+    "focus_nvfp4_act": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _I),
+    "focus_nvfp4_act_swizzled": ([_P, _I64, _I64, _P, _P, _P, _SZ, _P, _P], _I),
     "focus_mx_fwd": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _P], _I),
     "focus_mx_ste_bwd": ([_P, _P, _P, _P, _I64, _I64, _P, _P, _I, _P], _I),
     "focus_mx_step": ([_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, ctypes.POINTER(focus_hparams), _I64,
@@ -287,6 +289,24 @@ def focus_fouroversix_act_swizzled(X, token_scales, codes, scales_swz, Xq=None, 
     nbytes = scales_swz.numel() * scales_swz.element_size() if isinstance(scales_swz, torch.Tensor) else 1 << 62
     _check(_lib.focus_fouroversix_act_swizzled(_ptr(X), t, h, _ptr(token_scales), _ptr(codes), _ptr(scales_swz),
                                                nbytes, _ptr(Xq), _stream(stream)), "focus_fouroversix_act_swizzled")
+
+
+def focus_nvfp4_act(X, token_scales, codes, scales, Xq=None, stream=None, tokens=None, hidden=None):
+    """NVFP4 round to nearest with one scale per token (the target 6 alone); outputs
+    as focus_fouroversix_act."""
+    _bf16(X, "X"); _bf16(Xq, "Xq"); _f32(token_scales, "token_scales")
+    t, h = _shape(X, tokens, hidden)
+    _check(_lib.focus_nvfp4_act(_ptr(X), t, h, _ptr(token_scales), _ptr(codes), _ptr(scales), _ptr(Xq),
+                                _stream(stream)), "focus_nvfp4_act")
+
+
+def focus_nvfp4_act_swizzled(X, token_scales, codes, scales_swz, Xq=None, stream=None, tokens=None, hidden=None):
+    """As focus_nvfp4_act, the block scales in the 128x4-atom layout."""
+    _bf16(X, "X"); _bf16(Xq, "Xq"); _f32(token_scales, "token_scales")
+    t, h = _shape(X, tokens, hidden)
+    nbytes = scales_swz.numel() * scales_swz.element_size() if isinstance(scales_swz, torch.Tensor) else 1 << 62
+    _check(_lib.focus_nvfp4_act_swizzled(_ptr(X), t, h, _ptr(token_scales), _ptr(codes), _ptr(scales_swz), nbytes,
+                                         _ptr(Xq), _stream(stream)), "focus_nvfp4_act_swizzled")
 
 
 def focus_mx_fwd(W, m, q, Wq=None, codes=None, scales=None, stream=None, out=None, in_=None):

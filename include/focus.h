@@ -340,6 +340,19 @@ int focus_fouroversix_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hi
                                    uint8_t *codes, uint8_t *scales_swz, size_t scales_bytes, uint16_t *Xq,
                                    focus_stream_t stream);
 
+/* Plain NVFP4 round to nearest with one scale per token: the NVFP4 baseline
+ * of the card's section "Perplexity" (NVFP4 activations with one scale per
+ * token), read as the block equations with m = 1 and sigmoid = 1 and the
+ * token's scale s_t = fl(max_row |x| / 2688) in place of s2:
+ *   S_b = e4m3(clamp(fl(A_b / fl(6*s_t)), 2^-6, 448)) (x == 0 -> 1)
+ *   c_i = E2M1_rne(clamp(fl(x_i / fl(S_b*s_t)), -6, 6));  x'_i = bf16(fl(fl(c_i*S_b)*s_t))
+ * Arguments, layouts, the zero-row and non-finite rules exactly as
+ * focus_fouroversix_act / focus_fouroversix_act_swizzled. */
+int focus_nvfp4_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
+                    uint8_t *scales, uint16_t *Xq, focus_stream_t stream);
+int focus_nvfp4_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
+                             uint8_t *scales_swz, size_t scales_bytes, uint16_t *Xq, focus_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * MXFP4 variant: 32-element blocks with an E8M0 scale and four sub-blocks of
  * 8, no tensor scale.  "Technische Samenvatting: FOCUS ...", sections

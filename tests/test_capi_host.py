@@ -274,6 +274,13 @@ def test_fouroversix_checks(F):
     assert F.raw_call(sw, P, 4, 32, P, P, P, S(need), U, None) == 3
     assert F.raw_call(sw, P, 4, 32, P, P, P, S(need - 1), None, None) == 5
     assert F.raw_call(sw, P, 0, 32, P, P, P, S(0), None, None) == 0                # no tokens
+    # plain NVFP4 per token: the same checks
+    assert F.raw_call("focus_nvfp4_act", P, 4, 40, P, P, P, None, None) == 2
+    assert F.raw_call("focus_nvfp4_act", P, 4, 32, None, P, P, None, None) == 1
+    assert F.raw_call("focus_nvfp4_act", P, 4, 32, P, P, P, U, None) == 3
+    assert F.raw_call("focus_nvfp4_act", P, 0, 32, P, P, P, None, None) == 0
+    assert F.raw_call("focus_nvfp4_act_swizzled", P, 4, 32, P, P, P, S(need - 1), None, None) == 5
+    assert F.raw_call("focus_nvfp4_act_swizzled", P, 4, 32, P, P, None, S(need), None, None) == 1
 
 
 def test_table_prepare_fouroversix(F):
@@ -338,6 +345,7 @@ def test_maximum_tensor_size(F):
     assert F.raw_call("focus_fouroversix_act", P, rows, in16, P, P, P, None, None) == 2
     assert F.raw_call("focus_fouroversix_act_swizzled", P, rows, in16, P, P, P, ctypes.c_size_t(1 << 40), None,
                       None) == 2
+    assert F.raw_call("focus_nvfp4_act", P, rows, in16, P, P, P, None, None) == 2
     in32 = 32 * 65536                 # MXFP4: 65,536 32-blocks per row
     assert F.raw_call("focus_mx_fwd", P, P, P, rows, in32, P, None, None, None) == 2
     descs = (F.focus_tensor_desc * 1)()

@@ -112,6 +112,44 @@ def test_activations(F, tokens, hidden):
         assert host(ts)[-1] == 0 and np.all(host(scales)[-1] == 0x38)
 
 
+@pytest.mark.parametrize("tokens,hidden", [(1, 16), (5, 48), (33, 4096), (17, 14336), (300, 1040), (3, 64)])
+def test_nvfp4_activations(F, tokens, hidden):
+    """Plain NVFP4 round to nearest per token (focus_nvfp4_act) against the oracle's
+    fo_nvfp4_rows, bit for bit; one row carries a block far below the row maximum
+    (the lower scale clamp) when the shape allows."""
+    X = synth.activations(tokens, hidden, "cuda", seed=3 * tokens + hidden, zero_tokens=1 if tokens > 2 else 0)
+    if tokens > 1 and hidden >= 64:
+        X[0, 16:32] = 1e-4
+        X[0, 40] = 40.0
+    ts = torch.full((tokens,), -1.0, device="cuda")
+    codes, scales, Xq = outputs(tokens, hidden)
+    F.focus_nvfp4_act(X, ts, codes, scales, Xq)
+    assert F.focus_get_error() == 0
+    ref = oracle.nvfp4_rows(host_bits(X))
+    np.testing.assert_array_equal(host(ts), ref.row_scales)
+    assert_same(ref, codes, scales, Xq)
+    if tokens > 1 and hidden >= 64:
+        assert host(scales)[0, 1] == 0x08               # x below 2^-6: clamped to the smallest normal scale
+
+
+def test_nvfp4_activations_swizzled_and_nonfinite(F):
+    from tests.parity import unpack_codes as _unpack
+    tokens, hidden = 130, 1040
+    X = synth.activations(tokens, hidden, "cuda", seed=9)
+    ts = torch.empty(tokens, device="cuda")
+    codes = torch.empty((tokens, hidden // 2), dtype=torch.uint8, device="cuda")
+    sw = torch.full((F.focus_scales_swizzled_bytes(tokens, hidden // 16),), 0xAB, dtype=torch.uint8, device="cuda")
+    F.focus_nvfp4_act_swizzled(X, ts, codes, sw)
+    assert F.focus_get_error() == 0
+    ref = oracle.nvfp4_rows(host_bits(X))
+    np.testing.assert_array_equal(host(sw), oracle.scales_swizzle(ref.scales))
+    np.testing.assert_array_equal(_unpack(host(codes)), ref.codes)
+    X[7, 3] = float("nan")
+    codes2, scales2, _ = outputs(tokens, hidden)
+    F.focus_nvfp4_act(X, ts, codes2, scales2)
+    assert F.focus_get_error() == 7
+
+
 def test_worked_example_on_gpu(F):
     gold = json.load(open(os.path.join(HERE, "golden", "fouroversix_worked.json")))
     u = gold["unit"]
