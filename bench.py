@@ -352,6 +352,11 @@ def measure_next_rows(ents, dev, N, peaks, world):
     r["with_Wq"] = {"bytes_per_weight": 4.5625, **_roof(4.5625 * N, ms, peak)}
     r["Gelem_s"] = round(N * world / (r["ms"] * 1e-3) / 1e9, 2)
     out["fouroversix_weights_llama8b"] = r
+    # plain NVFP4 round to nearest of the weights (the target 6 alone), codes + scales
+    ms = _timed(t_cs.nvfp4_rtn, stream)
+    out["nvfp4_rtn_weights_llama8b"] = {"kernel": "pipe_kernel<KIND_F46> (rtn)", "bytes_per_weight": 2.5625,
+                                        "Gelem_s": round(N * world / (ms * 1e-3) / 1e9, 2),
+                                        **_roof(2.5625 * N, ms, peak)}
     # FourOverSix activations, one scale per token
     Xs = [synth.activations(4096, h, dev, seed=50 + j) for j, h in enumerate((4096, 4096, 4096, 14336))]
     bufs = [(torch.empty(X.shape[0], device=dev), torch.empty((X.shape[0], X.shape[1] // 2), dtype=torch.uint8,

@@ -15,6 +15,7 @@ _BINDING_NAMES = {"focus_s2", "focus_fwd", "focus_ste_bwd", "focus_adamw_step", 
                   "focus_fouroversix_weight", "focus_fouroversix_multi", "focus_fouroversix_act",
                   "focus_fouroversix_act_swizzled",
                   "focus_nvfp4_act", "focus_nvfp4_act_swizzled",
+                  "focus_nvfp4_weight", "focus_nvfp4_weight_multi",
                   "focus_scales_swizzle", "focus_scales_swizzled_bytes", "focus_mx_fwd", "focus_mx_ste_bwd",
                   "focus_mx_step", "focus_mx_fwd_multi", "focus_mx_ste_bwd_multi", "focus_mx_step_multi",
                   "focus_step_host", "focus_step_host_workspace_bytes",

@@ -581,8 +581,11 @@ int focus_pack_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_ti
     return launch_on<KIND_FWD>(a, (cudaStream_t)stream);
 }
 
-int focus_fouroversix_weight(const uint16_t *W, int64_t out, int64_t in, float s2, uint8_t *codes, uint8_t *scales,
-                             uint16_t *Wq, focus_stream_t stream) {
+}  // extern "C"
+
+namespace {
+int weight_f46(const uint16_t *W, int64_t out, int64_t in, float s2, uint8_t *codes, uint8_t *scales, uint16_t *Wq,
+               int rtn, cudaStream_t stream) {
     int rc = check_shape(out, in);
     if (rc) return rc;
     if ((rc = check_s2(s2))) return rc;
@@ -598,10 +601,11 @@ int focus_fouroversix_weight(const uint16_t *W, int64_t out, int64_t in, float s
     a.one_s2 = s2;
     a.n_tensors = 1;
     a.total_tiles = tiles_of(out, in);
-    return launch_on<KIND_F46>(a, (cudaStream_t)stream);
+    a.rtn = rtn;
+    return launch_on<KIND_F46>(a, stream);
 }
 
-int focus_fouroversix_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {
+int weight_f46_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, int rtn, cudaStream_t stream) {
     if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
     if (n == 0) return FOCUS_OK;
     if (!descs_dev) return FOCUS_ERR_NULL;
@@ -610,7 +614,29 @@ int focus_fouroversix_multi(const focus_tensor_desc *descs_dev, int n, int64_t t
     a.table = descs_dev;
     a.n_tensors = n;
     a.total_tiles = total_tiles;
-    return launch_on<KIND_F46>(a, (cudaStream_t)stream);
+    a.rtn = rtn;
+    return launch_on<KIND_F46>(a, stream);
+}
+}  // namespace
+
+extern "C" {
+
+int focus_fouroversix_weight(const uint16_t *W, int64_t out, int64_t in, float s2, uint8_t *codes, uint8_t *scales,
+                             uint16_t *Wq, focus_stream_t stream) {
+    return weight_f46(W, out, in, s2, codes, scales, Wq, 0, (cudaStream_t)stream);
+}
+
+int focus_fouroversix_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {
+    return weight_f46_multi(descs_dev, n, total_tiles, 0, (cudaStream_t)stream);
+}
+
+int focus_nvfp4_weight(const uint16_t *W, int64_t out, int64_t in, float s2, uint8_t *codes, uint8_t *scales,
+                       uint16_t *Wq, focus_stream_t stream) {
+    return weight_f46(W, out, in, s2, codes, scales, Wq, 1, (cudaStream_t)stream);
+}
+
+int focus_nvfp4_weight_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {
+    return weight_f46_multi(descs_dev, n, total_tiles, 1, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -80,6 +80,7 @@ struct Args {
     int write_grad;                  // step: FOCUS_STEP_WRITE_GRAD
     int pack_updated;                // step: FOCUS_STEP_PACK_UPDATED
     uint32_t *amax_ws;               // step: per-tensor max |w| (bf16 magnitude bits) for the next s2, or nullptr
+    int rtn;                         // KIND_F46: plain NVFP4 round to nearest (the target 6 alone) instead
     Hyper hp;
 };
 
@@ -413,9 +414,10 @@ __device__ __forceinline__ void wq_words(const uint32_t codes[2], uint32_t sbyte
     }
 }
 
-// FourOverSix of one block of a weight tensor (tensor scale s2 = T.s2).
+// FourOverSix (or, rtn, plain NVFP4 round to nearest) of one block of a weight
+// tensor (tensor scale s2 = T.s2).
 template <class TV>
-__device__ __forceinline__ void compute_block_f46(const TV &T, Block &B) {
+__device__ __forceinline__ void compute_block_f46(const TV &T, Block &B, bool rtn) {
     const uint32_t abits = block_amax_bits(B.w);
     const bool bad = B.valid && abits >= 0x7f80u;
     if (B.valid) {
@@ -423,7 +425,8 @@ __device__ __forceinline__ void compute_block_f46(const TV &T, Block &B) {
         sc.s = T.s2; sc.den6 = T.den; sc.rden6 = T.rden; sc.den4 = T.den4; sc.rden4 = T.rden4;
         sc.den_ok = T.den46_ok;
         uint32_t sb, codes[2];
-        f46_block(B.w, __uint_as_float(abits << 16), sc, sb, codes);
+        if (rtn) rtn_block(B.w, __uint_as_float(abits << 16), sc, sb, codes);
+        else f46_block(B.w, __uint_as_float(abits << 16), sc, sb, codes);
         if (T.d.codes) {
             reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = make_uint2(codes[0], codes[1]);
             T.d.scales[B.blk] = (uint8_t)sb;
@@ -447,7 +450,7 @@ __device__ __forceinline__ void compute_block_f46(const TV &T, Block &B) {
 template <int KIND, bool WQU, class TV>
 __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block &B) {
     if constexpr (KIND == KIND_F46) {
-        compute_block_f46(T, B);
+        compute_block_f46(T, B, a.rtn != 0);
         return;
     }
     // A_b = max |w| over the block: max of the bf16 magnitude bit patterns (a NaN

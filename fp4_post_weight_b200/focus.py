@@ -69,6 +69,8 @@ _SIGS = {
     "focus_ste_bwd_multi": ([_P, _I, _I64, _I, _P], _I),
     "focus_fouroversix_weight": ([_P, _I64, _I64, _F, _P, _P, _P, _P], _I),
     "focus_fouroversix_multi": ([_P, _I, _I64, _P], _I),
+    "focus_nvfp4_weight": ([_P, _I64, _I64, _F, _P, _P, _P, _P], _I),
+    "focus_nvfp4_weight_multi": ([_P, _I, _I64, _P], _I),
     "focus_fouroversix_act": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _I),
     "focus_fouroversix_act_swizzled": ([_P, _I64, _I64, _P, _P, _P, _SZ, _P, _P], _I),
     "focus_nvfp4_act": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _I),
@@ -268,6 +270,20 @@ def focus_fouroversix_weight(W, s2: float, codes, scales, Wq=None, stream=None, 
 def focus_fouroversix_multi(table_dev, n: int, total_tiles: int, stream=None):
     _check(_lib.focus_fouroversix_multi(_ptr(table_dev), int(n), int(total_tiles), _stream(stream)),
            "focus_fouroversix_multi")
+
+
+def focus_nvfp4_weight(W, s2: float, codes, scales, Wq=None, stream=None, out=None, in_=None):
+    """Plain NVFP4 round to nearest of a weight with tensor scale s2 (outputs as
+    focus_fouroversix_weight)."""
+    _bf16(W, "W"); _bf16(Wq, "Wq")
+    o, i = _shape(W, out, in_)
+    _check(_lib.focus_nvfp4_weight(_ptr(W), o, i, float(s2), _ptr(codes), _ptr(scales), _ptr(Wq), _stream(stream)),
+           "focus_nvfp4_weight")
+
+
+def focus_nvfp4_weight_multi(table_dev, n: int, total_tiles: int, stream=None):
+    _check(_lib.focus_nvfp4_weight_multi(_ptr(table_dev), int(n), int(total_tiles), _stream(stream)),
+           "focus_nvfp4_weight_multi")
 
 
 def focus_fouroversix_act(X, token_scales, codes, scales, Xq=None, stream=None, tokens=None, hidden=None):

@@ -95,6 +95,10 @@ class FocusTable:
     def fouroversix(self, stream=None):
         F.focus_fouroversix_multi(self.dev, self.n, self.total_tiles, stream)
 
+    def nvfp4_rtn(self, stream=None):
+        """Plain NVFP4 round to nearest of every entry (a table as for fouroversix)."""
+        F.focus_nvfp4_weight_multi(self.dev, self.n, self.total_tiles, stream)
+
     # MXFP4 (a table built with PURPOSE_MX)
     def mx_fwd(self, stream=None):
         F.focus_mx_fwd_multi(self.dev, self.n, self.total_tiles, stream)

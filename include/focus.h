@@ -318,6 +318,16 @@ int focus_fouroversix_weight(const uint16_t *W, int64_t out, int64_t in, float s
 int focus_fouroversix_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
                             focus_stream_t stream);
 
+/* Plain NVFP4 round to nearest of weights with the tensor scale s2 (the
+ * card's NVFP4 baseline, section "Perplexity": round-to-nearest NVFP4
+ * weights): the block equations with m = 1 and sigmoid = 1, i.e. the target 6
+ * alone; arguments and outputs exactly as focus_fouroversix_weight and
+ * focus_fouroversix_multi. */
+int focus_nvfp4_weight(const uint16_t *W, int64_t out, int64_t in, float s2, uint8_t *codes, uint8_t *scales,
+                       uint16_t *Wq, focus_stream_t stream);
+int focus_nvfp4_weight_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
+                             focus_stream_t stream);
+
 /* Activations with one scale per token: X [tokens, hidden] bf16, device
  * (hidden % 16 == 0); token_scales [tokens] float, device, receives
  * s_t = fl(max_row |x| / 2688); codes [tokens][hidden/2], scales

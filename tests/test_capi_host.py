@@ -255,6 +255,13 @@ def test_fouroversix_checks(F):
     assert F.raw_call("focus_fouroversix_multi", P, -1, 1, None) == 4
     assert F.raw_call("focus_fouroversix_multi", None, 1, 1, None) == 1
     assert F.raw_call("focus_fouroversix_multi", U, 1, 1, None) == 3
+    # plain NVFP4 weights: the same checks
+    assert F.raw_call("focus_nvfp4_weight", P, 4, 24, f32(1.0), P, P, None, None) == 2
+    assert F.raw_call("focus_nvfp4_weight", P, 4, 16, f32(0.0), P, P, None, None) == 4
+    assert F.raw_call("focus_nvfp4_weight", P, 4, 16, f32(1.0), None, None, None, None) == 1
+    assert F.raw_call("focus_nvfp4_weight", U, 4, 16, f32(1.0), P, P, None, None) == 3
+    assert F.raw_call("focus_nvfp4_weight_multi", P, -1, 1, None) == 4
+    assert F.raw_call("focus_nvfp4_weight_multi", None, 1, 1, None) == 1
     # activations: per-token scales, codes and scales are required
     assert F.raw_call("focus_fouroversix_act", P, 4, 40, P, P, P, None, None) == 2
     assert F.raw_call("focus_fouroversix_act", P, 4, 32, None, P, P, None, None) == 1

@@ -98,6 +98,53 @@ def test_weight_table(F):
         assert_same(oracle.fouroversix(Wb, s2), e.codes, e.scales, e.Wq)
 
 
+def _rtn_ref(Wb, s2):
+    """The oracle's forward with m = 1 and sigmoid(q) = 1 (q = 30): plain NVFP4 RTN."""
+    o, i = Wb.shape
+    return oracle.fwd(Wb, np.ones((o, i // 16), np.float32), np.full((o, i // 8), 30.0, np.float32), s2)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_nvfp4_weight(F, shape):
+    """Plain NVFP4 round to nearest of weights (focus_nvfp4_weight) against the
+    oracle's forward with unit parameters, bit for bit; outputs optional."""
+    W = weights(shape, 60 + shape[0])
+    Wb = host_bits(W)
+    s2 = oracle.s2(Wb)
+    codes, scales, Wq = outputs(*shape)
+    F.focus_nvfp4_weight(W, float(s2), codes, scales, Wq)
+    assert F.focus_get_error() == 0
+    ref = _rtn_ref(Wb, s2)
+    np.testing.assert_array_equal(host(scales), ref.scales)
+    np.testing.assert_array_equal(unpack_codes(host(codes)), ref.codes)
+    np.testing.assert_array_equal(host_bits(Wq), ref.Wq)
+    Wq2 = torch.full_like(Wq, 7.0)
+    F.focus_nvfp4_weight(W, float(s2), None, None, Wq2)
+    assert F.focus_get_error() == 0 and torch.equal(Wq2.view(torch.int16), Wq.view(torch.int16))
+
+
+def test_nvfp4_weight_table(F):
+    from fp4_post_weight_b200.table import Entry, FocusTable, PURPOSE_FOUROVERSIX
+    shapes = SHAPES + [(0, 32)]
+    ents = []
+    for j, sh in enumerate(shapes):
+        W = weights(sh, 80 + j) if sh[0] * sh[1] else torch.zeros(sh, dtype=torch.bfloat16, device="cuda")
+        c, s, q = outputs(*sh)
+        ents.append(Entry(W=W, m=None, q=None, s2=torch.zeros(1, device="cuda"), codes=c, scales=s, Wq=q))
+    tab = FocusTable(ents, PURPOSE_FOUROVERSIX)
+    tab.s2()
+    tab.nvfp4_rtn()
+    assert F.focus_get_error() == 0
+    for e in ents:
+        if e.W.numel() == 0:
+            continue
+        Wb = host_bits(e.W)
+        ref = _rtn_ref(Wb, oracle.s2(Wb))
+        np.testing.assert_array_equal(host(e.scales), ref.scales)
+        np.testing.assert_array_equal(unpack_codes(host(e.codes)), ref.codes)
+        np.testing.assert_array_equal(host_bits(e.Wq), ref.Wq)
+
+
 @pytest.mark.parametrize("tokens,hidden", [(1, 16), (5, 48), (33, 4096), (17, 14336), (300, 1040), (3, 64)])
 def test_activations(F, tokens, hidden):
     X = synth.activations(tokens, hidden, "cuda", seed=tokens + hidden, zero_tokens=1 if tokens > 2 else 0)
