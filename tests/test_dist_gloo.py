@@ -40,6 +40,17 @@ def _worker(rank, world, port, q):
         owned = D.shard([o * i for _, (o, i) in synth.LLAMA_8B.tensors()], world, rank)
         all_owned = [None] * world
         dist.all_gather_object(all_owned, owned)
+        # one tensor split by rows: each rank's s2 of its rows, then the max over
+        # ranks, is the s2 of the whole tensor (the oracle's, on the full tensor)
+        import numpy as np
+        import oracle
+        for out in (37, 1):                          # with one row, rank 1 owns none
+            W = synth.llama_1b_tensor(5, (out, 64), "cpu").W
+            r0, r1 = D.row_shard(out, world, rank)
+            bits = W.view(torch.int16).numpy().view(np.uint16)
+            local = oracle.s2(bits[r0:r1]) if r1 > r0 else np.float32(0)
+            s2 = D.s2_across_ranks(torch.tensor([float(local)], dtype=torch.float32))
+            assert float(s2.item()) == float(oracle.s2(bits)), (out, rank)
         q.put((rank, t, seeds[0], all_first, all_owned))
     finally:
         dist.destroy_process_group()
@@ -75,3 +86,12 @@ def test_single_process_defaults():
     assert D.min_over_ranks(3.0) == 3.0
     D.barrier()
     assert D.shard([5, 1, 1], 1, 0) == [0, 1, 2]
+    # row shards: contiguous, covering, sizes within one
+    for out, world in ((37, 2), (1, 2), (10, 4), (0, 3)):
+        spans = [D.row_shard(out, world, r) for r in range(world)]
+        assert spans[0][0] == 0 and spans[-1][1] == out
+        assert all(spans[i][1] == spans[i + 1][0] for i in range(world - 1))
+        sizes = [b - a for a, b in spans]
+        assert max(sizes) - min(sizes) <= 1
+    s2 = torch.tensor([0.25])
+    assert D.s2_across_ranks(s2) is s2 and float(s2) == 0.25
