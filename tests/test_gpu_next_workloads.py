@@ -6,6 +6,9 @@ configurations bench.py times:
   every other tensor, bit for bit against the oracle with each tensor's s2;
 * FourOverSix with one scale per token over one decoder layer's linear inputs
   for a micro-batch of 4096 tokens (four launches), in full;
+* plain NVFP4 round to nearest: the weights over all 224 linears in one launch
+  (layer 0 in full, a 1/64 row sample of the rest) and the same per-token
+  inputs, in full;
 * the MXFP4 fused step, one launch per tensor, on layer 0 of the 8B shapes
   with the benchmark's parameters (m = 1, q = 6, zero moments), a 1/16 row
   sample against the oracle, and the same step as one launch over a table of
@@ -139,3 +142,43 @@ def test_mx_step_table_llama_8b_sampled(F):
             assert_close(host(x[rows]), r, name)
         checked += Wb.size
     print(f"MXFP4 table step: {checked} weights checked over {len(ents)} tensors")
+
+
+def test_nvfp4_weights_llama_8b_one_launch(F):
+    """Plain NVFP4 round to nearest over all 224 8B linears in one launch (the bench's
+    line): layer 0 in full, a 1/64 row sample of every other tensor, against the
+    oracle's forward with m = 1, sigmoid = 1."""
+    from fp4_post_weight_b200.table import Entry, FocusTable, PURPOSE_FOUROVERSIX
+    ents, samples = [], []
+    for j, (_, (o, i)) in enumerate(synth.LLAMA_8B.tensors()):
+        t = synth.llama_8b_tensor(j, (o, i), "cuda", with_grad=False)
+        ents.append(Entry(W=t.W, m=None, q=None, s2=torch.zeros(1, device="cuda"),
+                          codes=torch.empty((o, i // 2), dtype=torch.uint8, device="cuda"),
+                          scales=torch.empty((o, i // 16), dtype=torch.uint8, device="cuda")))
+        samples.append(None if j < 7 else _rows(o, 64))
+    tab = FocusTable(ents, PURPOSE_FOUROVERSIX)
+    tab.s2()
+    tab.nvfp4_rtn()
+    assert F.focus_get_error() == 0
+    for e, rows in zip(ents, samples):
+        Wb = host_bits(e.W if rows is None else e.W[rows])
+        s2 = oracle.s2(host_bits(e.W))
+        o, i = Wb.shape
+        ref = oracle.fwd(Wb, np.ones((o, i // 16), np.float32), np.full((o, i // 8), 30.0, np.float32), s2)
+        sel = (lambda x: x) if rows is None else (lambda x: x[rows])
+        np.testing.assert_array_equal(host(sel(e.scales)), ref.scales)
+        np.testing.assert_array_equal(unpack_codes(host(sel(e.codes))), ref.codes)
+
+
+def test_nvfp4_activations_one_layer_4096_tokens(F):
+    for j, h in enumerate((4096, 4096, 4096, 14336)):
+        X = synth.activations(4096, h, "cuda", seed=50 + j)
+        ts = torch.empty(4096, device="cuda")
+        codes = torch.empty((4096, h // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((4096, h // 16), dtype=torch.uint8, device="cuda")
+        F.focus_nvfp4_act(X, ts, codes, scales)
+        assert F.focus_get_error() == 0
+        ref = oracle.nvfp4_rows(host_bits(X))
+        np.testing.assert_array_equal(host(ts), ref.row_scales)
+        np.testing.assert_array_equal(host(scales), ref.scales)
+        np.testing.assert_array_equal(unpack_codes(host(codes)), ref.codes)
