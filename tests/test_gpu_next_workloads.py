@@ -6,6 +6,8 @@ configurations bench.py times:
   every other tensor, bit for bit against the oracle with each tensor's s2;
 * FourOverSix with one scale per token over one decoder layer's linear inputs
   for a micro-batch of 4096 tokens (four launches), in full;
+* the calibration step over four micro-batches (bench order) on layer 0 of the
+  8B shapes, a 1/16 row sample;
 * plain NVFP4 round to nearest: the weights over all 224 linears in one launch
   (layer 0 in full, a 1/64 row sample of the rest) and the same per-token
   inputs, in full;
@@ -182,3 +184,54 @@ def test_nvfp4_activations_one_layer_4096_tokens(F):
         np.testing.assert_array_equal(host(ts), ref.row_scales)
         np.testing.assert_array_equal(host(scales), ref.scales)
         np.testing.assert_array_equal(unpack_codes(host(codes)), ref.codes)
+
+
+def test_micro_batch_step_llama_8b_layer0_sampled(F):
+    """The calibration step over four micro-batches as the bench times it (table
+    backward, two accumulating backward passes, then the accumulating step with the
+    next step's W') on layer 0 of the 8B shapes with the bench's parameters (m = 1,
+    q = 6, zero moments), a 1/16 row sample against the oracle."""
+    from fp4_post_weight_b200.table import Entry, FocusTable, hparams
+    from tests.parity import block_mask, check_forward
+    ents, grads, samples = [], [], []
+    g = torch.Generator(device="cuda").manual_seed(21)
+    for j, (_, (o, i)) in enumerate(synth.LLAMA_8B.tensors()[:7]):
+        t = synth.llama_8b_tensor(j, (o, i), "cuda")
+        ents.append(Entry(W=t.W, m=t.m, q=t.q, s2=torch.zeros(1, device="cuda"), dWq=t.dWq, Wq=torch.empty_like(t.W),
+                          m_exp_avg=torch.zeros_like(t.m), m_exp_avg_sq=torch.zeros_like(t.m),
+                          q_exp_avg=torch.zeros_like(t.q), q_exp_avg_sq=torch.zeros_like(t.q),
+                          dm=torch.zeros_like(t.m), dq=torch.zeros_like(t.q)))
+        grads.append([synth.normal_bf16((o, i), 1e-3, g, "cuda") for _ in range(4)])
+        samples.append(_rows(o, 16))
+    host_in = [(host_bits(e.W[r]), host(e.m[r]).copy(), host(e.q[r]).copy(), [host_bits(x[r]) for x in gs])
+               for e, gs, r in zip(ents, grads, samples)]
+    tab = FocusTable(ents)
+    tab.s2()
+    for j in range(3):
+        for e, gs in zip(ents, grads):
+            e.dWq.copy_(gs[j])
+        tab.bwd(accumulate=j > 0)
+    for e, gs in zip(ents, grads):
+        e.dWq.copy_(gs[3])
+    tab.step(1, hparams(), flags=F.FOCUS_STEP_ACCUMULATE | F.FOCUS_STEP_WRITE_GRAD | F.FOCUS_STEP_WQ_UPDATED)
+    assert F.focus_get_error() == 0
+    for e, r, (Wb, m, q, Gs) in zip(ents, samples, host_in):
+        s2 = host(e.s2)[0]
+        assert s2 == oracle.s2(host_bits(e.W))
+        skip = block_mask(check_forward(oracle.fwd(Wb, m, q, s2)))
+        dm, dq = oracle.ste_bwd(Wb, Gs[0], m, q, s2)
+        for j in (1, 2):
+            oracle.ste_bwd(Wb, Gs[j], m, q, s2, dm=dm, dq=dq)
+        z = [np.zeros_like(m), np.zeros_like(m), np.zeros_like(q), np.zeros_like(q)]
+        _, gm, gq = oracle.step(Wb, Gs[3], m, q, *z, s2, 1, want_wq=False, dm_acc=dm, dq_acc=dq)
+        skq = np.repeat(skip, 2, axis=1)
+        assert_close(host(e.dm[r]), gm, "dm over four micro-batches", skip)
+        assert_close(host(e.dq[r]), gq, "dq over four micro-batches", skq)
+        assert_close(host(e.m[r]), m, "m", skip)
+        assert_close(host(e.q[r]), q, "q", skq)
+        # W' of the updated parameters: the oracle's forward of the device's updated m
+        # and q; a value may differ only where its quotient lies in the 2^-20 band
+        ref = oracle.fwd(Wb, host(e.m[r]).copy(), host(e.q[r]).copy(), s2)
+        diff = host_bits(e.Wq[r]) != ref.Wq
+        assert not (diff & (ref.band == 0)).any()
+        assert diff.sum() <= 1e-6 * diff.size + 1
