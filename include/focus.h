@@ -469,7 +469,10 @@ int focus_scales_swizzle(const uint8_t *scales, int64_t rows, int64_t cols, uint
  *
  * BLOCKING: the call returns when every result is in host memory (it creates
  * and releases its two copy streams and its events).  The device flag is
- * reported by focus_get_error as for the other calls.
+ * reported by focus_get_error as for the other calls.  An entry the step
+ * skips (an all-zero W under FOCUS_HOST_S2_FIRST gives s2 = 0; the flag is
+ * set) gets its m, q and moments back unchanged and s2 = 0; its Wq, codes and
+ * scales are then undefined.
  * ------------------------------------------------------------------------- */
 #define FOCUS_HOST_S2_FIRST 16u   /* compute s2 from W in the slot before the step (first step) */
 size_t focus_step_host_workspace_bytes(const focus_tensor_desc *host_descs, int n_tensors);

@@ -78,7 +78,7 @@ def assert_same(dev_ents, host_ents, what):
         for name in FIELDS:
             a, b = getattr(d, name).cpu(), getattr(h, name)
             assert torch.equal(a.view(torch.uint8) if a.numel() else a, b.view(torch.uint8) if b.numel() else b), \
-                f"{what}: tensor {j} {SHAPES[j]} field {name} differs"
+                f"{what}: entry {j} {tuple(d.W.shape)} field {name} differs"
 
 
 @pytest.mark.parametrize("pinned", [True, False])
@@ -123,3 +123,28 @@ def test_host_step_computes_s2_first_and_matches_oracle(F):
     oracle.step(host_bits(W), host_bits(G), hm, hq, *hmo, s2, 1, want_wq=False)
     assert_close(hst[1].m.numpy(), hm, "m")
     assert_close(hst[1].q.numpy(), hq, "q")
+
+
+def test_host_step_both_updated_outputs_and_a_zero_tensor(F):
+    """Both updated outputs (export and next W') through the host executor, with an
+    all-zero tensor among the others and s2 computed in the call: that tensor's s2
+    is 0, so the step skips it and sets the device flag; every other tensor matches
+    the device-resident step bit for bit."""
+    from fp4_post_weight_b200.table import FocusTable, HostTable, hparams
+    st = state(13)
+    W0 = st[1][0]
+    W0.zero_()
+    flags = F.FOCUS_STEP_PACK_UPDATED | F.FOCUS_STEP_WQ_UPDATED
+    hst = host_entries(st)
+    m_before = hst[1].m.clone()
+    HostTable(hst).step(2, hparams(), F.FOCUS_HOST_S2_FIRST | flags)
+    assert F.focus_get_error() == 7
+    assert F.focus_get_error() == 0
+    assert hst[1].s2.item() == 0.0 and torch.equal(hst[1].m, m_before)
+    dev = device_entries(st)
+    tab = FocusTable(dev)
+    tab.s2()
+    tab.step_s2(2, hparams(), flags)
+    assert F.focus_get_error() == 7                  # the device-resident step skips it the same way
+    keep = [j for j in range(len(SHAPES)) if j != 1]
+    assert_same([dev[j] for j in keep], [hst[j] for j in keep], "both updated outputs")
