@@ -25,9 +25,10 @@
 // memory: W' as two 16-byte streaming stores per block, the codes as 8 bytes.
 //
 // Besides the FOCUS kinds (forward, backward, fused step) the same pipeline
-// runs FourOverSix round to nearest (KIND_F46, W alone is staged); the
-// per-token FourOverSix kernel, the scale relayout and the standalone AdamW
-// below are plain grid-stride kernels.
+// runs FourOverSix round to nearest and plain NVFP4 round to nearest of
+// weights (KIND_F46, W alone is staged; Args::rtn picks the latter); the
+// per-token kernel (FourOverSix or NVFP4, row-major or 128x4 scales), the
+// scale relayout and the standalone AdamW below are plain grid-stride kernels.
 //
 // Exactness.  Forward decisions (S_b, codes, w') are taken in binary32 with
 // explicit round-to-nearest intrinsics (__fmul_rn / __fdiv_rn cannot be fused
@@ -56,8 +57,9 @@ constexpr int TILE_BLOCKS = CONSUMERS;           // 16-blocks per tile (4096 wei
 constexpr unsigned FULL = 0xffffffffu;
 
 // Sticky error word read by focus_get_error(): bit 0 a non-finite input,
-// bit 1 an invalid tensor scale read from a table, bit 2 a non-finite
-// gradient, bit 3 a pipeline wait that ran out.
+// bit 1 a table entry skipped (an invalid tensor scale, or a pointer its
+// kernel needs missing), bit 2 a non-finite gradient, bit 3 a pipeline wait
+// that ran out.
 // (This header is compiled into exactly one translation unit.)
 __device__ unsigned int g_error_flags = 0;
 
