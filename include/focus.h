@@ -22,6 +22,13 @@
  * All arithmetic is IEEE binary32 with one rounding per operation; sigmoid is
  * the binary32 rounding of 1/(1+exp(-q)) evaluated in binary64.
  *
+ * Besides the FOCUS calls (s2, forward, straight-through backward, AdamW, the
+ * fused step, the NVFP4 pack; single tensors or a whole model as a table) the
+ * library has the rows around them: FourOverSix and plain NVFP4 round to
+ * nearest of weights and of activations with one scale per token, the MXFP4
+ * variant of FOCUS, the 128x4 scale layout of sm_100 block-scaled GEMMs, and
+ * the fused step over tensors held in host memory.
+ *
  * Conventions for every call:
  *  - Tensors are dense row-major.  W, dW' and W' are bf16, passed as uint16_t
  *    bit patterns.  m is float[out][in/16], q is float[out][in/8]: m[r][b]
@@ -29,13 +36,16 @@
  *  - Pointers named *_dev, and every tensor pointer, are device pointers
  *    (cudaMalloc / PyTorch CUDA memory) on the current device; their base
  *    addresses must be 16-byte aligned.  Parameters passed by value or through
- *    a host pointer are read before the call returns.
+ *    a host pointer are read before the call returns.  (focus_step_host is the
+ *    one exception: its tensors are in host memory; see there.)
  *  - The caller owns every buffer and the stream.  The library allocates no
- *    device or host memory; temporary storage is passed in as a workspace.
+ *    device or host memory of its own; temporary storage is passed in as a
+ *    workspace.
  *  - Every call only enqueues work on `stream` (a cudaStream_t; NULL is the
- *    legacy default stream) and returns at once.  The return value reports the
- *    argument checks (done on the host, before anything is enqueued) and the
- *    launch status; a failed check enqueues nothing.
+ *    legacy default stream) and returns at once, except focus_get_error and
+ *    focus_step_host, which block.  The return value reports the argument
+ *    checks (done on the host, before anything is enqueued) and the launch
+ *    status; a failed check enqueues nothing.
  *  - Non-finite values in W, m or q, and an invalid s2 read from device
  *    memory, are outside the contract: kernels never trap on them, they set a
  *    sticky device flag that focus_get_error() reports.  Every wait inside a
