@@ -14,7 +14,9 @@ configurations bench.py times:
 * the MXFP4 fused step, one launch per tensor, on layer 0 of the 8B shapes
   with the benchmark's parameters (m = 1, q = 6, zero moments), a 1/16 row
   sample against the oracle, and the same step as one launch over a table of
-  all 224 tensors (layer 0 at 1/16, the rest at 1/128 of the rows).
+  all 224 tensors (layer 0 at 1/16, the rest at 1/128 of the rows); the table
+  step with the export of the updated parameters on layer 0, against the
+  table forward after a plain step.
 """
 import numpy as np
 import pytest
@@ -235,3 +237,35 @@ def test_micro_batch_step_llama_8b_layer0_sampled(F):
         diff = host_bits(e.Wq[r]) != ref.Wq
         assert not (diff & (ref.band == 0)).any()
         assert diff.sum() <= 1e-6 * diff.size + 1
+
+
+def test_mx_step_export_llama_8b_layer0(F):
+    """The MXFP4 table step with the export of the updated parameters (the bench's
+    one_launch_export line) on layer 0 of the 8B shapes: codes, E8M0 scales and W'
+    bit for bit what the table forward writes after a plain step, and the updated
+    m, q and moments identical to the plain step's."""
+    from fp4_post_weight_b200.table import PURPOSE_MX, Entry, FocusTable, hparams
+
+    def table():
+        ents = []
+        for j, (_, (o, i)) in enumerate(synth.LLAMA_8B.tensors()[:7]):
+            t = synth.llama_8b_tensor(j, (o, i), "cuda")
+            m = torch.ones((o, i // 32), device="cuda")
+            q = torch.full((o, i // 8), 6.0, device="cuda")
+            ents.append(Entry(W=t.W, m=m, q=q, s2=None, dWq=t.dWq, Wq=torch.empty_like(t.W),
+                              m_exp_avg=torch.zeros_like(m), m_exp_avg_sq=torch.zeros_like(m),
+                              q_exp_avg=torch.zeros_like(q), q_exp_avg_sq=torch.zeros_like(q),
+                              codes=torch.empty((o, i // 2), dtype=torch.uint8, device="cuda"),
+                              scales=torch.empty((o, i // 32), dtype=torch.uint8, device="cuda")))
+        return FocusTable(ents, PURPOSE_MX)
+    ta = table()
+    ta.mx_step(1, hparams(), F.FOCUS_STEP_PACK_UPDATED | F.FOCUS_STEP_WQ_UPDATED)
+    assert F.focus_get_error() == 0
+    tb = table()
+    tb.mx_step(1, hparams())
+    tb.mx_fwd()
+    assert F.focus_get_error() == 0
+    for a, b in zip(ta.entries, tb.entries):
+        for name in ("codes", "scales", "Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"):
+            x, y = getattr(a, name), getattr(b, name)
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8)), name
