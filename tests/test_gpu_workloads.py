@@ -15,6 +15,9 @@
   tensor's maximum and its s2 after the step.
 * C5: Llama-3.1-70B layers 0, 40 and 79, one layer at a time: a 1/256 row
   sample.
+* A single tensor of more than 2^31 weights (byte offsets past 2^32): s2,
+  forward, pack and the fused step, s2 in full and rows at both ends and the
+  middle against the oracle.
 
 The export of the updated parameters is compared with the oracle's pack of the
 oracle's own updated m and q.  The two updates agree within the tolerance, not
@@ -288,3 +291,47 @@ def test_c5_llama_70b_layer_sampled(F, layer):
         for k, v in r.items():
             tot[k] = tot.get(k, 0) + v
     print(f"C5 layer {layer}: {tot}")
+
+
+def test_tensor_above_four_gigabytes(F):
+    """A single tensor of more than 2^31 weights (4.3 GB of bf16, byte offsets past
+    2^32): s2, forward and pack through the single-tensor calls, then the fused
+    step through a one-entry table; s2 over the whole tensor and a row sample at
+    the start, the middle and the end against the oracle."""
+    from fp4_post_weight_b200.table import Entry, FocusTable, hparams
+    o, i = 131072, 16512                              # 2,164,260,864 weights
+    g = torch.Generator(device="cuda").manual_seed(31)
+    W = synth.normal_bf16((o, i), 0.02, g, "cuda")
+    m = synth.uniform((o, i // 16), 0.8, 1.2, g, "cuda")
+    q = synth.normal((o, i // 8), 6.0, 2.0, g, "cuda")
+    ws = torch.empty(F.focus_s2_workspace_bytes(o, i), dtype=torch.uint8, device="cuda")
+    s2d = torch.zeros(1, device="cuda")
+    F.focus_s2(W, s2d, ws)
+    Wq = torch.empty_like(W)
+    s2 = float(host(s2d)[0])
+    F.focus_fwd(W, m, q, s2, Wq)
+    codes = torch.empty((o, i // 2), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((o, i // 16), dtype=torch.uint8, device="cuda")
+    F.focus_pack_nvfp4(W, m, q, s2, codes, scales, torch.zeros(1, device="cuda"))
+    assert F.focus_get_error() == 0
+    rows = torch.tensor([0, 1, o // 2, o // 2 + 1, o - 2, o - 1], device="cuda")
+    assert np.float32(s2) == oracle.s2(host_bits(W))
+    Wb, mb, qb = host_bits(W[rows]), host(m[rows]).copy(), host(q[rows]).copy()
+    ref = oracle.fwd(Wb, mb, qb, s2)
+    mism = check_forward(ref, Wq=host_bits(Wq[rows]), codes=unpack_codes(host(codes[rows])),
+                         scales=host(scales[rows]))
+    del Wq, codes, scales
+    torch.cuda.empty_cache()
+    # the fused step over the same tensor (dW' and the moments: another ~13 GB)
+    dW = synth.normal_bf16((o, i), 1e-3, g, "cuda")
+    Gb = host_bits(dW[rows])
+    e = Entry(W=W, m=m, q=q, s2=s2d, dWq=dW, Wq=None, m_exp_avg=torch.zeros_like(m), m_exp_avg_sq=torch.zeros_like(m),
+              q_exp_avg=torch.zeros_like(q), q_exp_avg_sq=torch.zeros_like(q))
+    tab = FocusTable([e])
+    tab.step(1, hparams())
+    assert F.focus_get_error() == 0
+    z = [np.zeros_like(mb), np.zeros_like(mb), np.zeros_like(qb), np.zeros_like(qb)]
+    oracle.step(Wb, Gb, mb, qb, *z, np.float32(s2), 1, want_wq=False)
+    skip = block_mask(mism)                           # blocks whose code sits in the 2^-20 band
+    assert_close(host(m[rows]), mb, "m", skip)
+    assert_close(host(q[rows]), qb, "q", np.repeat(skip, 2, axis=1))
