@@ -145,7 +145,8 @@ def test_nvfp4_weight_table(F):
         np.testing.assert_array_equal(host_bits(e.Wq), ref.Wq)
 
 
-@pytest.mark.parametrize("tokens,hidden", [(1, 16), (5, 48), (33, 4096), (17, 14336), (300, 1040), (3, 64)])
+@pytest.mark.parametrize("tokens,hidden", [(1, 16), (5, 48), (33, 4096), (17, 14336), (300, 1040), (3, 64),
+                                           (3, 262144)])
 def test_activations(F, tokens, hidden):
     X = synth.activations(tokens, hidden, "cuda", seed=tokens + hidden, zero_tokens=1 if tokens > 2 else 0)
     ts = torch.full((tokens,), -1.0, device="cuda")
@@ -159,7 +160,8 @@ def test_activations(F, tokens, hidden):
         assert host(ts)[-1] == 0 and np.all(host(scales)[-1] == 0x38)
 
 
-@pytest.mark.parametrize("tokens,hidden", [(1, 16), (5, 48), (33, 4096), (17, 14336), (300, 1040), (3, 64)])
+@pytest.mark.parametrize("tokens,hidden", [(1, 16), (5, 48), (33, 4096), (17, 14336), (300, 1040), (3, 64),
+                                           (3, 262144)])
 def test_nvfp4_activations(F, tokens, hidden):
     """Plain NVFP4 round to nearest per token (focus_nvfp4_act) against the oracle's
     fo_nvfp4_rows, bit for bit; one row carries a block far below the row maximum
