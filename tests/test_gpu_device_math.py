@@ -9,7 +9,8 @@
 * fl(c*S) through the mixed-precision FMA equals the binary32 product for
   every E2M1 value and every normal E4M3 scale, and c - y likewise.
 * The E2M1 conversion keeps the sign of negative values that round to zero
-  (code 0x8), which the kernels rely on for the signed-zero reading.
+  (code 0x8), which the kernels rely on for the signed-zero reading; the
+  four-pair form (codes packed by a byte move) equals four single pairs.
 * The reciprocal from the hardware approximation and one Newton step equals
   __frcp_rn for every significand; the twice-corrected quotient used for the
   scaled block maximum equals __fdiv_rn (every divisor significand for 1024
@@ -51,6 +52,8 @@ def lib():
                                  ctypes.POINTER(ctypes.c_float)]
     L.e2m1_raw_bytes.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     L.check_wait.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong)]
+    L.check_quad.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_ulonglong, ctypes.c_int,
+                             ctypes.POINTER(ctypes.c_ulonglong)]
     L.check_sigmoid_fast.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_float)]
     L.check_sigmoid_step.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_ulonglong),
                                      ctypes.POINTER(ctypes.c_float)]
@@ -82,6 +85,23 @@ def test_e2m1_conversion_zero_sign(lib):
     assert np.all(mags == 0)            # every value rounds to a zero magnitude
     want = (np.signbit(lo).astype(np.uint32) << 3) | (np.signbit(hi).astype(np.uint32) << 7)
     np.testing.assert_array_equal(out, want)
+
+
+def test_e2m1_quad_equals_pairs(lib):
+    """The four-pair conversion (FourOverSix) gives the word and the binary16 values
+    of four single-pair conversions, on 2^24 quadruples drawn from the E2M1 grid
+    values, the midpoints and their binary32 neighbours, signed zeros, tiny and
+    out-of-range values and random values."""
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, 6.5, 7], np.float32)
+    near = np.concatenate([np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(10))])
+    odd = np.array([1e-30, 1e-45, 6.0000005, 1e6, 3e38], np.float32)
+    rng = np.random.default_rng(5)
+    base = np.concatenate([grid, mids, near, odd, rng.uniform(-8, 8, 2000).astype(np.float32)])
+    vals = np.ascontiguousarray(np.concatenate([base, -base, np.array([0.0, -0.0], np.float32)]))
+    n = ctypes.c_ulonglong(0)
+    assert lib.check_quad(vals.ctypes.data, len(vals), 99, 1 << 16, ctypes.byref(n)) == 0
+    assert n.value == 0, f"{n.value} quadruples differ"
 
 
 @pytest.mark.parametrize("e", [0, -20, 20, -59, 59, -100, 100])
