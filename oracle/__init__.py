@@ -78,6 +78,8 @@ def lib():
         L.fo_pack.restype = ctypes.c_int
         L.fo_f46.argtypes = [_P, _I64, _I64, _F, ctypes.c_int, _P, _P, _P, _P, _P, _P]
         L.fo_f46.restype = ctypes.c_int
+        L.fo_f46_exact_sign.argtypes = [_P, _P, _P, ctypes.c_int]
+        L.fo_f46_exact_sign.restype = ctypes.c_int
         L.fo_nvfp4_rows.argtypes = [_P, _I64, _I64, _P, _P, _P, _P]; L.fo_nvfp4_rows.restype = ctypes.c_int
         L.fo_mx_fwd.argtypes = [_P, _P, _P, _I64, _I64, _P, _P, _P]; L.fo_mx_fwd.restype = ctypes.c_int
         L.fo_mx_ste_bwd.argtypes = [_P, _P, _P, _P, _I64, _I64, _P, _P, ctypes.c_int]
@@ -249,7 +251,7 @@ class FourOverSix:
     scales: np.ndarray      # uint8 [rows, cols/16], E4M3 byte of the chosen block scale
     Xq: np.ndarray          # uint16 bf16 bits [rows, cols], dequantized values
     four: np.ndarray        # uint8 [rows, cols/16], 1 where the target 4 was chosen
-    errs: np.ndarray        # float32 [rows, cols/16, 2], squared errors of the targets 6 and 4
+    errs: np.ndarray        # float64 [rows, cols/16, 2], squared errors of the targets 6 and 4 (binary64 sums)
     row_scales: np.ndarray | None   # float32 [rows] with one scale per row, else None
 
 
@@ -263,12 +265,20 @@ def fouroversix(X, s=None) -> FourOverSix:
     scales = np.empty((rows, nb), np.uint8)
     Xq = np.empty((rows, cols), np.uint16)
     four = np.empty((rows, nb), np.uint8)
-    errs = np.empty((rows, nb, 2), np.float32)
+    errs = np.empty((rows, nb, 2), np.float64)
     per_row = s is None
     rs = np.empty(rows, np.float32) if per_row else None
     _chk(lib().fo_f46(_p(X), rows, cols, 0.0 if per_row else float(s), 1 if per_row else 0, _p(codes),
                       _p(scales), _p(Xq), _p(four), _p(errs), _p(rs)))
     return FourOverSix(codes, scales, Xq, four, errs, rs)
+
+
+def f46_exact_sign(w, v4, v6) -> int:
+    """Sign of sum (w - v4)^2 - sum (w - v6)^2 over at most 16 binary64 values,
+    evaluated exactly (the comparison behind the FourOverSix choice)."""
+    w, v4, v6 = (_c(np.asarray(a, np.float64), np.float64) for a in (w, v4, v6))
+    assert w.shape == v4.shape == v6.shape and w.size <= 16
+    return int(lib().fo_f46_exact_sign(_p(w), _p(v4), _p(v6), w.size))
 
 
 def nvfp4_rows(X) -> FourOverSix:

@@ -523,17 +523,27 @@ int fo_pack(const uint16_t *W, const float *m, const float *q, float s2, int64_t
  *    m = 1, sigmoid = 1 and T in place of 6: x_T = fl(A / fl(T*s)); scale 1
  *    when x_T == 0; S_T = e4m3(clamp(x_T, 2^-6, 448)); D_T = fl(S_T*s);
  *    c_i = E2M1(clamp(fl(w_i/D_T), -6, 6)).  With T = 6 this is plain NVFP4
- *    round to nearest.
+ *    round to nearest.  These decisions are binary32, as every other
+ *    decision of the quantizer.
  *  - "error" is the squared error of the dequantized block,
- *    sum_i (w_i - c_i*S_T*s)^2.  The pages fix no precision for it; it
- *    decides an integer (the target), so it is evaluated in the kernels'
- *    precision, binary32, in this order: d_i = fl(w_i - (c_i*S_T)*s) with one
- *    rounding (c_i*S_T is exact, so this is one fused multiply-add); the even
- *    elements i = 0, 2, ..., 14 and the odd elements i = 1, 3, ..., 15 are
- *    summed separately, each as E <- fl(d_i*d_i + E) in index order from 0;
- *    the error is fl(E_even + E_odd).
- *  - The target 4 is taken only when its error is strictly lower; equal
- *    errors keep 6.
+ *        e_T = sum over i = 0..15 of (w_i - c_i*S_T*s)^2,
+ *    taken as a real number: the pages fix no precision for it, so the
+ *    definition itself is used, with no rounding.  w_i, c_i, S_T and s are
+ *    binary32 values, so every term is a dyadic rational and the comparison
+ *    e_4 < e_6 has one exact answer.
+ *  - The target 4 is taken only when e_4 < e_6 exactly; equal errors keep 6.
+ *  - How the comparison is evaluated (its result is the exact one either
+ *    way): both errors are first summed in binary64 in element order,
+ *    d_i = w_i - (c_i*S_T)*s (c_i*S_T is exact in binary32, its product with
+ *    s exact in binary64, one rounding in the difference), e <- e + d_i*d_i.
+ *    Each sum is then within gamma_18 = 18u/(1-18u) < 2^-48.8 of e_T
+ *    (u = 2^-53: one rounding in d_i, two in the square, at most fifteen in
+ *    the additions), so when the two binary64 sums differ by more than
+ *    2^-46 of their sum their order is the exact order.  Otherwise the
+ *    difference e_4 - e_6 is formed exactly as a floating-point expansion
+ *    and its sign read off (f46_exact_sign below).
+ *  - The errors reported are the binary64 sums (exact whenever every d_i^2
+ *    and partial sum fits 53 bits, e.g. the hand-derived examples).
  *  - The dequantized value is bf16(fl(fl(c*S)*s)), as w' of the card.
  *  - One scale per token: s_t = fl(A_row / 2688), the tensor scale's formula
  *    over one row.  A row whose maximum is 0 has s_t = 0; its blocks get
@@ -543,11 +553,89 @@ int fo_pack(const uint16_t *W, const float *m, const float *q, float s2, int64_t
 typedef struct {
     int sb[2];         /* E4M3 byte of S_T for T = 6 (index 0) and T = 4 (index 1) */
     int code[2][16];   /* E2M1 codes under each target */
-    float err[2];      /* squared error under each target */
+    double err[2];     /* squared error under each target (binary64 sum in element order) */
+    double cSs[2][16]; /* c_i*S_T*s of each element under each target (exact in binary64) */
     int four;          /* 1 when the target 4 is chosen */
 } fo_f46_block;
 
-static void f46_candidate(const float *w, float A, float s, float target, int *sb, int *code, float *err)
+/* Error-free transformations in binary64 (exact while nothing overflows and no
+ * product underflows): a + b = s + t (Knuth's two-sum), a*b = p + t (the
+ * rounding error of the product by one fused multiply-add). */
+static void two_sum(double a, double b, double *s, double *t)
+{
+    double x = a + b;
+    double bv = x - a;
+    double av = x - bv;
+    *s = x;
+    *t = (a - av) + (b - bv);
+}
+
+static void two_prod(double a, double b, double *p, double *t)
+{
+    double x = a * b;
+    *p = x;
+    *t = fma(a, b, -x);
+}
+
+/* Adds b to the expansion h[0..n) -- nonoverlapping components in increasing
+ * magnitude whose exact sum is the value -- and returns the new length; zero
+ * components are dropped.  Grow-Expansion of J. R. Shewchuk, "Adaptive
+ * Precision Floating-Point Arithmetic and Fast Robust Geometric Predicates",
+ * Discrete & Computational Geometry 18 (1997), with zero elimination.  The sum
+ * is exact; the largest component carries the sign of the value. */
+static int grow_expansion(double *h, int n, double b)
+{
+    double q = b;
+    int m = 0;
+    for (int i = 0; i < n; ++i) {
+        double s, t;
+        two_sum(q, h[i], &s, &t);
+        if (t != 0.0) h[m++] = t;
+        q = s;
+    }
+    if (q != 0.0) h[m++] = q;
+    return m;
+}
+
+/* Adds sign * (w - v)^2 to the expansion exactly (sign = +1 or -1):
+ * w - v = dh + dl exactly, (dh + dl)^2 = dh^2 + 2*dh*dl + dl^2, each product
+ * split into two doubles. */
+static int add_square(double *h, int n, double w, double v, double sign)
+{
+    double dh, dl, p, t;
+    two_sum(w, -v, &dh, &dl);
+    two_prod(dh, dh, &p, &t);
+    n = grow_expansion(h, n, sign * p);
+    n = grow_expansion(h, n, sign * t);
+    two_prod(2.0 * dh, dl, &p, &t);
+    n = grow_expansion(h, n, sign * p);
+    n = grow_expansion(h, n, sign * t);
+    two_prod(dl, dl, &p, &t);
+    n = grow_expansion(h, n, sign * p);
+    n = grow_expansion(h, n, sign * t);
+    return n;
+}
+
+/* Sign (-1, 0, +1) of e_4 - e_6 = sum_i (w_i - v4_i)^2 - sum_i (w_i - v6_i)^2,
+ * exactly.  Here w_i is a bf16 value (0 or at least 2^-133 in magnitude,
+ * at most 2^128) and v_i = c_i*S*s with at most 30 significant bits (0 or at
+ * least 2^-156: c >= 1/2, S >= 2^-6, s >= 2^-149), so every part of w_i - v_i
+ * is 0 or at least 2^-185 and every square at least 2^-370: far from
+ * binary64's underflow and overflow, where two_sum and two_prod are exact. */
+int fo_f46_exact_sign(const double *w, const double *v4, const double *v6, int n_el)
+{
+    double h[16 * 12 + 4];
+    int n = 0;
+    for (int i = 0; i < n_el && i < 16; ++i) {
+        n = add_square(h, n, w[i], v4[i], 1.0);
+        n = add_square(h, n, w[i], v6[i], -1.0);
+    }
+    if (n == 0) return 0;
+    return h[n - 1] > 0.0 ? 1 : -1;
+}
+
+static void f46_candidate(const float *w, float A, float s, float target, int *sb, int *code, double *cSs,
+                          double *err)
 {
     float den = target * s;
     float x = A / den;
@@ -557,32 +645,39 @@ static void f46_candidate(const float *w, float A, float s, float target, int *s
     *sb = fo_e4m3_encode(x);
     float S = (float)fo_e4m3_decode(*sb);
     float D = S * s;
-    float E[2] = {0.0f, 0.0f};      /* even and odd elements */
+    double e = 0.0;
     for (int i = 0; i < 16; ++i) {
         float u = w[i] / D;
         if (u < -6.0f) u = -6.0f;
         if (u > 6.0f) u = 6.0f;
         code[i] = fo_e2m1_encode(u);
         float cS = (float)fo_e2m1_decode(code[i]) * S;                 /* exact */
-        float d = fmaf(-cS, s, w[i]);
-        E[i & 1] = fmaf(d, d, E[i & 1]);
+        cSs[i] = (double)cS * (double)s;                               /* exact: at most 30 bits */
+        double d = (double)w[i] - cSs[i];
+        e = e + d * d;
     }
-    *err = E[0] + E[1];
+    *err = e;
 }
 
 /* Both candidates of one block of 16 bf16 values with scale s > 0, and the choice. */
 static void f46_block(const uint16_t *w16, float s, fo_f46_block *B)
 {
     float w[16];
+    double wd[16];
     float A = 0.0f;
     for (int i = 0; i < 16; ++i) {
         w[i] = fo_bf16_to_f32(w16[i]);
+        wd[i] = (double)w[i];
         float a = fabsf(w[i]);
         if (a > A) A = a;
     }
-    f46_candidate(w, A, s, 6.0f, &B->sb[0], B->code[0], &B->err[0]);
-    f46_candidate(w, A, s, 4.0f, &B->sb[1], B->code[1], &B->err[1]);
-    B->four = B->err[1] < B->err[0];
+    f46_candidate(w, A, s, 6.0f, &B->sb[0], B->code[0], B->cSs[0], &B->err[0]);
+    f46_candidate(w, A, s, 4.0f, &B->sb[1], B->code[1], B->cSs[1], &B->err[1]);
+    const double e6 = B->err[0], e4 = B->err[1];
+    if (fabs(e4 - e6) > 0x1p-46 * (e4 + e6))
+        B->four = e4 < e6;                                  /* the binary64 order is the exact order */
+    else
+        B->four = fo_f46_exact_sign(wd, B->cSs[1], B->cSs[0], 16) < 0;
 }
 
 /* FourOverSix over a row-major [rows, cols] bf16 tensor (cols % 16 == 0).
@@ -593,9 +688,9 @@ static void f46_block(const uint16_t *w16, float s, fo_f46_block *B)
  *   scales u8 [rows, cols/16]     E4M3 byte of the chosen scale
  *   Xq     bf16 bits [rows, cols] dequantized values
  *   four   u8 [rows, cols/16]     1 where the target 4 was chosen
- *   errs   f32 [rows, cols/16, 2] squared errors of the targets 6 and 4    */
+ *   errs   f64 [rows, cols/16, 2] squared errors of the targets 6 and 4    */
 int fo_f46(const uint16_t *X, int64_t rows, int64_t cols, float s, int per_row, uint8_t *codes,
-           uint8_t *scales, uint16_t *Xq, uint8_t *four, float *errs, float *row_scales)
+           uint8_t *scales, uint16_t *Xq, uint8_t *four, double *errs, float *row_scales)
 {
     int rc = check_shape(rows, cols);
     if (rc) return rc;
@@ -624,7 +719,7 @@ int fo_f46(const uint16_t *X, int64_t rows, int64_t cols, float s, int per_row, 
             if (sr == 0.0f) {           /* a row of zeros */
                 if (scales) scales[blk] = 0x38;
                 if (four) four[blk] = 0;
-                if (errs) { errs[2 * blk] = 0.0f; errs[2 * blk + 1] = 0.0f; }
+                if (errs) { errs[2 * blk] = 0.0; errs[2 * blk + 1] = 0.0; }
                 for (int i = 0; i < 16; ++i) {
                     if (codes) codes[e0 + i] = 0;
                     if (Xq) Xq[e0 + i] = 0;
