@@ -25,7 +25,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
     nvcc = os.environ.get("NVCC", "nvcc")
     cu = sorted(glob.glob(os.path.join(PKG, "csrc", "*.cu")))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, *cu, "-o", tmp]
+    # FOCUS_NVTX=0 builds the library without the NVTX ranges around its entry points
+    extra = ["-DFOCUS_NO_NVTX"] if os.environ.get("FOCUS_NVTX", "1") == "0" else []
+    cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", INCLUDE, *cu, "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)

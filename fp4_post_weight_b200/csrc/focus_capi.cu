@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include "focus.h"
+#include "focus_trace.cuh"
 #include "focus_kernels.cuh"
 #include "focus_mx.cuh"
 
@@ -268,9 +269,26 @@ static_assert(NOALLOC_TILES * TILE_BLOCKS * 16 == FOCUS_S2_NOALLOC_MAX_WEIGHTS, 
 
 static __device__ __align__(256) uint32_t g_s2_noalloc_scratch[NOALLOC_TILES];
 
-std::once_flag g_noalloc_once[MAX_DEVICES];
-uint32_t *g_noalloc_ptr[MAX_DEVICES];
-cudaError_t g_noalloc_status[MAX_DEVICES];
+std::mutex g_noalloc_mutex;
+uint32_t *g_noalloc_ptr[MAX_DEVICES];   // the array's device address on each device, once found
+
+// The scratch array's device address on device `dev` (current), or nullptr when
+// the lookup fails.  A successful lookup is kept; a failed one (for instance
+// inside a stream capture, where the lookup may be refused) is retried by the
+// next call, and its error is taken off the runtime's error state so that the
+// next entry point does not report it as its own launch failure.
+uint32_t *noalloc_scratch(int dev) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_s2_noalloc_scratch) == cudaSuccess) {
+            g_noalloc_ptr[dev] = static_cast<uint32_t *>(p);
+        } else {
+            (void)cudaGetLastError();
+        }
+    }
+    return g_noalloc_ptr[dev];
+}
 
 }  // namespace
 
@@ -301,6 +319,7 @@ size_t focus_s2_workspace_bytes(int64_t out, int64_t in) {
 
 int focus_s2(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, void *ws_dev, size_t ws_bytes,
              focus_stream_t stream) {
+    FOCUS_RANGE();
     int rc = check_shape(out, in);
     if (rc) return rc;
     if (!s2_dev || !ws_dev || (!W && out * in > 0)) return FOCUS_ERR_NULL;
@@ -315,6 +334,7 @@ int focus_s2(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, void *ws
 }
 
 int focus_s2_noalloc(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, focus_stream_t stream) {
+    FOCUS_RANGE();
     int rc = check_shape(out, in);
     if (rc) return rc;
     if (!s2_dev || (!W && out * in > 0)) return FOCUS_ERR_NULL;
@@ -325,22 +345,19 @@ int focus_s2_noalloc(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, 
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return FOCUS_ERR_CUDA;
     // The first call on a device, with that device current, looks up the device
     // address of the scratch array (its name in host code is only a stand-in).
-    std::call_once(g_noalloc_once[dev], [dev] {
-        void *p = nullptr;
-        g_noalloc_status[dev] = cudaGetSymbolAddress(&p, g_s2_noalloc_scratch);
-        g_noalloc_ptr[dev] = static_cast<uint32_t *>(p);
-    });
-    if (g_noalloc_status[dev] != cudaSuccess || g_noalloc_ptr[dev] == nullptr) return FOCUS_ERR_CUDA;
+    uint32_t *scratch = noalloc_scratch(dev);
+    if (scratch == nullptr) return FOCUS_ERR_CUDA;
     Args a{};
     a.table = nullptr;
     a.n_tensors = 1;
     a.one = one_desc(W, nullptr, nullptr, nullptr, nullptr, out, in);
     a.total_tiles = tiles;
-    return launch_s2(a, g_noalloc_ptr[dev], s2_dev, 1, (cudaStream_t)stream);
+    return launch_s2(a, scratch, s2_dev, 1, (cudaStream_t)stream);
 }
 
 int focus_fwd(const uint16_t *W, const float *m, const float *q, float s2, int64_t out, int64_t in, uint16_t *Wq,
               focus_stream_t stream) {
+    FOCUS_RANGE();
     int rc = check_shape(out, in);
     if (rc) return rc;
     if ((rc = check_s2(s2))) return rc;
@@ -358,6 +375,7 @@ int focus_fwd(const uint16_t *W, const float *m, const float *q, float s2, int64
 
 int focus_pack_nvfp4(const uint16_t *W, const float *m, const float *q, float s2, int64_t out, int64_t in,
                      uint8_t *codes, uint8_t *scales, float *tensor_scale_dev, focus_stream_t stream) {
+    FOCUS_RANGE();
     int rc = check_shape(out, in);
     if (rc) return rc;
     if ((rc = check_s2(s2))) return rc;
@@ -380,6 +398,7 @@ int focus_pack_nvfp4(const uint16_t *W, const float *m, const float *q, float s2
 
 int focus_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, const float *q, float s2, int64_t out,
                   int64_t in, float *dm, float *dq, int accumulate, focus_stream_t stream) {
+    FOCUS_RANGE();
     int rc = check_shape(out, in);
     if (rc) return rc;
     if ((rc = check_s2(s2))) return rc;
@@ -401,6 +420,7 @@ int focus_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, const 
 
 int focus_adamw_step(float *p, const float *g, float *exp_avg, float *exp_avg_sq, int64_t n, float lr, float beta1,
                      float beta2, float eps, float weight_decay, int64_t step, focus_stream_t stream) {
+    FOCUS_RANGE();
     if (n < 0) return FOCUS_ERR_SHAPE;
     int rc = check_hyper(lr, beta1, beta2, eps, weight_decay, step);
     if (rc) return rc;
@@ -418,6 +438,7 @@ int focus_adamw_step(float *p, const float *g, float *exp_avg, float *exp_avg_sq
 }
 
 int focus_table_prepare(focus_tensor_desc *d, int n, int purpose, int64_t *total_tiles) {
+    FOCUS_RANGE();
     if (!d || !total_tiles) return FOCUS_ERR_NULL;
     if (n < 0 || purpose < 0 || purpose > FOCUS_PURPOSE_MX) return FOCUS_ERR_VALUE;
     int64_t tiles = 0, blocks = 0;
@@ -480,6 +501,7 @@ size_t focus_s2_multi_workspace_bytes(int64_t total_tiles) {
 
 int focus_s2_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, void *ws_dev, size_t ws_bytes,
                    focus_stream_t stream) {
+    FOCUS_RANGE();
     if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
     if (n == 0) return FOCUS_OK;
     if (!descs_dev || !ws_dev) return FOCUS_ERR_NULL;
@@ -521,17 +543,20 @@ static int step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_t
 
 int focus_step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, const focus_hparams *hp,
                      int64_t step, unsigned flags, focus_stream_t stream) {
+    FOCUS_RANGE();
     return step_fused(descs_dev, n, total_tiles, hp, step, flags, nullptr, stream);
 }
 
 int focus_step_fused_amax(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, const focus_hparams *hp,
                           int64_t step, unsigned flags, uint32_t *amax_ws, focus_stream_t stream) {
+    FOCUS_RANGE();
     if (n > 0 && !amax_ws) return FOCUS_ERR_NULL;
     if (!aligned16(amax_ws)) return FOCUS_ERR_ALIGN;
     return step_fused(descs_dev, n, total_tiles, hp, step, flags, amax_ws, stream);
 }
 
 int focus_s2_from_amax(const focus_tensor_desc *descs_dev, int n, uint32_t *amax_ws, focus_stream_t stream) {
+    FOCUS_RANGE();
     if (n < 0) return FOCUS_ERR_VALUE;
     if (n == 0) return FOCUS_OK;
     if (!descs_dev || !amax_ws) return FOCUS_ERR_NULL;
@@ -542,6 +567,7 @@ int focus_s2_from_amax(const focus_tensor_desc *descs_dev, int n, uint32_t *amax
 }
 
 int focus_fwd_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {
+    FOCUS_RANGE();
     if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
     if (n == 0) return FOCUS_OK;
     if (!descs_dev) return FOCUS_ERR_NULL;
@@ -556,6 +582,7 @@ int focus_fwd_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_til
 
 int focus_ste_bwd_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, int accumulate,
                         focus_stream_t stream) {
+    FOCUS_RANGE();
     if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
     if (accumulate != 0 && accumulate != 1) return FOCUS_ERR_VALUE;
     if (n == 0) return FOCUS_OK;
@@ -570,6 +597,7 @@ int focus_ste_bwd_multi(const focus_tensor_desc *descs_dev, int n, int64_t total
 }
 
 int focus_pack_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {
+    FOCUS_RANGE();
     if (n < 0 || total_tiles < 0) return FOCUS_ERR_VALUE;
     if (n == 0) return FOCUS_OK;
     if (!descs_dev) return FOCUS_ERR_NULL;
@@ -623,19 +651,23 @@ extern "C" {
 
 int focus_fouroversix_weight(const uint16_t *W, int64_t out, int64_t in, float s2, uint8_t *codes, uint8_t *scales,
                              uint16_t *Wq, focus_stream_t stream) {
+    FOCUS_RANGE();
     return weight_f46(W, out, in, s2, codes, scales, Wq, 0, (cudaStream_t)stream);
 }
 
 int focus_fouroversix_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {
+    FOCUS_RANGE();
     return weight_f46_multi(descs_dev, n, total_tiles, 0, (cudaStream_t)stream);
 }
 
 int focus_nvfp4_weight(const uint16_t *W, int64_t out, int64_t in, float s2, uint8_t *codes, uint8_t *scales,
                        uint16_t *Wq, focus_stream_t stream) {
+    FOCUS_RANGE();
     return weight_f46(W, out, in, s2, codes, scales, Wq, 1, (cudaStream_t)stream);
 }
 
 int focus_nvfp4_weight_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, focus_stream_t stream) {
+    FOCUS_RANGE();
     return weight_f46_multi(descs_dev, n, total_tiles, 1, (cudaStream_t)stream);
 }
 
@@ -675,29 +707,34 @@ extern "C" {
 
 int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
                           uint8_t *scales, uint16_t *Xq, focus_stream_t stream) {
+    FOCUS_RANGE();
     return act_rows(X, tokens, hidden, token_scales, codes, scales, 0, Xq, false, false, (cudaStream_t)stream);
 }
 
 int focus_fouroversix_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales,
                                    uint8_t *codes, uint8_t *scales_swz, size_t scales_bytes, uint16_t *Xq,
                                    focus_stream_t stream) {
+    FOCUS_RANGE();
     return act_rows(X, tokens, hidden, token_scales, codes, scales_swz, scales_bytes, Xq, false, true,
                     (cudaStream_t)stream);
 }
 
 int focus_nvfp4_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
                     uint8_t *scales, uint16_t *Xq, focus_stream_t stream) {
+    FOCUS_RANGE();
     return act_rows(X, tokens, hidden, token_scales, codes, scales, 0, Xq, true, false, (cudaStream_t)stream);
 }
 
 int focus_nvfp4_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
                              uint8_t *scales_swz, size_t scales_bytes, uint16_t *Xq, focus_stream_t stream) {
+    FOCUS_RANGE();
     return act_rows(X, tokens, hidden, token_scales, codes, scales_swz, scales_bytes, Xq, true, true,
                     (cudaStream_t)stream);
 }
 
 int focus_mx_fwd(const uint16_t *W, const float *m, const float *q, int64_t out, int64_t in, uint16_t *Wq,
                  uint8_t *codes, uint8_t *scales, focus_stream_t stream) {
+    FOCUS_RANGE();
     int rc = check_shape_mx(out, in);
     if (rc) return rc;
     if ((codes == nullptr) != (scales == nullptr)) return FOCUS_ERR_NULL;
@@ -715,6 +752,7 @@ int focus_mx_fwd(const uint16_t *W, const float *m, const float *q, int64_t out,
 
 int focus_mx_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, const float *q, int64_t out, int64_t in,
                      float *dm, float *dq, int accumulate, focus_stream_t stream) {
+    FOCUS_RANGE();
     int rc = check_shape_mx(out, in);
     if (rc) return rc;
     if (accumulate != 0 && accumulate != 1) return FOCUS_ERR_VALUE;
@@ -732,6 +770,7 @@ int focus_mx_ste_bwd(const uint16_t *W, const uint16_t *dWq, const float *m, con
 int focus_mx_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, float *m_exp_avg, float *m_exp_avg_sq,
                   float *q_exp_avg, float *q_exp_avg_sq, int64_t out, int64_t in, const focus_hparams *hp,
                   int64_t step, unsigned flags, uint16_t *Wq, float *dm, float *dq, focus_stream_t stream) {
+    FOCUS_RANGE();
     int rc = check_shape_mx(out, in);
     if (rc) return rc;
     if (!hp) return FOCUS_ERR_NULL;
@@ -761,11 +800,13 @@ int focus_mx_step(const uint16_t *W, const uint16_t *dWq, float *m, float *q, fl
 
 int focus_mx_fwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
                        focus_stream_t stream) {
+    FOCUS_RANGE();
     return launch_mx_multi<KIND_FWD>(descs_dev, n_tensors, total_tiles, 0, 0, Hyper{}, (cudaStream_t)stream);
 }
 
 int focus_mx_ste_bwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles, int accumulate,
                            focus_stream_t stream) {
+    FOCUS_RANGE();
     if (accumulate != 0 && accumulate != 1) return FOCUS_ERR_VALUE;
     return launch_mx_multi<KIND_BWD>(descs_dev, n_tensors, total_tiles, accumulate, 0, Hyper{},
                                      (cudaStream_t)stream);
@@ -773,6 +814,7 @@ int focus_mx_ste_bwd_multi(const focus_tensor_desc *descs_dev, int n_tensors, in
 
 int focus_mx_step_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_tiles,
                         const focus_hparams *hp, int64_t step, unsigned flags, focus_stream_t stream) {
+    FOCUS_RANGE();
     if (!hp) return FOCUS_ERR_NULL;
     int rc;
     if ((rc = check_hyper(hp->lr_m, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step))) return rc;
@@ -795,6 +837,7 @@ size_t focus_scales_swizzled_bytes(int64_t rows, int64_t cols) {
 
 int focus_scales_swizzle(const uint8_t *scales, int64_t rows, int64_t cols, uint8_t *out, size_t out_bytes,
                          focus_stream_t stream) {
+    FOCUS_RANGE();
     if (rows < 0 || cols < 0) return FOCUS_ERR_SHAPE;
     const size_t need = focus_scales_swizzled_bytes(rows, cols);
     if (need == 0) return FOCUS_OK;
@@ -812,6 +855,7 @@ int focus_scales_swizzle(const uint8_t *scales, int64_t rows, int64_t cols, uint
 }
 
 int focus_get_error(focus_stream_t stream) {
+    FOCUS_RANGE();
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return FOCUS_ERR_CUDA;
     unsigned int flags = 0;
     if (cudaMemcpyFromSymbol(&flags, g_error_flags, sizeof flags) != cudaSuccess) return FOCUS_ERR_CUDA;

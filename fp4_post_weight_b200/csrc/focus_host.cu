@@ -16,6 +16,7 @@
 #include <cuda_runtime.h>
 
 #include "focus.h"
+#include "focus_trace.cuh"
 
 namespace {
 
@@ -109,6 +110,7 @@ size_t focus_step_host_workspace_bytes(const focus_tensor_desc *host_descs, int 
 
 int focus_step_host(const focus_tensor_desc *h, int n, const focus_hparams *hp, int64_t step, unsigned flags,
                     void *ws_dev, size_t ws_bytes, focus_stream_t stream) {
+    FOCUS_RANGE();
     if (n < 0) return FOCUS_ERR_VALUE;
     if (!hp) return FOCUS_ERR_NULL;
     if (flags & ~(unsigned)(FOCUS_STEP_PACK_UPDATED | FOCUS_STEP_WQ_UPDATED | FOCUS_HOST_S2_FIRST))

@@ -349,10 +349,56 @@ __device__ __forceinline__ void f46_both(const uint32_t *w, const F46Target &t6,
     e4 = __fadd_rn(f2_lo(E4), f2_hi(E4));
 }
 
+// Whether the target 4's squared error is strictly below the target 6's, decided
+// exactly.  With alpha_i = c6_i*S6 and beta_i = c4_i*S4 (exact in binary32), the
+// dequantized values are alpha_i*s and beta_i*s, and
+//   e4 - e6 = sum_i (w_i - beta_i s)^2 - (w_i - alpha_i s)^2 = s (2P - sQ),
+//   P = sum_i (alpha_i - beta_i) w_i,   Q = sum_i (alpha_i^2 - beta_i^2).
+// S4 >= S6 and its exponent is E or E + 1, E the exponent of S6, so alpha_i and
+// beta_i are integers below 2^9 times 2^(E-4): alpha - beta has at most 10
+// significant bits, each term of P at most 18 (w is bf16), each term of Q at
+// most 19 units of 2^(2E-8) and Q at most 23.  So every product here is exact
+// in binary64, Q and s*Q (47 bits) are exact, and P is exact whenever the
+// elements with a nonzero code span at most 2^31 in magnitude (always, unless
+// the block scale is clamped far away from the block maximum): then 2P < sQ is
+// the exact comparison.  Called for the rare near-tie blocks only, hence out of
+// line.
+__device__ __noinline__ bool f46_four_exact(uint4 wa, uint4 wb, uint32_t c6_0, uint32_t c6_1, uint32_t S6_h,
+                                            uint32_t c4_0, uint32_t c4_1, uint32_t S4_h, float s) {
+    const uint32_t w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+    double P = 0.0, Q = 0.0;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t h6 = e2m1_pair_f16x2(((k ? c6_1 : c6_0) >> (8 * j)) & 0xffu);
+            const uint32_t h4 = e2m1_pair_f16x2(((k ? c4_1 : c4_0) >> (8 * j)) & 0xffu);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const double al = mul_f16_exact(h ? hi16(h6) : lo16(h6), (uint16_t)S6_h);
+                const double be = mul_f16_exact(h ? hi16(h4) : lo16(h4), (uint16_t)S4_h);
+                const double wv = h ? bf16_hi(w[4 * k + j]) : bf16_lo(w[4 * k + j]);
+                P = __dadd_rn(P, __dmul_rn(__dsub_rn(al, be), wv));
+                Q = __dadd_rn(Q, __dsub_rn(__dmul_rn(al, al), __dmul_rn(be, be)));
+            }
+        }
+    }
+    return __dmul_rn(2.0, P) < __dmul_rn((double)s, Q);
+}
+
 // FourOverSix of one block with block maximum A (bf16 magnitude, exact) and
-// scale sc.s > 0.  The error of each target is fl(E_even + E_odd).  Returns
-// true when the target 4 is chosen (its error strictly lower); sb and codes
-// receive the choice.
+// scale sc.s > 0.  Returns true when the target 4 is chosen (its squared error
+// strictly lower than the target 6's; a tie keeps 6); sb and codes receive the
+// choice.
+//
+// The choice is screened with the binary32 sums e = fl(E_even + E_odd) of
+// f46_both.  Each is within gamma_11 < 2^-20.5 relative of the exact error
+// (one rounding in every d, two in every fused square-and-add of a lane, one in
+// the final add), plus at most 2^-144 absolute where values are subnormal.  So
+// when |e4 - e6| exceeds 2^-19 (e4 + e6) + 2^-140 the binary32 order is the
+// exact order.  Otherwise -- a near tie, an exact tie (they occur: about one
+// block in 10^7 of Gaussian weights), or a non-finite sum -- the choice is
+// taken by f46_four_exact.
 __device__ __forceinline__ bool f46_block(const uint32_t *w, float A, const F46Scale &sc, uint32_t &sb,
                                           uint32_t codes[2]) {
     const F46Target t6 = f46_target(f46_x(A, sc.den6, sc.rden6, sc.den_ok), sc.s, A);
@@ -361,7 +407,11 @@ __device__ __forceinline__ bool f46_block(const uint32_t *w, float A, const F46S
     float e6, e4;
     if (t6.fast && t4.fast) f46_both<true>(w, t6, t4, sc.s, c6, c4, e6, e4);
     else f46_both<false>(w, t6, t4, sc.s, c6, c4, e6, e4);
-    const bool four = e4 < e6;
+    bool four = e4 < e6;
+    if (!(fabsf(e4 - e6) > fmaf(0x1p-19f, e4 + e6, 0x1p-140f))) {
+        const uint4 wa = make_uint4(w[0], w[1], w[2], w[3]), wb = make_uint4(w[4], w[5], w[6], w[7]);
+        four = f46_four_exact(wa, wb, c6[0], c6[1], t6.S_h, c4[0], c4[1], t4.S_h, sc.s);
+    }
     sb = four ? t4.sb : t6.sb;
     codes[0] = four ? c4[0] : c6[0];
     codes[1] = four ? c4[1] : c6[1];

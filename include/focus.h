@@ -105,14 +105,21 @@ int focus_s2(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, void *ws
  * can synchronize the device).  The pages describe nothing like it; it only
  * changes where the per-tile maxima live: in a 256 KB array inside the
  * library's device image, held on every GPU that loads the library until the
- * process exits.  This call allocates nothing.
+ * process exits.  This call allocates nothing.  (The CUDA runtime loads the
+ * library's device code on a device when any of its entry points first runs
+ * there, which reserves its device globals, this array among them, and may
+ * synchronize; a caller that must avoid that on its critical path makes one
+ * warm-up call beforehand.  Later calls allocate nothing.)
  *   W       [out, in] bf16, device; at most FOCUS_S2_NOALLOC_MAX_WEIGHTS
- *           weights, else FOCUS_ERR_WORKSPACE and nothing is enqueued
+ *           weights, else FOCUS_ERR_WORKSPACE and nothing is enqueued;
+ *           out = 0 gives s2 = 0, as focus_s2
  *   s2_dev  one float, device, written
  * The first call on a device (with that device current) looks up the array's
- * device address; make that first call before any stream capture.  All calls
- * share the array: calls whose work may overlap on the GPU (different streams
- * without ordering between them) race and must not be issued.
+ * device address; make that first call before any stream capture.  If the
+ * lookup fails the call returns FOCUS_ERR_CUDA and the next call tries again.
+ * All calls share the array: calls whose work may overlap on the GPU
+ * (different streams without ordering between them) race and must not be
+ * issued.
  * ------------------------------------------------------------------------- */
 #define FOCUS_S2_NOALLOC_MAX_WEIGHTS 268435456 /* 65,536 tiles of 4096 weights */
 int focus_s2_noalloc(const uint16_t *W, int64_t out, int64_t in, float *s2_dev, focus_stream_t stream);
@@ -308,10 +315,11 @@ int focus_pack_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t 
  * Per block, for the targets T = 6 and T = 4 (s the tensor or token scale):
  *   x_T = fl(A_b / fl(T*s));  x_T == 0 -> 1;  S_T = e4m3_rne(clamp(x_T, 2^-6, 448))
  *   c_i = E2M1_rne(clamp(fl(w_i / fl(S_T*s)), -6, 6))
- *   err_T = fl(E_even + E_odd), E over the even / odd elements in index
- *           order, E <- fma(d_i, d_i, E), d_i = fma(-(c_i*S_T), s, w_i)
- * The target 4 is taken when err_4 < err_6 (a tie keeps 6); the dequantized
- * value is bf16(fl(fl(c_i*S)*s)).  Outputs use the focus_pack_nvfp4 layout
+ *   err_T = sum_i (w_i - c_i*S_T*s)^2, the exact squared error
+ * The target 4 is taken when err_4 < err_6 exactly (a tie keeps 6; exact ties
+ * occur, about one block in 10^7 of Gaussian weights).  The kernels screen the
+ * choice with binary32 sums and decide the blocks within 2^-19 of a tie by an
+ * exact comparison.  The dequantized value is bf16(fl(fl(c_i*S)*s)).  Outputs use the focus_pack_nvfp4 layout
  * (codes [rows][cols/2], element 2j in the low nibble; scales [rows][cols/16]).
  * ------------------------------------------------------------------------- */
 

@@ -26,3 +26,16 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """One line per workload with the parity counts the GPU tests recorded: elements
+    (or blocks) checked, the populations of the rounding bands and the mismatches,
+    which the tests hold at or below 1e-6 of the elements."""
+    from tests.parity import RECORD
+    if not RECORD:
+        return
+    terminalreporter.write_sep("-", "parity counts")
+    for name in sorted(RECORD):
+        c = RECORD[name]
+        terminalreporter.write_line(name + ": " + ", ".join(f"{k} {v}" for k, v in c.items()))

@@ -6,6 +6,13 @@ or of +-6 (the oracle's band flag 1; exact midpoints, flag 2, must match), and
 such mismatches below 1e-6 of the elements; w' bit-exact wherever the code
 matches; gradients, parameters and moments within
 |gpu - ref| <= 1e-7 + 1e-5 * |ref|.
+
+FourOverSix: the oracle's choice between the targets 6 and 4 is the exact
+order of the two squared errors.  The kernels take it from binary32 sums and,
+inside their certified screen band, from binary64 sums, which can order a
+block otherwise only when |e4 - e6| <= 2^-47 (e4 + e6).  A block's outputs
+(scale byte, codes, dequantized values) must therefore match bit for bit
+except inside that band, and such blocks must stay below 1e-6 of the blocks.
 """
 from __future__ import annotations
 
@@ -15,6 +22,17 @@ import torch
 RTOL = 1e-5
 ATOL = 1e-7
 MAX_MISMATCH_FRAC = 1e-6
+
+# Counts the parity tests record (elements checked, band populations, mismatches),
+# printed once at the end of the run by tests/conftest.py.
+RECORD: dict[str, dict] = {}
+
+
+def record(name: str, counts: dict) -> None:
+    """Adds counts to the run's parity record under `name` (summed over calls)."""
+    acc = RECORD.setdefault(name, {})
+    for k, v in counts.items():
+        acc[k] = acc.get(k, 0) + int(v)
 
 
 def host_bits(t: torch.Tensor) -> np.ndarray:
@@ -56,6 +74,14 @@ def check_forward(ref, Wq=None, codes=None, scales=None):
     return mism
 
 
+def forward_counts(ref, mism: np.ndarray | None = None) -> dict:
+    """Counts of an oracle forward (oracle.Forward.stats) with the code mismatches found."""
+    st = ref.stats
+    return {"elements": int(ref.codes.size), "band": st["band"], "exact_ties": st["exact_ties"],
+            "code_mismatch": 0 if mism is None else int(mism.sum()), "zero_blocks": st["zero_blocks"],
+            "clamp_low": st["clamp_low"], "clamp_high": st["clamp_high"], "out_of_range": st["out_of_range"]}
+
+
 def block_mask(mism: np.ndarray) -> np.ndarray:
     """Blocks [out, in/16] that contain a tolerated code mismatch."""
     o, i = mism.shape
@@ -75,3 +101,35 @@ def assert_close(gpu: np.ndarray, ref: np.ndarray, name: str, skip: np.ndarray |
         idx = np.argwhere(bad)[:5]
         raise AssertionError(f"{name}: {int(bad.sum())} of {gpu.size} outside tolerance; e.g. "
                              + ", ".join(f"{tuple(i)}: gpu {gpu[tuple(i)]!r} ref {ref[tuple(i)]!r}" for i in idx))
+
+
+F46_SCREEN = 2.0 ** -19     # the kernels' binary32 screen: inside it the choice is taken from binary64 sums
+F46_BAND = 2.0 ** -47       # the binary64 sums' bound: only inside it may a kernel's choice differ
+
+
+def f46_counts(ref) -> dict:
+    """Band populations of a FourOverSix oracle result (exact errors, reported as binary64 sums)."""
+    e6, e4 = ref.errs[..., 0], ref.errs[..., 1]
+    gap, tot = np.abs(e4 - e6), e4 + e6
+    return {"blocks": int(e6.size), "target4": int(ref.four.sum()),
+            "screen_band": int((gap <= F46_SCREEN * tot).sum()),
+            "ties_nonzero": int(((gap == 0) & (tot > 0)).sum()),
+            "band_2^-47": int((gap <= F46_BAND * tot).sum())}
+
+
+def check_fouroversix(ref, codes: np.ndarray, scales: np.ndarray, Xq: np.ndarray | None) -> dict:
+    """ref: oracle.FourOverSix; codes unpacked uint8 [rows, cols]; scales uint8 [rows, cols/16];
+    Xq uint16 bits or None.  Asserts the bar above and returns the counts with the mismatches."""
+    rows, nb = ref.scales.shape
+    bad = scales != ref.scales
+    bad |= (codes != ref.codes).reshape(rows, nb, 16).any(-1)
+    if Xq is not None:
+        bad |= (Xq != ref.Xq).reshape(rows, nb, 16).any(-1)
+    c = f46_counts(ref)
+    c["mismatched_blocks"] = n = int(bad.sum())
+    if n:
+        e6, e4 = ref.errs[..., 0], ref.errs[..., 1]
+        assert np.all(np.abs(e4 - e6)[bad] <= F46_BAND * (e4 + e6)[bad]), \
+            f"{n} FourOverSix blocks differ outside the 2^-47 band of the exact errors"
+        assert n <= MAX_MISMATCH_FRAC * bad.size, f"{n} FourOverSix blocks differ in {bad.size}"
+    return c
