@@ -48,7 +48,7 @@ WORKLOAD = "Llama-3.1-8B all 224 linear weights (32 layers x q,o[4096,4096] k,v[
 BYTES_STEP = 11.0625
 KERNEL_SOURCES = ("fp4_post_weight_b200/csrc/focus_kernels.cuh", "fp4_post_weight_b200/csrc/focus_device.cuh",
                   "fp4_post_weight_b200/csrc/focus_pipeline.cuh", "fp4_post_weight_b200/csrc/focus_capi.cu")
-TRAFFIC_RECORD = "profiles/focus_step_fused_export_llama8b_2layers.md"
+TRAFFIC_RECORD = "profiles/step_traffic.json"
 
 
 def kernel_source_hash() -> str:
@@ -76,12 +76,11 @@ def measured_peaks() -> dict:
 
 def recorded_traffic():
     """DRAM bytes per launch of the fused step kernel on the full workload, from the
-    `bench-traffic:` line of the committed ncu summary; None once the kernel sources
-    differ from those the counters were taken with."""
+    committed record of an ncu capture (profiles/step_traffic.json); None once the
+    kernel sources differ from those the counters were taken with."""
     try:
         with open(os.path.join(ROOT, TRAFFIC_RECORD)) as f:
-            line = next(l for l in f if l.startswith("bench-traffic:"))
-        d = json.loads(line.split(":", 1)[1])
+            d = json.load(f)
     except Exception:
         return None
     if d.get("kernel_source_hash") != kernel_source_hash():
@@ -221,8 +220,17 @@ def run_ours(args, world, rank, local):
 
     step_tab.s2()                  # s2 of every tensor before the first step
     amax_ws = torch.zeros(max(step_tab.n, 4), dtype=torch.int32, device=dev)
-    for _ in range(args.warmup):
+    # The CPU baseline times the oracle on a row sample of this workload; its
+    # outputs are checked against what the first warm-up step computed for the
+    # same rows (the inputs are the generator's, taken before that step).
+    do_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    sample = None
+    if do_cpu:
+        sample = ParitySample(ents, int(_oracle_rate() * args.cpu_seconds))
+    for w in range(args.warmup):
         one_step()
+        if w == 0 and sample is not None:
+            sample.read_outputs(ents)
     st = F.focus_get_error()
     if st != 0:
         raise SystemExit(f"device status after warm-up: {F.focus_status_string(st)}")
@@ -270,9 +278,9 @@ def run_ours(args, world, rank, local):
     rows = None
     if not args.no_rows:
         rows = measure_next_rows(ents, dev, N, peaks, world)
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.cpu_seconds)
+    cpu = parity = None
+    if sample is not None:
+        cpu, parity = cpu_baseline(ents, sample)
     if rank == 0:
         line = {"metric": METRIC, "value": round(value, 2), "unit": "Gelem/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -284,10 +292,15 @@ def run_ours(args, world, rank, local):
                            "l2": f"inputs larger than L2 ({N * 8.25 / 1e9:.1f} GB resident per GPU vs 126 MB L2)",
                            "parallelism": f"dp{world} (one model per GPU, no collective)",
                            "bytes_per_elem_step": BYTES_STEP},
-                "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "next_rows": rows,
+                "roofline": roof, "cpu_baseline": cpu, "parity": parity, "e2e": e2e, "next_rows": rows,
                 "gpu_launches": 2 * args.steps, "clocks": clk,
                 "kernel_ms": {"fused_step": round(step_kernel_ms, 4), "fused_step_min": round(min(kms), 4),
-                              "fused_step_max": round(max(kms), 4), "fused_step_each": [round(x, 3) for x in kms]}}
+                              "fused_step_max": round(max(kms), 4),
+                              "fused_step_median": round(statistics.median(kms), 4),
+                              "fused_step_last5_mean": round(sum(kms[-5:]) / len(kms[-5:]), 4),
+                              "fused_step_each": [round(x, 3) for x in kms],
+                              "fused_step_ms_x_median_sm_mhz": (round(step_kernel_ms * clk["sm_mhz"], 1)
+                                                                if clk.get("sm_mhz") else None)}}
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -639,18 +652,182 @@ def _oracle_rate() -> float:
     return n / max(time.time() - t0, 1e-6)
 
 
-def cpu_baseline(seconds: float) -> dict:
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            return next(l.split(":", 1)[1].strip() for l in f if l.startswith("model name"))
+    except Exception:
+        return "unknown"
+
+
+class ParitySample:
+    """A row sample of the benchmark's own tensors: every `stride`-th row of each
+    of them (from an offset that varies by tensor), about `target` weights.  The
+    inputs (W, dW', m, q, the moments) are taken from the device before the first
+    step -- they are the seeded generator's -- and the first step's outputs for
+    the same rows are read back right after it, outside any timed region."""
+
+    def __init__(self, ents, target: int):
+        import math
+
+        import torch
+        N = sum(e.W.numel() for e in ents)
+        self.N = N
+        self.stride = max(1, math.ceil(N / max(target, 1)))
+        self.rows = []
+        for j, e in enumerate(ents):
+            o = e.W.shape[0]
+            off = j % self.stride if j % self.stride < o else 0
+            self.rows.append(torch.arange(off, o, self.stride, device=e.W.device))
+        self.inputs = [self._take(e, r, ("W", "dWq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg",
+                                          "q_exp_avg_sq")) for e, r in zip(ents, self.rows)]
+        self.s2_before = [float(e.s2.item()) for e in ents]
+        self.outputs = None
+
+    @staticmethod
+    def _take(e, rows, names):
+        import numpy as np
+        import torch
+        out = {}
+        for n in names:
+            t = getattr(e, n).index_select(0, rows)
+            if t.dtype == torch.bfloat16:
+                out[n] = t.view(torch.int16).cpu().numpy().view(np.uint16)
+            else:
+                out[n] = t.cpu().numpy()
+        return out
+
+    def read_outputs(self, ents):
+        import torch
+        torch.cuda.synchronize()
+        self.outputs = [self._take(e, r, ("Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg",
+                                          "q_exp_avg_sq", "codes", "scales")) for e, r in zip(ents, self.rows)]
+        self.s2_after = [float(e.s2.item()) for e in ents]
+
+
+def _near_e4m3_boundary(x):
+    """x (float64 array of scaled block maxima) within 2^-20 relative of an E4M3
+    rounding boundary (a midpoint between neighbouring normal values) or of a
+    clamp edge."""
+    import numpy as np
+    mids = []
+    for b in range(0x08, 0x7E):
+        e, mn = (b >> 3) & 15, b & 7
+        e2, mn2 = (e, mn + 1) if mn < 7 else (e + 1, 0)
+        mids.append(((1 + mn / 8) * 2.0 ** (e - 7) + (1 + mn2 / 8) * 2.0 ** (e2 - 7)) / 2)
+    edges = np.array(mids + [2.0 ** -6, 448.0])
+    edges.sort()
+    x = np.asarray(x, np.float64)
+    j = np.clip(np.searchsorted(edges, x), 1, len(edges) - 1)
+    d = np.minimum(np.abs(x - edges[j - 1]), np.abs(x - edges[j]))
+    return d <= 2.0 ** -20 * np.abs(x)
+
+
+def cpu_baseline(ents, sample: ParitySample):
+    """The CPU oracle on the host cores, on the benchmark's own workload: s2 of
+    every tensor over all its weights, then on the sampled rows the forward (W',
+    codes, rounding bands), the straight-through backward with AdamW at step 1,
+    and the NVFP4 export of the updated m and q.  Reported as weights per second
+    of the whole path, a1 charged per weight of the model and the rest per
+    sampled weight.  Its outputs are then compared (outside the timing) with what
+    the first GPU step wrote for the same rows, which gives the parity counts
+    the method's correctness bar asks for: codes (seen through W', which the step
+    writes from the forward's codes and scale bytes) may differ from the oracle's
+    only where y lies within 2^-20 relative of a rounding boundary, and at most
+    1e-6 of the elements; s2 not at all; the updated parameters and
+    moments within |gpu - ref| <= 1e-7 + 1e-5 |ref|; the export of the updated
+    parameters (compared with the oracle's pack of its own update, which agrees
+    within that tolerance) may differ in a scale byte only where x_b lies within
+    2^-20 of an E4M3 rounding boundary and in a code only inside the band."""
+    import numpy as np
+
     import oracle
+    import synth
     oracle.build()
     threads = oracle.num_threads()
-    target = int(_oracle_rate() * seconds)
-    sample, layers, frac = oracle_sample_inputs(target)
+    # single-threaded: W[2048, 2048] ~ N(0, 0.02), m = 1, q = 6, forward + pack
+    c1 = synth.single_2048("cpu")
+    W1 = synth.bits(c1.W)
+    oracle.set_threads(1)
     t0 = time.time()
-    n = oracle_step(sample)
-    dt = time.time() - t0
-    return {"value": round(n / dt / 1e9, 5), "unit": "Gelem/s", "cores": threads, "kind": "oracle",
-            "sample": f"{frac:.3f} of the rows of each Llama-3.1-8B projection shape over {layers} layer(s) "
-                      f"({n} weights): s2 + fwd + STE-bwd + AdamW + pack, {dt:.1f} s on {threads} OpenMP threads"}
+    s21 = oracle.s2(W1)
+    oracle.fwd(W1, c1.m.numpy(), c1.q.numpy(), s21, want_y=False)
+    oracle.pack(W1, c1.m.numpy(), c1.q.numpy(), s21)
+    t_c1 = time.time() - t0
+    oracle.set_threads(threads)
+    # s2 of every tensor over all its rows
+    import torch
+    t_s2 = 0.0
+    s2s = []
+    for e in ents:
+        wb = e.W.view(torch.int16).cpu().numpy().view(np.uint16)
+        t0 = time.time()
+        s2s.append(oracle.s2(wb))
+        t_s2 += time.time() - t0
+        del wb
+    # the path on the sampled rows, each tensor's outputs compared (untimed) with
+    # what the first GPU step wrote for the same rows
+    tol = lambda g, r: np.abs(g.astype(np.float64) - r) > 1e-7 + 1e-5 * np.abs(r.astype(np.float64))
+    c = {k: 0 for k in ("elements", "blocks", "band", "exact_ties", "code_mismatch", "code_mismatch_outside_band",
+                        "s2_mismatch", "state_outside_tolerance", "export_scale_mismatch",
+                        "export_scale_mismatch_off_boundary", "export_code_mismatch",
+                        "export_code_mismatch_outside_band", "zero_blocks", "clamp_low", "clamp_high",
+                        "out_of_range")}
+    n = 0
+    t_path = 0.0
+    for j, (inp, out, s2) in enumerate(zip(sample.inputs, sample.outputs, s2s)):
+        W, G = inp["W"], inp["dWq"]
+        m, q = inp["m"].copy(), inp["q"].copy()
+        mo = [inp[k].copy() for k in ("m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq")]
+        t0 = time.time()
+        fwd = oracle.fwd(W, m, q, s2, want_y=False)
+        oracle.step(W, G, m, q, *mo, s2, 1, want_wq=False)
+        exp = oracle.fwd(W, m, q, s2, want_y=False)
+        t_path += time.time() - t0
+        n += W.size
+        c["s2_mismatch"] += int(np.float32(sample.s2_before[j]) != s2) + int(np.float32(sample.s2_after[j]) != s2)
+        c["elements"] += W.size
+        c["blocks"] += W.size // 16
+        for k in ("band", "exact_ties", "zero_blocks", "clamp_low", "clamp_high", "out_of_range"):
+            c[k] += fwd.stats[k]
+        # W' is the forward's (before the update): it differs only where a code does
+        wbad = out["Wq"] != fwd.Wq
+        c["code_mismatch"] += int(wbad.sum())
+        c["code_mismatch_outside_band"] += int((wbad & (fwd.band != 1)).sum())
+        skip = wbad.reshape(W.shape[0], -1, 16).any(-1)
+        for g, r, sk in zip(("m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"), [m, q] + mo,
+                            (1, 2, 1, 1, 2, 2)):
+            c["state_outside_tolerance"] += int((tol(out[g], r) & ~np.repeat(skip, sk, axis=1)).sum())
+        # the export of the updated parameters
+        sbad = out["scales"] != exp.scales
+        if sbad.any():
+            A = ((W.astype(np.uint32) & 0x7FFF) << 16).view(np.float32).reshape(W.shape[0], -1, 16).max(-1)
+            x = (A * m) / (np.float32(6) * np.float32(s2))
+            c["export_scale_mismatch_off_boundary"] += int((~_near_e4m3_boundary(x[sbad])).sum())
+        c["export_scale_mismatch"] += int(sbad.sum())
+        codes = np.empty(W.shape, np.uint8)
+        codes[:, 0::2], codes[:, 1::2] = out["codes"] & 0xF, out["codes"] >> 4
+        cbad = (codes != exp.codes) & ~np.repeat(sbad, 16, axis=1)
+        c["export_code_mismatch"] += int(cbad.sum())
+        c["export_code_mismatch_outside_band"] += int((cbad & (exp.band != 1)).sum())
+        del fwd, exp, codes
+    value = n / (t_path + t_s2 * n / sample.N) / 1e9
+    cpu = {"value": round(value, 5), "unit": "Gelem/s", "cores": threads, "kind": "oracle",
+           "cpu_model": _cpu_model(), "nproc": os.cpu_count(),
+           "sample": f"the benchmark's own weights: s2 of all {sample.N} weights ({t_s2:.1f} s), then every "
+                     f"{sample.stride}th row of each of the {len(ents)} tensors ({n} weights): forward, "
+                     f"STE-bwd + AdamW and the NVFP4 export of the update ({t_path:.1f} s), on {threads} "
+                     f"OpenMP threads; s2 time charged per weight of the model",
+           "single_thread_c1": {"value": round(W1.size / t_c1 / 1e9, 5), "unit": "Gelem/s", "seconds": round(t_c1, 3),
+                                "work": "W[2048,2048] ~ N(0,0.02), m = 1, q = 6: s2 + forward + pack, 1 thread"}}
+    c["meets_bar"] = bool(c["code_mismatch_outside_band"] == 0 and c["code_mismatch"] <= 1e-6 * c["elements"]
+                          and c["s2_mismatch"] == 0
+                          and c["state_outside_tolerance"] == 0 and c["export_scale_mismatch_off_boundary"] == 0
+                          and c["export_code_mismatch_outside_band"] == 0
+                          and 16 * c["export_scale_mismatch"] + c["export_code_mismatch"] <= 1e-6 * c["elements"])
+    c["what"] = ("first GPU step of this run (the benchmarked launch) on every "
+                 f"{sample.stride}th row of the {len(ents)} tensors, against the oracle of the CPU baseline")
+    return cpu, c
 
 
 def run_reference(args, world, rank):
@@ -698,7 +875,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="skip the next-row measurements")
-    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-seconds", type=float, default=4.0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -5,7 +5,8 @@
   for bit (signed zeros included),
   for every bf16 significand of w (both signs, and +-0) and every binary32
   significand of D, at several exponent pairs inside the range the kernels
-  use it for.
+  use it for; where the quotient falls below the normal range (tiny w, large
+  D) it is within one unit of 2^-149 with the same sign and E2M1 code.
 * fl(c*S) through the mixed-precision FMA equals the binary32 product for
   every E2M1 value and every normal E4M3 scale, and c - y likewise.
 * The E2M1 conversion keeps the sign of negative values that round to zero
@@ -67,6 +68,21 @@ def test_division_exhaustive(lib, we, de, variant):
     n = ctypes.c_ulonglong(0)
     ex = (ctypes.c_float * 4)()
     assert lib.check_div(we, de, ctypes.byref(n), ex, variant) == 0
+    assert n.value == 0, f"{n.value} quotients differ, e.g. w={ex[0]!r} D={ex[1]!r} got {ex[2]!r} want {ex[3]!r}"
+
+
+@pytest.mark.parametrize("variant", [0, 2], ids=["scalar", "packed"])
+@pytest.mark.parametrize("we,de", [(-126, 0), (-126, 5), (-133, 0), (-90, 40), (-110, 30), (-100, 59), (-126, 59),
+                                   (-133, 59), (-120, -3)])
+def test_division_tiny_quotients(lib, we, de, variant):
+    """Tiny w over a large D (the kernels take the fast quotient whenever D lies in
+    [2^-60, 2^60], whatever |w|): where the IEEE quotient is normal the bits agree;
+    below the normal range the result may be one unit of 2^-149 off, with the same
+    sign, so its E2M1 code is the same signed zero and its share of a gradient sum
+    is below 2^-149 |g|."""
+    n = ctypes.c_ulonglong(0)
+    ex = (ctypes.c_float * 4)()
+    assert lib.check_div(we, de, ctypes.byref(n), ex, variant | 4) == 0
     assert n.value == 0, f"{n.value} quotients differ, e.g. w={ex[0]!r} D={ex[1]!r} got {ex[2]!r} want {ex[3]!r}"
 
 
