@@ -334,7 +334,8 @@ def measure_next_rows(ents, dev, N, peaks, world):
         and scales, and codes, scales and W');
       * FourOverSix with one scale per token over one decoder layer's linear
         inputs for a micro-batch of 4096 tokens (q/k/v, o and gate/up inputs
-        [4096, 4096], the down input [4096, 14336]: 208 MB);
+        [4096, 4096], the down input [4096, 14336]: 208 MB), one launch over
+        the four tensors (and, for comparison, one launch per width);
       * a calibration step over four micro-batches: three table backward passes
         (the first overwriting dm/dq, then accumulating) and the fused step
         with FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WQ_UPDATED;
@@ -370,44 +371,46 @@ def measure_next_rows(ents, dev, N, peaks, world):
     out["nvfp4_rtn_weights_llama8b"] = {"kernel": "pipe_kernel<KIND_F46> (rtn)", "bytes_per_weight": 2.5625,
                                         "Gelem_s": round(N * world / (ms * 1e-3) / 1e9, 2),
                                         **_roof(2.5625 * N, ms, peak)}
-    # FourOverSix activations, one scale per token
+    # FourOverSix activations, one scale per token: one launch over the layer's four
+    # activation tensors (rows staged in shared memory)
+    from fp4_post_weight_b200.table import ActTable, act_entry
     Xs = [synth.activations(4096, h, dev, seed=50 + j) for j, h in enumerate((4096, 4096, 4096, 14336))]
     bufs = [(torch.empty(X.shape[0], device=dev), torch.empty((X.shape[0], X.shape[1] // 2), dtype=torch.uint8,
                                                                 device=dev),
              torch.empty((X.shape[0], X.shape[1] // 16), dtype=torch.uint8, device=dev)) for X in Xs]
     n_act = sum(X.numel() for X in Xs)
     b_act = sum(X.numel() * (2 + 0.5 + 0.0625) + 4 * X.shape[0] for X in Xs)
-
-    def act():
-        for X, (ts, c, sc) in zip(Xs, bufs):
-            F.focus_fouroversix_act(X, ts, c, sc)
-    ms = _timed(act, stream)
-    out["fouroversix_act_4096_tokens_one_layer"] = {"kernel": "f46_rows_kernel", "launches": 4,
+    act_tab = ActTable([act_entry(X, ts, c, sc) for X, (ts, c, sc) in zip(Xs, bufs)])
+    ms = _timed(act_tab.fouroversix, stream)
+    out["fouroversix_act_4096_tokens_one_layer"] = {"kernel": "rows_staged_kernel", "launches": 1,
                                                      "elements": n_act, "bytes_per_elem": 2.5625,
                                                      "Gelem_s": round(n_act / (ms * 1e-3) / 1e9, 2),
                                                      **_roof(b_act, ms, peak)}
+    # the same, one launch per width (the three 4096-wide tensors, then the 14336-wide one)
+    t_a = ActTable([act_entry(X, ts, c, sc) for X, (ts, c, sc) in zip(Xs[:3], bufs[:3])])
+    t_b = ActTable([act_entry(Xs[3], *bufs[3])])
+
+    def act_by_width():
+        t_a.fouroversix()
+        t_b.fouroversix()
+    ms = _timed(act_by_width, stream)
+    out["fouroversix_act_4096_tokens_one_layer"]["by_width"] = {
+        "launches": 2, "Gelem_s": round(n_act / (ms * 1e-3) / 1e9, 2), **_roof(b_act, ms, peak)}
     # the same writing the scales in the 128x4 layout of sm_100 block-scaled GEMMs
     # (4096 tokens and hidden/16 columns: no padding, the same bytes)
     swz = [torch.empty(F.focus_scales_swizzled_bytes(X.shape[0], X.shape[1] // 16), dtype=torch.uint8, device=dev)
            for X in Xs]
-
-    def act_swz():
-        for X, (ts, c, _), sw in zip(Xs, bufs, swz):
-            F.focus_fouroversix_act_swizzled(X, ts, c, sw)
-    ms = _timed(act_swz, stream)
+    swz_tab = ActTable([act_entry(X, ts, c, sw) for X, (ts, c, _), sw in zip(Xs, bufs, swz)], swizzled=True)
+    ms = _timed(swz_tab.fouroversix, stream)
     out["fouroversix_act_4096_tokens_one_layer"]["scales_128x4"] = {
-        "kernel": "f46_rows_kernel<SWZ>", "Gelem_s": round(n_act / (ms * 1e-3) / 1e9, 2), **_roof(b_act, ms, peak)}
+        "kernel": "rows_staged_kernel<SWZ>", "Gelem_s": round(n_act / (ms * 1e-3) / 1e9, 2), **_roof(b_act, ms, peak)}
     # plain NVFP4 round to nearest per token (the target 6 alone), same inputs and bytes
-
-    def act_rtn():
-        for X, (ts, c, sc) in zip(Xs, bufs):
-            F.focus_nvfp4_act(X, ts, c, sc)
-    ms = _timed(act_rtn, stream)
-    out["nvfp4_act_4096_tokens_one_layer"] = {"kernel": "f46_rows_kernel<RTN>", "launches": 4, "elements": n_act,
+    ms = _timed(act_tab.nvfp4, stream)
+    out["nvfp4_act_4096_tokens_one_layer"] = {"kernel": "rows_staged_kernel<RTN>", "launches": 1, "elements": n_act,
                                                "bytes_per_elem": 2.5625,
                                                "Gelem_s": round(n_act / (ms * 1e-3) / 1e9, 2),
                                                **_roof(b_act, ms, peak)}
-    del Xs, bufs, swz
+    del Xs, bufs, swz, act_tab, swz_tab, t_a, t_b
     # the calibration step over four micro-batches
     for e in ents:
         e.dm = torch.zeros_like(e.m)

@@ -15,6 +15,7 @@
 #include "focus_trace.cuh"
 #include "focus_kernels.cuh"
 #include "focus_mx.cuh"
+#include "focus_rows.cuh"
 
 namespace focus {
 
@@ -440,8 +441,31 @@ int focus_adamw_step(float *p, const float *g, float *exp_avg, float *exp_avg_sq
 int focus_table_prepare(focus_tensor_desc *d, int n, int purpose, int64_t *total_tiles) {
     FOCUS_RANGE();
     if (!d || !total_tiles) return FOCUS_ERR_NULL;
-    if (n < 0 || purpose < 0 || purpose > FOCUS_PURPOSE_MX) return FOCUS_ERR_VALUE;
+    if (n < 0 || purpose < 0 || purpose > FOCUS_PURPOSE_ACT_SWIZZLED) return FOCUS_ERR_VALUE;
     int64_t tiles = 0, blocks = 0;
+    if (purpose == FOCUS_PURPOSE_ACT || purpose == FOCUS_PURPOSE_ACT_SWIZZLED) {
+        // activation tensors for the per-token calls: W = X, s2 = token scales;
+        // tile_begin is the entry's first row (rows padded to 128 for the 128x4 layout)
+        int64_t rows = 0;
+        for (int i = 0; i < n; ++i) {
+            focus_tensor_desc &e = d[i];
+            int rc = check_shape(e.out, e.in);
+            if (rc) return rc;
+            if (e.in > RS_MAX_HIDDEN) return FOCUS_ERR_SHAPE;
+            if (e.out * e.in > 0) {
+                if (!e.W || !e.s2 || !e.codes || !e.scales) return FOCUS_ERR_NULL;
+                const void *ptrs[] = {e.W, e.s2, e.codes, e.scales, e.Wq};
+                for (const void *p : ptrs)
+                    if (p && !aligned16(p)) return FOCUS_ERR_ALIGN;
+            }
+            e.block_begin = blocks;
+            e.tile_begin = rows;
+            blocks += e.out * (e.in / 16);
+            if (e.out * e.in > 0) rows += purpose == FOCUS_PURPOSE_ACT_SWIZZLED ? (e.out + 127) / 128 * 128 : e.out;
+        }
+        *total_tiles = rows;
+        return FOCUS_OK;
+    }
     if (purpose == FOCUS_PURPOSE_MX) {
         for (int i = 0; i < n; ++i) {
             focus_tensor_desc &e = d[i];
@@ -674,6 +698,53 @@ int focus_nvfp4_weight_multi(const focus_tensor_desc *descs_dev, int n, int64_t 
 }  // extern "C"
 
 namespace {
+// The staged per-token kernel over the rows of `a` (one entry or a device
+// table), buffers sized for rows of a.max_in values.
+template <bool SWZ, bool RTN>
+int launch_rows_staged_t(const RowArgs &a, cudaStream_t stream) {
+    static std::once_flag once[MAX_DEVICES];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return FOCUS_ERR_CUDA;
+    std::call_once(once[dev], [] {
+        cudaFuncSetAttribute(rows_staged_kernel<SWZ, RTN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(2 * RS_MAX_HIDDEN * 2));
+    });
+    DeviceInfo *di;
+    int rc = device_info(&di);
+    if (rc) return rc;
+    const uint32_t stage = (uint32_t)((a.max_in * 2 + 127) / 128 * 128);
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rows_staged_kernel<SWZ, RTN>, RS_THREADS, 2 * stage) !=
+            cudaSuccess || occ <= 0)
+        return FOCUS_ERR_CUDA;
+    const int64_t grid = grid_for(a.total_rows, di->sms, occ);
+    if (grid <= 0) return FOCUS_OK;
+    rows_staged_kernel<SWZ, RTN><<<(unsigned)grid, RS_THREADS, 2 * stage, stream>>>(a, stage);
+    return launch_status();
+}
+
+int launch_rows_staged(const RowArgs &a, bool rtn, bool swz, cudaStream_t stream) {
+    if (swz && rtn) return launch_rows_staged_t<true, true>(a, stream);
+    if (swz) return launch_rows_staged_t<true, false>(a, stream);
+    if (rtn) return launch_rows_staged_t<false, true>(a, stream);
+    return launch_rows_staged_t<false, false>(a, stream);
+}
+
+// The per-token quantizers over a prepared table of activation tensors.
+int act_rows_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_rows, int64_t max_hidden, bool rtn,
+                   bool swz, cudaStream_t stream) {
+    if (n < 0 || total_rows < 0) return FOCUS_ERR_VALUE;
+    if (n == 0 || total_rows == 0) return FOCUS_OK;
+    if (!descs_dev) return FOCUS_ERR_NULL;
+    if (max_hidden < 16 || max_hidden % 16 != 0 || max_hidden > RS_MAX_HIDDEN) return FOCUS_ERR_SHAPE;
+    RowArgs a{};
+    a.table = descs_dev;
+    a.n_tensors = n;
+    a.total_rows = total_rows;
+    a.max_in = max_hidden;
+    return launch_rows_staged(a, rtn, swz, stream);
+}
+
 // The per-token quantizers: FourOverSix or NVFP4 round to nearest (rtn), the
 // block scales row-major or in the 128x4-atom layout (swz: scales_bytes is
 // the caller's buffer size).
@@ -686,6 +757,18 @@ int act_rows(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_sca
     if (!aligned16(X) || !aligned16(token_scales) || !aligned16(codes) || !aligned16(scales) || !aligned16(Xq))
         return FOCUS_ERR_ALIGN;
     if (swz && scales_bytes < focus_scales_swizzled_bytes(tokens, hidden / 16)) return FOCUS_ERR_WORKSPACE;
+    if (hidden <= RS_MAX_HIDDEN) {                  // rows staged in shared memory
+        RowArgs a{};
+        a.table = nullptr;
+        a.n_tensors = 1;
+        a.total_rows = swz ? (tokens + 127) / 128 * 128 : tokens;
+        a.max_in = hidden;
+        a.one = one_desc(X, nullptr, Xq, nullptr, nullptr, tokens, hidden);
+        a.one.s2 = token_scales;
+        a.one.codes = codes;
+        a.one.scales = scales;
+        return launch_rows_staged(a, rtn, swz, stream);
+    }
     DeviceInfo *di;
     if ((rc = device_info(&di))) return rc;
     const int64_t rows_out = swz ? (tokens + 127) / 128 * 128 : tokens;
@@ -730,6 +813,18 @@ int focus_nvfp4_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hidden, 
     FOCUS_RANGE();
     return act_rows(X, tokens, hidden, token_scales, codes, scales_swz, scales_bytes, Xq, true, true,
                     (cudaStream_t)stream);
+}
+
+int focus_fouroversix_act_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_rows,
+                                int64_t max_hidden, int swizzled, focus_stream_t stream) {
+    FOCUS_RANGE();
+    return act_rows_multi(descs_dev, n_tensors, total_rows, max_hidden, false, swizzled != 0, (cudaStream_t)stream);
+}
+
+int focus_nvfp4_act_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_rows, int64_t max_hidden,
+                          int swizzled, focus_stream_t stream) {
+    FOCUS_RANGE();
+    return act_rows_multi(descs_dev, n_tensors, total_rows, max_hidden, true, swizzled != 0, (cudaStream_t)stream);
 }
 
 int focus_mx_fwd(const uint16_t *W, const float *m, const float *q, int64_t out, int64_t in, uint16_t *Wq,

@@ -259,7 +259,12 @@ __device__ __forceinline__ void store_wq_from_codes(const TV &T, uint32_t blk, c
 struct F46Scale {
     float s, den6, rden6, den4, rden4;
     bool den_ok;
+    bool fast;   // den_ok and s in [2^-54, 2^51], so that every D = S*s (S in [2^-6, 448]) is in [2^-60, 2^60]
 };
+
+__device__ __forceinline__ bool f46_scale_fast(bool den_ok, float s) {
+    return den_ok && s >= 0x1p-54f && s <= 0x1p51f;
+}
 
 __device__ __forceinline__ F46Scale f46_scale(float s) {
     F46Scale c;
@@ -269,6 +274,7 @@ __device__ __forceinline__ F46Scale f46_scale(float s) {
     c.den_ok = c.den6 >= 0x1p-60f && c.den6 <= 0x1p60f && c.den4 >= 0x1p-60f && c.den4 <= 0x1p60f;
     c.rden6 = c.den_ok ? rcp_rn(c.den6) : 0.0f;
     c.rden4 = c.den_ok ? rcp_rn(c.den4) : 0.0f;
+    c.fast = f46_scale_fast(c.den_ok, s);
     return c;
 }
 
@@ -297,6 +303,40 @@ __device__ __forceinline__ F46Target f46_target(float x, float s, float A) {
     t.fast = t.D >= 0x1p-60f && t.D <= 0x1p60f && A <= 0x1p60f;
     t.nr = t.fast ? -rcp_rn(t.D) : 0.0f;
     return t;
+}
+
+// Both targets of a block whose scale is fast (sc.fast) and whose maximum A
+// lies in [2^-60, 2^60] or is 0, bit for bit what f46_target(f46_x(...)) gives
+// each: the two scaled maxima x_6 = fl(A/fl(6s)), x_4 = fl(A/fl(4s)) as one
+// packed pair (div_full's Markstein steps, lane by lane), 1 for a zero block,
+// clamped below at 2^-6 (the conversion's saturation is the clamp at 448),
+// both E4M3 bytes from one conversion, and D_T = fl(S_T*s) as one packed
+// product, which lies in [2^-60, 2^60] by sc.fast.
+__device__ __forceinline__ void f46_targets_fast(float A, const F46Scale &sc, F46Target &t6, F46Target &t4) {
+    const uint64_t A2 = f2_pack(A, A);
+    const uint64_t r2 = f2_pack(sc.rden6, sc.rden4);
+    const uint64_t nd2 = f2_pack(-sc.den6, -sc.den4);
+    uint64_t q = f2_mul(A2, r2);
+    uint64_t e = f2_fma(q, nd2, A2);
+    q = f2_fma(e, r2, q);
+    e = f2_fma(q, nd2, A2);
+    q = f2_fma(e, r2, q);
+    float x6 = f2_lo(q), x4 = f2_hi(q);
+    if (A == 0.0f) x6 = x4 = 1.0f;
+    x6 = fmaxf(x6, 0x1p-6f);
+    x4 = fmaxf(x4, 0x1p-6f);
+    uint16_t sbs;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sbs) : "f"(x4), "f"(x6));
+    t6.sb = (uint32_t)sbs & 0xffu;
+    t4.sb = (uint32_t)sbs >> 8;
+    t6.S_h = (uint16_t)e4m3_normal_f16_bits(t6.sb);
+    t4.S_h = (uint16_t)e4m3_normal_f16_bits(t4.sb);
+    const uint64_t D2 = f2_mul(f2_pack(e4m3_normal_f32(t6.sb), e4m3_normal_f32(t4.sb)), f2_pack(sc.s, sc.s));
+    t6.D = f2_lo(D2);
+    t4.D = f2_hi(D2);
+    t6.nr = -rcp_rn(t6.D);
+    t4.nr = -rcp_rn(t4.D);
+    t6.fast = t4.fast = true;
 }
 
 // The quotient pair y = w / D of one pair of weights under a target.  FAST:
@@ -396,19 +436,30 @@ __device__ __noinline__ bool f46_four_exact(uint4 wa, uint4 wb, uint32_t c6_0, u
 // (one rounding in every d, two in every fused square-and-add of a lane, one in
 // the final add), plus at most 2^-144 absolute where values are subnormal.  So
 // when |e4 - e6| exceeds 2^-19 (e4 + e6) + 2^-140 the binary32 order is the
-// exact order.  Otherwise -- a near tie, an exact tie (they occur: about one
-// block in 10^7 of Gaussian weights), or a non-finite sum -- the choice is
-// taken by f46_four_exact.
+// exact order.  Otherwise -- a near tie, an exact tie between different
+// candidates (they occur: about one block in 10^7 of Gaussian weights), or a
+// non-finite sum -- the choice is taken by f46_four_exact, unless the two
+// candidates are the same (equal scale bytes).
 __device__ __forceinline__ bool f46_block(const uint32_t *w, float A, const F46Scale &sc, uint32_t &sb,
                                           uint32_t codes[2]) {
-    const F46Target t6 = f46_target(f46_x(A, sc.den6, sc.rden6, sc.den_ok), sc.s, A);
-    const F46Target t4 = f46_target(f46_x(A, sc.den4, sc.rden4, sc.den_ok), sc.s, A);
+    F46Target t6, t4;
     uint32_t c6[2], c4[2];
     float e6, e4;
-    if (t6.fast && t4.fast) f46_both<true>(w, t6, t4, sc.s, c6, c4, e6, e4);
-    else f46_both<false>(w, t6, t4, sc.s, c6, c4, e6, e4);
+    if (sc.fast && A <= 0x1p60f && (A >= 0x1p-60f || A == 0.0f)) {
+        f46_targets_fast(A, sc, t6, t4);
+        f46_both<true>(w, t6, t4, sc.s, c6, c4, e6, e4);
+    } else {
+        t6 = f46_target(f46_x(A, sc.den6, sc.rden6, sc.den_ok), sc.s, A);
+        t4 = f46_target(f46_x(A, sc.den4, sc.rden4, sc.den_ok), sc.s, A);
+        if (t6.fast && t4.fast) f46_both<true>(w, t6, t4, sc.s, c6, c4, e6, e4);
+        else f46_both<false>(w, t6, t4, sc.s, c6, c4, e6, e4);
+    }
     bool four = e4 < e6;
-    if (!(fabsf(e4 - e6) > fmaf(0x1p-19f, e4 + e6, 0x1p-140f))) {
+    // Equal scale bytes make the two candidates identical (an exact tie: 6 is
+    // kept, and e4 < e6 is false); this is the block of a tensor's or token's
+    // maximum, where both scales clamp at 448.  Any other near tie is decided
+    // exactly.
+    if (t4.sb != t6.sb && !(fabsf(e4 - e6) > fmaf(0x1p-19f, e4 + e6, 0x1p-140f))) {
         const uint4 wa = make_uint4(w[0], w[1], w[2], w[3]), wb = make_uint4(w[4], w[5], w[6], w[7]);
         four = f46_four_exact(wa, wb, c6[0], c6[1], t6.S_h, c4[0], c4[1], t4.S_h, sc.s);
     }
@@ -422,7 +473,18 @@ __device__ __forceinline__ bool f46_block(const uint32_t *w, float A, const F46S
 // equations with m = 1 and sigmoid = 1) with block maximum A and scale sc.s > 0.
 __device__ __forceinline__ void rtn_block(const uint32_t *w, float A, const F46Scale &sc, uint32_t &sb,
                                           uint32_t codes[2]) {
-    const F46Target t6 = f46_target(f46_x(A, sc.den6, sc.rden6, sc.den_ok), sc.s, A);
+    F46Target t6;
+    if (sc.fast && A <= 0x1p60f && (A >= 0x1p-60f || A == 0.0f)) {
+        // as f46_target(f46_x(...)), without the range checks sc.fast makes redundant
+        float x = (A == 0.0f) ? 1.0f : div_full(A, sc.den6, sc.rden6);
+        t6.sb = e4m3_byte(fmaxf(x, 0x1p-6f));           // the conversion saturates at 448
+        t6.S_h = (uint16_t)e4m3_normal_f16_bits(t6.sb);
+        t6.D = __fmul_rn(e4m3_normal_f32(t6.sb), sc.s);
+        t6.nr = -rcp_rn(t6.D);
+        t6.fast = true;
+    } else {
+        t6 = f46_target(f46_x(A, sc.den6, sc.rden6, sc.den_ok), sc.s, A);
+    }
     sb = t6.sb;
     const uint64_t D6 = f2_pack(t6.D, t6.D), n6 = f2_pack(t6.nr, t6.nr);
 #pragma unroll
@@ -476,6 +538,7 @@ __device__ __forceinline__ void compute_block_f46(const TV &T, Block &B, bool rt
         F46Scale sc;
         sc.s = T.s2; sc.den6 = T.den; sc.rden6 = T.rden; sc.den4 = T.den4; sc.rden4 = T.rden4;
         sc.den_ok = T.den46_ok;
+        sc.fast = f46_scale_fast(sc.den_ok, sc.s);
         uint32_t sb, codes[2];
         if (rtn) rtn_block(B.w, __uint_as_float(abits << 16), sc, sb, codes);
         else f46_block(B.w, __uint_as_float(abits << 16), sc, sb, codes);

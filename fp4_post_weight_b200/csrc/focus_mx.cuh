@@ -63,12 +63,22 @@ __device__ __forceinline__ float pow2f(int e) {           // 2^e for e in [-127,
 // The export of one 32-block from the UPDATED m and q (qn): the same
 // arithmetic as the forward below, so the result is bit for bit what the
 // forward writes when run after the step.  Codes and scale when pack_updated,
-// W' when wq_updated.
-__device__ __forceinline__ void mx_encode(const MxArgs &a, int64_t blk, const uint32_t *w, float A, float m,
-                                          const float *qn) {
+// W' when wq_updated.  The block's W is read again here (the step's first
+// read left it in L1) rather than held in sixteen registers across the
+// update.
+__device__ __forceinline__ void mx_encode(const MxArgs &a, int64_t blk, float A, float m, const float *qn) {
     const bool want_codes = a.pack_updated && a.codes != nullptr;
     const bool want_wq = a.wq_updated && a.Wq != nullptr;
     if (!want_codes && !want_wq) return;
+    uint32_t w[16];
+    {
+        const uint4 *Wp = reinterpret_cast<const uint4 *>(a.W) + 4 * blk;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 v = __ldg(Wp + j);
+            w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+        }
+    }
     if (!finitef(m) || !finitef(qn[0]) || !finitef(qn[1]) || !finitef(qn[2]) || !finitef(qn[3]))
         atomicOr(&g_error_flags, 1u);
     const float x = __fmul_rn(A, m);
@@ -122,7 +132,7 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
         const uint4 *Wp = reinterpret_cast<const uint4 *>(a.W) + 4 * blk;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const uint4 v = __ldcs(Wp + j);
+            const uint4 v = EXPORT ? __ldg(Wp + j) : __ldcs(Wp + j);    // the export reads it again
             w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
         }
         if (KIND != KIND_FWD) {
@@ -233,7 +243,7 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
                 reinterpret_cast<float4 *>(a.q_eas)[blk] = make_float4(f2_lo(b01), f2_hi(b01), f2_lo(b23), f2_hi(b23));
                 if (EXPORT) {
                     const float qn[4] = {f2_lo(p01), f2_hi(p01), f2_lo(p23), f2_hi(p23)};
-                    mx_encode(a, blk, w, A, m, qn);
+                    mx_encode(a, blk, A, m, qn);
                 }
             }
         }
@@ -271,7 +281,7 @@ struct MxMultiArgs {
 };
 
 template <int KIND, bool EXPORT = false>
-__global__ void __launch_bounds__(MX_TILE_BLOCKS) mx_multi_kernel(const MxMultiArgs g) {
+__global__ void __launch_bounds__(MX_TILE_BLOCKS, 7) mx_multi_kernel(const MxMultiArgs g) {
     __shared__ MxArgs sa;
     __shared__ int64_t s_range[2];          // tiles [first, end) of the current tensor
     int t = 0;                              // thread 0's table cursor

@@ -1,0 +1,225 @@
+// focus_rows.cuh -- the per-token quantizers (FourOverSix, or plain NVFP4 round
+// to nearest) over one or more activation tensors in one launch, rows staged
+// in shared memory.
+//
+// Model card "FOCUS NVFP4 scales for Llama-3.2-1B-Instruct (our
+// reproduction)", section "Calibration" (activation bullet: FourOverSix with
+// one FP32 scale per token) and section "Perplexity" (the NVFP4 baseline: one
+// scale per token).  For every row (token) r of X [tokens, hidden]:
+//   s_r = fl(max_row |x| / 2688);  every 16-block as the weights' quantizer
+//   with s_r in place of s2 (FourOverSix: the target 6 or 4 of the lower
+//   squared error; NVFP4: the target 6);  a row of zeros has s_r = 0, scale
+//   bytes 0x38, codes 0 and values 0.
+//
+// Work decomposition.  A CTA takes rows R = blockIdx.x, blockIdx.x + grid,
+// ... of the table's rows (each entry's rows in order; with the 128x4 scale
+// layout an entry's rows are padded to a multiple of 128 and a padding row
+// only writes its scale words 0).  Thread 0 stages a row in shared memory with
+// one 1-D bulk copy (completion counted in bytes on an mbarrier) while the
+// CTA quantizes the previous one from the other buffer, so X is read from HBM
+// once and both passes over a row read shared memory: the first computes the
+// block maxima and their row maximum, the second
+// quantizes every block.  Thread t owns the blocks t, t + RS_THREADS, ...
+// (consecutive threads, consecutive 32-byte blocks) and keeps their maxima
+// in its own slots of a shared array between the passes.  Rows up to
+// RS_MAX_HIDDEN values; longer rows take f46_rows_kernel.
+//
+// Every wait is bounded (focus_pipeline.cuh); the decision to stop is made
+// uniformly through the row's barrier, and a CTA that stops waits (bounded)
+// for its last copy before it exits.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "focus.h"
+#include "focus_kernels.cuh"
+#include "focus_pipeline.cuh"
+
+namespace focus {
+
+constexpr int RS_THREADS = 256;                           // 8 warps per CTA
+constexpr int RS_BPT = 4;                                 // blocks per thread at most
+constexpr int64_t RS_MAX_HIDDEN = 16 * RS_THREADS * RS_BPT;   // 16384 values per row
+
+// The activation tensors of one launch.  Each entry uses focus_tensor_desc
+// fields as: W = X [out = tokens, in = hidden] bf16, s2 = token scales
+// [tokens] (written), codes [tokens][hidden/2], scales (row-major
+// [tokens][hidden/16], or the 128x4-atom buffer), Wq = X' (nullable),
+// tile_begin = the entry's first row in the launch's row numbering.
+struct RowArgs {
+    const focus_tensor_desc *table;  // device table, or nullptr: use `one`
+    int n_tensors;
+    int64_t total_rows;
+    int64_t max_in;                  // the staging buffers hold rows of at most this many values
+    focus_tensor_desc one;
+};
+
+// The record of a staged row, written by thread 0 before it completes the
+// stage's barrier phase and read by every thread after waiting on it.
+struct RowStage {
+    float *ts;          // token scales of the row's entry
+    uint8_t *codes;
+    uint8_t *scales;
+    uint16_t *xq;
+    int64_t r;          // row within its entry
+    int64_t nb;         // 16-blocks per row
+    int64_t groups;     // column groups of 4 scales (128x4 layout)
+    uint32_t mode;      // ROW_SKIP, ROW_DATA or ROW_PAD
+};
+enum : uint32_t { ROW_SKIP = 0, ROW_DATA = 1, ROW_PAD = 2 };
+
+// Thread 0: fill the record of global row R and stage the row into `dst`
+// (one bulk copy of hidden*2 bytes, completion on `bar`); for a padding row,
+// a skipped or an empty one, complete the barrier's phase without data.  An
+// entry wider than the buffers is skipped and reported.
+// (The entry of R is found by scanning the table forward from entry t, which
+// the caller keeps: a CTA's rows only increase.  The descriptor is read again
+// for every row rather than held in registers across the loop.)
+template <bool SWZ>
+__device__ __forceinline__ void stage_row(const RowArgs &a, int64_t R, int &t, unsigned char *dst, uint64_t *bar,
+                                          RowStage &rec) {
+    const uint32_t b = smem_u32(bar);
+    const int n = a.table ? a.n_tensors : 1;
+    focus_tensor_desc d;
+    int64_t end;
+    for (;;) {
+        d = a.table ? a.table[t] : a.one;
+        end = d.tile_begin + (SWZ ? (d.out + 127) / 128 * 128 : d.out);
+        if (R < end || t + 1 >= n) break;
+        ++t;
+    }
+    rec.mode = ROW_SKIP;
+    if (R < end) {
+        const int64_t r = R - d.tile_begin;
+        rec.ts = d.s2;
+        rec.codes = d.codes;
+        rec.scales = d.scales;
+        rec.xq = d.Wq;
+        rec.r = r;
+        rec.nb = d.in / 16;
+        rec.groups = (d.in / 16 + 3) / 4;
+        if (d.in > a.max_in) {
+            if (r == 0) atomicOr(&g_error_flags, 2u);
+        } else if (r >= d.out) {
+            rec.mode = ROW_PAD;
+        } else if (d.in > 0) {
+            rec.mode = ROW_DATA;
+            const uint32_t bytes = (uint32_t)(d.in * 2);
+            mbar_arrive_expect_tx(b, bytes);
+            bulk_g2s(smem_u32(dst), d.W + r * d.in, bytes, b);
+            return;
+        }
+    }
+    mbar_arrive(b);
+}
+
+template <bool SWZ, bool RTN>
+__global__ void __launch_bounds__(RS_THREADS) rows_staged_kernel(const RowArgs a, uint32_t stage_bytes) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full[2];
+    __shared__ RowStage info[2];
+    __shared__ uint32_t red[2][RS_THREADS / 32];
+    __shared__ uint32_t amax_s[RS_BPT * RS_THREADS];   // block maxima; each thread keeps only its own
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        mbar_init(smem_u32(&full[0]), 1);
+        mbar_init(smem_u32(&full[1]), 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    int tn = 0;                 // thread 0's cursor over the table
+    if (tid == 0 && (int64_t)blockIdx.x < a.total_rows)
+        stage_row<SWZ>(a, blockIdx.x, tn, smem, &full[0], info[0]);
+    bool stopped = false;
+    uint32_t i = 0, st = 0, ph = 0;
+    for (int64_t R = blockIdx.x; R < a.total_rows; R += gridDim.x, ++i) {
+        st = i & 1u;
+        ph = (i >> 1) & 1u;
+        const unsigned char *row = smem + st * stage_bytes;
+        // pass 1: the block maxima of this thread's blocks and their maximum
+        const bool ok = mbar_wait(smem_u32(&full[st]), ph);
+        const RowStage &rec = info[st];
+        const uint32_t mode = ok ? rec.mode : ROW_SKIP;
+        const int64_t nb = rec.nb;
+        uint32_t mx = 0u;
+        if (mode == ROW_DATA) {
+#pragma unroll 2
+            for (int j = 0; j < RS_BPT; ++j) {
+                const int64_t b = tid + (int64_t)j * RS_THREADS;
+                if (b < nb) {
+                    const uint4 *p = reinterpret_cast<const uint4 *>(row) + 2 * b;
+                    const uint4 v0 = p[0], v1 = p[1];
+                    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                    const uint32_t ab = block_amax_bits(w);
+                    amax_s[j * RS_THREADS + tid] = ab;
+                    mx = max(mx, ab);
+                }
+            }
+        }
+        mx = __reduce_max_sync(FULL, mx);
+        if (lane == 0) red[st][warp] = mx;
+        if (__syncthreads_or(!ok)) {           // a wait ran out: every thread stops here
+            if (tid == 0) atomicOr(&g_error_flags, 8u);
+            stopped = true;
+            break;
+        }
+        // every thread is done with the other buffer and its record (the previous
+        // row): stage the next row there
+        if (tid == 0 && R + gridDim.x < a.total_rows)
+            stage_row<SWZ>(a, R + gridDim.x, tn, smem + (st ^ 1u) * stage_bytes, &full[st ^ 1u], info[st ^ 1u]);
+        if (mode == ROW_SKIP) continue;
+        const int64_t r = rec.r;
+        if (mode == ROW_PAD) {                  // a padding row of the 128x4 layout: its words are 0
+            if (SWZ)
+                for (int64_t g = tid; g < rec.groups; g += RS_THREADS)
+                    *reinterpret_cast<uint32_t *>(rec.scales + swizzled_offset(r, 4 * g, rec.groups)) = 0u;
+            continue;
+        }
+        uint32_t amax = 0u;
+#pragma unroll
+        for (int w = 0; w < RS_THREADS / 32; ++w) amax = max(amax, red[st][w]);
+        if (amax >= 0x7f80u) {                  // a non-finite value: flag it, write nothing of the row
+            if (tid == 0) atomicOr(&g_error_flags, 1u);
+            continue;
+        }
+        const float s = __fdiv_rn(__uint_as_float(amax << 16), 2688.0f);
+        if (tid == 0) rec.ts[r] = s;
+        const F46Scale sc = f46_scale(s);
+        // pass 2: quantize every block of this thread
+#pragma unroll 1
+        for (int j = 0; j < RS_BPT; ++j) {
+            const int64_t b = tid + (int64_t)j * RS_THREADS;
+            if (b < nb) {
+                const int64_t blk = r * nb + b;
+                uint32_t sb = 0x38u, cw[2] = {0u, 0u};
+                uint4 o[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
+                uint16_t *xq = rec.xq;
+                if (s != 0.0f) {
+                    const uint4 *p = reinterpret_cast<const uint4 *>(row) + 2 * b;
+                    const uint4 v0 = p[0], v1 = p[1];
+                    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                    const float Ab = __uint_as_float(amax_s[j * RS_THREADS + tid] << 16);
+                    if (RTN) rtn_block(w, Ab, sc, sb, cw);
+                    else f46_block(w, Ab, sc, sb, cw);
+                    if (xq) wq_words(cw, sb, s, o);
+                }
+                reinterpret_cast<uint2 *>(rec.codes)[blk] = make_uint2(cw[0], cw[1]);
+                rec.scales[SWZ ? swizzled_offset(r, b, rec.groups) : blk] = (uint8_t)sb;
+                if (xq) {
+                    __stcs(reinterpret_cast<uint4 *>(xq) + 2 * blk, o[0]);
+                    __stcs(reinterpret_cast<uint4 *>(xq) + 2 * blk + 1, o[1]);
+                }
+            }
+        }
+        if (SWZ)                                // the row's padding columns (at most 3)
+            for (int64_t c = nb + tid; c < 4 * rec.groups; c += RS_THREADS)
+                rec.scales[swizzled_offset(r, c, rec.groups)] = 0u;
+    }
+    // After a wait ran out, the copy into the current buffer may still be in
+    // flight: it must land before the CTA's shared memory is released.
+    if (stopped && tid == 0)
+        if (!mbar_wait(smem_u32(&full[st]), ph)) atomicOr(&g_error_flags, 8u);
+}
+
+}  // namespace focus

@@ -30,6 +30,8 @@ FOCUS_STEP_WRITE_GRAD = 2
 FOCUS_STEP_PACK_UPDATED = 4
 FOCUS_STEP_WQ_UPDATED = 8
 FOCUS_PURPOSE_MX = 4
+FOCUS_PURPOSE_ACT = 5
+FOCUS_PURPOSE_ACT_SWIZZLED = 6
 FOCUS_HOST_S2_FIRST = 16
 
 
@@ -75,6 +77,8 @@ _SIGS = {
     "focus_fouroversix_act_swizzled": ([_P, _I64, _I64, _P, _P, _P, _SZ, _P, _P], _I),
     "focus_nvfp4_act": ([_P, _I64, _I64, _P, _P, _P, _P, _P], _I),
     "focus_nvfp4_act_swizzled": ([_P, _I64, _I64, _P, _P, _P, _SZ, _P, _P], _I),
+    "focus_fouroversix_act_multi": ([_P, _I, _I64, _I64, _I, _P], _I),
+    "focus_nvfp4_act_multi": ([_P, _I, _I64, _I64, _I, _P], _I),
     "focus_mx_fwd": ([_P, _P, _P, _I64, _I64, _P, _P, _P, _P], _I),
     "focus_mx_ste_bwd": ([_P, _P, _P, _P, _I64, _I64, _P, _P, _I, _P], _I),
     "focus_mx_step": ([_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, ctypes.POINTER(focus_hparams), _I64,
@@ -265,6 +269,20 @@ def focus_fouroversix_weight(W, s2: float, codes, scales, Wq=None, stream=None, 
     o, i = _shape(W, out, in_)
     _check(_lib.focus_fouroversix_weight(_ptr(W), o, i, float(s2), _ptr(codes), _ptr(scales), _ptr(Wq),
                                          _stream(stream)), "focus_fouroversix_weight")
+
+
+def focus_fouroversix_act_multi(table_dev, n: int, total_rows: int, max_hidden: int, swizzled: bool = False,
+                                stream=None):
+    """FourOverSix with one scale per token over a table of activation tensors
+    (prepared with FOCUS_PURPOSE_ACT, or FOCUS_PURPOSE_ACT_SWIZZLED and swizzled)."""
+    _check(_lib.focus_fouroversix_act_multi(_ptr(table_dev), int(n), int(total_rows), int(max_hidden),
+                                            1 if swizzled else 0, _stream(stream)), "focus_fouroversix_act_multi")
+
+
+def focus_nvfp4_act_multi(table_dev, n: int, total_rows: int, max_hidden: int, swizzled: bool = False, stream=None):
+    """NVFP4 round to nearest with one scale per token over a table of activation tensors."""
+    _check(_lib.focus_nvfp4_act_multi(_ptr(table_dev), int(n), int(total_rows), int(max_hidden),
+                                      1 if swizzled else 0, _stream(stream)), "focus_nvfp4_act_multi")
 
 
 def focus_fouroversix_multi(table_dev, n: int, total_tiles: int, stream=None):

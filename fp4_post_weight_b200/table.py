@@ -21,6 +21,8 @@ PURPOSE_STEP = 1
 PURPOSE_BACKWARD = 2
 PURPOSE_FOUROVERSIX = 3
 PURPOSE_MX = 4                                # the MXFP4 calls (focus_mx_*_multi): in % 32 == 0, no s2
+PURPOSE_ACT = 5                               # activations for the per-token calls, scales row-major
+PURPOSE_ACT_SWIZZLED = 6                      # the same, scales in the 128x4-atom layout
 
 
 @dataclass
@@ -137,3 +139,28 @@ class HostTable:
 
     def step(self, step: int, hp: F.focus_hparams | None = None, flags: int = 0, stream=None):
         F.focus_step_host(self.descs, self.n, hp or hparams(), step, flags, self.ws, stream)
+
+
+def act_entry(X: torch.Tensor, token_scales: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+              Xq: torch.Tensor | None = None) -> Entry:
+    """An activation tensor X [tokens, hidden] bf16 for an ActTable: token_scales [tokens]
+    f32, codes [tokens, hidden/2] u8, scales (row-major [tokens, hidden/16] u8, or the
+    128x4-atom buffer), Xq bf16 (optional)."""
+    return Entry(W=X, m=None, q=None, s2=token_scales, codes=codes, scales=scales, Wq=Xq)
+
+
+class ActTable(FocusTable):
+    """Activation tensors (act_entry) quantized per token in one launch: FourOverSix or
+    plain NVFP4, the block scales row-major or (swizzled) in the 128x4-atom layout."""
+
+    def __init__(self, entries: list[Entry], swizzled: bool = False):
+        self.swizzled = bool(swizzled)
+        super().__init__(entries, PURPOSE_ACT_SWIZZLED if swizzled else PURPOSE_ACT)
+        self.total_rows = self.total_tiles
+        self.max_hidden = max([int(e.W.shape[1]) for e in self.entries] + [16])
+
+    def fouroversix(self, stream=None):
+        F.focus_fouroversix_act_multi(self.dev, self.n, self.total_rows, self.max_hidden, self.swizzled, stream)
+
+    def nvfp4(self, stream=None):
+        F.focus_nvfp4_act_multi(self.dev, self.n, self.total_rows, self.max_hidden, self.swizzled, stream)

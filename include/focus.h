@@ -226,6 +226,11 @@ typedef struct focus_hparams {
 
 /* focus_table_prepare purpose of a table for the MXFP4 multi-tensor calls. */
 #define FOCUS_PURPOSE_MX 4
+/* focus_table_prepare purposes of a table of activation tensors for the
+ * per-token calls focus_fouroversix_act_multi / focus_nvfp4_act_multi: block
+ * scales row-major (5) or in the 128x4-atom layout (6). */
+#define FOCUS_PURPOSE_ACT 5
+#define FOCUS_PURPOSE_ACT_SWIZZLED 6
 
 /* Flags of focus_step_fused. */
 #define FOCUS_STEP_ACCUMULATE 1u  /* add dm/dq (earlier micro-batches) to this step's gradients */
@@ -243,11 +248,18 @@ typedef struct focus_hparams {
  * FourOverSix only (W and s2; m and q may be NULL; codes+scales or Wq),
  * FOCUS_PURPOSE_MX (4) = the MXFP4 calls focus_mx_*_multi (in % 32 == 0; W,
  * m and q present; s2 unused; the other pointers optional here and checked by
- * the kernels: an entry lacking one its call needs is skipped and flagged))
+ * the kernels: an entry lacking one its call needs is skipped and flagged),
+ * FOCUS_PURPOSE_ACT (5) and FOCUS_PURPOSE_ACT_SWIZZLED (6) = the per-token
+ * calls focus_*_act_multi (W = X [tokens = out, hidden = in] with hidden at
+ * most 16384, s2 = the token scales [tokens], codes and scales present, Wq =
+ * X' optional))
  * and fills block_begin and tile_begin (for purpose 4 in 32-blocks and tiles
- * of 128 of them: 4096 weights, as for the other purposes).  Host memory in,
- * host memory out.
- * *total_tiles receives the number of work tiles, passed to the calls below.
+ * of 128 of them: 4096 weights, as for the other purposes; for purposes 5 and
+ * 6 tile_begin is the entry's first row, and the rows of every entry count
+ * padded to a multiple of 128 for purpose 6).  Host memory in, host memory
+ * out.
+ * *total_tiles receives the number of work tiles (for purposes 5 and 6: of
+ * rows), passed to the calls below.
  * A device-resident table cannot be checked again at call time: a kernel that
  * meets an entry lacking a pointer it needs skips that entry and sets the
  * device flag (FOCUS_ERR_NONFINITE_INPUT from focus_get_error). */
@@ -368,6 +380,20 @@ int focus_fouroversix_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hi
                                    uint8_t *codes, uint8_t *scales_swz, size_t scales_bytes, uint16_t *Xq,
                                    focus_stream_t stream);
 
+/* The same over every entry of a table of activation tensors prepared with
+ * FOCUS_PURPOSE_ACT (block scales row-major; swizzled = 0) or
+ * FOCUS_PURPOSE_ACT_SWIZZLED (the 128x4-atom layout, each entry's scales
+ * buffer at least focus_scales_swizzled_bytes(tokens, hidden/16) bytes;
+ * swizzled = 1), in one launch: total_rows as focus_table_prepare returned it,
+ * max_hidden at least every entry's hidden (a multiple of 16, at most 16384,
+ * else FOCUS_ERR_SHAPE; an entry wider than max_hidden is skipped and sets
+ * the device flag).  Every entry as the single-tensor call: desc.W = X,
+ * desc.s2 = token scales (written), desc.codes, desc.scales, desc.Wq = X'
+ * (nullable).  Rows of up to 16384 values are staged in shared memory, so X
+ * is read from HBM once. */
+int focus_fouroversix_act_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_rows,
+                                int64_t max_hidden, int swizzled, focus_stream_t stream);
+
 /* Plain NVFP4 round to nearest with one scale per token: the NVFP4 baseline
  * of the card's section "Perplexity" (NVFP4 activations with one scale per
  * token), read as the block equations with m = 1 and sigmoid = 1 and the
@@ -380,6 +406,9 @@ int focus_nvfp4_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *to
                     uint8_t *scales, uint16_t *Xq, focus_stream_t stream);
 int focus_nvfp4_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales, uint8_t *codes,
                              uint8_t *scales_swz, size_t scales_bytes, uint16_t *Xq, focus_stream_t stream);
+/* ... and over a table, as focus_fouroversix_act_multi. */
+int focus_nvfp4_act_multi(const focus_tensor_desc *descs_dev, int n_tensors, int64_t total_rows, int64_t max_hidden,
+                          int swizzled, focus_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * MXFP4 variant: 32-element blocks with an E8M0 scale and four sub-blocks of

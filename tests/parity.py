@@ -117,6 +117,21 @@ def f46_counts(ref) -> dict:
             "band_2^-47": int((gap <= F46_BAND * tot).sum())}
 
 
+def f46_tie_counts(ref, X_bits: np.ndarray, s) -> dict:
+    """Of the blocks whose two exact errors tie (nonzero), how many have identical
+    candidates (equal scale bytes S6 == S4: the block of the row's or tensor's maximum,
+    where both scales clamp at 448) -- recomputed here from X and the scale(s)."""
+    e6, e4 = ref.errs[..., 0], ref.errs[..., 1]
+    tie = (e6 == e4) & (e6 + e4 > 0)
+    rows, nb = ref.scales.shape
+    A = ((X_bits.astype(np.uint32) & 0x7FFF) << 16).view(np.float32).reshape(rows, nb, 16).max(-1)
+    s = np.broadcast_to(np.asarray(s, np.float32).reshape(-1, 1), (rows, nb))
+    x6 = (A / (np.float32(6) * s)).astype(np.float32)
+    x4 = (A / (np.float32(4) * s)).astype(np.float32)
+    same = (x6 >= np.float32(432)) & (x4 >= np.float32(432))    # both E4M3 bytes round to 448
+    return {"ties_same_candidate": int((tie & same).sum()), "ties_different_candidates": int((tie & ~same).sum())}
+
+
 def check_fouroversix(ref, codes: np.ndarray, scales: np.ndarray, Xq: np.ndarray | None) -> dict:
     """ref: oracle.FourOverSix; codes unpacked uint8 [rows, cols]; scales uint8 [rows, cols/16];
     Xq uint16 bits or None.  Asserts the bar above and returns the counts with the mismatches."""

@@ -99,7 +99,7 @@ def test_table_prepare_on_host(F):
         F.focus_table_prepare(descs, 1)
     assert e.value.status == 1
     assert F.focus_table_prepare(descs, 0) == tiles
-    # a table backward needs dW', dm and dq; purposes beyond 3 do not exist
+    # a table backward needs dW', dm and dq; purposes beyond 6 do not exist
     with pytest.raises(F.FocusError) as e:
         F.focus_table_prepare(descs, 2)
     assert e.value.status == 1
@@ -108,7 +108,7 @@ def test_table_prepare_on_host(F):
         descs[i].dq = P + 65536 * (i + 1) + 4096
     assert F.focus_table_prepare(descs, 2) == tiles
     with pytest.raises(F.FocusError) as e:
-        F.focus_table_prepare(descs, 5)
+        F.focus_table_prepare(descs, 7)
     assert e.value.status == 4
     with pytest.raises(F.FocusError) as e:      # MXFP4: in must be a multiple of 32
         F.focus_table_prepare(descs, F.FOCUS_PURPOSE_MX)
@@ -372,3 +372,36 @@ def test_step_amax_checks(F):
     assert F.raw_call("focus_s2_from_amax", P, 1, None, None) == 1
     assert F.raw_call("focus_s2_from_amax", U, 1, P, None) == 3
     assert F.raw_call("focus_s2_from_amax", P, 0, P, None) == 0
+
+
+def test_activation_table_prepare_on_host():
+    """Purposes 5 and 6 (activation tables for the per-token calls): tile_begin is
+    each entry's first row (rows padded to 128 for the 128x4 layout), the total is
+    the row count, an empty entry adds no rows, rows above 16384 values and entries
+    without codes, scales or token scales are refused."""
+    from fp4_post_weight_b200 import focus as F
+    P = 1 << 20
+    shapes = [(33, 4096), (0, 64), (130, 1040), (5, 16384)]
+    descs = (F.focus_tensor_desc * len(shapes))()
+    for i, (t, h) in enumerate(shapes):
+        d = descs[i]
+        d.W, d.s2, d.codes, d.scales = P + (i << 24), P + (i << 24) + 4096, P + (i << 24) + 8192, P + (i << 24) + 16384
+        d.out, d.in_ = t, h
+    assert F.focus_table_prepare(descs, F.FOCUS_PURPOSE_ACT) == 33 + 130 + 5
+    assert [descs[i].tile_begin for i in range(4)] == [0, 33, 33, 163]
+    assert F.focus_table_prepare(descs, F.FOCUS_PURPOSE_ACT_SWIZZLED) == 128 + 256 + 128
+    assert [descs[i].tile_begin for i in range(4)] == [0, 128, 128, 384]
+    descs[2].codes = None
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, F.FOCUS_PURPOSE_ACT)
+    assert e.value.status == 1
+    descs[2].codes = P + (2 << 24) + 8192
+    descs[3].in_ = 16400
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, F.FOCUS_PURPOSE_ACT)
+    assert e.value.status == 2
+    descs[3].in_ = 16384
+    descs[0].s2 = P + 2                                # token scales not 16-byte aligned
+    with pytest.raises(F.FocusError) as e:
+        F.focus_table_prepare(descs, F.FOCUS_PURPOSE_ACT)
+    assert e.value.status == 3

@@ -5,8 +5,8 @@
   for bit (signed zeros included),
   for every bf16 significand of w (both signs, and +-0) and every binary32
   significand of D, at several exponent pairs inside the range the kernels
-  use it for; where the quotient falls below the normal range (tiny w, large
-  D) it is within one unit of 2^-149 with the same sign and E2M1 code.
+  use it for; where the quotient is below 2^-100 (tiny w, large D) it is
+  within one unit in the last place with the same sign and E2M1 code.
 * fl(c*S) through the mixed-precision FMA equals the binary32 product for
   every E2M1 value and every normal E4M3 scale, and c - y likewise.
 * The E2M1 conversion keeps the sign of negative values that round to zero
@@ -76,10 +76,11 @@ def test_division_exhaustive(lib, we, de, variant):
                                    (-133, 59), (-120, -3)])
 def test_division_tiny_quotients(lib, we, de, variant):
     """Tiny w over a large D (the kernels take the fast quotient whenever D lies in
-    [2^-60, 2^60], whatever |w|): where the IEEE quotient is normal the bits agree;
-    below the normal range the result may be one unit of 2^-149 off, with the same
-    sign, so its E2M1 code is the same signed zero and its share of a gradient sum
-    is below 2^-149 |g|."""
+    [2^-60, 2^60], whatever |w|): for quotients of at least 2^-100 the bits agree;
+    below that the remainder of the correction need not be representable and the
+    result may be one unit in the last place off, with the same sign, so its E2M1
+    code is the same signed zero and its share of a gradient sum is below
+    2^-123 |g|."""
     n = ctypes.c_ulonglong(0)
     ex = (ctypes.c_float * 4)()
     assert lib.check_div(we, de, ctypes.byref(n), ex, variant | 4) == 0

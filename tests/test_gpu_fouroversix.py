@@ -185,6 +185,85 @@ def test_nvfp4_activations(F, tokens, hidden):
         assert host(scales)[0, 1] == 0x08               # x below 2^-6: clamped to the smallest normal scale
 
 
+@pytest.mark.parametrize("swizzled", [False, True], ids=["row-major", "128x4"])
+@pytest.mark.parametrize("rtn", [False, True], ids=["fouroversix", "nvfp4"])
+def test_activation_table_one_launch(F, rtn, swizzled):
+    """Activation tensors of mixed widths in one launch (focus_*_act_multi): a zero
+    row, rows of one block, ragged widths, an empty tensor, a token count not a
+    multiple of 128 (padding rows of the 128x4 layout), and the widest staged row;
+    every tensor against the oracle (row scales, scale bytes, codes, X')."""
+    from fp4_post_weight_b200.table import ActTable, act_entry
+    shapes = [(33, 4096), (5, 48), (0, 64), (130, 1040), (17, 14336), (3, 16), (7, 16384)]
+    ents, Xs = [], []
+    for j, (t, h) in enumerate(shapes):
+        X = synth.activations(t, h, "cuda", seed=90 + j, zero_tokens=1 if t > 2 else 0) if t else \
+            torch.zeros((0, h), dtype=torch.bfloat16, device="cuda")
+        nsc = F.focus_scales_swizzled_bytes(t, h // 16) if swizzled else t * (h // 16)
+        ents.append(act_entry(X, torch.full((max(t, 1),), -1.0, device="cuda"),
+                              torch.empty((max(t, 1), h // 2), dtype=torch.uint8, device="cuda"),
+                              torch.full((max(nsc, 16),), 0xAB, dtype=torch.uint8, device="cuda"),
+                              torch.empty_like(X) if t else None))
+        Xs.append(X)
+    tab = ActTable(ents, swizzled=swizzled)
+    assert tab.total_rows == sum(((t + 127) // 128 * 128 if swizzled else t) for t, h in shapes if t)
+    tab.nvfp4() if rtn else tab.fouroversix()
+    assert F.focus_get_error() == 0
+    for (t, h), X, e in zip(shapes, Xs, ents):
+        if t == 0:
+            continue
+        ref = oracle.nvfp4_rows(host_bits(X)) if rtn else oracle.fouroversix(host_bits(X))
+        np.testing.assert_array_equal(host(e.s2)[:t], ref.row_scales)
+        codes = unpack_codes(host(e.codes))
+        if swizzled:
+            nsc = F.focus_scales_swizzled_bytes(t, h // 16)
+            np.testing.assert_array_equal(host(e.scales)[:nsc], oracle.scales_swizzle(ref.scales))
+            lin = None
+        else:
+            lin = host(e.scales)[:t * (h // 16)].reshape(t, h // 16)
+        if rtn:
+            np.testing.assert_array_equal(codes, ref.codes)
+            np.testing.assert_array_equal(host_bits(e.Wq), ref.Xq)
+            if lin is not None:
+                np.testing.assert_array_equal(lin, ref.scales)
+        else:
+            sc = lin if lin is not None else ref.scales      # the 128x4 bytes were checked above
+            c = check_fouroversix(ref, codes, sc, host_bits(e.Wq))
+            assert c["mismatched_blocks"] == 0, c
+
+
+def test_activation_table_rejects_and_flags(F):
+    """A row holding infinity in a table sets the device flag and leaves that row
+    unwritten while the other rows and tensors match the oracle; a table entry wider
+    than max_hidden is skipped and flagged; shapes above 16384 values per row are
+    refused by the table preparation."""
+    from fp4_post_weight_b200.table import ActTable, act_entry
+    Xa = synth.activations(9, 1024, "cuda", seed=5, zero_tokens=0)
+    Xb = synth.activations(4, 2048, "cuda", seed=6, zero_tokens=0)
+    Xa[4, 100] = float("inf")
+    mk = lambda X: act_entry(X, torch.zeros(X.shape[0], device="cuda"),
+                             torch.zeros((X.shape[0], X.shape[1] // 2), dtype=torch.uint8, device="cuda"),
+                             torch.zeros((X.shape[0], X.shape[1] // 16), dtype=torch.uint8, device="cuda"))
+    ents = [mk(Xa), mk(Xb)]
+    tab = ActTable(ents)
+    assert F.focus_get_error() == 0
+    tab.fouroversix()
+    assert F.focus_get_error() == 7
+    good = [r for r in range(9) if r != 4]
+    ref = oracle.fouroversix(host_bits(Xa)[good])
+    np.testing.assert_array_equal(host(ents[0].scales)[good], ref.scales)
+    assert not host(ents[0].scales)[4].any() and not host(ents[0].codes)[4].any()
+    refb = oracle.fouroversix(host_bits(Xb))
+    np.testing.assert_array_equal(host(ents[1].scales), refb.scales)
+    # max_hidden below an entry's width: that entry is skipped and reported
+    tab2 = ActTable([mk(Xb)])
+    F.focus_fouroversix_act_multi(tab2.dev, 1, tab2.total_rows, 1024)
+    assert F.focus_get_error() == 7
+    with pytest.raises(F.FocusError):
+        ActTable([mk(torch.zeros((2, 16400), dtype=torch.bfloat16, device="cuda"))])
+    with pytest.raises(F.FocusError):
+        F.focus_fouroversix_act_multi(tab.dev, 2, tab.total_rows, 16400)
+
+
 def test_nvfp4_activations_swizzled_and_nonfinite(F):
     from tests.parity import unpack_codes as _unpack
     tokens, hidden = 130, 1040

@@ -5,12 +5,12 @@ configurations bench.py times:
   launch (codes, scales and W'), layer 0 in full and a 1/64 row sample of
   every other tensor, bit for bit against the oracle with each tensor's s2;
 * FourOverSix with one scale per token over one decoder layer's linear inputs
-  for a micro-batch of 4096 tokens (four launches), in full;
+  for a micro-batch of 4096 tokens (one launch over the four tensors), in full;
 * the calibration step over four micro-batches (bench order) on layer 0 of the
   8B shapes, a 1/16 row sample;
 * plain NVFP4 round to nearest: the weights over all 224 linears in one launch
   (layer 0 in full, a 1/64 row sample of the rest) and the same per-token
-  inputs, in full;
+  inputs in one launch, in full;
 * the MXFP4 fused step, one launch per tensor, on layer 0 of the 8B shapes
   with the benchmark's parameters (m = 1, q = 6, zero moments), a 1/16 row
   sample against the oracle, and the same step as one launch over a table of
@@ -24,7 +24,8 @@ import torch
 
 import oracle
 import synth
-from tests.parity import MAX_MISMATCH_FRAC, assert_close, check_fouroversix, host, host_bits, record, unpack_codes
+from tests.parity import (MAX_MISMATCH_FRAC, assert_close, check_fouroversix, f46_tie_counts, host, host_bits,
+                          record, unpack_codes)
 
 pytestmark = pytest.mark.gpu
 
@@ -63,25 +64,36 @@ def test_fouroversix_weights_llama_8b_one_launch(F):
         sel = (lambda x: x) if rows is None else (lambda x: x[rows])
         ref = oracle.fouroversix(host_bits(sel(e.W)), s2)
         c = check_fouroversix(ref, unpack_codes(host(sel(e.codes))), host(sel(e.scales)), host_bits(sel(e.Wq)))
+        c.update(f46_tie_counts(ref, host_bits(sel(e.W)), s2))
         for k, v in c.items():
             total[k] = total.get(k, 0) + v
     assert total["mismatched_blocks"] <= MAX_MISMATCH_FRAC * total["blocks"]
     record("FourOverSix weights, Llama-3.1-8B layer 0 full + 1/64 rows (blocks)", total)
 
 
-def test_fouroversix_activations_one_layer_4096_tokens(F):
+def _layer_inputs():
+    """One decoder layer's linear inputs for 4096 tokens (q/k/v, o, gate/up, down), as one
+    activation table (the benchmark's launch), with X' written."""
+    from fp4_post_weight_b200.table import ActTable, act_entry
+    ents = []
     for j, h in enumerate((4096, 4096, 4096, 14336)):
         X = synth.activations(4096, h, "cuda", seed=50 + j)
-        ts = torch.empty(4096, device="cuda")
-        codes = torch.empty((4096, h // 2), dtype=torch.uint8, device="cuda")
-        scales = torch.empty((4096, h // 16), dtype=torch.uint8, device="cuda")
-        Xq = torch.empty_like(X)
-        F.focus_fouroversix_act(X, ts, codes, scales, Xq)
-        assert F.focus_get_error() == 0
-        ref = oracle.fouroversix(host_bits(X))
-        np.testing.assert_array_equal(host(ts), ref.row_scales)
-        c = check_fouroversix(ref, unpack_codes(host(codes)), host(scales), host_bits(Xq))
+        ents.append(act_entry(X, torch.empty(4096, device="cuda"),
+                              torch.empty((4096, h // 2), dtype=torch.uint8, device="cuda"),
+                              torch.empty((4096, h // 16), dtype=torch.uint8, device="cuda"), torch.empty_like(X)))
+    return ents, ActTable(ents)
+
+
+def test_fouroversix_activations_one_layer_4096_tokens(F):
+    ents, tab = _layer_inputs()
+    tab.fouroversix()
+    assert F.focus_get_error() == 0
+    for e in ents:
+        ref = oracle.fouroversix(host_bits(e.W))
+        np.testing.assert_array_equal(host(e.s2), ref.row_scales)
+        c = check_fouroversix(ref, unpack_codes(host(e.codes)), host(e.scales), host_bits(e.Wq))
         assert c["mismatched_blocks"] <= MAX_MISMATCH_FRAC * c["blocks"], c
+        c.update(f46_tie_counts(ref, host_bits(e.W), ref.row_scales))
         record("FourOverSix per token, one 8B layer's inputs, 4096 tokens (blocks)", c)
 
 
@@ -174,17 +186,15 @@ def test_nvfp4_weights_llama_8b_one_launch(F):
 
 
 def test_nvfp4_activations_one_layer_4096_tokens(F):
-    for j, h in enumerate((4096, 4096, 4096, 14336)):
-        X = synth.activations(4096, h, "cuda", seed=50 + j)
-        ts = torch.empty(4096, device="cuda")
-        codes = torch.empty((4096, h // 2), dtype=torch.uint8, device="cuda")
-        scales = torch.empty((4096, h // 16), dtype=torch.uint8, device="cuda")
-        F.focus_nvfp4_act(X, ts, codes, scales)
-        assert F.focus_get_error() == 0
-        ref = oracle.nvfp4_rows(host_bits(X))
-        np.testing.assert_array_equal(host(ts), ref.row_scales)
-        np.testing.assert_array_equal(host(scales), ref.scales)
-        np.testing.assert_array_equal(unpack_codes(host(codes)), ref.codes)
+    ents, tab = _layer_inputs()
+    tab.nvfp4()
+    assert F.focus_get_error() == 0
+    for e in ents:
+        ref = oracle.nvfp4_rows(host_bits(e.W))
+        np.testing.assert_array_equal(host(e.s2), ref.row_scales)
+        np.testing.assert_array_equal(host(e.scales), ref.scales)
+        np.testing.assert_array_equal(unpack_codes(host(e.codes)), ref.codes)
+        np.testing.assert_array_equal(host_bits(e.Wq), ref.Xq)
 
 
 def test_micro_batch_step_llama_8b_layer0_sampled(F):
