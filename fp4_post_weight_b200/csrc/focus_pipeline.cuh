@@ -9,8 +9,9 @@
 //
 // Every wait is bounded: after WAIT_LIMIT_NS of wall time (read from
 // %globaltimer), or a hard iteration cap, it gives up and returns false; the
-// caller then records an error and leaves its loop, so a kernel never spins
-// forever.
+// caller then records an error and leaves its loop, so a kernel never waits
+// forever.  Between its tests a waiting thread is suspended by the hardware
+// (the try_wait suspend-time hint) rather than polling.
 #pragma once
 
 #include <cstdint>
@@ -54,21 +55,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test, but a thread whose phase is not yet complete is suspended by
+// the hardware until it completes or about HINT_NS nanoseconds have passed:
+// a waiting warp then takes no issue slots from the warps that compute.
+template <uint32_t HINT_NS>
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "n"(HINT_NS)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
 
-// Waits until the phase of parity `parity` of the barrier has completed.
-// Returns false if that does not happen within `limit_ns` of wall time (or
-// WAIT_MAX_ITERS polls).
+// Waits until the phase of parity `parity` of the barrier has completed,
+// suspended (not polling) between tests.  Returns false if that does not
+// happen within `limit_ns` of wall time (or WAIT_MAX_ITERS tests).
+constexpr uint32_t WAIT_SLEEP_NS = 1000;
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns = WAIT_LIMIT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t i = 1; i < WAIT_MAX_ITERS; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0 && global_ns() - t0 > limit_ns) return false;
+        if (mbar_try_wait_sleep<WAIT_SLEEP_NS>(bar, parity)) return true;
+        if ((i & 15u) == 0 && global_ns() - t0 > limit_ns) return false;
     }
     return false;
 }
