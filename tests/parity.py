@@ -126,9 +126,10 @@ def f46_tie_counts(ref, X_bits: np.ndarray, s) -> dict:
     rows, nb = ref.scales.shape
     A = ((X_bits.astype(np.uint32) & 0x7FFF) << 16).view(np.float32).reshape(rows, nb, 16).max(-1)
     s = np.broadcast_to(np.asarray(s, np.float32).reshape(-1, 1), (rows, nb))
-    x6 = (A / (np.float32(6) * s)).astype(np.float32)
-    x4 = (A / (np.float32(4) * s)).astype(np.float32)
-    same = (x6 >= np.float32(432)) & (x4 >= np.float32(432))    # both E4M3 bytes round to 448
+    with np.errstate(divide="ignore", invalid="ignore"):      # a zero row (s = 0) has no tie
+        x6 = (A / (np.float32(6) * s)).astype(np.float32)
+        x4 = (A / (np.float32(4) * s)).astype(np.float32)
+    same = (s > 0) & (x6 >= np.float32(432)) & (x4 >= np.float32(432))    # both E4M3 bytes round to 448
     return {"ties_same_candidate": int((tie & same).sum()), "ties_different_candidates": int((tie & ~same).sum())}
 
 
