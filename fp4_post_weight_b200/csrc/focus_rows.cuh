@@ -41,6 +41,7 @@ namespace focus {
 constexpr int RS_THREADS = 256;                           // 8 warps per CTA
 constexpr int RS_BPT = 4;                                 // blocks per thread at most
 constexpr int64_t RS_MAX_HIDDEN = 16 * RS_THREADS * RS_BPT;   // 16384 values per row
+constexpr float RCP_2688 = 1.0f / 2688.0f;                    // correctly rounded (evaluated at compile time)
 
 // The activation tensors of one launch.  Each entry uses focus_tensor_desc
 // fields as: W = X [out = tokens, in = hidden] bf16, s2 = token scales
@@ -146,9 +147,9 @@ __global__ void __launch_bounds__(RS_THREADS) rows_staged_kernel(const RowArgs a
         if (mode == ROW_DATA) {
 #pragma unroll 2
             for (int j = 0; j < RS_BPT; ++j) {
-                const int64_t b = tid + (int64_t)j * RS_THREADS;
-                if (b < nb) {
-                    const uint4 *p = reinterpret_cast<const uint4 *>(row) + 2 * b;
+                const uint32_t b = (uint32_t)tid + (uint32_t)j * RS_THREADS;
+                if (b < (uint32_t)nb) {
+                    const uint4 *p = reinterpret_cast<const uint4 *>(row) + 2u * b;
                     const uint4 v0 = p[0], v1 = p[1];
                     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                     const uint32_t ab = block_amax_bits(w);
@@ -183,32 +184,49 @@ __global__ void __launch_bounds__(RS_THREADS) rows_staged_kernel(const RowArgs a
             if (tid == 0) atomicOr(&g_error_flags, 1u);
             continue;
         }
-        const float s = __fdiv_rn(__uint_as_float(amax << 16), 2688.0f);
+        const float A_row = __uint_as_float(amax << 16);
+        // s = fl(A_row / 2688): the twice-corrected quotient by the correctly rounded
+        // 1/2688 (bit-identical to the IEEE division while nothing underflows)
+        const float s = A_row >= 0x1p-100f ? div_full(A_row, 2688.0f, RCP_2688) : __fdiv_rn(A_row, 2688.0f);
         if (tid == 0) rec.ts[r] = s;
-        const F46Scale sc = f46_scale(s);
-        // pass 2: quantize every block of this thread
-#pragma unroll 1
-        for (int j = 0; j < RS_BPT; ++j) {
-            const int64_t b = tid + (int64_t)j * RS_THREADS;
-            if (b < nb) {
-                const int64_t blk = r * nb + b;
-                uint32_t sb = 0x38u, cw[2] = {0u, 0u};
-                uint4 o[2] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u)};
-                uint16_t *xq = rec.xq;
-                if (s != 0.0f) {
-                    const uint4 *p = reinterpret_cast<const uint4 *>(row) + 2 * b;
-                    const uint4 v0 = p[0], v1 = p[1];
-                    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                    const float Ab = __uint_as_float(amax_s[j * RS_THREADS + tid] << 16);
-                    if (RTN) rtn_block(w, Ab, sc, sb, cw);
-                    else f46_block(w, Ab, sc, sb, cw);
-                    if (xq) wq_words(cw, sb, s, o);
-                }
-                reinterpret_cast<uint2 *>(rec.codes)[blk] = make_uint2(cw[0], cw[1]);
-                rec.scales[SWZ ? swizzled_offset(r, b, rec.groups) : blk] = (uint8_t)sb;
+        // pass 2: this thread's blocks (b = tid + j*RS_THREADS, j < jn; a tensor holds
+        // fewer than 2^31 blocks, so block indices fit 32 bits)
+        const uint32_t nbu = (uint32_t)nb;
+        const uint32_t jn = (uint32_t)tid < nbu ? (nbu - 1u - (uint32_t)tid) / RS_THREADS + 1u : 0u;
+        const uint32_t base = (uint32_t)r * nbu;
+        uint2 *const codes = reinterpret_cast<uint2 *>(rec.codes);
+        uint8_t *const scales = rec.scales;
+        uint4 *const xq = reinterpret_cast<uint4 *>(rec.xq);
+        const int64_t groups = rec.groups;
+        if (s == 0.0f) {                        // a row of zeros: scale bytes 0x38, codes 0, values 0
+            for (uint32_t j = 0; j < jn; ++j) {
+                const uint32_t b = (uint32_t)tid + j * RS_THREADS, blk = base + b;
+                codes[blk] = make_uint2(0u, 0u);
+                scales[SWZ ? swizzled_offset(r, b, groups) : (int64_t)blk] = 0x38u;
                 if (xq) {
-                    __stcs(reinterpret_cast<uint4 *>(xq) + 2 * blk, o[0]);
-                    __stcs(reinterpret_cast<uint4 *>(xq) + 2 * blk + 1, o[1]);
+                    __stcs(xq + 2ull * blk, make_uint4(0u, 0u, 0u, 0u));
+                    __stcs(xq + 2ull * blk + 1, make_uint4(0u, 0u, 0u, 0u));
+                }
+            }
+        } else {
+            const F46Scale sc = f46_scale(s);
+#pragma unroll 1
+            for (uint32_t j = 0; j < jn; ++j) {
+                const uint32_t b = (uint32_t)tid + j * RS_THREADS, blk = base + b;
+                const uint4 *p = reinterpret_cast<const uint4 *>(row) + 2u * b;
+                const uint4 v0 = p[0], v1 = p[1];
+                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                const float Ab = __uint_as_float(amax_s[j * RS_THREADS + tid] << 16);
+                uint32_t sb, cw[2];
+                if (RTN) rtn_block(w, Ab, sc, sb, cw);
+                else f46_block(w, Ab, sc, sb, cw);
+                codes[blk] = make_uint2(cw[0], cw[1]);
+                scales[SWZ ? swizzled_offset(r, b, groups) : (int64_t)blk] = (uint8_t)sb;
+                if (xq) {
+                    uint4 o[2];
+                    wq_words(cw, sb, s, o);
+                    __stcs(xq + 2ull * blk, o[0]);
+                    __stcs(xq + 2ull * blk + 1, o[1]);
                 }
             }
         }

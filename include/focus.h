@@ -364,7 +364,9 @@ int focus_nvfp4_weight_multi(const focus_tensor_desc *descs_dev, int n_tensors, 
  * [tokens][hidden/16] and Xq [tokens, hidden] bf16 (nullable) are device
  * outputs.  A row whose maximum is 0 gets s_t = 0, scale bytes 0x38, codes 0
  * and values 0.  A row holding a non-finite value sets the device flag and
- * its outputs are left unwritten.  One launch, X read once from HBM. */
+ * its outputs are left unwritten.  One launch; X is read from HBM once
+ * (rows of up to 16384 values are staged in shared memory, longer rows are
+ * read a second time from L2). */
 int focus_fouroversix_act(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_scales,
                           uint8_t *codes, uint8_t *scales, uint16_t *Xq, focus_stream_t stream);
 
