@@ -861,7 +861,7 @@ def run_reference(args, world, rank):
             "impl": "reference",
             "config": {"workload": WORKLOAD, "sample_weights_per_step": n // args.steps},
             "cpu_baseline": {"value": round(value, 5), "unit": "Gelem/s", "cores": threads, "kind": "oracle",
-                             "sample": desc},
+                             "cpu_model": _cpu_model(), "nproc": os.cpu_count(), "sample": desc},
             "e2e": {"value": round(value, 5), "unit": "Gelem/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
