@@ -445,7 +445,8 @@ int focus_table_prepare(focus_tensor_desc *d, int n, int purpose, int64_t *total
     int64_t tiles = 0, blocks = 0;
     if (purpose == FOCUS_PURPOSE_ACT || purpose == FOCUS_PURPOSE_ACT_SWIZZLED) {
         // activation tensors for the per-token calls: W = X, s2 = token scales;
-        // tile_begin is the entry's first row (rows padded to 128 for the 128x4 layout)
+        // tile_begin is the entry's first bundle of rows (rows padded to 128 for the
+        // 128x4 layout; rs_bundles gives an entry's bundles)
         int64_t rows = 0;
         for (int i = 0; i < n; ++i) {
             focus_tensor_desc &e = d[i];
@@ -461,7 +462,8 @@ int focus_table_prepare(focus_tensor_desc *d, int n, int purpose, int64_t *total
             e.block_begin = blocks;
             e.tile_begin = rows;
             blocks += e.out * (e.in / 16);
-            if (e.out * e.in > 0) rows += purpose == FOCUS_PURPOSE_ACT_SWIZZLED ? (e.out + 127) / 128 * 128 : e.out;
+            if (e.out * e.in > 0)
+                rows += rs_bundles(purpose == FOCUS_PURPOSE_ACT_SWIZZLED ? (e.out + 127) / 128 * 128 : e.out, e.in / 16);
         }
         *total_tiles = rows;
         return FOCUS_OK;
@@ -712,7 +714,8 @@ int launch_rows_staged_t(const RowArgs &a, cudaStream_t stream) {
     DeviceInfo *di;
     int rc = device_info(&di);
     if (rc) return rc;
-    const uint32_t stage = (uint32_t)((a.max_in * 2 + 127) / 128 * 128);
+    // one stage holds a bundle of rows: at most RS_BPT * RS_THREADS blocks (32 KB)
+    const uint32_t stage = (uint32_t)(RS_MAX_HIDDEN * 2);
     int occ = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rows_staged_kernel<SWZ, RTN>, RS_THREADS, 2 * stage) !=
             cudaSuccess || occ <= 0)
@@ -761,7 +764,7 @@ int act_rows(const uint16_t *X, int64_t tokens, int64_t hidden, float *token_sca
         RowArgs a{};
         a.table = nullptr;
         a.n_tensors = 1;
-        a.total_rows = swz ? (tokens + 127) / 128 * 128 : tokens;
+        a.total_rows = rs_bundles(swz ? (tokens + 127) / 128 * 128 : tokens, hidden / 16);
         a.max_in = hidden;
         a.one = one_desc(X, nullptr, Xq, nullptr, nullptr, tokens, hidden);
         a.one.s2 = token_scales;

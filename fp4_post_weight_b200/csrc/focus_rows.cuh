@@ -11,21 +11,23 @@
 //   squared error; NVFP4: the target 6);  a row of zeros has s_r = 0, scale
 //   bytes 0x38, codes 0 and values 0.
 //
-// Work decomposition.  A CTA takes rows R = blockIdx.x, blockIdx.x + grid,
-// ... of the table's rows (each entry's rows in order; with the 128x4 scale
-// layout an entry's rows are padded to a multiple of 128 and a padding row
-// only writes its scale words 0).  Thread 0 stages a row in shared memory with
-// one 1-D bulk copy (completion counted in bytes on an mbarrier) while the
-// CTA quantizes the previous one from the other buffer, so X is read from HBM
-// once and both passes over a row read shared memory: the first computes the
-// block maxima and their row maximum, the second
-// quantizes every block.  Thread t owns the blocks t, t + RS_THREADS, ...
-// (consecutive threads, consecutive 32-byte blocks) and keeps their maxima
-// in its own slots of a shared array between the passes.  Rows up to
-// RS_MAX_HIDDEN values; longer rows take f46_rows_kernel.
+// Work decomposition.  A CTA takes bundles U = blockIdx.x, blockIdx.x + grid,
+// ... of the table's rows: consecutive rows of one entry, as many as fit 256
+// threads with at most 4 blocks each (4 rows of 4096 values, 1 of 14336; with
+// the 128x4 scale layout an entry's rows are padded to a multiple of 128 and a
+// padding row only writes its scale words 0).  Thread 0 stages a bundle in
+// shared memory with one 1-D bulk copy (completion counted in bytes on an
+// mbarrier) while the CTA quantizes the previous one from the other buffer,
+// so X is read from HBM once and both passes over a row read shared memory:
+// the first computes the block maxima and each row's maximum (warp reduction,
+// one barrier per bundle), the second quantizes every block.  The threads of
+// a row own its blocks in turn (consecutive threads, consecutive 32-byte
+// blocks) and keep their maxima in their own slots of a shared array between
+// the passes.  Rows up to RS_MAX_HIDDEN values; longer rows take
+// f46_rows_kernel.
 //
 // Every wait is bounded (focus_pipeline.cuh); the decision to stop is made
-// uniformly through the row's barrier, and a CTA that stops waits (bounded)
+// uniformly through the bundle's barrier, and a CTA that stops waits (bounded)
 // for its last copy before it exits.
 #pragma once
 
@@ -47,69 +49,95 @@ constexpr float RCP_2688 = 1.0f / 2688.0f;                    // correctly round
 // fields as: W = X [out = tokens, in = hidden] bf16, s2 = token scales
 // [tokens] (written), codes [tokens][hidden/2], scales (row-major
 // [tokens][hidden/16], or the 128x4-atom buffer), Wq = X' (nullable),
-// tile_begin = the entry's first row in the launch's row numbering.
+// tile_begin = the entry's first bundle in the launch's numbering (below).
 struct RowArgs {
     const focus_tensor_desc *table;  // device table, or nullptr: use `one`
     int n_tensors;
-    int64_t total_rows;
+    int64_t total_rows;              // bundles of rows (rs_bundles) over all entries
     int64_t max_in;                  // the staging buffers hold rows of at most this many values
     focus_tensor_desc one;
 };
 
-// The record of a staged row, written by thread 0 before it completes the
+// Rows are taken in bundles of consecutive rows of one entry: a row of nb
+// blocks gets rs_tpr(nb) threads (a power of two from 32 to RS_THREADS, at
+// most RS_BPT blocks each), and a bundle holds RS_THREADS / rs_tpr(nb) rows,
+// at most RS_BPT * RS_THREADS blocks (32 KB of X).  A row of 4096 values is
+// one of a bundle of 4 (64 threads each); a row of 14336 is a bundle of its
+// own.  The entries' tile_begin count bundles.
+__host__ __device__ constexpr int64_t rs_tpr(int64_t nb) {
+    int64_t t = 32;
+    while (t < RS_THREADS && t * RS_BPT < nb) t *= 2;
+    return t;
+}
+__host__ __device__ constexpr int64_t rs_rows_per_bundle(int64_t nb) { return RS_THREADS / rs_tpr(nb); }
+__host__ __device__ constexpr int64_t rs_bundles(int64_t rows_out, int64_t nb) {
+    return (rows_out + rs_rows_per_bundle(nb) - 1) / rs_rows_per_bundle(nb);
+}
+
+// The record of a staged bundle, written by thread 0 before it completes the
 // stage's barrier phase and read by every thread after waiting on it.
 struct RowStage {
-    float *ts;          // token scales of the row's entry
+    float *ts;          // token scales of the bundle's entry
     uint8_t *codes;
     uint8_t *scales;
     uint16_t *xq;
-    int64_t r;          // row within its entry
+    int64_t r0;         // first row of the bundle within its entry
     int64_t nb;         // 16-blocks per row
     int64_t groups;     // column groups of 4 scales (128x4 layout)
-    uint32_t mode;      // ROW_SKIP, ROW_DATA or ROW_PAD
+    uint32_t rows;      // rows in the bundle (data rows, then padding rows of the 128x4 layout)
+    uint32_t data;      // data rows in the bundle (staged)
+    uint32_t tpr;       // threads per row
+    uint32_t skip;      // 1: nothing to do (an entry wider than the buffers, or past the table)
 };
-enum : uint32_t { ROW_SKIP = 0, ROW_DATA = 1, ROW_PAD = 2 };
 
-// Thread 0: fill the record of global row R and stage the row into `dst`
-// (one bulk copy of hidden*2 bytes, completion on `bar`); for a padding row,
-// a skipped or an empty one, complete the barrier's phase without data.  An
-// entry wider than the buffers is skipped and reported.
-// (The entry of R is found by scanning the table forward from entry t, which
-// the caller keeps: a CTA's rows only increase.  The descriptor is read again
-// for every row rather than held in registers across the loop.)
+// Thread 0: fill the record of bundle U and stage its data rows into `dst`
+// (one bulk copy, the rows being consecutive in X; completion on `bar`); for
+// a bundle without data rows, or a skipped one, complete the barrier's phase
+// without data.  An entry wider than the buffers is skipped and reported.
+// (The entry of U is found by scanning the table forward from entry t, which
+// the caller keeps: a CTA's bundles only increase.  The descriptor is read
+// again for every bundle rather than held in registers across the loop.)
 template <bool SWZ>
-__device__ __forceinline__ void stage_row(const RowArgs &a, int64_t R, int &t, unsigned char *dst, uint64_t *bar,
-                                          RowStage &rec) {
+__device__ __forceinline__ void stage_bundle(const RowArgs &a, int64_t U, int &t, unsigned char *dst, uint64_t *bar,
+                                             RowStage &rec) {
     const uint32_t b = smem_u32(bar);
     const int n = a.table ? a.n_tensors : 1;
     focus_tensor_desc d;
-    int64_t end;
+    int64_t rows_out = 0, end;
     for (;;) {
         d = a.table ? a.table[t] : a.one;
-        end = d.tile_begin + (SWZ ? (d.out + 127) / 128 * 128 : d.out);
-        if (R < end || t + 1 >= n) break;
+        rows_out = (d.out > 0 && d.in > 0) ? (SWZ ? (d.out + 127) / 128 * 128 : d.out) : 0;
+        end = d.tile_begin + rs_bundles(rows_out, d.in / 16);
+        if (U < end || t + 1 >= n) break;
         ++t;
     }
-    rec.mode = ROW_SKIP;
-    if (R < end) {
-        const int64_t r = R - d.tile_begin;
+    rec.skip = 1u;
+    if (U < end) {
+        const int64_t nb = d.in / 16;
+        const int64_t rpb = rs_rows_per_bundle(nb);
+        const int64_t r0 = (U - d.tile_begin) * rpb;
+        const int64_t rows = rows_out - r0 < rpb ? rows_out - r0 : rpb;
+        const int64_t data = d.out - r0 < 0 ? 0 : (d.out - r0 < rows ? d.out - r0 : rows);
         rec.ts = d.s2;
         rec.codes = d.codes;
         rec.scales = d.scales;
         rec.xq = d.Wq;
-        rec.r = r;
-        rec.nb = d.in / 16;
-        rec.groups = (d.in / 16 + 3) / 4;
+        rec.r0 = r0;
+        rec.nb = nb;
+        rec.groups = (nb + 3) / 4;
+        rec.rows = (uint32_t)rows;
+        rec.data = (uint32_t)data;
+        rec.tpr = (uint32_t)rs_tpr(nb);
         if (d.in > a.max_in) {
-            if (r == 0) atomicOr(&g_error_flags, 2u);
-        } else if (r >= d.out) {
-            rec.mode = ROW_PAD;
-        } else if (d.in > 0) {
-            rec.mode = ROW_DATA;
-            const uint32_t bytes = (uint32_t)(d.in * 2);
-            mbar_arrive_expect_tx(b, bytes);
-            bulk_g2s(smem_u32(dst), d.W + r * d.in, bytes, b);
-            return;
+            if (r0 == 0) atomicOr(&g_error_flags, 2u);
+        } else {
+            rec.skip = 0u;
+            if (data > 0) {
+                const uint32_t bytes = (uint32_t)(data * d.in * 2);
+                mbar_arrive_expect_tx(b, bytes);
+                bulk_g2s(smem_u32(dst), d.W + r0 * d.in, bytes, b);
+                return;
+            }
         }
     }
     mbar_arrive(b);
@@ -131,24 +159,29 @@ __global__ void __launch_bounds__(RS_THREADS) rows_staged_kernel(const RowArgs a
     __syncthreads();
     int tn = 0;                 // thread 0's cursor over the table
     if (tid == 0 && (int64_t)blockIdx.x < a.total_rows)
-        stage_row<SWZ>(a, blockIdx.x, tn, smem, &full[0], info[0]);
+        stage_bundle<SWZ>(a, blockIdx.x, tn, smem, &full[0], info[0]);
     bool stopped = false;
     uint32_t i = 0, st = 0, ph = 0;
-    for (int64_t R = blockIdx.x; R < a.total_rows; R += gridDim.x, ++i) {
+    for (int64_t U = blockIdx.x; U < a.total_rows; U += gridDim.x, ++i) {
         st = i & 1u;
         ph = (i >> 1) & 1u;
-        const unsigned char *row = smem + st * stage_bytes;
-        // pass 1: the block maxima of this thread's blocks and their maximum
+        const unsigned char *bundle = smem + st * stage_bytes;
         const bool ok = mbar_wait(smem_u32(&full[st]), ph);
         const RowStage &rec = info[st];
-        const uint32_t mode = ok ? rec.mode : ROW_SKIP;
-        const int64_t nb = rec.nb;
+        const bool skip = !ok || rec.skip != 0u;
+        // this thread's row of the bundle and its place in it
+        const uint32_t tpr = rec.tpr;
+        const uint32_t ri = (uint32_t)tid / tpr, li = (uint32_t)tid % tpr;
+        const uint32_t nbu = (uint32_t)rec.nb;
+        const bool data = !skip && ri < rec.data;
+        const unsigned char *row = bundle + (size_t)ri * nbu * 32u;
+        // pass 1: the block maxima of this thread's blocks and their maximum
         uint32_t mx = 0u;
-        if (mode == ROW_DATA) {
+        if (data) {
 #pragma unroll 2
             for (int j = 0; j < RS_BPT; ++j) {
-                const uint32_t b = (uint32_t)tid + (uint32_t)j * RS_THREADS;
-                if (b < (uint32_t)nb) {
+                const uint32_t b = li + (uint32_t)j * tpr;
+                if (b < nbu) {
                     const uint4 *p = reinterpret_cast<const uint4 *>(row) + 2u * b;
                     const uint4 v0 = p[0], v1 = p[1];
                     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
@@ -158,7 +191,7 @@ __global__ void __launch_bounds__(RS_THREADS) rows_staged_kernel(const RowArgs a
                 }
             }
         }
-        mx = __reduce_max_sync(FULL, mx);
+        mx = __reduce_max_sync(FULL, mx);       // a warp's lanes belong to one row (tpr >= 32)
         if (lane == 0) red[st][warp] = mx;
         if (__syncthreads_or(!ok)) {           // a wait ran out: every thread stops here
             if (tid == 0) atomicOr(&g_error_flags, 8u);
@@ -166,41 +199,41 @@ __global__ void __launch_bounds__(RS_THREADS) rows_staged_kernel(const RowArgs a
             break;
         }
         // every thread is done with the other buffer and its record (the previous
-        // row): stage the next row there
-        if (tid == 0 && R + gridDim.x < a.total_rows)
-            stage_row<SWZ>(a, R + gridDim.x, tn, smem + (st ^ 1u) * stage_bytes, &full[st ^ 1u], info[st ^ 1u]);
-        if (mode == ROW_SKIP) continue;
-        const int64_t r = rec.r;
-        if (mode == ROW_PAD) {                  // a padding row of the 128x4 layout: its words are 0
+        // bundle): stage the next bundle there
+        if (tid == 0 && U + gridDim.x < a.total_rows)
+            stage_bundle<SWZ>(a, U + gridDim.x, tn, smem + (st ^ 1u) * stage_bytes, &full[st ^ 1u],
+                              info[st ^ 1u]);
+        if (skip || ri >= rec.rows) continue;
+        const int64_t r = rec.r0 + ri;
+        const int64_t groups = rec.groups;
+        uint8_t *const scales = rec.scales;
+        if (!data) {                            // a padding row of the 128x4 layout: its words are 0
             if (SWZ)
-                for (int64_t g = tid; g < rec.groups; g += RS_THREADS)
-                    *reinterpret_cast<uint32_t *>(rec.scales + swizzled_offset(r, 4 * g, rec.groups)) = 0u;
+                for (int64_t g = li; g < groups; g += tpr)
+                    *reinterpret_cast<uint32_t *>(scales + swizzled_offset(r, 4 * g, groups)) = 0u;
             continue;
         }
         uint32_t amax = 0u;
-#pragma unroll
-        for (int w = 0; w < RS_THREADS / 32; ++w) amax = max(amax, red[st][w]);
+        const uint32_t wpr = tpr / 32u, w0 = ri * wpr;
+        for (uint32_t w = 0; w < wpr; ++w) amax = max(amax, red[st][w0 + w]);
         if (amax >= 0x7f80u) {                  // a non-finite value: flag it, write nothing of the row
-            if (tid == 0) atomicOr(&g_error_flags, 1u);
+            if (li == 0) atomicOr(&g_error_flags, 1u);
             continue;
         }
         const float A_row = __uint_as_float(amax << 16);
         // s = fl(A_row / 2688): the twice-corrected quotient by the correctly rounded
         // 1/2688 (bit-identical to the IEEE division while nothing underflows)
         const float s = A_row >= 0x1p-100f ? div_full(A_row, 2688.0f, RCP_2688) : __fdiv_rn(A_row, 2688.0f);
-        if (tid == 0) rec.ts[r] = s;
-        // pass 2: this thread's blocks (b = tid + j*RS_THREADS, j < jn; a tensor holds
-        // fewer than 2^31 blocks, so block indices fit 32 bits)
-        const uint32_t nbu = (uint32_t)nb;
-        const uint32_t jn = (uint32_t)tid < nbu ? (nbu - 1u - (uint32_t)tid) / RS_THREADS + 1u : 0u;
+        if (li == 0) rec.ts[r] = s;
+        // pass 2: this thread's blocks (b = li + j*tpr, j < jn; a tensor holds fewer
+        // than 2^31 blocks, so block indices fit 32 bits)
+        const uint32_t jn = li < nbu ? (nbu - 1u - li) / tpr + 1u : 0u;
         const uint32_t base = (uint32_t)r * nbu;
         uint2 *const codes = reinterpret_cast<uint2 *>(rec.codes);
-        uint8_t *const scales = rec.scales;
         uint4 *const xq = reinterpret_cast<uint4 *>(rec.xq);
-        const int64_t groups = rec.groups;
         if (s == 0.0f) {                        // a row of zeros: scale bytes 0x38, codes 0, values 0
             for (uint32_t j = 0; j < jn; ++j) {
-                const uint32_t b = (uint32_t)tid + j * RS_THREADS, blk = base + b;
+                const uint32_t b = li + j * tpr, blk = base + b;
                 codes[blk] = make_uint2(0u, 0u);
                 scales[SWZ ? swizzled_offset(r, b, groups) : (int64_t)blk] = 0x38u;
                 if (xq) {
@@ -212,7 +245,7 @@ __global__ void __launch_bounds__(RS_THREADS) rows_staged_kernel(const RowArgs a
             const F46Scale sc = f46_scale(s);
 #pragma unroll 1
             for (uint32_t j = 0; j < jn; ++j) {
-                const uint32_t b = (uint32_t)tid + j * RS_THREADS, blk = base + b;
+                const uint32_t b = li + j * tpr, blk = base + b;
                 const uint4 *p = reinterpret_cast<const uint4 *>(row) + 2u * b;
                 const uint4 v0 = p[0], v1 = p[1];
                 const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
@@ -231,8 +264,8 @@ __global__ void __launch_bounds__(RS_THREADS) rows_staged_kernel(const RowArgs a
             }
         }
         if (SWZ)                                // the row's padding columns (at most 3)
-            for (int64_t c = nb + tid; c < 4 * rec.groups; c += RS_THREADS)
-                rec.scales[swizzled_offset(r, c, rec.groups)] = 0u;
+            for (int64_t c = nbu + li; c < 4 * groups; c += tpr)
+                scales[swizzled_offset(r, c, groups)] = 0u;
     }
     // After a wait ran out, the copy into the current buffer may still be in
     // flight: it must land before the CTA's shared memory is released.

@@ -255,11 +255,13 @@ typedef struct focus_hparams {
  * X' optional))
  * and fills block_begin and tile_begin (for purpose 4 in 32-blocks and tiles
  * of 128 of them: 4096 weights, as for the other purposes; for purposes 5 and
- * 6 tile_begin is the entry's first row, and the rows of every entry count
- * padded to a multiple of 128 for purpose 6).  Host memory in, host memory
- * out.
- * *total_tiles receives the number of work tiles (for purposes 5 and 6: of
- * rows), passed to the calls below.
+ * 6 the work unit is a bundle of consecutive rows of one entry -- as many as
+ * 256 threads cover with at most 4 blocks each, e.g. 4 rows of 4096 values, 1
+ * of 14336 -- tile_begin is the entry's first bundle, and the rows of every
+ * entry count padded to a multiple of 128 for purpose 6).  Host memory in,
+ * host memory out.
+ * *total_tiles receives the number of work units (tiles; for purposes 5 and
+ * 6 bundles of rows), passed to the calls below.
  * A device-resident table cannot be checked again at call time: a kernel that
  * meets an entry lacking a pointer it needs skips that entry and sets the
  * device flag (FOCUS_ERR_NONFINITE_INPUT from focus_get_error). */
@@ -386,7 +388,8 @@ int focus_fouroversix_act_swizzled(const uint16_t *X, int64_t tokens, int64_t hi
  * FOCUS_PURPOSE_ACT (block scales row-major; swizzled = 0) or
  * FOCUS_PURPOSE_ACT_SWIZZLED (the 128x4-atom layout, each entry's scales
  * buffer at least focus_scales_swizzled_bytes(tokens, hidden/16) bytes;
- * swizzled = 1), in one launch: total_rows as focus_table_prepare returned it,
+ * swizzled = 1), in one launch: total_rows = the work count
+ * focus_table_prepare returned (bundles of rows),
  * max_hidden at least every entry's hidden (a multiple of 16, at most 16384,
  * else FOCUS_ERR_SHAPE; an entry wider than max_hidden is skipped and sets
  * the device flag).  Every entry as the single-tensor call: desc.W = X,

@@ -376,9 +376,9 @@ def test_step_amax_checks(F):
 
 def test_activation_table_prepare_on_host():
     """Purposes 5 and 6 (activation tables for the per-token calls): tile_begin is
-    each entry's first row (rows padded to 128 for the 128x4 layout), the total is
-    the row count, an empty entry adds no rows, rows above 16384 values and entries
-    without codes, scales or token scales are refused."""
+    each entry's first bundle of rows (rows padded to 128 for the 128x4 layout),
+    the total is the bundle count, an empty entry adds none, rows above 16384
+    values and entries without codes, scales or token scales are refused."""
     from fp4_post_weight_b200 import focus as F
     P = 1 << 20
     shapes = [(33, 4096), (0, 64), (130, 1040), (5, 16384)]
@@ -387,10 +387,12 @@ def test_activation_table_prepare_on_host():
         d = descs[i]
         d.W, d.s2, d.codes, d.scales = P + (i << 24), P + (i << 24) + 4096, P + (i << 24) + 8192, P + (i << 24) + 16384
         d.out, d.in_ = t, h
-    assert F.focus_table_prepare(descs, F.FOCUS_PURPOSE_ACT) == 33 + 130 + 5
-    assert [descs[i].tile_begin for i in range(4)] == [0, 33, 33, 163]
-    assert F.focus_table_prepare(descs, F.FOCUS_PURPOSE_ACT_SWIZZLED) == 128 + 256 + 128
-    assert [descs[i].tile_begin for i in range(4)] == [0, 128, 128, 384]
+    # work units are bundles of rows: 4 rows of 4096 values (64 threads each), 8 of 1040
+    # (32 threads each, at most 4 blocks per thread), 1 of 16384
+    assert F.focus_table_prepare(descs, F.FOCUS_PURPOSE_ACT) == 9 + 17 + 5
+    assert [descs[i].tile_begin for i in range(4)] == [0, 9, 9, 26]
+    assert F.focus_table_prepare(descs, F.FOCUS_PURPOSE_ACT_SWIZZLED) == 32 + 32 + 128
+    assert [descs[i].tile_begin for i in range(4)] == [0, 32, 32, 64]
     descs[2].codes = None
     with pytest.raises(F.FocusError) as e:
         F.focus_table_prepare(descs, F.FOCUS_PURPOSE_ACT)

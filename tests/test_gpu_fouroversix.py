@@ -190,8 +190,9 @@ def test_nvfp4_activations(F, tokens, hidden):
 def test_activation_table_one_launch(F, rtn, swizzled):
     """Activation tensors of mixed widths in one launch (focus_*_act_multi): a zero
     row, rows of one block, ragged widths, an empty tensor, a token count not a
-    multiple of 128 (padding rows of the 128x4 layout), and the widest staged row;
-    every tensor against the oracle (row scales, scale bytes, codes, X')."""
+    multiple of 128 (padding rows of the 128x4 layout), the widest staged row, and
+    bundles of several rows ending short of a full bundle; every tensor against the
+    oracle (row scales, scale bytes, codes, X')."""
     from fp4_post_weight_b200.table import ActTable, act_entry
     shapes = [(33, 4096), (5, 48), (0, 64), (130, 1040), (17, 14336), (3, 16), (7, 16384)]
     ents, Xs = [], []
@@ -205,7 +206,13 @@ def test_activation_table_one_launch(F, rtn, swizzled):
                               torch.empty_like(X) if t else None))
         Xs.append(X)
     tab = ActTable(ents, swizzled=swizzled)
-    assert tab.total_rows == sum(((t + 127) // 128 * 128 if swizzled else t) for t, h in shapes if t)
+
+    def bundles(rows, nb):            # rows per bundle: 256 threads, at most 4 blocks per thread
+        tpr = 32
+        while tpr < 256 and 4 * tpr < nb:
+            tpr *= 2
+        return -(-rows // (256 // tpr))
+    assert tab.total_rows == sum(bundles((t + 127) // 128 * 128 if swizzled else t, h // 16) for t, h in shapes if t)
     tab.nvfp4() if rtn else tab.fouroversix()
     assert F.focus_get_error() == 0
     for (t, h), X, e in zip(shapes, Xs, ents):
