@@ -334,7 +334,7 @@ def measure_next_rows(ents, dev, N, peaks, world):
         and scales, and codes, scales and W');
       * FourOverSix with one scale per token over one decoder layer's linear
         inputs for a micro-batch of 4096 tokens (q/k/v, o and gate/up inputs
-        [4096, 4096], the down input [4096, 14336]: 208 MB), one launch over
+        [4096, 4096], the down input [4096, 14336]: 218 MB), one launch over
         the four tensors (and, for comparison, one launch per width);
       * a calibration step over four micro-batches: three table backward passes
         (the first overwriting dm/dq, then accumulating) and the fused step

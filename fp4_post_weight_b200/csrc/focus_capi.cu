@@ -25,9 +25,36 @@ namespace {
 
 constexpr int MAX_DEVICES = 64;
 
+static_assert(SF_ACC == (int)FOCUS_STEP_ACCUMULATE && SF_WRITE_GRAD == (int)FOCUS_STEP_WRITE_GRAD &&
+                  SF_PACK == (int)FOCUS_STEP_PACK_UPDATED && (SF_AMAX & 15) == 0,
+              "the step kernels' option bits are the FOCUS_STEP_* flags, plus one for the tensor maxima");
+
+// The step kernels: one per FOCUS_STEP_WQ_UPDATED setting that reads the other
+// options at run time, and ones compiled for the option sets of a calibration
+// loop: the step with the export and the tensor maxima, with either alone or
+// neither, and the last micro-batch's step (accumulate, W' of the update).
+constexpr int STEP_KERNELS = 7;
+template <bool WQU, int SF>
+constexpr int step_kernel_index() {
+    return !WQU ? (SF == SF_RUNTIME ? 0 : SF == (SF_PACK | SF_AMAX) ? 2 : SF == SF_PACK ? 3 : SF == SF_AMAX ? 4
+                                                                                      : SF == 0 ? 5 : -1)
+                : (SF == SF_RUNTIME ? 1 : SF == SF_ACC ? 6 : -1);
+}
+
+template <int KIND, bool WQU = false, int SF = SF_RUNTIME>
+int pipe_occupancy() {
+    cudaFuncSetAttribute(pipe_kernel<KIND, WQU, SF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)stage_smem_bytes<KIND>());
+    int occ = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, pipe_kernel<KIND, WQU, SF>, CTA_THREADS,
+                                                  stage_smem_bytes<KIND>());
+    return occ;
+}
+
 struct DeviceInfo {
     int sms = 0;
-    int occ_fwd = 0, occ_bwd = 0, occ_step = 0, occ_step_wqu = 0, occ_f46 = 0,
+    int occ_step[STEP_KERNELS] = {};   // by step_kernel_index
+    int occ_fwd = 0, occ_bwd = 0, occ_f46 = 0,
         occ_rows = 0, occ_rows_swz = 0, occ_amax = 0, occ_adam = 0;
     int occ_rows_rtn[2] = {0, 0};   // per-token NVFP4: row-major scales, 128x4 layout
     int occ_mx[3] = {0, 0, 0}, occ_mx_multi[3] = {0, 0, 0}, occ_mx_export = 0, occ_mx_multi_export = 0;
@@ -42,26 +69,16 @@ int device_info(DeviceInfo **out) {
     std::call_once(g_once[dev], [dev] {
         DeviceInfo &d = g_info[dev];
         cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
-        cudaFuncSetAttribute(pipe_kernel<KIND_FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)stage_smem_bytes<KIND_FWD>());
-        cudaFuncSetAttribute(pipe_kernel<KIND_BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)stage_smem_bytes<KIND_BWD>());
-        cudaFuncSetAttribute(pipe_kernel<KIND_STEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)stage_smem_bytes<KIND_STEP>());
-        cudaFuncSetAttribute(pipe_kernel<KIND_STEP, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)stage_smem_bytes<KIND_STEP>());
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_fwd, pipe_kernel<KIND_FWD>, CTA_THREADS,
-                                                      stage_smem_bytes<KIND_FWD>());
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_bwd, pipe_kernel<KIND_BWD>, CTA_THREADS,
-                                                      stage_smem_bytes<KIND_BWD>());
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_step, pipe_kernel<KIND_STEP>, CTA_THREADS,
-                                                      stage_smem_bytes<KIND_STEP>());
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_step_wqu, pipe_kernel<KIND_STEP, true>, CTA_THREADS,
-                                                      stage_smem_bytes<KIND_STEP>());
-        cudaFuncSetAttribute(pipe_kernel<KIND_F46>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)stage_smem_bytes<KIND_F46>());
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_f46, pipe_kernel<KIND_F46>, CTA_THREADS,
-                                                      stage_smem_bytes<KIND_F46>());
+        d.occ_fwd = pipe_occupancy<KIND_FWD>();
+        d.occ_bwd = pipe_occupancy<KIND_BWD>();
+        d.occ_f46 = pipe_occupancy<KIND_F46>();
+        d.occ_step[step_kernel_index<false, SF_RUNTIME>()] = pipe_occupancy<KIND_STEP, false, SF_RUNTIME>();
+        d.occ_step[step_kernel_index<true, SF_RUNTIME>()] = pipe_occupancy<KIND_STEP, true, SF_RUNTIME>();
+        d.occ_step[step_kernel_index<false, SF_PACK | SF_AMAX>()] = pipe_occupancy<KIND_STEP, false, SF_PACK | SF_AMAX>();
+        d.occ_step[step_kernel_index<false, SF_PACK>()] = pipe_occupancy<KIND_STEP, false, SF_PACK>();
+        d.occ_step[step_kernel_index<false, SF_AMAX>()] = pipe_occupancy<KIND_STEP, false, SF_AMAX>();
+        d.occ_step[step_kernel_index<false, 0>()] = pipe_occupancy<KIND_STEP, false, 0>();
+        d.occ_step[step_kernel_index<true, SF_ACC>()] = pipe_occupancy<KIND_STEP, true, SF_ACC>();
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows, f46_rows_kernel<false>, ROW_THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows_swz, f46_rows_kernel<true>, ROW_THREADS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_rows_rtn[0], f46_rows_kernel<false, true>, ROW_THREADS, 0);
@@ -82,7 +99,9 @@ int device_info(DeviceInfo **out) {
                                                       MX_TILE_BLOCKS, 0);
     });
     DeviceInfo &d = g_info[dev];
-    if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || d.occ_step <= 0 || d.occ_step_wqu <= 0 || d.occ_f46 <= 0 ||
+    bool step_ok = true;
+    for (int k = 0; k < STEP_KERNELS; ++k) step_ok = step_ok && d.occ_step[k] > 0;
+    if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || !step_ok || d.occ_f46 <= 0 ||
         d.occ_rows <= 0 || d.occ_rows_swz <= 0 || d.occ_rows_rtn[0] <= 0 || d.occ_rows_rtn[1] <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 ||
         d.occ_mx[1] <= 0 || d.occ_mx[2] <= 0 || d.occ_mx_multi[0] <= 0 || d.occ_mx_multi[1] <= 0 ||
         d.occ_mx_multi[2] <= 0 || d.occ_mx_export <= 0 || d.occ_mx_multi_export <= 0)
@@ -166,19 +185,20 @@ int check_hyper(float lr, float beta1, float beta2, float eps, float wd, int64_t
 using namespace focus;
 
 namespace {
-template <int KIND, bool WQU = false>
+template <int KIND, bool WQU = false, int SF = SF_RUNTIME>
 int launch_on(const Args &a, cudaStream_t s) {
+    static_assert(KIND == KIND_STEP ? step_kernel_index<WQU, SF>() >= 0 : (!WQU && SF == SF_RUNTIME),
+                  "a pipe_kernel instance that device_info does not set up");
     DeviceInfo *di;
     int rc = device_info(&di);
     if (rc) return rc;
     if (a.total_tiles == 0 && !a.one_scale_out) return FOCUS_OK;
-    const int occ = KIND == KIND_FWD ? di->occ_fwd
-                    : KIND == KIND_BWD ? di->occ_bwd
-                    : KIND == KIND_F46 ? di->occ_f46
-                    : (WQU ? di->occ_step_wqu : di->occ_step);
+    int occ;
+    if constexpr (KIND == KIND_STEP) occ = di->occ_step[step_kernel_index<WQU, SF>()];
+    else occ = KIND == KIND_FWD ? di->occ_fwd : KIND == KIND_BWD ? di->occ_bwd : di->occ_f46;
     int64_t grid = grid_for(a.total_tiles, di->sms, occ);
     if (grid < 1) grid = 1;   // the pack of an empty tensor still writes its tensor scale
-    pipe_kernel<KIND, WQU><<<(unsigned)grid, CTA_THREADS, stage_smem_bytes<KIND>(), s>>>(a);
+    pipe_kernel<KIND, WQU, SF><<<(unsigned)grid, CTA_THREADS, stage_smem_bytes<KIND>(), s>>>(a);
     return launch_status();
 }
 
@@ -563,8 +583,22 @@ static int step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_t
     a.pack_updated = (flags & FOCUS_STEP_PACK_UPDATED) ? 1 : 0;
     a.amax_ws = amax_ws;
     a.hp = make_hyper(hp->lr_m, hp->lr_q, hp->beta1, hp->beta2, hp->eps, hp->weight_decay, step);
-    if (flags & FOCUS_STEP_WQ_UPDATED) return launch_on<KIND_STEP, true>(a, (cudaStream_t)stream);
-    return launch_on<KIND_STEP>(a, (cudaStream_t)stream);
+    // the kernel compiled for these options where there is one (FOCUS_STEP_WRITE_GRAD
+    // always takes the kernel that reads them at run time)
+    const cudaStream_t s = (cudaStream_t)stream;
+    const int sf = (int)(flags & (FOCUS_STEP_ACCUMULATE | FOCUS_STEP_WRITE_GRAD | FOCUS_STEP_PACK_UPDATED)) |
+                   (amax_ws ? SF_AMAX : 0);
+    if (flags & FOCUS_STEP_WQ_UPDATED) {
+        if (sf == SF_ACC) return launch_on<KIND_STEP, true, SF_ACC>(a, s);
+        return launch_on<KIND_STEP, true>(a, s);
+    }
+    switch (sf) {
+    case SF_PACK | SF_AMAX: return launch_on<KIND_STEP, false, SF_PACK | SF_AMAX>(a, s);
+    case SF_PACK: return launch_on<KIND_STEP, false, SF_PACK>(a, s);
+    case SF_AMAX: return launch_on<KIND_STEP, false, SF_AMAX>(a, s);
+    case 0: return launch_on<KIND_STEP, false, 0>(a, s);
+    default: return launch_on<KIND_STEP>(a, s);
+    }
 }
 
 int focus_step_fused(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, const focus_hparams *hp,

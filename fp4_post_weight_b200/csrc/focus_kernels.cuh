@@ -86,6 +86,29 @@ struct Args {
     Hyper hp;
 };
 
+// The step's options fixed at compile time: SF is a mask of the SF_* bits
+// (FOCUS_STEP_ACCUMULATE, _WRITE_GRAD, _PACK_UPDATED and the tensor maxima of
+// focus_step_fused_amax), or SF_RUNTIME to read them from Args.  The launcher
+// picks a kernel compiled for the caller's options where one exists; the
+// specialised kernels carry neither the run-time tests nor the registers of
+// the inputs their options leave unused (3% of the step's time, measured).
+// FOCUS_STEP_WQ_UPDATED is the separate template argument WQU.
+enum : int { SF_ACC = 1, SF_WRITE_GRAD = 2, SF_PACK = 4, SF_AMAX = 16, SF_RUNTIME = -1 };
+
+template <int SF>
+struct StepOpt {
+    static __device__ __forceinline__ bool acc(const Args &a) { return SF < 0 ? a.accumulate != 0 : (SF & SF_ACC) != 0; }
+    static __device__ __forceinline__ bool write_grad(const Args &a) {
+        return SF < 0 ? a.write_grad != 0 : (SF & SF_WRITE_GRAD) != 0;
+    }
+    static __device__ __forceinline__ bool pack(const Args &a) {
+        return SF < 0 ? a.pack_updated != 0 : (SF & SF_PACK) != 0;
+    }
+    static __device__ __forceinline__ bool amax(const Args &a) {
+        return SF < 0 ? a.amax_ws != nullptr : (SF & SF_AMAX) != 0;
+    }
+};
+
 // ---------------------------------------------------------------------------
 // tensor lookup
 // ---------------------------------------------------------------------------
@@ -139,7 +162,7 @@ struct Block {
 };
 
 // A block's inputs straight from global memory (ragged tiles).
-template <int KIND, class TV>
+template <int KIND, int SF, class TV>
 __device__ __forceinline__ void load_block_global(const TV &T, const Args &a, Block &B, uint32_t blk) {
     B.blk = blk;
     B.valid = blk < (uint32_t)T.nblk;
@@ -173,7 +196,7 @@ __device__ __forceinline__ void load_block_global(const TV &T, const Args &a, Bl
         const float2 v2 = reinterpret_cast<const float2 *>(T.d.q_exp_avg_sq)[blk];
         B.qv1[0] = v1.x; B.qv1[1] = v1.y; B.qv2[0] = v2.x; B.qv2[1] = v2.y;
     }
-    if (has_grad(KIND) && a.accumulate) {
+    if (has_grad(KIND) && StepOpt<SF>::acc(a)) {
         B.gm_in = T.d.dm[blk];
         const float2 gq = reinterpret_cast<const float2 *>(T.d.dq)[blk];
         B.gq_in[0] = gq.x; B.gq_in[1] = gq.y;
@@ -562,8 +585,9 @@ __device__ __forceinline__ void compute_block_f46(const TV &T, Block &B, bool rt
 // TV is any view of a tensor with members d (descriptor), s2, den and nblk:
 // the consumer warps pass the stage record in shared memory, so the
 // descriptor's pointers are read where used instead of held in registers.
-template <int KIND, bool WQU, class TV>
+template <int KIND, bool WQU, int SF, class TV>
 __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block &B) {
+    using O = StepOpt<SF>;
     if constexpr (KIND == KIND_F46) {
         compute_block_f46(T, B, a.rtn != 0);
         return;
@@ -580,7 +604,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
     // maximum of the block maxima (the blocks past a ragged end have w = 0) into the
     // stage record in shared memory; the producer folds the stage maxima of a tensor
     // and writes them out (T is the stage record here).
-    if (KIND == KIND_STEP && a.amax_ws != nullptr) {
+    if (KIND == KIND_STEP && O::amax(a)) {
         const uint32_t wm = __reduce_max_sync(FULL, abits);
         if ((threadIdx.x & 31) == 0 && wm != 0u) atomicMax(const_cast<uint32_t *>(&T.amax), wm);
     }
@@ -595,7 +619,8 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
     const uint16_t S_h = (uint16_t)e4m3_normal_f16_bits(sbyte);
     const uint64_t s2_2 = f2_pack(T.s2, T.s2);
 
-    const bool want_wq = KIND != KIND_BWD && !WQU && a.write_wq && T.d.Wq != nullptr && B.valid;
+    // (the step always writes W' where the descriptor has it)
+    const bool want_wq = KIND != KIND_BWD && !WQU && (KIND == KIND_STEP || a.write_wq) && T.d.Wq != nullptr && B.valid;
     float sig[2], sq[2];
     double s64[2];                              // the forward's binary64 sigmoids, reused by the export
     uint64_t sm2 = 0ull;                        // sum of g * (in ? c - y : c), pairwise
@@ -652,11 +677,11 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
                 sm2 = f2_fma(g2, t2, sm2);
                 sq2 = f2_fma(g2, f2_pack(ilo, ihi), sq2);
             }
-            sq[k] = f2_lo(sq2) + f2_hi(sq2);
+            sq[k] = __fadd_rn(f2_lo(sq2), f2_hi(sq2));
         }
     }
     // the forward's NVFP4 codes and scale (unless the step exports the updated parameters instead)
-    if (B.valid && !(KIND == KIND_STEP && a.pack_updated)) {
+    if (B.valid && !(KIND == KIND_STEP && O::pack(a))) {
         if (T.d.codes) {
             uint2 cc; cc.x = codes[0]; cc.y = codes[1];
             reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
@@ -666,16 +691,18 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
 
     if (has_grad(KIND)) {
         // dL/dm = inS*(A/6)*sum g*t;  dL/dq_k = -(1 - sigma_k)*S*s2*sum_k g*y_in
-        float gm = inS ? (A * (1.0f / 6.0f)) * (f2_lo(sm2) + f2_hi(sm2)) : 0.0f;
-        float gq0 = -((((1.0f - sig[0]) * S) * T.s2) * sq[0]);
-        float gq1 = -((((1.0f - sig[1]) * S) * T.s2) * sq[1]);
-        if (a.accumulate) {
-            gm = B.gm_in + gm;
-            gq0 = B.gq_in[0] + gq0;
-            gq1 = B.gq_in[1] + gq1;
+        // (every operation rounded on its own, never contracted into a fused
+        // multiply-add, so that every build of the step gives the same bits)
+        float gm = inS ? __fmul_rn(__fmul_rn(A, 1.0f / 6.0f), __fadd_rn(f2_lo(sm2), f2_hi(sm2))) : 0.0f;
+        float gq0 = -__fmul_rn(__fmul_rn(__fmul_rn(__fsub_rn(1.0f, sig[0]), S), T.s2), sq[0]);
+        float gq1 = -__fmul_rn(__fmul_rn(__fmul_rn(__fsub_rn(1.0f, sig[1]), S), T.s2), sq[1]);
+        if (O::acc(a)) {
+            gm = __fadd_rn(B.gm_in, gm);
+            gq0 = __fadd_rn(B.gq_in[0], gq0);
+            gq1 = __fadd_rn(B.gq_in[1], gq1);
         }
         if (B.valid && !bad && !(finitef(gm) && finitef(gq0) && finitef(gq1))) atomicOr(&g_error_flags, 4u);
-        if (B.valid && (KIND == KIND_BWD || a.write_grad)) {
+        if (B.valid && (KIND == KIND_BWD || O::write_grad(a))) {
             T.d.dm[B.blk] = gm;
             reinterpret_cast<float2 *>(T.d.dq)[B.blk] = make_float2(gq0, gq1);
         }
@@ -695,7 +722,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
             }
             // the forward of the updated m and q: NVFP4 export (what a pack after this
             // step would write) and/or W' for the next step's forward
-            const bool exp_codes = a.pack_updated && T.d.codes != nullptr;
+            const bool exp_codes = O::pack(a) && T.d.codes != nullptr;
             const bool exp_wq = WQU && T.d.Wq != nullptr;
             if (B.valid && (exp_codes || exp_wq)) {
                 uint32_t sb2, codes2[2];
@@ -789,7 +816,7 @@ struct AmaxFold {
 };
 
 // A block's inputs from a staged tile (local block lb of the tile).
-template <int KIND>
+template <int KIND, int SF>
 __device__ __forceinline__ void load_block_smem(const Args &a, const unsigned char *stage, Block &B, uint32_t lb,
                                                 uint32_t blk) {
     using L = Layout<KIND>;
@@ -817,7 +844,7 @@ __device__ __forceinline__ void load_block_smem(const Args &a, const unsigned ch
         const float2 v2 = reinterpret_cast<const float2 *>(stage + L::QV2)[lb];
         B.qv1[0] = v1.x; B.qv1[1] = v1.y; B.qv2[0] = v2.x; B.qv2[1] = v2.y;
     }
-    if (has_grad(KIND) && a.accumulate) {
+    if (has_grad(KIND) && StepOpt<SF>::acc(a)) {
         B.gm_in = reinterpret_cast<const float *>(stage + L::GM)[lb];
         const float2 gq = reinterpret_cast<const float2 *>(stage + L::GQ)[lb];
         B.gq_in[0] = gq.x; B.gq_in[1] = gq.y;
@@ -842,10 +869,11 @@ __device__ __forceinline__ bool seek_tensor(const Args &a, int64_t tile, int &t,
 }
 
 // The producer: one thread feeding the ring.
-template <int KIND>
+template <int KIND, int SF>
 __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint64_t *full, uint64_t *empty,
                                         StageInfo *info) {
     using L = Layout<KIND>;
+    using O = StepOpt<SF>;
     constexpr int S = Depth<KIND>::STAGES;
     int t = 0;
     TensorRef T;
@@ -865,7 +893,7 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
         }
         pending &= ~(1u << st);       // the consumers released it: its copies have landed
         StageInfo &inf = info[st];
-        if (KIND == KIND_STEP && a.amax_ws != nullptr) {
+        if (KIND == KIND_STEP && O::amax(a)) {
             if (it >= (uint32_t)S) fold.add(a.amax_ws, inf.tensor, inf.amax);   // the stage's previous tile
             inf.amax = 0u;
         }
@@ -877,7 +905,7 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
         // another purpose) is skipped and reported, never dereferenced
         bool complete = T.d.W != nullptr && (!has_mq(KIND) || (T.d.m != nullptr && T.d.q != nullptr));
         if (has_grad(KIND)) complete = complete && T.d.dWq != nullptr;
-        if (KIND == KIND_BWD || a.accumulate || a.write_grad) complete = complete && T.d.dm != nullptr && T.d.dq != nullptr;
+        if (KIND == KIND_BWD || O::acc(a) || O::write_grad(a)) complete = complete && T.d.dm != nullptr && T.d.dq != nullptr;
         if (KIND == KIND_STEP)
             complete = complete && T.d.m_exp_avg && T.d.m_exp_avg_sq && T.d.q_exp_avg && T.d.q_exp_avg_sq;
         if (KIND != KIND_BWD && T.d.codes != nullptr) complete = complete && T.d.scales != nullptr;
@@ -901,7 +929,7 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
         if (mode == MODE_BULK) {
             unsigned char *stage = smem + st * L::BYTES;
             const uint32_t f = first;
-            mbar_arrive_expect_tx(bar, L::tx_bytes(a.accumulate != 0));
+            mbar_arrive_expect_tx(bar, L::tx_bytes(O::acc(a)));
             bulk_g2s(smem_u32(stage + L::W), reinterpret_cast<const uint4 *>(T.d.W) + 2u * f, TILE_BLOCKS * 32, bar);
             if (has_grad(KIND))
                 bulk_g2s(smem_u32(stage + L::G), reinterpret_cast<const uint4 *>(T.d.dWq) + 2u * f, TILE_BLOCKS * 32,
@@ -916,7 +944,7 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
                 bulk_g2s(smem_u32(stage + L::QV1), T.d.q_exp_avg + 2u * f, TILE_BLOCKS * 8, bar);
                 bulk_g2s(smem_u32(stage + L::QV2), T.d.q_exp_avg_sq + 2u * f, TILE_BLOCKS * 8, bar);
             }
-            if (has_grad(KIND) && a.accumulate) {
+            if (has_grad(KIND) && O::acc(a)) {
                 bulk_g2s(smem_u32(stage + L::GM), T.d.dm + f, TILE_BLOCKS * 4, bar);
                 bulk_g2s(smem_u32(stage + L::GQ), T.d.dq + 2u * f, TILE_BLOCKS * 8, bar);
             }
@@ -928,7 +956,7 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
     }
     // The tensor maxima of the last uses of the stages: wait (bounded) until the
     // consumers have released them, fold them in and write the running maximum.
-    if (KIND == KIND_STEP && a.amax_ws != nullptr && !timed_out) {
+    if (KIND == KIND_STEP && O::amax(a) && !timed_out) {
         for (uint32_t j = it > (uint32_t)S ? it - (uint32_t)S : 0u; j < it; ++j) {
             const uint32_t st = j % S;
             if (!mbar_wait(smem_u32(&empty[st]), (j / S) & 1u)) {
@@ -947,7 +975,7 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
 }
 
 // The consumers: NC_WARPS warps computing from the ring.
-template <int KIND, bool WQU>
+template <int KIND, bool WQU, int SF>
 __device__ __forceinline__ void consume(const Args &a, const unsigned char *smem, uint64_t *full, uint64_t *empty,
                                         const StageInfo *info) {
     using L = Layout<KIND>;
@@ -967,16 +995,16 @@ __device__ __forceinline__ void consume(const Args &a, const unsigned char *smem
             const unsigned char *stage = smem + st * L::BYTES;
             const uint32_t lb = threadIdx.x;
             Block B;
-            if (mode == MODE_BULK) load_block_smem<KIND>(a, stage, B, lb, inf.first + lb);
-            else load_block_global<KIND>(inf, a, B, inf.first + lb);
-            compute_block<KIND, WQU>(inf, a, B);
+            if (mode == MODE_BULK) load_block_smem<KIND, SF>(a, stage, B, lb, inf.first + lb);
+            else load_block_global<KIND, SF>(inf, a, B, inf.first + lb);
+            compute_block<KIND, WQU, SF>(inf, a, B);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
     }
 }
 
-template <int KIND, bool WQU = false>
+template <int KIND, bool WQU = false, int SF = SF_RUNTIME>
 __global__ void __launch_bounds__(CTA_THREADS, Depth<KIND>::MIN_CTAS) pipe_kernel(const Args a) {
     constexpr int S = Depth<KIND>::STAGES;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -993,10 +1021,10 @@ __global__ void __launch_bounds__(CTA_THREADS, Depth<KIND>::MIN_CTAS) pipe_kerne
     }
     __syncthreads();
     if (threadIdx.x >= CONSUMERS) {
-        if (threadIdx.x == CONSUMERS) produce<KIND>(a, smem, full, empty, info);
+        if (threadIdx.x == CONSUMERS) produce<KIND, SF>(a, smem, full, empty, info);
         return;
     }
-    consume<KIND, WQU>(a, smem, full, empty, info);
+    consume<KIND, WQU, SF>(a, smem, full, empty, info);
 }
 
 // ---------------------------------------------------------------------------

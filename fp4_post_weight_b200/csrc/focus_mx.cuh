@@ -205,7 +205,7 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
             codes[k] = code;
             if (KIND != KIND_BWD && a.Wq && !(EXPORT && a.wq_updated))
                 __stcs(reinterpret_cast<uint4 *>(a.Wq) + 4 * blk + k, make_uint4(o[0], o[1], o[2], o[3]));
-            sq[k] = (KIND != KIND_FWD) ? f2_lo(sq2) + f2_hi(sq2) : 0.0f;
+            sq[k] = (KIND != KIND_FWD) ? __fadd_rn(f2_lo(sq2), f2_hi(sq2)) : 0.0f;
         }
         if (KIND != KIND_BWD && a.codes && !(EXPORT && a.pack_updated)) {
             reinterpret_cast<uint4 *>(a.codes)[blk] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
@@ -215,11 +215,12 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
             float gm = inS ? (float)((double)A * 0.25 * sm) : 0.0f;
             float gq[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) gq[k] = -(((1.0f - sig[k]) * S) * sq[k]);
+            for (int k = 0; k < 4; ++k) gq[k] = -__fmul_rn(__fmul_rn(__fsub_rn(1.0f, sig[k]), S), sq[k]);
             if (a.accumulate) {
-                gm = a.dm[blk] + gm;
+                gm = __fadd_rn(a.dm[blk], gm);
                 const float4 p = reinterpret_cast<const float4 *>(a.dq)[blk];
-                gq[0] = p.x + gq[0]; gq[1] = p.y + gq[1]; gq[2] = p.z + gq[2]; gq[3] = p.w + gq[3];
+                gq[0] = __fadd_rn(p.x, gq[0]); gq[1] = __fadd_rn(p.y, gq[1]);
+                gq[2] = __fadd_rn(p.z, gq[2]); gq[3] = __fadd_rn(p.w, gq[3]);
             }
             if (!bad && !(finitef(gm) && finitef(gq[0]) && finitef(gq[1]) && finitef(gq[2]) && finitef(gq[3])))
                 atomicOr(&g_error_flags, 4u);

@@ -234,6 +234,49 @@ def test_step_with_both_updated_outputs(F):
         assert np.array_equal(host_bits(a.Wq), host_bits(b.Wq))
 
 
+@pytest.mark.parametrize("acc", [False, True])
+@pytest.mark.parametrize("pack", [False, True])
+@pytest.mark.parametrize("wqu", [False, True])
+@pytest.mark.parametrize("amax", [False, True])
+def test_step_kernels_for_fixed_options_match_the_runtime_one(F, acc, pack, wqu, amax):
+    """The step runs in a kernel compiled for the caller's options where one
+    exists (the export with or without the tensor maxima, either alone,
+    neither, the accumulating step with W' of the update) and otherwise in the
+    kernel that reads them at run time, which FOCUS_STEP_WRITE_GRAD always
+    selects.  For every combination of the other options, both kernels leave
+    bit-identical parameters, moments, W', codes, scales and tensor maxima from
+    the same inputs (the run-time kernel is checked against the oracle by the
+    tests above)."""
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    shapes = [(37, 1040), (64, 512), (3, 48), (0, 32), (9, 4096)]
+    flags = ((F.FOCUS_STEP_ACCUMULATE if acc else 0) | (F.FOCUS_STEP_PACK_UPDATED if pack else 0)
+             | (F.FOCUS_STEP_WQ_UPDATED if wqu else 0))
+    ea, eb = _entries(shapes, 210, warm=True), _entries(shapes, 210, warm=True)
+    g = torch.Generator(device="cuda").manual_seed(11)
+    for a, b in zip(ea, eb):
+        a.dm.copy_(synth.normal(a.dm.shape, 0, 1e-5, g, "cuda")); b.dm.copy_(a.dm)
+        a.dq.copy_(synth.normal(a.dq.shape, 0, 1e-7, g, "cuda")); b.dq.copy_(a.dq)
+    ta, tb = FocusTable(ea), FocusTable(eb)
+    ta.s2(); tb.s2()
+    wa = torch.zeros(8, dtype=torch.int32, device="cuda")
+    wb = torch.zeros(8, dtype=torch.int32, device="cuda")
+    hp = hparams()
+    if amax:
+        F.focus_step_fused_amax(ta.dev, ta.n, ta.total_tiles, hp, 4, wa, flags)
+        F.focus_step_fused_amax(tb.dev, tb.n, tb.total_tiles, hp, 4, wb, flags | F.FOCUS_STEP_WRITE_GRAD)
+    else:
+        ta.step(4, hp, flags)
+        tb.step(4, hp, flags | F.FOCUS_STEP_WRITE_GRAD)
+    assert F.focus_get_error() == 0
+    assert torch.equal(wa, wb)
+    if amax:
+        assert int(wa[:5].ne(0).sum()) == 4            # every non-empty tensor got its maximum
+    for a, b in zip(ea, eb):
+        for name in ("codes", "scales", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"):
+            assert torch.equal(getattr(a, name), getattr(b, name)), name
+        assert np.array_equal(host_bits(a.Wq), host_bits(b.Wq))
+
+
 def test_pack_multi_leaves_wq_alone(F):
     from fp4_post_weight_b200.table import FocusTable
     ents = _entries([(16, 256)], 60)
