@@ -26,7 +26,8 @@ namespace {
 constexpr int MAX_DEVICES = 64;
 
 static_assert(SF_ACC == (int)FOCUS_STEP_ACCUMULATE && SF_WRITE_GRAD == (int)FOCUS_STEP_WRITE_GRAD &&
-                  SF_PACK == (int)FOCUS_STEP_PACK_UPDATED && (SF_AMAX & 15) == 0,
+                  SF_PACK == (int)FOCUS_STEP_PACK_UPDATED && SF_WQU == (int)FOCUS_STEP_WQ_UPDATED &&
+                  (SF_AMAX & 15) == 0,
               "the step kernels' option bits are the FOCUS_STEP_* flags, plus one for the tensor maxima");
 
 // The step kernels: one per FOCUS_STEP_WQ_UPDATED setting that reads the other
@@ -57,7 +58,8 @@ struct DeviceInfo {
     int occ_fwd = 0, occ_bwd = 0, occ_f46 = 0,
         occ_rows = 0, occ_rows_swz = 0, occ_amax = 0, occ_adam = 0;
     int occ_rows_rtn[2] = {0, 0};   // per-token NVFP4: row-major scales, 128x4 layout
-    int occ_mx[3] = {0, 0, 0}, occ_mx_multi[3] = {0, 0, 0}, occ_mx_export = 0, occ_mx_multi_export = 0;
+    int occ_mx[3] = {0, 0, 0}, occ_mx_multi[3] = {0, 0, 0}, occ_mx_export = 0;
+    int occ_mx_multi_export[3] = {0, 0, 0};   // run-time options; export and W' of the update; export alone
 };
 
 std::once_flag g_once[MAX_DEVICES];
@@ -95,7 +97,12 @@ int device_info(DeviceInfo **out) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi[2], mx_multi_kernel<KIND_STEP>,
                                                       MX_TILE_BLOCKS, 0);
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_export, mx_kernel<KIND_STEP, true>, THREADS, 0);
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi_export, mx_multi_kernel<KIND_STEP, true>,
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi_export[1],
+                                                      mx_multi_kernel<KIND_STEP, true, SF_PACK | SF_WQU>,
+                                                      MX_TILE_BLOCKS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi_export[2], mx_multi_kernel<KIND_STEP, true, SF_PACK>,
+                                                      MX_TILE_BLOCKS, 0);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&d.occ_mx_multi_export[0], mx_multi_kernel<KIND_STEP, true>,
                                                       MX_TILE_BLOCKS, 0);
     });
     DeviceInfo &d = g_info[dev];
@@ -104,7 +111,8 @@ int device_info(DeviceInfo **out) {
     if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || !step_ok || d.occ_f46 <= 0 ||
         d.occ_rows <= 0 || d.occ_rows_swz <= 0 || d.occ_rows_rtn[0] <= 0 || d.occ_rows_rtn[1] <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 ||
         d.occ_mx[1] <= 0 || d.occ_mx[2] <= 0 || d.occ_mx_multi[0] <= 0 || d.occ_mx_multi[1] <= 0 ||
-        d.occ_mx_multi[2] <= 0 || d.occ_mx_export <= 0 || d.occ_mx_multi_export <= 0)
+        d.occ_mx_multi[2] <= 0 || d.occ_mx_export <= 0 || d.occ_mx_multi_export[0] <= 0 ||
+        d.occ_mx_multi_export[1] <= 0 || d.occ_mx_multi_export[2] <= 0)
         return FOCUS_ERR_CUDA;
     *out = &d;
     return FOCUS_OK;
@@ -241,8 +249,13 @@ int launch_mx_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_til
     a.hp = hp;
     if constexpr (KIND == KIND_STEP) {
         if (pack_updated || wq_updated) {
-            const int64_t grid = grid_for(total_tiles, di->sms, di->occ_mx_multi_export);
-            mx_multi_kernel<KIND, true><<<(unsigned)grid, MX_TILE_BLOCKS, 0, s>>>(a);
+            // the export kernels compiled for the options of a calibration loop where
+            // they apply (no accumulation, no gradient output), else the run-time one
+            const int v = (accumulate || write_grad || !pack_updated) ? 0 : (wq_updated ? 1 : 2);
+            const int64_t grid = grid_for(total_tiles, di->sms, di->occ_mx_multi_export[v]);
+            if (v == 1) mx_multi_kernel<KIND, true, SF_PACK | SF_WQU><<<(unsigned)grid, MX_TILE_BLOCKS, 0, s>>>(a);
+            else if (v == 2) mx_multi_kernel<KIND, true, SF_PACK><<<(unsigned)grid, MX_TILE_BLOCKS, 0, s>>>(a);
+            else mx_multi_kernel<KIND, true><<<(unsigned)grid, MX_TILE_BLOCKS, 0, s>>>(a);
             return launch_status();
         }
     }

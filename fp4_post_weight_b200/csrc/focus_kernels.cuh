@@ -92,8 +92,9 @@ struct Args {
 // picks a kernel compiled for the caller's options where one exists; the
 // specialised kernels carry neither the run-time tests nor the registers of
 // the inputs their options leave unused (3% of the step's time, measured).
-// FOCUS_STEP_WQ_UPDATED is the separate template argument WQU.
-enum : int { SF_ACC = 1, SF_WRITE_GRAD = 2, SF_PACK = 4, SF_AMAX = 16, SF_RUNTIME = -1 };
+// FOCUS_STEP_WQ_UPDATED is the separate template argument WQU here, and the
+// bit SF_WQU in the MXFP4 kernels.
+enum : int { SF_ACC = 1, SF_WRITE_GRAD = 2, SF_PACK = 4, SF_WQU = 8, SF_AMAX = 16, SF_RUNTIME = -1 };
 
 template <int SF>
 struct StepOpt {

@@ -49,6 +49,23 @@ struct MxArgs {
     Hyper hp;
 };
 
+// The MXFP4 step's options fixed at compile time (SF: the SF_* bits of the
+// NVFP4 step, SF_WQU for FOCUS_STEP_WQ_UPDATED) or read from MxArgs
+// (SF_RUNTIME); see StepOpt.
+template <int SF>
+struct MxOpt {
+    static __device__ __forceinline__ bool acc(const MxArgs &a) { return SF < 0 ? a.accumulate != 0 : (SF & SF_ACC) != 0; }
+    static __device__ __forceinline__ bool write_grad(const MxArgs &a) {
+        return SF < 0 ? a.write_grad != 0 : (SF & SF_WRITE_GRAD) != 0;
+    }
+    static __device__ __forceinline__ bool pack(const MxArgs &a) {
+        return SF < 0 ? a.pack_updated != 0 : (SF & SF_PACK) != 0;
+    }
+    static __device__ __forceinline__ bool wqu(const MxArgs &a) {
+        return SF < 0 ? a.wq_updated != 0 : (SF & SF_WQU) != 0;
+    }
+};
+
 // E8M0 exponent of the scaled maximum x (see the header comment) and S = 2^e.
 __device__ __forceinline__ int mx_exponent(float x) {
     if (x == 0.0f) return 0;
@@ -66,9 +83,10 @@ __device__ __forceinline__ float pow2f(int e) {           // 2^e for e in [-127,
 // W' when wq_updated.  The block's W is read again here (the step's first
 // read left it in L1) rather than held in sixteen registers across the
 // update.
+template <int SF>
 __device__ __forceinline__ void mx_encode(const MxArgs &a, int64_t blk, float A, float m, const float *qn) {
-    const bool want_codes = a.pack_updated && a.codes != nullptr;
-    const bool want_wq = a.wq_updated && a.Wq != nullptr;
+    const bool want_codes = MxOpt<SF>::pack(a) && a.codes != nullptr;
+    const bool want_wq = MxOpt<SF>::wqu(a) && a.Wq != nullptr;
     if (!want_codes && !want_wq) return;
     uint32_t w[16];
     {
@@ -125,8 +143,9 @@ __device__ __forceinline__ void mx_encode(const MxArgs &a, int64_t blk, float A,
 // One 32-block of the tensor `a` describes.  EXPORT (step only): the codes,
 // scale and/or W' are those of the updated m and q (mx_encode) instead of the
 // forward's, a compile-time choice so that the plain step keeps its registers.
-template <int KIND, bool EXPORT = false>
+template <int KIND, bool EXPORT = false, int SF = SF_RUNTIME>
 __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
+    using O = MxOpt<SF>;
     {
         uint32_t w[16], g[16];
         const uint4 *Wp = reinterpret_cast<const uint4 *>(a.W) + 4 * blk;
@@ -203,11 +222,11 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
                 }
             }
             codes[k] = code;
-            if (KIND != KIND_BWD && a.Wq && !(EXPORT && a.wq_updated))
+            if (KIND != KIND_BWD && a.Wq && !(EXPORT && O::wqu(a)))
                 __stcs(reinterpret_cast<uint4 *>(a.Wq) + 4 * blk + k, make_uint4(o[0], o[1], o[2], o[3]));
             sq[k] = (KIND != KIND_FWD) ? __fadd_rn(f2_lo(sq2), f2_hi(sq2)) : 0.0f;
         }
-        if (KIND != KIND_BWD && a.codes && !(EXPORT && a.pack_updated)) {
+        if (KIND != KIND_BWD && a.codes && !(EXPORT && O::pack(a))) {
             reinterpret_cast<uint4 *>(a.codes)[blk] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
             a.scales[blk] = (uint8_t)(e + 127);
         }
@@ -216,7 +235,7 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
             float gq[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) gq[k] = -__fmul_rn(__fmul_rn(__fsub_rn(1.0f, sig[k]), S), sq[k]);
-            if (a.accumulate) {
+            if (O::acc(a)) {
                 gm = __fadd_rn(a.dm[blk], gm);
                 const float4 p = reinterpret_cast<const float4 *>(a.dq)[blk];
                 gq[0] = __fadd_rn(p.x, gq[0]); gq[1] = __fadd_rn(p.y, gq[1]);
@@ -224,7 +243,7 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
             }
             if (!bad && !(finitef(gm) && finitef(gq[0]) && finitef(gq[1]) && finitef(gq[2]) && finitef(gq[3])))
                 atomicOr(&g_error_flags, 4u);
-            if (KIND == KIND_BWD || a.write_grad) {
+            if (KIND == KIND_BWD || O::write_grad(a)) {
                 a.dm[blk] = gm;
                 reinterpret_cast<float4 *>(a.dq)[blk] = make_float4(gq[0], gq[1], gq[2], gq[3]);
             }
@@ -244,7 +263,7 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
                 reinterpret_cast<float4 *>(a.q_eas)[blk] = make_float4(f2_lo(b01), f2_hi(b01), f2_lo(b23), f2_hi(b23));
                 if (EXPORT) {
                     const float qn[4] = {f2_lo(p01), f2_hi(p01), f2_lo(p23), f2_hi(p23)};
-                    mx_encode(a, blk, A, m, qn);
+                    mx_encode<SF>(a, blk, A, m, qn);
                 }
             }
         }
@@ -281,8 +300,10 @@ struct MxMultiArgs {
     Hyper hp;
 };
 
-template <int KIND, bool EXPORT = false>
+template <int KIND, bool EXPORT = false, int SF = SF_RUNTIME>
 __global__ void __launch_bounds__(MX_TILE_BLOCKS, 7) mx_multi_kernel(const MxMultiArgs g) {
+    const bool acc = SF < 0 ? g.accumulate != 0 : (SF & SF_ACC) != 0;
+    const bool write_grad = SF < 0 ? g.write_grad != 0 : (SF & SF_WRITE_GRAD) != 0;
     __shared__ MxArgs sa;
     __shared__ int64_t s_range[2];          // tiles [first, end) of the current tensor
     int t = 0;                              // thread 0's table cursor
@@ -305,7 +326,7 @@ __global__ void __launch_bounds__(MX_TILE_BLOCKS, 7) mx_multi_kernel(const MxMul
                 if (KIND != KIND_FWD) ok = ok && d.dWq != nullptr;
                 if (KIND == KIND_STEP)
                     ok = ok && d.m_exp_avg && d.m_exp_avg_sq && d.q_exp_avg && d.q_exp_avg_sq;
-                if (KIND == KIND_BWD || g.accumulate || g.write_grad) ok = ok && d.dm && d.dq;
+                if (KIND == KIND_BWD || acc || write_grad) ok = ok && d.dm && d.dq;
                 if ((d.codes == nullptr) != (d.scales == nullptr)) ok = false;
                 if (!ok && nb > 0) atomicOr(&g_error_flags, 2u);
                 sa.W = d.W; sa.dWq = d.dWq; sa.Wq = d.Wq;
@@ -328,7 +349,7 @@ __global__ void __launch_bounds__(MX_TILE_BLOCKS, 7) mx_multi_kernel(const MxMul
             if (tile >= end) break;         // past the last tensor (uniform): nothing left
         }
         const int64_t blk = (tile - first) * MX_TILE_BLOCKS + threadIdx.x;
-        if (tile >= first && blk < sa.nblk) mx_block<KIND, EXPORT>(sa, blk);
+        if (tile >= first && blk < sa.nblk) mx_block<KIND, EXPORT, SF>(sa, blk);
     }
 }
 

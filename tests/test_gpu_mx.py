@@ -257,3 +257,23 @@ def test_mx_step_wq_of_the_update(F):
     assert F.focus_get_error() == 0
     assert torch.equal(m, m2) and torch.equal(q, q2)
     assert torch.equal(Wq_a.view(torch.int16), Wq_b.view(torch.int16))
+
+
+@pytest.mark.parametrize("wqu", [False, True])
+def test_mx_export_kernels_for_fixed_options_match_the_runtime_one(F, wqu):
+    """The table step with the export runs in a kernel compiled for its options
+    (the export with or without W' of the update, no accumulation, no gradient
+    output) and otherwise in the kernel that reads them at run time, which
+    FOCUS_STEP_WRITE_GRAD selects: both leave bit-identical parameters,
+    moments, W', codes and scales from the same inputs."""
+    from fp4_post_weight_b200.table import hparams
+    flags = F.FOCUS_STEP_PACK_UPDATED | (F.FOCUS_STEP_WQ_UPDATED if wqu else 0)
+    ta, _ = mx_table(F, 720, "warm")
+    tb, _ = mx_table(F, 720, "warm")
+    ta.mx_step(3, hparams(), flags)
+    tb.mx_step(3, hparams(), flags | F.FOCUS_STEP_WRITE_GRAD)
+    assert F.focus_get_error() == 0
+    for a, b in zip(ta.entries, tb.entries):
+        for name in ("codes", "scales", "Wq", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"):
+            x, y = getattr(a, name), getattr(b, name)
+            assert torch.equal(x.view(torch.uint8), y.view(torch.uint8)), name
