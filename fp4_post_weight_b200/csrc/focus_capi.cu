@@ -764,12 +764,13 @@ int launch_rows_staged_t(const RowArgs &a, cudaStream_t stream) {
     // one stage holds a bundle of rows: at most RS_BPT * RS_THREADS blocks (32 KB)
     const uint32_t stage = (uint32_t)(RS_MAX_HIDDEN * 2);
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rows_staged_kernel<SWZ, RTN>, RS_THREADS, 2 * stage) !=
-            cudaSuccess || occ <= 0)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rows_staged_kernel<SWZ, RTN>, RS_CTA_THREADS,
+                                                      2 * stage) != cudaSuccess ||
+        occ <= 0)
         return FOCUS_ERR_CUDA;
     const int64_t grid = grid_for(a.total_rows, di->sms, occ);
     if (grid <= 0) return FOCUS_OK;
-    rows_staged_kernel<SWZ, RTN><<<(unsigned)grid, RS_THREADS, 2 * stage, stream>>>(a, stage);
+    rows_staged_kernel<SWZ, RTN><<<(unsigned)grid, RS_CTA_THREADS, 2 * stage, stream>>>(a, stage);
     return launch_status();
 }
 
