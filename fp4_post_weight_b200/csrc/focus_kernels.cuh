@@ -213,14 +213,15 @@ __device__ __forceinline__ float scaled_max(const TV &T, float A, float m) {
     const float Am = __fmul_rn(A, m);
     const float aAm = fabsf(Am);
     if (T.den_ok && aAm <= 0x1p60f && (aAm >= 0x1p-60f || aAm == 0.0f)) return div_full(Am, T.den, T.rden);
-    return __fdiv_rn(Am, T.den);
+    return div_rn_slow(Am, T.den);
 }
 
 // NVFP4 codes and E4M3 scale byte of one block for block factor m and
 // sub-block logits q0, q1 (the forward's decisions only).
 // The sub-block sigmoids come from sigmoid_step with the forward's binary64
 // sigmoids (s0, s1 at the logits q0_old, q1_old), bit-identical to evaluating
-// them afresh.
+// them afresh.  (A warp vote per sub-block between this checked code and an
+// unchecked fast path, as the forward has, measured no faster here.)
 template <class TV>
 __device__ __forceinline__ void encode_block(const TV &T, const uint32_t *w, float A, float m, float q0, float q1,
                                              double s0, double s1, float q0_old, float q1_old, uint32_t &sbyte,
@@ -246,7 +247,7 @@ __device__ __forceinline__ void encode_block(const TV &T, const uint32_t *w, flo
         } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                code |= e2m1_pair(__fdiv_rn(bf16_lo(w[4 * k + j]), D), __fdiv_rn(bf16_hi(w[4 * k + j]), D)) << (8 * j);
+                code |= e2m1_pair(div_rn_slow(bf16_lo(w[4 * k + j]), D), div_rn_slow(bf16_hi(w[4 * k + j]), D)) << (8 * j);
         }
         codes[k] = code;
     }
@@ -306,7 +307,7 @@ __device__ __forceinline__ F46Scale f46_scale(float s) {
 // the IEEE division elsewhere.
 __device__ __forceinline__ float f46_x(float A, float den, float rden, bool den_ok) {
     if (den_ok && A <= 0x1p60f && (A >= 0x1p-60f || A == 0.0f)) return div_full(A, den, rden);
-    return __fdiv_rn(A, den);
+    return div_rn_slow(A, den);
 }
 
 // Scale byte, its value, its binary16 bits and D = fl(S*s) of target x.
@@ -369,7 +370,7 @@ __device__ __forceinline__ void f46_targets_fast(float A, const F46Scale &sc, F4
 template <bool FAST>
 __device__ __forceinline__ uint64_t f46_quot(uint64_t nw, uint32_t wv, float D, uint64_t D2, uint64_t nr2) {
     if (FAST) return div_by_f2(nw, D2, nr2);
-    return f2_pack(__fdiv_rn(bf16_lo(wv), D), __fdiv_rn(bf16_hi(wv), D));
+    return f2_pack(div_rn_slow(bf16_lo(wv), D), div_rn_slow(bf16_hi(wv), D));
 }
 
 // A pair's contribution to a target's squared error from its code values h2
@@ -450,6 +451,12 @@ __device__ __noinline__ bool f46_four_exact(uint4 wa, uint4 wb, uint32_t c6_0, u
     return __dmul_rn(2.0, P) < __dmul_rn((double)s, Q);
 }
 
+// Whether a block with maximum A takes the fast arithmetic under scale sc:
+// the scale is fast and A lies in [2^-60, 2^60] or is 0.
+__device__ __forceinline__ bool f46_fast_range(float A, const F46Scale &sc) {
+    return sc.fast && A <= 0x1p60f && (A >= 0x1p-60f || A == 0.0f);
+}
+
 // FourOverSix of one block with block maximum A (bf16 magnitude, exact) and
 // scale sc.s > 0.  Returns true when the target 4 is chosen (its squared error
 // strictly lower than the target 6's; a tie keeps 6); sb and codes receive the
@@ -464,12 +471,14 @@ __device__ __noinline__ bool f46_four_exact(uint4 wa, uint4 wb, uint32_t c6_0, u
 // candidates (they occur: about one block in 10^7 of Gaussian weights), or a
 // non-finite sum -- the choice is taken by f46_four_exact, unless the two
 // candidates are the same (equal scale bytes).
+// (The warp vote on the range that rtn_block's callers take measured 2-3%
+// slower here: the two-target code has more to lose in registers.)
 __device__ __forceinline__ bool f46_block(const uint32_t *w, float A, const F46Scale &sc, uint32_t &sb,
                                           uint32_t codes[2]) {
     F46Target t6, t4;
     uint32_t c6[2], c4[2];
     float e6, e4;
-    if (sc.fast && A <= 0x1p60f && (A >= 0x1p-60f || A == 0.0f)) {
+    if (f46_fast_range(A, sc)) {
         f46_targets_fast(A, sc, t6, t4);
         f46_both<true>(w, t6, t4, sc.s, c6, c4, e6, e4);
     } else {
@@ -495,10 +504,13 @@ __device__ __forceinline__ bool f46_block(const uint32_t *w, float A, const F46S
 
 // NVFP4 round to nearest of one block (the target 6 alone: the card's block
 // equations with m = 1 and sigmoid = 1) with block maximum A and scale sc.s > 0.
+// FAST: the caller has found f46_fast_range true for this block, for every
+// lane of its warp, so that the general code is not compiled into the path.
+template <bool FAST = false>
 __device__ __forceinline__ void rtn_block(const uint32_t *w, float A, const F46Scale &sc, uint32_t &sb,
                                           uint32_t codes[2]) {
     F46Target t6;
-    if (sc.fast && A <= 0x1p60f && (A >= 0x1p-60f || A == 0.0f)) {
+    if (FAST || f46_fast_range(A, sc)) {
         // as f46_target(f46_x(...)), without the range checks sc.fast makes redundant
         float x = (A == 0.0f) ? 1.0f : div_full(A, sc.den6, sc.rden6);
         t6.sb = e4m3_byte(fmaxf(x, 0x1p-6f));           // the conversion saturates at 448
@@ -518,8 +530,8 @@ __device__ __forceinline__ void rtn_block(const uint32_t *w, float A, const F46S
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint32_t wv = w[4 * k + j];
-            y[j] = t6.fast ? f46_quot<true>(bf16x2_neg_f2(wv), wv, t6.D, D6, n6)
-                           : f46_quot<false>(bf16x2_neg_f2(wv), wv, t6.D, D6, n6);
+            y[j] = (FAST || t6.fast) ? f46_quot<true>(bf16x2_neg_f2(wv), wv, t6.D, D6, n6)
+                                     : f46_quot<false>(bf16x2_neg_f2(wv), wv, t6.D, D6, n6);
         }
         codes[k] = e2m1_quad(y, h);
     }
@@ -554,18 +566,24 @@ __device__ __forceinline__ void wq_words(const uint32_t codes[2], uint32_t sbyte
 
 // FourOverSix (or, rtn, plain NVFP4 round to nearest) of one block of a weight
 // tensor (tensor scale s2 = T.s2).
+// Every lane of the warp calls it (past a ragged end with B.valid false): for
+// plain round to nearest, when every valid block of the warp is in the fast
+// range, the warp runs the fast code alone.
 template <class TV>
 __device__ __forceinline__ void compute_block_f46(const TV &T, Block &B, bool rtn) {
     const uint32_t abits = block_amax_bits(B.w);
+    const float A = __uint_as_float(abits << 16);
     const bool bad = B.valid && abits >= 0x7f80u;
+    F46Scale sc;
+    sc.s = T.s2; sc.den6 = T.den; sc.rden6 = T.rden; sc.den4 = T.den4; sc.rden4 = T.rden4;
+    sc.den_ok = T.den46_ok;
+    sc.fast = f46_scale_fast(sc.den_ok, sc.s);
+    const bool fast = rtn && __all_sync(FULL, !B.valid || f46_fast_range(A, sc));
     if (B.valid) {
-        F46Scale sc;
-        sc.s = T.s2; sc.den6 = T.den; sc.rden6 = T.rden; sc.den4 = T.den4; sc.rden4 = T.rden4;
-        sc.den_ok = T.den46_ok;
-        sc.fast = f46_scale_fast(sc.den_ok, sc.s);
         uint32_t sb, codes[2];
-        if (rtn) rtn_block(B.w, __uint_as_float(abits << 16), sc, sb, codes);
-        else f46_block(B.w, __uint_as_float(abits << 16), sc, sb, codes);
+        if (!rtn) f46_block(B.w, A, sc, sb, codes);
+        else if (fast) rtn_block<true>(B.w, A, sc, sb, codes);
+        else rtn_block(B.w, A, sc, sb, codes);
         if (T.d.codes) {
             reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = make_uint2(codes[0], codes[1]);
             T.d.scales[B.blk] = (uint8_t)sb;
@@ -580,43 +598,65 @@ __device__ __forceinline__ void compute_block_f46(const TV &T, Block &B, bool rt
     if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_error_flags, 1u);
 }
 
-// The forward, the straight-through gradients and the AdamW update of one block.
-// WQU (step only, FOCUS_STEP_WQ_UPDATED): W' is that of the updated m and q,
-// a compile-time choice so that the other step variants keep its registers.
-// TV is any view of a tensor with members d (descriptor), s2, den and nblk:
-// the consumer warps pass the stage record in shared memory, so the
-// descriptor's pointers are read where used instead of held in registers.
-template <int KIND, bool WQU, int SF, class TV>
-__device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block &B) {
-    using O = StepOpt<SF>;
-    if constexpr (KIND == KIND_F46) {
-        compute_block_f46(T, B, a.rtn != 0);
-        return;
-    }
-    // A_b = max |w| over the block: max of the bf16 magnitude bit patterns (a NaN
-    // or an infinity sorts above every finite magnitude, which is how it is found)
-    uint32_t am = 0u;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) am = __vmaxu2(am, B.w[j] & 0x7fff7fffu);
-    const uint32_t abits = max(am & 0xffffu, am >> 16);
-    const float A = __uint_as_float(abits << 16);
-    const bool bad = B.valid && (abits >= 0x7f80u || !finitef(B.m) || !finitef(B.q[0]) || !finitef(B.q[1]));
-    // The tensor maximum for the next step's s2 (focus_step_fused_amax): the warp's
-    // maximum of the block maxima (the blocks past a ragged end have w = 0) into the
-    // stage record in shared memory; the producer folds the stage maxima of a tensor
-    // and writes them out (T is the stage record here).
-    if (KIND == KIND_STEP && O::amax(a)) {
-        const uint32_t wm = __reduce_max_sync(FULL, abits);
-        if ((threadIdx.x & 31) == 0 && wm != 0u) atomicMax(const_cast<uint32_t *>(&T.amax), wm);
-    }
+// The forward's per-block scalars: the scaled maximum, the scale byte and
+// value, and the sub-blocks' sigmoids (binary32, and the binary64 values the
+// export starts from).  The divisors D = fl(fl(S*sigma)*s2) are recomputed
+// where used rather than held.
+struct BlockScalars {
+    float x, S;
+    uint32_t sbyte;
+    float sig[2];
+    double s64[2];
+};
 
-    // S_b = e4m3(clamp(fl(fl(A*m)/fl(6*s2)), 2^-6, 448)), scale 1 when the scaled max is 0
-    const float x = scaled_max(T, A, B.m);
-    const bool inS = (x != 0.0f) && (x >= 0x1p-6f) && (x <= 448.0f);
-    float xc = (x == 0.0f) ? 1.0f : x;
+// The forward's scalars on the fast path, with no branch: returns whether
+// each is the one the general code computes and lies where the fast
+// arithmetic that follows is exact -- the scaled maximum by the reciprocal,
+// the sigmoids decided, A <= 2^60 and both D in [2^-60, 2^60].  When it
+// returns false the values are unspecified (never a fault) and the caller
+// takes the general code.
+template <class TV>
+__device__ __forceinline__ bool block_scalars_fast(const TV &T, float A, float m, float q0, float q1,
+                                                   BlockScalars &f) {
+    const float Am = __fmul_rn(A, m);
+    const float aAm = fabsf(Am);
+    bool ok = T.den_ok && aAm <= 0x1p60f && (aAm >= 0x1p-60f || aAm == 0.0f) && A <= 0x1p60f;
+    f.x = div_full(Am, T.den, T.rden);
+    float xc = (f.x == 0.0f) ? 1.0f : f.x;
     xc = fminf(fmaxf(xc, 0x1p-6f), 448.0f);
-    const uint32_t sbyte = e4m3_byte(xc);
-    const float S = e4m3_normal_f32(sbyte);
+    f.sbyte = e4m3_byte(xc);
+    f.S = e4m3_normal_f32(f.sbyte);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        ok = sigmoid_fast_try(k ? q1 : q0, f.sig[k], f.s64[k]) && ok;
+        const float D = __fmul_rn(__fmul_rn(f.S, f.sig[k]), T.s2);
+        ok = ok && D >= 0x1p-60f && D <= 0x1p60f;
+    }
+    return ok;
+}
+
+// Everything of compute_block after the block maximum.  FAST: the forward's
+// scalars f come from block_scalars_fast, which held for every lane of the
+// warp, so the forward's per-element work runs with no range test and no
+// branch.  Otherwise (a lane outside the fast range: rare) the general code,
+// which tests each quantity where it is used.  Both give the same bits.
+template <int KIND, bool WQU, int SF, bool FAST, class TV>
+__device__ __forceinline__ void block_body(const TV &T, const Args &a, Block &B, float A, bool bad,
+                                           const BlockScalars &f) {
+    using O = StepOpt<SF>;
+    // S_b = e4m3(clamp(fl(fl(A*m)/fl(6*s2)), 2^-6, 448)), scale 1 when the scaled max is 0
+    float x, S;
+    uint32_t sbyte;
+    if constexpr (FAST) {
+        x = f.x; S = f.S; sbyte = f.sbyte;
+    } else {
+        x = scaled_max(T, A, B.m);
+        float xc = (x == 0.0f) ? 1.0f : x;
+        xc = fminf(fmaxf(xc, 0x1p-6f), 448.0f);
+        sbyte = e4m3_byte(xc);
+        S = e4m3_normal_f32(sbyte);
+    }
+    const bool inS = (x != 0.0f) && (x >= 0x1p-6f) && (x <= 448.0f);
     const uint16_t S_h = (uint16_t)e4m3_normal_f16_bits(sbyte);
     const uint64_t s2_2 = f2_pack(T.s2, T.s2);
 
@@ -629,10 +669,14 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
         // D_k = fl(fl(S*sigmoid(q_k))*s2); y_i = fl(w_i/D_k); c_i = E2M1(clamp(y_i, -6, 6))
-        sig[k] = sigmoid_fast(B.q[k], s64[k]);
+        if constexpr (FAST) {
+            sig[k] = f.sig[k]; s64[k] = f.s64[k];
+        } else {
+            sig[k] = sigmoid_fast(B.q[k], s64[k]);
+        }
         const float D = __fmul_rn(__fmul_rn(S, sig[k]), T.s2);
         uint64_t y2[4];
-        if (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f) {
+        if (FAST || (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f)) {
             const float nr = -rcp_rn(D);
             const uint64_t D2 = f2_pack(D, D), nr2 = f2_pack(nr, nr);
 #pragma unroll
@@ -640,7 +684,7 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
         } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                y2[j] = f2_pack(__fdiv_rn(bf16_lo(B.w[4 * k + j]), D), __fdiv_rn(bf16_hi(B.w[4 * k + j]), D));
+                y2[j] = f2_pack(div_rn_slow(bf16_lo(B.w[4 * k + j]), D), div_rn_slow(bf16_hi(B.w[4 * k + j]), D));
         }
         uint32_t code = 0u;
         uint32_t ch2[4];
@@ -737,6 +781,44 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
             }
         }
     }
+}
+
+// The forward, the straight-through gradients and the AdamW update of one block.
+// WQU (step only, FOCUS_STEP_WQ_UPDATED): W' is that of the updated m and q,
+// a compile-time choice so that the other step variants keep its registers.
+// TV is any view of a tensor with members d (descriptor), s2, den and nblk:
+// the consumer warps pass the stage record in shared memory, so the
+// descriptor's pointers are read where used instead of held in registers.
+// Every lane of the warp calls it (past a ragged end with B.valid false).
+template <int KIND, bool WQU, int SF, class TV>
+__device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block &B) {
+    using O = StepOpt<SF>;
+    if constexpr (KIND == KIND_F46) {
+        compute_block_f46(T, B, a.rtn != 0);
+        return;
+    }
+    // A_b = max |w| over the block: max of the bf16 magnitude bit patterns (a NaN
+    // or an infinity sorts above every finite magnitude, which is how it is found)
+    uint32_t am = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) am = __vmaxu2(am, B.w[j] & 0x7fff7fffu);
+    const uint32_t abits = max(am & 0xffffu, am >> 16);
+    const float A = __uint_as_float(abits << 16);
+    const bool bad = B.valid && (abits >= 0x7f80u || !finitef(B.m) || !finitef(B.q[0]) || !finitef(B.q[1]));
+    // The tensor maximum for the next step's s2 (focus_step_fused_amax): the warp's
+    // maximum of the block maxima (the blocks past a ragged end have w = 0) into the
+    // stage record in shared memory; the producer folds the stage maxima of a tensor
+    // and writes them out (T is the stage record here).
+    if (KIND == KIND_STEP && O::amax(a)) {
+        const uint32_t wm = __reduce_max_sync(FULL, abits);
+        if ((threadIdx.x & 31) == 0 && wm != 0u) atomicMax(const_cast<uint32_t *>(&T.amax), wm);
+    }
+    // the forward's scalars on the fast path; a warp with a lane outside it takes
+    // the general code (the lanes of a warp hold neighbouring blocks of one tile)
+    BlockScalars f;
+    const bool fast = block_scalars_fast(T, A, B.m, B.q[0], B.q[1], f);
+    if (__all_sync(FULL, fast)) block_body<KIND, WQU, SF, true>(T, a, B, A, bad, f);
+    else block_body<KIND, WQU, SF, false>(T, a, B, A, bad, f);
     if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_error_flags, 1u);
 }
 

@@ -116,7 +116,7 @@ __device__ __forceinline__ void mx_encode(const MxArgs &a, int64_t blk, float A,
         } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                y2[j] = f2_pack(__fdiv_rn(bf16_lo(w[4 * k + j]), D), __fdiv_rn(bf16_hi(w[4 * k + j]), D));
+                y2[j] = f2_pack(div_rn_slow(bf16_lo(w[4 * k + j]), D), div_rn_slow(bf16_hi(w[4 * k + j]), D));
         }
         uint32_t code = 0u, o[4];
 #pragma unroll
@@ -197,7 +197,7 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
             } else {
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    y2[j] = f2_pack(__fdiv_rn(bf16_lo(w[4 * k + j]), D), __fdiv_rn(bf16_hi(w[4 * k + j]), D));
+                    y2[j] = f2_pack(div_rn_slow(bf16_lo(w[4 * k + j]), D), div_rn_slow(bf16_hi(w[4 * k + j]), D));
             }
             uint32_t code = 0u, o[4];
             uint64_t sq2 = 0ull;

@@ -197,7 +197,7 @@ __device__ __forceinline__ void quantize_row_part(const RowStage &rec, const uns
     const float A_row = __uint_as_float(amax << 16);
     // s = fl(A_row / 2688): the twice-corrected quotient by the correctly rounded
     // 1/2688 (bit-identical to the IEEE division while nothing underflows)
-    const float s = A_row >= 0x1p-100f ? div_full(A_row, 2688.0f, RCP_2688) : __fdiv_rn(A_row, 2688.0f);
+    const float s = A_row >= 0x1p-100f ? div_full(A_row, 2688.0f, RCP_2688) : div_rn_slow(A_row, 2688.0f);
     if (li == 0) rec.ts[r] = s;
     // this thread's blocks (a tensor holds fewer than 2^31 blocks, so block
     // indices fit 32 bits)
@@ -217,16 +217,23 @@ __device__ __forceinline__ void quantize_row_part(const RowStage &rec, const uns
         }
     } else {
         const F46Scale sc = f46_scale(s);
+        // the warp's lanes take the same number of iterations (the first lane's,
+        // the most), so that for round to nearest each can vote for the fast code
+        const uint32_t jw = RTN ? __shfl_sync(FULL, jn, 0) : jn;
 #pragma unroll 1
-        for (uint32_t j = 0; j < jn; ++j) {
+        for (uint32_t j = 0; j < jw; ++j) {
             const uint32_t b = li + j * tpr, blk = base + b;
+            const bool mine = j < jn;
+            const float Ab = mine ? __uint_as_float(amax_s[j * RS_THREADS + tid] << 16) : 0.0f;
+            const bool fast = RTN && __all_sync(FULL, !mine || f46_fast_range(Ab, sc));
+            if (!mine) continue;
             const uint4 *p = reinterpret_cast<const uint4 *>(row) + 2u * b;
             const uint4 v0 = p[0], v1 = p[1];
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            const float Ab = __uint_as_float(amax_s[j * RS_THREADS + tid] << 16);
             uint32_t sb, cw[2];
-            if (RTN) rtn_block(w, Ab, sc, sb, cw);
-            else f46_block(w, Ab, sc, sb, cw);
+            if (!RTN) f46_block(w, Ab, sc, sb, cw);
+            else if (fast) rtn_block<true>(w, Ab, sc, sb, cw);
+            else rtn_block(w, Ab, sc, sb, cw);
             codes[blk] = make_uint2(cw[0], cw[1]);
             scales[SWZ ? swizzled_offset32(r, b, groups) : blk] = (uint8_t)sb;
             if (xq) {
