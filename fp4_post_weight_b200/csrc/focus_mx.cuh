@@ -104,9 +104,22 @@ __device__ __forceinline__ void mx_encode(const MxArgs &a, int64_t blk, float A,
     const float S = pow2f(e);
     const uint64_t S2 = f2_pack(S, S);
     uint32_t codes[4];
+    float sg[4];                                  // as in mx_block: one warp vote for the fast sigmoids
+    {
+        bool ok = true;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            double s64u;
+            ok = sigmoid_fast_try(qn[k], sg[k], s64u) && ok;
+        }
+        if (!__all_sync(__activemask(), ok)) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sg[k] = sigmoid_rn(qn[k]);
+        }
+    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const float D = __fmul_rn(S, sigmoid_rn(qn[k]));
+        const float D = __fmul_rn(S, sg[k]);
         uint64_t y2[4];
         if (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f) {
             const float nr = -rcp_rn(D);
@@ -180,13 +193,31 @@ __device__ __forceinline__ void mx_block(const MxArgs &a, int64_t blk) {
         const bool inS = x >= 0x1p-125f;
         const uint64_t S2 = f2_pack(S, S);
 
+        // the sub-blocks' sigmoids: in the step, the table-driven evaluation when it
+        // decides the rounding for every sub-block of every active lane (one warp
+        // vote), else the direct binary64 evaluation for the warp (the same bits
+        // either way; the forward and backward kernels keep the direct one, which
+        // fits their registers better)
         float sig[4], sq[4];
+        {
+            bool ok = KIND == KIND_STEP;
+            if (KIND == KIND_STEP) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    double s64u;
+                    ok = sigmoid_fast_try(qk[k], sig[k], s64u) && ok;
+                }
+            }
+            if (!__all_sync(__activemask(), ok)) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) sig[k] = sigmoid_rn(qk[k]);
+            }
+        }
         double sm = 0.0;              // sum of g*(in ? c - y : c): exact products, binary64 sum (a block's
                                       // gradient may nearly cancel, and AdamW at step 1 compares it with eps)
         uint32_t codes[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            sig[k] = sigmoid_rn(qk[k]);
             const float D = __fmul_rn(S, sig[k]);
             uint64_t y2[4];
             if (D >= 0x1p-60f && D <= 0x1p60f && A <= 0x1p60f) {
