@@ -55,7 +55,7 @@ int pipe_occupancy() {
 struct DeviceInfo {
     int sms = 0;
     int occ_step[STEP_KERNELS] = {};   // by step_kernel_index
-    int occ_fwd = 0, occ_bwd = 0, occ_f46 = 0,
+    int occ_fwd = 0, occ_bwd = 0, occ_f46 = 0, occ_rtn = 0,
         occ_rows = 0, occ_rows_swz = 0, occ_amax = 0, occ_adam = 0;
     int occ_rows_rtn[2] = {0, 0};   // per-token NVFP4: row-major scales, 128x4 layout
     int occ_mx[3] = {0, 0, 0}, occ_mx_multi[3] = {0, 0, 0}, occ_mx_export = 0;
@@ -74,6 +74,7 @@ int device_info(DeviceInfo **out) {
         d.occ_fwd = pipe_occupancy<KIND_FWD>();
         d.occ_bwd = pipe_occupancy<KIND_BWD>();
         d.occ_f46 = pipe_occupancy<KIND_F46>();
+        d.occ_rtn = pipe_occupancy<KIND_RTN>();
         d.occ_step[step_kernel_index<false, SF_RUNTIME>()] = pipe_occupancy<KIND_STEP, false, SF_RUNTIME>();
         d.occ_step[step_kernel_index<true, SF_RUNTIME>()] = pipe_occupancy<KIND_STEP, true, SF_RUNTIME>();
         d.occ_step[step_kernel_index<false, SF_PACK | SF_AMAX>()] = pipe_occupancy<KIND_STEP, false, SF_PACK | SF_AMAX>();
@@ -108,7 +109,7 @@ int device_info(DeviceInfo **out) {
     DeviceInfo &d = g_info[dev];
     bool step_ok = true;
     for (int k = 0; k < STEP_KERNELS; ++k) step_ok = step_ok && d.occ_step[k] > 0;
-    if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || !step_ok || d.occ_f46 <= 0 ||
+    if (d.sms <= 0 || d.occ_fwd <= 0 || d.occ_bwd <= 0 || !step_ok || d.occ_f46 <= 0 || d.occ_rtn <= 0 ||
         d.occ_rows <= 0 || d.occ_rows_swz <= 0 || d.occ_rows_rtn[0] <= 0 || d.occ_rows_rtn[1] <= 0 || d.occ_amax <= 0 || d.occ_adam <= 0 || d.occ_mx[0] <= 0 ||
         d.occ_mx[1] <= 0 || d.occ_mx[2] <= 0 || d.occ_mx_multi[0] <= 0 || d.occ_mx_multi[1] <= 0 ||
         d.occ_mx_multi[2] <= 0 || d.occ_mx_export <= 0 || d.occ_mx_multi_export[0] <= 0 ||
@@ -203,7 +204,8 @@ int launch_on(const Args &a, cudaStream_t s) {
     if (a.total_tiles == 0 && !a.one_scale_out) return FOCUS_OK;
     int occ;
     if constexpr (KIND == KIND_STEP) occ = di->occ_step[step_kernel_index<WQU, SF>()];
-    else occ = KIND == KIND_FWD ? di->occ_fwd : KIND == KIND_BWD ? di->occ_bwd : di->occ_f46;
+    else occ = KIND == KIND_FWD ? di->occ_fwd : KIND == KIND_BWD ? di->occ_bwd : KIND == KIND_RTN ? di->occ_rtn
+                                                                                             : di->occ_f46;
     int64_t grid = grid_for(a.total_tiles, di->sms, occ);
     if (grid < 1) grid = 1;   // the pack of an empty tensor still writes its tensor scale
     pipe_kernel<KIND, WQU, SF><<<(unsigned)grid, CTA_THREADS, stage_smem_bytes<KIND>(), s>>>(a);
@@ -702,8 +704,7 @@ int weight_f46(const uint16_t *W, int64_t out, int64_t in, float s2, uint8_t *co
     a.one_s2 = s2;
     a.n_tensors = 1;
     a.total_tiles = tiles_of(out, in);
-    a.rtn = rtn;
-    return launch_on<KIND_F46>(a, stream);
+    return rtn ? launch_on<KIND_RTN>(a, stream) : launch_on<KIND_F46>(a, stream);
 }
 
 int weight_f46_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_tiles, int rtn, cudaStream_t stream) {
@@ -715,8 +716,7 @@ int weight_f46_multi(const focus_tensor_desc *descs_dev, int n, int64_t total_ti
     a.table = descs_dev;
     a.n_tensors = n;
     a.total_tiles = total_tiles;
-    a.rtn = rtn;
-    return launch_on<KIND_F46>(a, stream);
+    return rtn ? launch_on<KIND_RTN>(a, stream) : launch_on<KIND_F46>(a, stream);
 }
 }  // namespace
 

@@ -26,7 +26,7 @@
 //
 // Besides the FOCUS kinds (forward, backward, fused step) the same pipeline
 // runs FourOverSix round to nearest and plain NVFP4 round to nearest of
-// weights (KIND_F46, W alone is staged; Args::rtn picks the latter); the
+// weights (KIND_F46 and KIND_RTN: W alone is staged); the
 // per-token kernel (FourOverSix or NVFP4, row-major or 128x4 scales), the
 // scale relayout and the standalone AdamW below are plain grid-stride kernels.
 //
@@ -63,12 +63,13 @@ constexpr unsigned FULL = 0xffffffffu;
 // (This header is compiled into exactly one translation unit.)
 __device__ unsigned int g_error_flags = 0;
 
-enum Kind : int { KIND_FWD = 0, KIND_BWD = 1, KIND_STEP = 2, KIND_F46 = 3 };
+enum Kind : int { KIND_FWD = 0, KIND_BWD = 1, KIND_STEP = 2, KIND_F46 = 3, KIND_RTN = 4 };
 
 // Which inputs a kind reads besides W: dW' (and the gradient accumulators),
-// and the scale parameters m and q.  FourOverSix reads W alone.
+// and the scale parameters m and q.  FourOverSix and plain round to nearest
+// read W alone.
 __host__ __device__ constexpr bool has_grad(int kind) { return kind == KIND_BWD || kind == KIND_STEP; }
-__host__ __device__ constexpr bool has_mq(int kind) { return kind != KIND_F46; }
+__host__ __device__ constexpr bool has_mq(int kind) { return kind != KIND_F46 && kind != KIND_RTN; }
 
 struct Args {
     const focus_tensor_desc *table;  // device table, or nullptr: use `one`
@@ -82,7 +83,6 @@ struct Args {
     int write_grad;                  // step: FOCUS_STEP_WRITE_GRAD
     int pack_updated;                // step: FOCUS_STEP_PACK_UPDATED
     uint32_t *amax_ws;               // step: per-tensor max |w| (bf16 magnitude bits) for the next s2, or nullptr
-    int rtn;                         // KIND_F46: plain NVFP4 round to nearest (the target 6 alone) instead
     Hyper hp;
 };
 
@@ -793,8 +793,8 @@ __device__ __forceinline__ void block_body(const TV &T, const Args &a, Block &B,
 template <int KIND, bool WQU, int SF, class TV>
 __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block &B) {
     using O = StepOpt<SF>;
-    if constexpr (KIND == KIND_F46) {
-        compute_block_f46(T, B, a.rtn != 0);
+    if constexpr (KIND == KIND_F46 || KIND == KIND_RTN) {
+        compute_block_f46(T, B, KIND == KIND_RTN);
         return;
     }
     // A_b = max |w| over the block: max of the bf16 magnitude bit patterns (a NaN
@@ -853,6 +853,7 @@ template <> struct Depth<KIND_FWD> { static constexpr int STAGES = 6, MIN_CTAS =
 template <> struct Depth<KIND_BWD> { static constexpr int STAGES = 3, MIN_CTAS = 3; };
 template <> struct Depth<KIND_STEP> { static constexpr int STAGES = 2, MIN_CTAS = 3; };
 template <> struct Depth<KIND_F46> { static constexpr int STAGES = 8, MIN_CTAS = 3; };
+template <> struct Depth<KIND_RTN> { static constexpr int STAGES = 8, MIN_CTAS = 3; };
 
 template <int KIND>
 constexpr uint32_t stage_smem_bytes() { return Depth<KIND>::STAGES * Layout<KIND>::BYTES; }
