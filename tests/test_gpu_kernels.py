@@ -277,6 +277,100 @@ def test_step_kernels_for_fixed_options_match_the_runtime_one(F, acc, pack, wqu,
         assert np.array_equal(host_bits(a.Wq), host_bits(b.Wq))
 
 
+def _outside_fast_range_entries(seed):
+    """Entries whose blocks leave the step's fast range in each way it has:
+    logits above 80 (the direct sigmoid; sigma rounds to 1), logits near -50
+    (sigma ~ 2^-72, so D = S*sigma*s2 is normal but below 2^-60: the IEEE
+    quotient), a tensor whose weights reach 2^60 (A > 2^60), next to ordinary
+    blocks in the same warps."""
+    ents = _entries([(64, 512), (48, 256)], seed, warm=True)
+    e0, e1 = ents
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    q = e0.q
+    q[0:2] = torch.where(torch.rand(q[0:2].shape, generator=g, device="cuda") < 0.5, 95.0, 110.0)
+    q[2:4, ::3] = 81.5
+    q[4:8] = synth.normal(q[4:8].shape, -50.0, 2.0, g, "cuda")
+    e1.W.copy_((e1.W.float() * 2.0 ** 66).to(torch.bfloat16))      # |w| ~ 0.02 * 2^66 > 2^60
+    return ents
+
+
+def test_step_blocks_outside_the_fast_range(F):
+    """Warps with a block outside the fast range take the general code: the
+    forward (W', codes, scales) bit for bit the oracle's outside the rounding
+    band, m, q and the moments within tolerance, through the kernel compiled for
+    the plain step.  The gradients of the 2^66-scaled tensor are 2^66 times an
+    ordinary tensor's, so its moments are compared in units of 2^66 (2^132 for
+    the second moments), where the tolerances mean what they do elsewhere."""
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    ents = _outside_fast_range_entries(230)
+    host_in = [(host_bits(e.W), host_bits(e.dWq), host(e.m).copy(), host(e.q).copy(),
+                [host(x).copy() for x in (e.m_exp_avg, e.m_exp_avg_sq, e.q_exp_avg, e.q_exp_avg_sq)])
+               for e in ents]
+    tab = FocusTable(ents)
+    tab.s2()
+    tab.step(3, hparams())
+    assert F.focus_get_error() == 0
+    for e, (Wb, Gb, m, q, st), f in zip(ents, host_in, (1.0, 2.0 ** 66)):
+        s2 = oracle.s2(Wb)
+        ref_f = oracle.fwd(Wb, m, q, s2)
+        mism = check_forward(ref_f, Wq=host_bits(e.Wq), codes=unpack_codes(host(e.codes)), scales=host(e.scales))
+        skip = block_mask(mism)
+        skq = np.repeat(skip, 2, axis=1)
+        oracle.step(Wb, Gb, m, q, *st, s2, 3, want_wq=False)
+        assert_close(host(e.m), m, "m", skip)
+        assert_close(host(e.q), q, "q", skq)
+        d64 = lambda x: np.asarray(x, np.float64)              # 2^132 does not fit binary32
+        assert_close(d64(host(e.m_exp_avg)) / f, d64(st[0]) / f, "m exp_avg", skip)
+        assert_close(d64(host(e.m_exp_avg_sq)) / f ** 2, d64(st[1]) / f ** 2, "m exp_avg_sq", skip)
+        assert_close(d64(host(e.q_exp_avg)) / f, d64(st[2]) / f, "q exp_avg", skq)
+        assert_close(d64(host(e.q_exp_avg_sq)) / f ** 2, d64(st[3]) / f ** 2, "q exp_avg_sq", skq)
+
+
+def test_step_export_outside_the_fast_range(F):
+    """The same blocks with FOCUS_STEP_PACK_UPDATED (and the tensor maxima): the
+    exported codes and scales are bit for bit what focus_pack_multi writes after
+    a plain step, and W' of the forward and the parameters agree bit for bit."""
+    from fp4_post_weight_b200.table import FocusTable, hparams
+    ea, eb = _outside_fast_range_entries(240), _outside_fast_range_entries(240)
+    ta, tb = FocusTable(ea), FocusTable(eb)
+    ta.s2(); tb.s2()
+    ta.step_s2(2, hparams(), F.FOCUS_STEP_PACK_UPDATED)
+    tb.step(2, hparams())
+    tb.pack()
+    assert F.focus_get_error() == 0
+    for a, b in zip(ea, eb):
+        for name in ("codes", "scales", "m", "q", "m_exp_avg", "m_exp_avg_sq", "q_exp_avg", "q_exp_avg_sq"):
+            assert torch.equal(getattr(a, name), getattr(b, name)), name
+        assert np.array_equal(host_bits(a.Wq), host_bits(b.Wq))
+
+
+def test_round_to_nearest_weights_outside_the_fast_range(F):
+    """Plain NVFP4 round to nearest of weights (its kernel takes the fast code
+    for a warp whose blocks are all in range, else the general one): a tensor
+    with blocks of 2^61-sized weights next to ordinary ones, and a tensor scale
+    outside the fast range, bit for bit the oracle's RTN."""
+    from fp4_post_weight_b200.table import PURPOSE_FOUROVERSIX, Entry, FocusTable
+    g = torch.Generator(device="cuda").manual_seed(250)
+    W0 = synth.normal_bf16((64, 512), 0.02, g, "cuda")
+    W0[::7] = (W0[::7].float() * 2.0 ** 66).to(torch.bfloat16)      # some rows far above the rest
+    W1 = (synth.normal_bf16((16, 256), 0.02, g, "cuda").float() * 2.0 ** -110).to(torch.bfloat16)  # tiny s2
+    ents = [Entry(W=W, m=None, q=None, s2=torch.zeros(1, device="cuda"),
+                  codes=torch.empty((W.shape[0], W.shape[1] // 2), dtype=torch.uint8, device="cuda"),
+                  scales=torch.empty((W.shape[0], W.shape[1] // 16), dtype=torch.uint8, device="cuda"))
+            for W in (W0, W1)]
+    tab = FocusTable(ents, PURPOSE_FOUROVERSIX)
+    tab.s2()
+    tab.nvfp4_rtn()
+    assert F.focus_get_error() == 0
+    for e in ents:
+        Wb = host_bits(e.W)
+        s2 = oracle.s2(Wb)
+        ref = oracle.fwd(Wb, np.ones((Wb.shape[0], Wb.shape[1] // 16), np.float32),
+                         np.full((Wb.shape[0], Wb.shape[1] // 8), 30.0, np.float32), s2)
+        np.testing.assert_array_equal(host(e.scales), ref.scales)
+        np.testing.assert_array_equal(unpack_codes(host(e.codes)), ref.codes)
+
+
 def test_pack_multi_leaves_wq_alone(F):
     from fp4_post_weight_b200.table import FocusTable
     ents = _entries([(16, 256)], 60)
