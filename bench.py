@@ -368,7 +368,7 @@ def measure_next_rows(ents, dev, N, peaks, world):
     out["fouroversix_weights_llama8b"] = r
     # plain NVFP4 round to nearest of the weights (the target 6 alone), codes + scales
     ms = _timed(t_cs.nvfp4_rtn, stream)
-    out["nvfp4_rtn_weights_llama8b"] = {"kernel": "pipe_kernel<KIND_F46> (rtn)", "bytes_per_weight": 2.5625,
+    out["nvfp4_rtn_weights_llama8b"] = {"kernel": "pipe_kernel<KIND_RTN>", "bytes_per_weight": 2.5625,
                                         "Gelem_s": round(N * world / (ms * 1e-3) / 1e9, 2),
                                         **_roof(2.5625 * N, ms, peak)}
     # FourOverSix activations, one scale per token: one launch over the layer's four
