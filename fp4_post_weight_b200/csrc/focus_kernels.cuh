@@ -21,8 +21,13 @@
 // Inside a tile each 16-block is owned by one consumer thread: it takes the
 // block's 32 bytes of W (and of dW') from the stage, its m, its two q and
 // their moments, and does the block's work (A_b, x_b, S_b, the m-gradient and
-// its AdamW update) once.  Outputs go from registers straight to global
-// memory: W' as two 16-byte streaming stores per block, the codes as 8 bytes.
+// its AdamW update) once.  The forward and backward kinds store their outputs
+// from registers straight to global memory (W' as two 16-byte streaming
+// stores per block, the codes as 8 bytes).  The step leaves its outputs in the
+// block's slots of the stage (W' over W, m, q and the moments over theirs, the
+// codes and scales in two regions of their own); the producer writes a full
+// tile out with one bulk copy per array once the consumers release the stage,
+// and each thread of a ragged tile copies its block's out itself.
 //
 // Besides the FOCUS kinds (forward, backward, fused step) the same pipeline
 // runs FourOverSix round to nearest and plain NVFP4 round to nearest of
@@ -70,6 +75,10 @@ enum Kind : int { KIND_FWD = 0, KIND_BWD = 1, KIND_STEP = 2, KIND_F46 = 3, KIND_
 // read W alone.
 __host__ __device__ constexpr bool has_grad(int kind) { return kind == KIND_BWD || kind == KIND_STEP; }
 __host__ __device__ constexpr bool has_mq(int kind) { return kind != KIND_F46 && kind != KIND_RTN; }
+
+// The byte offsets of the input and output regions of one shared-memory stage
+// (defined with the tile engine below).
+template <int KIND> struct Layout;
 
 struct Args {
     const focus_tensor_desc *table;  // device table, or nullptr: use `one`
@@ -253,9 +262,11 @@ __device__ __forceinline__ void encode_block(const TV &T, const uint32_t *w, flo
     }
 }
 
-// w' = bf16(fl(fl(c*S)*s2)) of one block from its two code words and scale byte.
-template <class TV>
-__device__ __forceinline__ void store_wq_from_codes(const TV &T, uint32_t blk, const uint32_t codes[2], uint32_t sbyte) {
+// w' = bf16(fl(fl(c*S)*s2)) of one block from its two code words and scale byte,
+// to global memory, or (SO) to the block's W slot of the stage at so.
+template <bool SO = false, int KIND = KIND_STEP, class TV>
+__device__ __forceinline__ void store_wq_from_codes(const TV &T, uint32_t blk, const uint32_t codes[2], uint32_t sbyte,
+                                                    unsigned char *so = nullptr, uint32_t lb = 0) {
     const uint16_t S_h = (uint16_t)e4m3_normal_f16_bits(sbyte);
     const uint64_t s2_2 = f2_pack(T.s2, T.s2);
 #pragma unroll
@@ -267,7 +278,10 @@ __device__ __forceinline__ void store_wq_from_codes(const TV &T, uint32_t blk, c
             const uint64_t p = f2_mul(f2_pack(mul_f16_exact(lo16(h2), S_h), mul_f16_exact(hi16(h2), S_h)), s2_2);
             o[j] = pack_bf16x2(f2_lo(p), f2_hi(p));
         }
-        __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + (2u * blk + (uint32_t)k), make_uint4(o[0], o[1], o[2], o[3]));
+        if constexpr (SO)
+            reinterpret_cast<uint4 *>(so + Layout<KIND>::W)[2u * lb + (uint32_t)k] = make_uint4(o[0], o[1], o[2], o[3]);
+        else
+            __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + (2u * blk + (uint32_t)k), make_uint4(o[0], o[1], o[2], o[3]));
     }
 }
 
@@ -640,10 +654,11 @@ __device__ __forceinline__ bool block_scalars_fast(const TV &T, float A, float m
 // warp, so the forward's per-element work runs with no range test and no
 // branch.  Otherwise (a lane outside the fast range: rare) the general code,
 // which tests each quantity where it is used.  Both give the same bits.
-template <int KIND, bool WQU, int SF, bool FAST, class TV>
+template <int KIND, bool WQU, int SF, bool FAST, bool SO, class TV>
 __device__ __forceinline__ void block_body(const TV &T, const Args &a, Block &B, float A, bool bad,
-                                           const BlockScalars &f) {
+                                           const BlockScalars &f, unsigned char *so, uint32_t lb) {
     using O = StepOpt<SF>;
+    using L = Layout<KIND>;
     // S_b = e4m3(clamp(fl(fl(A*m)/fl(6*s2)), 2^-6, 448)), scale 1 when the scaled max is 0
     float x, S;
     uint32_t sbyte;
@@ -705,7 +720,8 @@ __device__ __forceinline__ void block_body(const TV &T, const Args &a, Block &B,
             p = f2_mul(cs2[1], s2_2); o.y = pack_bf16x2(f2_lo(p), f2_hi(p));
             p = f2_mul(cs2[2], s2_2); o.z = pack_bf16x2(f2_lo(p), f2_hi(p));
             p = f2_mul(cs2[3], s2_2); o.w = pack_bf16x2(f2_lo(p), f2_hi(p));
-            __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + (2u * B.blk + (uint32_t)k), o);
+            if constexpr (SO) reinterpret_cast<uint4 *>(so + L::W)[2u * lb + (uint32_t)k] = o;
+            else __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + (2u * B.blk + (uint32_t)k), o);
         }
         sq[k] = 0.0f;
         if (has_grad(KIND)) {
@@ -727,11 +743,16 @@ __device__ __forceinline__ void block_body(const TV &T, const Args &a, Block &B,
     }
     // the forward's NVFP4 codes and scale (unless the step exports the updated parameters instead)
     if (B.valid && !(KIND == KIND_STEP && O::pack(a))) {
-        if (T.d.codes) {
-            uint2 cc; cc.x = codes[0]; cc.y = codes[1];
-            reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
+        if constexpr (SO) {
+            reinterpret_cast<uint2 *>(so + L::CODES)[lb] = make_uint2(codes[0], codes[1]);
+            so[L::SCALES + lb] = (uint8_t)sbyte;
+        } else {
+            if (T.d.codes) {
+                uint2 cc; cc.x = codes[0]; cc.y = codes[1];
+                reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
+            }
+            if (T.d.scales) T.d.scales[B.blk] = (uint8_t)sbyte;
         }
-        if (T.d.scales) T.d.scales[B.blk] = (uint8_t)sbyte;
     }
 
     if (has_grad(KIND)) {
@@ -757,7 +778,14 @@ __device__ __forceinline__ void block_body(const TV &T, const Args &a, Block &B,
             uint64_t qp = f2_pack(B.q[0], B.q[1]);
             uint64_t v1 = f2_pack(B.qv1[0], B.qv1[1]), v2 = f2_pack(B.qv2[0], B.qv2[1]);
             adamw_pair(qp, f2_pack(gq0, gq1), v1, v2, a.hp.lr_q_step, a.hp.decay_q, a.hp);
-            if (B.valid) {
+            if constexpr (SO) {                          // over the block's input slots
+                reinterpret_cast<float *>(so + L::M)[lb] = B.m;
+                reinterpret_cast<float *>(so + L::MV1)[lb] = B.mv1;
+                reinterpret_cast<float *>(so + L::MV2)[lb] = B.mv2;
+                reinterpret_cast<uint64_t *>(so + L::Q)[lb] = qp;
+                reinterpret_cast<uint64_t *>(so + L::QV1)[lb] = v1;
+                reinterpret_cast<uint64_t *>(so + L::QV2)[lb] = v2;
+            } else if (B.valid) {
                 T.d.m[B.blk] = B.m;
                 T.d.m_exp_avg[B.blk] = B.mv1;
                 T.d.m_exp_avg_sq[B.blk] = B.mv2;
@@ -773,11 +801,16 @@ __device__ __forceinline__ void block_body(const TV &T, const Args &a, Block &B,
                 uint32_t sb2, codes2[2];
                 encode_block(T, B.w, A, B.m, f2_lo(qp), f2_hi(qp), s64[0], s64[1], q_old0, q_old1, sb2, codes2);
                 if (exp_codes) {
-                    uint2 cc; cc.x = codes2[0]; cc.y = codes2[1];
-                    reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
-                    T.d.scales[B.blk] = (uint8_t)sb2;
+                    if constexpr (SO) {
+                        reinterpret_cast<uint2 *>(so + L::CODES)[lb] = make_uint2(codes2[0], codes2[1]);
+                        so[L::SCALES + lb] = (uint8_t)sb2;
+                    } else {
+                        uint2 cc; cc.x = codes2[0]; cc.y = codes2[1];
+                        reinterpret_cast<uint2 *>(T.d.codes)[B.blk] = cc;
+                        T.d.scales[B.blk] = (uint8_t)sb2;
+                    }
                 }
-                if (exp_wq) store_wq_from_codes(T, B.blk, codes2, sb2);
+                if (exp_wq) store_wq_from_codes<SO>(T, B.blk, codes2, sb2, so, lb);
             }
         }
     }
@@ -790,8 +823,12 @@ __device__ __forceinline__ void block_body(const TV &T, const Args &a, Block &B,
 // the consumer warps pass the stage record in shared memory, so the
 // descriptor's pointers are read where used instead of held in registers.
 // Every lane of the warp calls it (past a ragged end with B.valid false).
-template <int KIND, bool WQU, int SF, class TV>
-__device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block &B) {
+// SO (the step's full tiles): the outputs go to the block's slots of the stage
+// at so (local block lb), which the producer writes out with bulk copies;
+// otherwise straight to global memory.
+template <int KIND, bool WQU, int SF, bool SO = false, class TV>
+__device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block &B, unsigned char *so = nullptr,
+                                              uint32_t lb = 0) {
     using O = StepOpt<SF>;
     if constexpr (KIND == KIND_F46 || KIND == KIND_RTN) {
         compute_block_f46(T, B, KIND == KIND_RTN);
@@ -817,8 +854,8 @@ __device__ __forceinline__ void compute_block(const TV &T, const Args &a, Block 
     // the general code (the lanes of a warp hold neighbouring blocks of one tile)
     BlockScalars f;
     const bool fast = block_scalars_fast(T, A, B.m, B.q[0], B.q[1], f);
-    if (__all_sync(FULL, fast)) block_body<KIND, WQU, SF, true>(T, a, B, A, bad, f);
-    else block_body<KIND, WQU, SF, false>(T, a, B, A, bad, f);
+    if (__all_sync(FULL, fast)) block_body<KIND, WQU, SF, true, SO>(T, a, B, A, bad, f, so, lb);
+    else block_body<KIND, WQU, SF, false, SO>(T, a, B, A, bad, f, so, lb);
     if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_error_flags, 1u);
 }
 
@@ -841,10 +878,14 @@ struct Layout {
     static constexpr uint32_t QV2 = QV1 + (ST ? TILE_BLOCKS * 8 : 0);
     static constexpr uint32_t GM = QV2 + (ST ? TILE_BLOCKS * 8 : 0);
     static constexpr uint32_t GQ = GM + (G_ ? TILE_BLOCKS * 4 : 0);
-    static constexpr uint32_t BYTES = GQ + (G_ ? TILE_BLOCKS * 8 : 0);   // one stage
+    static constexpr uint32_t IN_END = GQ + (G_ ? TILE_BLOCKS * 8 : 0);  // end of the inputs
+    // the step's outputs that have no input slot to take over: codes and scales
+    static constexpr uint32_t CODES = IN_END;
+    static constexpr uint32_t SCALES = CODES + (ST ? TILE_BLOCKS * 8 : 0);
+    static constexpr uint32_t BYTES = SCALES + (ST ? TILE_BLOCKS : 0);     // one stage
     // bytes the bulk copies of one full tile deliver
     static __device__ __forceinline__ uint32_t tx_bytes(bool accumulate) {
-        return (accumulate || !G_) ? BYTES : GM;
+        return (accumulate || !G_) ? IN_END : GM;
     }
 };
 
@@ -952,7 +993,30 @@ __device__ __forceinline__ bool seek_tensor(const Args &a, int64_t tile, int &t,
     return tile < T.tile_end;
 }
 
-// The producer: one thread feeding the ring.
+// The outputs a full tile of the step left in its stage, written to global
+// memory with bulk copies (one group): W' over W, the parameters and moments
+// over theirs, the codes and scales from their own regions.  Each array the
+// descriptor has is written whole: the step writes every block of a full tile.
+__device__ __forceinline__ void store_step_tile(const StageInfo &inf, const unsigned char *stage) {
+    using L = Layout<KIND_STEP>;
+    const focus_tensor_desc &d = inf.d;
+    const uint32_t f = inf.first;
+    if (d.Wq) bulk_s2g(reinterpret_cast<uint4 *>(d.Wq) + 2u * f, smem_u32(stage + L::W), TILE_BLOCKS * 32);
+    if (d.codes) {
+        bulk_s2g(d.codes + 8u * f, smem_u32(stage + L::CODES), TILE_BLOCKS * 8);
+        bulk_s2g(d.scales + f, smem_u32(stage + L::SCALES), TILE_BLOCKS);
+    }
+    bulk_s2g(d.m + f, smem_u32(stage + L::M), TILE_BLOCKS * 4);
+    bulk_s2g(d.m_exp_avg + f, smem_u32(stage + L::MV1), TILE_BLOCKS * 4);
+    bulk_s2g(d.m_exp_avg_sq + f, smem_u32(stage + L::MV2), TILE_BLOCKS * 4);
+    bulk_s2g(d.q + 2u * f, smem_u32(stage + L::Q), TILE_BLOCKS * 8);
+    bulk_s2g(d.q_exp_avg + 2u * f, smem_u32(stage + L::QV1), TILE_BLOCKS * 8);
+    bulk_s2g(d.q_exp_avg_sq + 2u * f, smem_u32(stage + L::QV2), TILE_BLOCKS * 8);
+    bulk_commit();
+}
+
+// The producer: one thread feeding the ring (and, for the step, writing the
+// outputs of each full tile from its stage before the stage takes the next).
 template <int KIND, int SF>
 __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint64_t *full, uint64_t *empty,
                                         StageInfo *info) {
@@ -980,6 +1044,11 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
         if (KIND == KIND_STEP && O::amax(a)) {
             if (it >= (uint32_t)S) fold.add(a.amax_ws, inf.tensor, inf.amax);   // the stage's previous tile
             inf.amax = 0u;
+        }
+        if (KIND == KIND_STEP && it >= (uint32_t)S && inf.mode == MODE_BULK) {
+            // the previous tile's outputs leave the stage before it is filled again
+            store_step_tile(inf, smem + st * L::BYTES);
+            bulk_wait_read();
         }
         const bool found = seek_tensor(a, tile, t, T, have);
         const uint32_t first = found ? (uint32_t)(tile - T.d.tile_begin) * TILE_BLOCKS : 0u;
@@ -1038,19 +1107,23 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
             mbar_arrive(bar);
         }
     }
-    // The tensor maxima of the last uses of the stages: wait (bounded) until the
-    // consumers have released them, fold them in and write the running maximum.
-    if (KIND == KIND_STEP && O::amax(a) && !timed_out) {
+    // The last uses of the stages: wait (bounded) until the consumers have
+    // released them, fold in their tensor maxima and write the running maximum,
+    // and write the outputs of the full tiles; then wait until every bulk store
+    // has completed.
+    if (KIND == KIND_STEP && !timed_out) {
         for (uint32_t j = it > (uint32_t)S ? it - (uint32_t)S : 0u; j < it; ++j) {
             const uint32_t st = j % S;
             if (!mbar_wait(smem_u32(&empty[st]), (j / S) & 1u)) {
                 atomicOr(&g_error_flags, 8u);
                 break;
             }
-            fold.add(a.amax_ws, info[st].tensor, info[st].amax);
+            if (O::amax(a)) fold.add(a.amax_ws, info[st].tensor, info[st].amax);
+            if (info[st].mode == MODE_BULK) store_step_tile(info[st], smem + st * L::BYTES);
         }
-        fold.flush(a.amax_ws);
+        if (O::amax(a)) fold.flush(a.amax_ws);
     }
+    if (KIND == KIND_STEP) bulk_wait_all();
     // Before the CTA may exit, every bulk copy it issued must have landed (normally
     // the consumers already waited for all of them; this matters after a timeout).
     for (int st = 0; st < S; ++st)
@@ -1058,9 +1131,34 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
             if (!mbar_wait(smem_u32(&full[st]), (pending_parity >> st) & 1u)) atomicOr(&g_error_flags, 8u);
 }
 
+// A ragged tile's block of the step: its outputs, left in the block's slots
+// of the stage, to global memory (what store_step_tile does for a full tile;
+// nothing for the blocks past the tensor's end).
+template <bool WQU, int SF>
+__device__ __forceinline__ void copy_out_step_block(const StageInfo &T, const Args &a, const Block &B,
+                                                    const unsigned char *so, uint32_t lb) {
+    using L = Layout<KIND_STEP>;
+    if (!B.valid) return;
+    const uint32_t blk = B.blk;
+    if (T.d.Wq) {
+        __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + 2u * blk, reinterpret_cast<const uint4 *>(so + L::W)[2u * lb]);
+        __stcs(reinterpret_cast<uint4 *>(T.d.Wq) + 2u * blk + 1u, reinterpret_cast<const uint4 *>(so + L::W)[2u * lb + 1u]);
+    }
+    if (T.d.codes) {
+        reinterpret_cast<uint2 *>(T.d.codes)[blk] = reinterpret_cast<const uint2 *>(so + L::CODES)[lb];
+        T.d.scales[blk] = so[L::SCALES + lb];
+    }
+    T.d.m[blk] = reinterpret_cast<const float *>(so + L::M)[lb];
+    T.d.m_exp_avg[blk] = reinterpret_cast<const float *>(so + L::MV1)[lb];
+    T.d.m_exp_avg_sq[blk] = reinterpret_cast<const float *>(so + L::MV2)[lb];
+    reinterpret_cast<uint64_t *>(T.d.q)[blk] = reinterpret_cast<const uint64_t *>(so + L::Q)[lb];
+    reinterpret_cast<uint64_t *>(T.d.q_exp_avg)[blk] = reinterpret_cast<const uint64_t *>(so + L::QV1)[lb];
+    reinterpret_cast<uint64_t *>(T.d.q_exp_avg_sq)[blk] = reinterpret_cast<const uint64_t *>(so + L::QV2)[lb];
+}
+
 // The consumers: NC_WARPS warps computing from the ring.
 template <int KIND, bool WQU, int SF>
-__device__ __forceinline__ void consume(const Args &a, const unsigned char *smem, uint64_t *full, uint64_t *empty,
+__device__ __forceinline__ void consume(const Args &a, unsigned char *smem, uint64_t *full, uint64_t *empty,
                                         const StageInfo *info) {
     using L = Layout<KIND>;
     constexpr int S = Depth<KIND>::STAGES;
@@ -1076,12 +1174,21 @@ __device__ __forceinline__ void consume(const Args &a, const unsigned char *smem
         const StageInfo &inf = info[st];
         const uint32_t mode = inf.mode;
         if (mode != MODE_SKIP) {
-            const unsigned char *stage = smem + st * L::BYTES;
+            unsigned char *stage = smem + st * L::BYTES;
             const uint32_t lb = threadIdx.x;
             Block B;
             if (mode == MODE_BULK) load_block_smem<KIND, SF>(a, stage, B, lb, inf.first + lb);
             else load_block_global<KIND, SF>(inf, a, B, inf.first + lb);
-            compute_block<KIND, WQU, SF>(inf, a, B);
+            if constexpr (KIND == KIND_STEP) {
+                // the step leaves its outputs in the stage: the producer writes a
+                // full tile out with bulk copies, each thread a ragged tile's block
+                // (the stage is free: a ragged tile was read from global memory)
+                compute_block<KIND, WQU, SF, true>(inf, a, B, stage, lb);
+                if (mode == MODE_BULK) fence_proxy_async_smem();
+                else copy_out_step_block<WQU, SF>(inf, a, B, stage, lb);
+            } else {
+                compute_block<KIND, WQU, SF>(inf, a, B);
+            }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&empty[st]));

@@ -4,8 +4,11 @@
 // producer thread issues 1-D bulk asynchronous copies (cp.async.bulk, global
 // to shared, completion counted in bytes on an mbarrier) and consumer warps
 // compute from the staged data, releasing each stage through a second
-// mbarrier.  No copy uses cluster multicast: every copy reads this GPU's own
-// global memory into the issuing CTA's shared memory.
+// mbarrier.  Where the consumers leave their outputs in the stage, the
+// producer writes them out with bulk copies the other way (shared to global,
+// completion tracked by bulk groups) before it fills the stage again.  No copy
+// uses cluster multicast: every copy reads or writes this GPU's own global
+// memory and the issuing CTA's shared memory.
 //
 // Every wait is bounded: after WAIT_LIMIT_NS of wall time (read from
 // %globaltimer), or a hard iteration cap, it gives up and returns false; the
@@ -96,6 +99,25 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from
+// this CTA's shared memory to global memory, in the thread's current bulk
+// group.
+__device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until every bulk group of this thread has finished reading its shared
+// memory source (the stage may then be written again).
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until every bulk group of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Makes this thread's writes to shared memory visible to later bulk copies
+// (the asynchronous proxy) that read it.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 }  // namespace focus
