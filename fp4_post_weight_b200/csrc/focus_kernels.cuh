@@ -1045,10 +1045,12 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
             if (it >= (uint32_t)S) fold.add(a.amax_ws, inf.tensor, inf.amax);   // the stage's previous tile
             inf.amax = 0u;
         }
+        // the previous tile's outputs leave the stage before those regions are
+        // filled again (the regions no output uses are refilled at once)
+        bool read_wait = false;
         if (KIND == KIND_STEP && it >= (uint32_t)S && inf.mode == MODE_BULK) {
-            // the previous tile's outputs leave the stage before it is filled again
             store_step_tile(inf, smem + st * L::BYTES);
-            bulk_wait_read();
+            read_wait = true;
         }
         const bool found = seek_tensor(a, tile, t, T, have);
         const uint32_t first = found ? (uint32_t)(tile - T.d.tile_begin) * TILE_BLOCKS : 0u;
@@ -1083,10 +1085,15 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
             unsigned char *stage = smem + st * L::BYTES;
             const uint32_t f = first;
             mbar_arrive_expect_tx(bar, L::tx_bytes(O::acc(a)));
-            bulk_g2s(smem_u32(stage + L::W), reinterpret_cast<const uint4 *>(T.d.W) + 2u * f, TILE_BLOCKS * 32, bar);
             if (has_grad(KIND))
                 bulk_g2s(smem_u32(stage + L::G), reinterpret_cast<const uint4 *>(T.d.dWq) + 2u * f, TILE_BLOCKS * 32,
                          bar);
+            if (has_grad(KIND) && O::acc(a)) {
+                bulk_g2s(smem_u32(stage + L::GM), T.d.dm + f, TILE_BLOCKS * 4, bar);
+                bulk_g2s(smem_u32(stage + L::GQ), T.d.dq + 2u * f, TILE_BLOCKS * 8, bar);
+            }
+            if (read_wait) bulk_wait_read();
+            bulk_g2s(smem_u32(stage + L::W), reinterpret_cast<const uint4 *>(T.d.W) + 2u * f, TILE_BLOCKS * 32, bar);
             if (has_mq(KIND)) {
                 bulk_g2s(smem_u32(stage + L::M), T.d.m + f, TILE_BLOCKS * 4, bar);
                 bulk_g2s(smem_u32(stage + L::Q), T.d.q + 2u * f, TILE_BLOCKS * 8, bar);
@@ -1097,13 +1104,11 @@ __device__ __forceinline__ void produce(const Args &a, unsigned char *smem, uint
                 bulk_g2s(smem_u32(stage + L::QV1), T.d.q_exp_avg + 2u * f, TILE_BLOCKS * 8, bar);
                 bulk_g2s(smem_u32(stage + L::QV2), T.d.q_exp_avg_sq + 2u * f, TILE_BLOCKS * 8, bar);
             }
-            if (has_grad(KIND) && O::acc(a)) {
-                bulk_g2s(smem_u32(stage + L::GM), T.d.dm + f, TILE_BLOCKS * 4, bar);
-                bulk_g2s(smem_u32(stage + L::GQ), T.d.dq + 2u * f, TILE_BLOCKS * 8, bar);
-            }
             pending |= 1u << st;
             pending_parity = (pending_parity & ~(1u << st)) | (ph << st);
         } else {
+            // (a ragged tile's consumers write their outputs into the stage)
+            if (read_wait) bulk_wait_read();
             mbar_arrive(bar);
         }
     }
